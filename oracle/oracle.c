@@ -1,0 +1,517 @@
+/*
+ * oracle.c - plain, slow CPU oracle for the skew-resilient routed-expert MoE
+ * layer: router top-k and gating, expert-load histogram, greedy replication
+ * planner, tile layout, row maps, dispatch, SwiGLU expert FFN and weighted
+ * combine, plus a dense compute-every-expert-then-mask reference.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg load this library. It shares no code with the
+ * CUDA library and neither one calls the other.
+ *
+ * Sources, cited by page title and section:
+ *   [MegaFlux]  "MegaFlux: Skew-Resilient MoE Megakernels via Pipelined
+ *               Expert Replication"
+ *   [MoonEP]    "MoonEP routing flow - live" (an explainer of MoonEP's
+ *               planning kernel)
+ *
+ * Where the pages leave a step open, the reading taken is marked READING.
+ * Single-threaded plain loops; floating point in fp64. Rounding points
+ * (round_mode) mirror where the GPU path stores a narrower type:
+ *   ORC_ROUND_NONE  no rounding anywhere (pure fp64),
+ *   ORC_ROUND_F32   H, Yp and out stored as fp32,
+ *   ORC_ROUND_BF16  H, Yp and out rounded to bf16 (nearest even).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { ORC_BF16 = 0, ORC_FP32 = 1 };
+enum { ORC_GATE_SOFTMAX_TOPK = 0, ORC_GATE_SIGMOID_TOPK = 1 };
+enum { ORC_ROUND_NONE = 0, ORC_ROUND_F32 = 1, ORC_ROUND_BF16 = 2 };
+enum { ORC_PLAN_INEXACT = 1u };
+enum { ORC_OK = 0, ORC_ERR_ARG = 1, ORC_ERR_INTERNAL = 2 };
+
+typedef struct { int32_t expert, rank, start, len, row0; } orc_piece;
+typedef struct { int32_t expert, row0, valid, rank; } orc_block;
+
+/* ---------------------------------------------------------------- numbers */
+
+static double bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+/* Round a double to the nearest bf16 (8 significant bits), ties to even. */
+static uint16_t double_to_bf16(double v)
+{
+    if (v == 0.0) {
+        float z = (float)v; /* keeps the sign of zero */
+        uint32_t u;
+        memcpy(&u, &z, 4);
+        return (uint16_t)(u >> 16);
+    }
+    int e;
+    double m = frexp(v, &e);            /* |m| in [0.5, 1) */
+    double r = nearbyint(ldexp(m, 8));  /* 8 significant bits, ties to even */
+    float f = (float)ldexp(r, e - 8);   /* exact: r has at most 9 bits */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    return (uint16_t)(u >> 16);
+}
+
+static double round_as(double v, int round_mode)
+{
+    if (round_mode == ORC_ROUND_BF16) return bf16_to_double(double_to_bf16(v));
+    if (round_mode == ORC_ROUND_F32) return (double)(float)v;
+    return v;
+}
+
+static double load_elem(const void* p, int64_t i, int dtype)
+{
+    if (dtype == ORC_BF16) return bf16_to_double(((const uint16_t*)p)[i]);
+    return (double)((const float*)p)[i];
+}
+
+static void store_elem(void* p, int64_t i, int dtype, double v)
+{
+    if (dtype == ORC_BF16) ((uint16_t*)p)[i] = double_to_bf16(v);
+    else ((float*)p)[i] = (float)v;
+}
+
+/* ------------------------------------------------- top-k and gating (A1, A2)
+ * [MegaFlux] §1: a learned router selects a small set of experts per token
+ * and their outputs are combined by the routing weights; §4.1 "Routing
+ * workload construction": each token has k distinct experts.
+ * READING: the K largest logits, in descending order, ties to the lower
+ * expert id. Gating (softmax or sigmoid, normalised over the chosen k) is
+ * taken on the same logits that choose the experts.
+ */
+int orc_topk_gate(int64_t T, int32_t E, int32_t K, int32_t gating,
+                  const float* logits, int32_t* idx, float* w)
+{
+    if (T < 0 || E <= 0 || K <= 0 || K > E) return ORC_ERR_ARG;
+    char* taken = (char*)malloc((size_t)E);
+    double* g = (double*)malloc(sizeof(double) * (size_t)K);
+    if (!taken || !g) { free(taken); free(g); return ORC_ERR_INTERNAL; }
+    for (int64_t t = 0; t < T; ++t) {
+        const float* l = logits + t * E;
+        memset(taken, 0, (size_t)E);
+        for (int k = 0; k < K; ++k) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || l[e] > l[best]) best = e;   /* strict: lower id wins ties */
+            }
+            taken[best] = 1;
+            idx[t * K + k] = best;
+        }
+        double sum = 0.0;
+        for (int k = 0; k < K; ++k) {
+            double lk = (double)l[idx[t * K + k]];
+            if (gating == ORC_GATE_SOFTMAX_TOPK) {
+                g[k] = exp(lk - (double)l[idx[t * K]]);     /* softmax, renormalised over top-k */
+            } else {
+                g[k] = 1.0 / (1.0 + exp(-lk));              /* sigmoid, normalised over top-k */
+            }
+            sum += g[k];
+        }
+        for (int k = 0; k < K; ++k) w[t * K + k] = (float)(g[k] / sum);
+    }
+    free(taken);
+    free(g);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- histogram (A3)
+ * [MegaFlux] §3.1 and App. A.1: the planner's input is the routing profile,
+ * the per-expert load. Here the load is counted in routed entries.
+ */
+int orc_histogram(int64_t n_entries, int32_t E, const int32_t* idx, int32_t* counts)
+{
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t i = 0; i < n_entries; ++i) {
+        if (idx[i] < 0 || idx[i] >= E) return ORC_ERR_ARG;
+        counts[idx[i]] += 1;
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- planner (A4) and layout
+ * [MoonEP] "Per-expert breakdown": every rank's capacity is S*K entries and
+ * its surplus is the sum of its experts' loads minus that capacity.
+ * [MoonEP] "The greedy balance, step by step": each move refills the
+ * currently hungriest rank in one shot from the currently biggest donor; the
+ * donor may overshoot into deficit and is then refilled by a later move; a
+ * move slices off the donor's biggest experts; every slice of a foreign
+ * expert ships one weight copy.
+ * [MegaFlux] §3.1 "Bounded greedy search" / App. A.1: the search starts from
+ * the no-replica assignment (every expert on its owner); §4.1: each GPU has
+ * capacity for a fixed number of extra replicas (the budget).
+ * [MegaFlux] §3.1 "Problem formulation": token blocks of at most beta rows
+ * match the FC1/FC2 token tile.
+ *
+ * READINGS:
+ *  - owner(e) = e / (E/R) (contiguous expert ownership).
+ *  - hungriest = lowest load, biggest donor = highest load, biggest expert =
+ *    largest remaining rows; every tie goes to the lowest index.
+ *  - a slice is the tail of the rows the donor still holds of that expert,
+ *    so the owner keeps a prefix; pieces of one expert partition its list.
+ *  - a receiver that has used its budget takes no new slice; if the
+ *    hungriest rank can take nothing, planning stops and the plan is
+ *    flagged inexact (still a valid partition of all entries).
+ *  - cut points are per entry (every rank gets exactly S*K entries when the
+ *    plan is exact); each piece is then padded to whole beta-row tiles at a
+ *    beta-aligned row, pieces laid out in (rank, expert) order.
+ */
+int orc_plan(int64_t T, int32_t E, int32_t K, int32_t R, int32_t tile, int32_t budget,
+             const int32_t* counts,
+             orc_piece* pieces, int32_t* n_pieces,
+             orc_block* blocks, int32_t* n_blocks,
+             int64_t* rank_load, int32_t* rank_replicas, int64_t* rank_row0,
+             int32_t* moves_out, uint32_t* status)
+{
+    if (R <= 0 || E <= 0 || E % R != 0 || T % R != 0 || tile <= 0 || budget < 0)
+        return ORC_ERR_ARG;
+    const int64_t C = (T / R) * (int64_t)K;       /* per-rank capacity S*K */
+    const int32_t per = E / R;                    /* experts owned per rank */
+
+    int64_t* rem = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+    int64_t* L = (int64_t*)calloc((size_t)R, sizeof(int64_t));
+    int32_t* used = (int32_t*)calloc((size_t)R, sizeof(int32_t));
+    int64_t* p_start = (int64_t*)calloc((size_t)R * E, sizeof(int64_t));
+    int64_t* p_len = (int64_t*)calloc((size_t)R * E, sizeof(int64_t));
+    if (!rem || !L || !used || !p_start || !p_len) {
+        free(rem); free(L); free(used); free(p_start); free(p_len);
+        return ORC_ERR_INTERNAL;
+    }
+    int rc = ORC_OK;
+    uint32_t st = 0;
+
+    /* no-replica start: every expert's whole list is held by its owner */
+    for (int e = 0; e < E; ++e) {
+        rem[e] = counts[e];
+        L[e / per] += counts[e];
+    }
+
+    int32_t moves = 0;
+    const int32_t cap = R * R + E;               /* backstop; a move settles a rank */
+    for (;;) {
+        int recv = 0;
+        for (int r = 1; r < R; ++r) if (L[r] < L[recv]) recv = r;
+        if (L[recv] >= C) break;                 /* sum is R*C, so all equal C */
+        if (moves == cap) { st |= ORC_PLAN_INEXACT; break; }
+        int donor = 0;
+        for (int r = 1; r < R; ++r) if (L[r] > L[donor]) donor = r;
+
+        int64_t phi_before = 0;
+        for (int r = 0; r < R; ++r) phi_before += llabs(L[r] - C);
+
+        int64_t need = C - L[recv];
+        int64_t gave = 0;
+        while (need > 0) {
+            int e_best = -1;
+            for (int e = donor * per; e < (donor + 1) * per; ++e) {
+                if (rem[e] <= 0) continue;
+                if (e_best < 0 || rem[e] > rem[e_best]) e_best = e;
+            }
+            if (e_best < 0) break;               /* donor has nothing left */
+            if (used[recv] >= budget) break;     /* a new replica is not allowed */
+            if (p_len[(size_t)recv * E + e_best] != 0) { rc = ORC_ERR_INTERNAL; goto done; }
+            int64_t x = rem[e_best] < need ? rem[e_best] : need;
+            p_start[(size_t)recv * E + e_best] = rem[e_best] - x;
+            p_len[(size_t)recv * E + e_best] = x;
+            used[recv] += 1;
+            rem[e_best] -= x;
+            need -= x;
+            L[donor] -= x;
+            L[recv] += x;
+            gave += x;
+        }
+        if (gave == 0) { st |= ORC_PLAN_INEXACT; break; }
+        moves += 1;
+
+        int64_t phi_after = 0;
+        for (int r = 0; r < R; ++r) phi_after += llabs(L[r] - C);
+        if (phi_after >= phi_before) { rc = ORC_ERR_INTERNAL; goto done; }
+    }
+
+    /* what the owners still hold: a prefix of each expert's list */
+    for (int e = 0; e < E; ++e) {
+        if (rem[e] > 0) {
+            int o = e / per;
+            p_start[(size_t)o * E + e] = 0;
+            p_len[(size_t)o * E + e] = rem[e];
+        }
+    }
+
+    /* tile layout: pieces in (rank, expert) order, each padded to whole tiles */
+    {
+        int32_t np = 0, nb = 0;
+        int64_t row = 0;
+        for (int r = 0; r < R; ++r) {
+            rank_row0[r] = row;
+            rank_load[r] = 0;
+            rank_replicas[r] = used[r];
+            for (int e = 0; e < E; ++e) {
+                int64_t len = p_len[(size_t)r * E + e];
+                if (len == 0) continue;
+                orc_piece* p = &pieces[np++];
+                p->expert = e;
+                p->rank = r;
+                p->start = (int32_t)p_start[(size_t)r * E + e];
+                p->len = (int32_t)len;
+                p->row0 = (int32_t)row;
+                int64_t ntiles = (len + tile - 1) / tile;
+                for (int64_t i = 0; i < ntiles; ++i) {
+                    orc_block* b = &blocks[nb++];
+                    b->expert = e;
+                    b->row0 = (int32_t)(row + i * tile);
+                    b->valid = (int32_t)((len - i * tile) < tile ? (len - i * tile) : tile);
+                    b->rank = r;
+                }
+                row += ntiles * tile;
+                rank_load[r] += len;
+            }
+        }
+        rank_row0[R] = row;
+        *n_pieces = np;
+        *n_blocks = nb;
+    }
+    *moves_out = moves;
+    *status = st;
+done:
+    free(rem); free(L); free(used); free(p_start); free(p_len);
+    return rc;
+}
+
+/* ------------------------------------------------- row maps (A5)
+ * [MegaFlux] App. A.2 "Mapping blocks to routed assignments": within each
+ * expert, routed assignments are ordered by source GPU and then local
+ * (token, top-k position), and cut into the planned blocks. READING: the
+ * source rank of token t is t / S, so the order is plain (t, k) order.
+ * pos(t,k) = number of earlier entries with the same expert; the entry goes
+ * to the piece of its expert whose [start, start+len) holds pos.
+ */
+int orc_row_maps(int64_t T, int32_t K, int32_t E, const int32_t* idx,
+                 const orc_piece* pieces, int32_t n_pieces,
+                 int64_t rows_cap, int32_t* row_of, int32_t* src_of)
+{
+    int64_t* seen = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+    if (!seen) return ORC_ERR_INTERNAL;
+    for (int64_t r = 0; r < rows_cap; ++r) src_of[r] = -1;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int k = 0; k < K; ++k) {
+            int e = idx[t * K + k];
+            int64_t pos = seen[e]++;
+            int found = -1;
+            for (int p = 0; p < n_pieces; ++p) {
+                if (pieces[p].expert == e && pieces[p].start <= pos &&
+                    pos < (int64_t)pieces[p].start + pieces[p].len) { found = p; break; }
+            }
+            if (found < 0) { free(seen); return ORC_ERR_ARG; }
+            int64_t row = pieces[found].row0 + (pos - pieces[found].start);
+            if (row >= rows_cap) { free(seen); return ORC_ERR_ARG; }
+            row_of[t * K + k] = (int32_t)row;
+            src_of[row] = (int32_t)t;
+        }
+    }
+    free(seen);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- dispatch (A6)
+ * [MegaFlux] §1: routed activations are sent to the GPUs hosting the
+ * selected experts. On one GPU the send is a copy of token rows into the
+ * expert-major buffer; padding rows are zero.
+ */
+int orc_dispatch(int64_t rows, int32_t d, int32_t dtype, const void* x,
+                 const int32_t* src_of, void* xp)
+{
+    const size_t eb = dtype == ORC_BF16 ? 2 : 4;   /* a copy of the element's bytes */
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t i = 0; i < d; ++i) {
+            char* dst = (char*)xp + ((size_t)r * d + i) * eb;
+            if (src_of[r] >= 0)
+                memcpy(dst, (const char*)x + ((size_t)src_of[r] * d + i) * eb, eb);
+            else
+                memset(dst, 0, eb);
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- expert FFN (A7, A8)
+ * [MegaFlux] §4.1: SwiGLU experts; §2.1 and §3.2 "Forward": FC1 (input
+ * projection, W1) then FC2 (output projection, W2) per token block.
+ * READING: W1 = [gate; up] stacked as w_gate_up[e] of shape [2F, d], rows
+ * 0..F-1 gate and F..2F-1 up; W2 = w_down[e] of shape [d, F];
+ * h = silu(x.gate) * (x.up), silu(a) = a / (1 + exp(-a)); y = h . W2.
+ * One row of the expert FFN in fp64; h and y are rounded per round_mode.
+ */
+static void ffn_row(int32_t d, int32_t F, int32_t dtype, int32_t round_mode,
+                    const void* xrow_src, int64_t xrow_off,
+                    const void* w_gu, const void* w_down, int32_t e,
+                    double* h /*[F]*/, double* y /*[d]*/)
+{
+    const int64_t gu_base = (int64_t)e * 2 * F * d;
+    const int64_t dn_base = (int64_t)e * d * F;
+    for (int32_t j = 0; j < F; ++j) {
+        double a = 0.0, g = 0.0;
+        for (int32_t i = 0; i < d; ++i) {
+            double xv = load_elem(xrow_src, xrow_off + i, dtype);
+            a += xv * load_elem(w_gu, gu_base + (int64_t)j * d + i, dtype);
+            g += xv * load_elem(w_gu, gu_base + (int64_t)(F + j) * d + i, dtype);
+        }
+        double silu = a / (1.0 + exp(-a));
+        h[j] = round_as(silu * g, round_mode);
+    }
+    for (int32_t i = 0; i < d; ++i) {
+        double s = 0.0;
+        for (int32_t j = 0; j < F; ++j)
+            s += h[j] * load_elem(w_down, dn_base + (int64_t)i * F + j, dtype);
+        y[i] = round_as(s, round_mode);
+    }
+}
+
+/* H and Yp for every row of every planned block; padding rows are zero. */
+int orc_expert_ffn(int32_t d, int32_t F, int32_t dtype, int32_t round_mode, int32_t tile,
+                   const orc_block* blocks, int32_t n_blocks,
+                   const void* xp, const void* w_gu, const void* w_down,
+                   void* h_out, void* yp_out)
+{
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    double* y = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!h || !y) { free(h); free(y); return ORC_ERR_INTERNAL; }
+    for (int32_t b = 0; b < n_blocks; ++b) {
+        for (int32_t r = 0; r < tile; ++r) {
+            int64_t row = (int64_t)blocks[b].row0 + r;
+            if (r < blocks[b].valid) {
+                ffn_row(d, F, dtype, round_mode, xp, row * d, w_gu, w_down,
+                        blocks[b].expert, h, y);
+            } else {
+                for (int32_t j = 0; j < F; ++j) h[j] = 0.0;
+                for (int32_t i = 0; i < d; ++i) y[i] = 0.0;
+            }
+            for (int32_t j = 0; j < F; ++j) store_elem(h_out, row * F + j, dtype, h[j]);
+            for (int32_t i = 0; i < d; ++i) store_elem(yp_out, row * d + i, dtype, y[i]);
+        }
+    }
+    free(h);
+    free(y);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- combine (A9)
+ * [MegaFlux] §1: expert outputs are combined according to the routing
+ * weights; §2.1: the final top-k sum is its own launch.
+ * out[t] = sum over k, in k order, of w[t,k] * Yp[row_of(t,k)].
+ */
+int orc_combine(int64_t T, int32_t K, int32_t d, int32_t dtype, int32_t round_mode,
+                const void* yp, const int32_t* row_of, const float* w, void* out)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int32_t k = 0; k < K; ++k)
+                s += (double)w[t * K + k] * load_elem(yp, (int64_t)row_of[t * K + k] * d + i, dtype);
+            store_elem(out, t * d + i, dtype, round_as(s, round_mode));
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- one token's layer output
+ * The same arithmetic as dispatch + FFN + combine for one token, taken
+ * straight from x: the plan only decides which rows hold a token's copies,
+ * never their values. Used to check sampled tokens of large layers.
+ */
+int orc_token_out(int32_t d, int32_t F, int32_t K, int32_t dtype, int32_t round_mode,
+                  int64_t n_tok, const int64_t* tokens,
+                  const void* x, const int32_t* idx, const float* w,
+                  const void* w_gu, const void* w_down, double* out /*[n_tok, d]*/)
+{
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    double* y = (double*)malloc(sizeof(double) * (size_t)d * K);
+    if (!h || !y) { free(h); free(y); return ORC_ERR_INTERNAL; }
+    for (int64_t n = 0; n < n_tok; ++n) {
+        int64_t t = tokens[n];
+        for (int32_t k = 0; k < K; ++k)
+            ffn_row(d, F, dtype, round_mode, x, t * d, w_gu, w_down, idx[t * K + k], h,
+                    y + (size_t)k * d);
+        for (int32_t i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int32_t k = 0; k < K; ++k) s += (double)w[t * K + k] * y[(size_t)k * d + i];
+            out[n * d + i] = round_as(s, round_mode);
+        }
+    }
+    free(h);
+    free(y);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------- dense reference
+ * The plain definition of the routed layer: run every expert on every
+ * token in fp64 and add expert e's output with weight gate(t,e) when e is
+ * among the token's top-k, else zero. Membership is decided by rank
+ * counting (e is chosen when fewer than K experts beat it, a higher logit
+ * or an equal logit at a lower id), and the weight is the full softmax (or
+ * the sigmoid) renormalised over the chosen set. Inputs are fp64 arrays.
+ */
+int orc_dense_layer(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32_t gating,
+                    const double* logits, const double* x, const double* w_gu,
+                    const double* w_down, double* out)
+{
+    double* p = (double*)malloc(sizeof(double) * (size_t)E);
+    char* chosen = (char*)malloc((size_t)E);
+    double* h = (double*)malloc(sizeof(double) * (size_t)F);
+    if (!p || !chosen || !h) { free(p); free(chosen); free(h); return ORC_ERR_INTERNAL; }
+    for (int64_t t = 0; t < T; ++t) {
+        const double* l = logits + t * E;
+        double mx = l[0];
+        for (int e = 1; e < E; ++e) if (l[e] > mx) mx = l[e];
+        double z = 0.0;
+        for (int e = 0; e < E; ++e) {
+            p[e] = gating == ORC_GATE_SOFTMAX_TOPK ? exp(l[e] - mx) : 1.0 / (1.0 + exp(-l[e]));
+            z += p[e];
+        }
+        if (gating == ORC_GATE_SOFTMAX_TOPK) for (int e = 0; e < E; ++e) p[e] /= z;
+        double zsel = 0.0;
+        for (int e = 0; e < E; ++e) {
+            int beaten_by = 0;
+            for (int j = 0; j < E; ++j)
+                if (l[j] > l[e] || (l[j] == l[e] && j < e)) beaten_by++;
+            chosen[e] = beaten_by < K;
+            if (chosen[e]) zsel += p[e];
+        }
+        for (int32_t i = 0; i < d; ++i) out[t * d + i] = 0.0;
+        for (int e = 0; e < E; ++e) {
+            double gate = chosen[e] ? p[e] / zsel : 0.0;
+            const double* wg = w_gu + (int64_t)e * 2 * F * d;
+            const double* wd = w_down + (int64_t)e * d * F;
+            for (int32_t j = 0; j < F; ++j) {
+                double a = 0.0, g = 0.0;
+                for (int32_t i = 0; i < d; ++i) {
+                    a += x[t * d + i] * wg[(int64_t)j * d + i];
+                    g += x[t * d + i] * wg[(int64_t)(F + j) * d + i];
+                }
+                h[j] = a / (1.0 + exp(-a)) * g;
+            }
+            for (int32_t i = 0; i < d; ++i) {
+                double s = 0.0;
+                for (int32_t j = 0; j < F; ++j) s += h[j] * wd[(int64_t)i * F + j];
+                out[t * d + i] += gate * s;
+            }
+        }
+    }
+    free(p);
+    free(chosen);
+    free(h);
+    return ORC_OK;
+}
+
+/* bf16 rounding exposed for pins of the rounding helper itself */
+uint16_t orc_double_to_bf16(double v) { return double_to_bf16(v); }

@@ -1,0 +1,274 @@
+"""Python face of the CPU oracle (``oracle.c``), over numpy arrays.
+
+TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+benchmark's CPU-baseline leg import this module. The product path (the CUDA
+library and its binding) never imports it, and it imports nothing from the
+product package.
+
+bf16 tensors travel as uint16 arrays of bf16 bit patterns, fp32 tensors as
+float32 arrays. ``dtype`` is 0 for bf16 and 1 for fp32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import time
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+BF16, FP32 = 0, 1
+ROUND_NONE, ROUND_F32, ROUND_BF16 = 0, 1, 2
+PLAN_INEXACT = 1
+
+_PIECE_FIELDS = ("expert", "rank", "start", "len", "row0")
+_BLOCK_FIELDS = ("expert", "row0", "valid", "rank")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so with gcc (plain -O2, no fast-math, no FMA contraction)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < os.path.getmtime(SRC):
+        tmp = f"{LIB}.{os.getpid()}.tmp"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+                               "-ffp-contract=off", "-Wall", "-o", tmp, SRC, "-lm"])
+        os.replace(tmp, LIB)
+    return LIB
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(LIB)
+        P = ctypes.c_void_p
+        i32, i64 = ctypes.c_int32, ctypes.c_int64
+        L.orc_topk_gate.argtypes = [i64, i32, i32, i32, P, P, P]
+        L.orc_histogram.argtypes = [i64, i32, P, P]
+        L.orc_plan.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P]
+        L.orc_row_maps.argtypes = [i64, i32, i32, P, P, i32, i64, P, P]
+        L.orc_dispatch.argtypes = [i64, i32, i32, P, P, P]
+        L.orc_expert_ffn.argtypes = [i32, i32, i32, i32, i32, P, i32, P, P, P, P, P]
+        L.orc_combine.argtypes = [i64, i32, i32, i32, i32, P, P, P, P]
+        L.orc_token_out.argtypes = [i32, i32, i32, i32, i32, i64, P, P, P, P, P, P, P]
+        L.orc_dense_layer.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P]
+        L.orc_double_to_bf16.argtypes = [ctypes.c_double]
+        L.orc_double_to_bf16.restype = ctypes.c_uint16
+        for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_row_maps", "orc_dispatch",
+                  "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"], "oracle arrays must be C-contiguous"
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"oracle {what} failed with code {rc}")
+
+
+def _elem_dtype(dtype: int):
+    return np.uint16 if dtype == BF16 else np.float32
+
+
+# ---------------------------------------------------------------- layout sizes
+
+def rows_capacity(N: int, E: int, R: int, budget: int, tile: int) -> int:
+    """Rows the padded expert-major buffer can need: every piece wastes < tile rows."""
+    return N + (E + R * budget) * tile
+
+
+def max_pieces(E: int, R: int, budget: int) -> int:
+    return E + R * budget
+
+
+def max_blocks(N: int, E: int, R: int, budget: int, tile: int) -> int:
+    return -(-N // tile) + max_pieces(E, R, budget)
+
+
+# ---------------------------------------------------------------- steps
+
+def topk_gate(logits: np.ndarray, K: int, gating: int):
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = logits.shape
+    idx = np.empty((T, K), np.int32)
+    w = np.empty((T, K), np.float32)
+    _check(lib().orc_topk_gate(T, E, K, gating, _p(logits), _p(idx), _p(w)), "topk_gate")
+    return idx, w
+
+
+def histogram(idx: np.ndarray, E: int) -> np.ndarray:
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    counts = np.empty(E, np.int32)
+    _check(lib().orc_histogram(idx.size, E, _p(idx), _p(counts)), "histogram")
+    return counts
+
+
+def plan(T: int, E: int, K: int, R: int, tile: int, budget: int, counts: np.ndarray) -> dict:
+    counts = np.ascontiguousarray(counts, dtype=np.int32)
+    N = T * K
+    pieces = np.zeros((max_pieces(E, R, budget), 5), np.int32)
+    blocks = np.zeros((max_blocks(N, E, R, budget, tile), 4), np.int32)
+    npc = np.zeros(1, np.int32)
+    nbl = np.zeros(1, np.int32)
+    rank_load = np.zeros(R, np.int64)
+    rank_rep = np.zeros(R, np.int32)
+    rank_row0 = np.zeros(R + 1, np.int64)
+    moves = np.zeros(1, np.int32)
+    status = np.zeros(1, np.uint32)
+    _check(lib().orc_plan(T, E, K, R, tile, budget, _p(counts), _p(pieces), _p(npc), _p(blocks),
+                          _p(nbl), _p(rank_load), _p(rank_rep), _p(rank_row0), _p(moves),
+                          _p(status)), "plan")
+    return {"pieces": pieces[:npc[0]].copy(), "blocks": blocks[:nbl[0]].copy(),
+            "rank_load": rank_load, "rank_replicas": rank_rep, "rank_row0": rank_row0,
+            "moves": int(moves[0]), "status": int(status[0]),
+            "total_rows": int(rank_row0[R])}
+
+
+def row_maps(idx: np.ndarray, E: int, pieces: np.ndarray, rows_cap: int):
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    T, K = idx.shape
+    pieces = np.ascontiguousarray(pieces, dtype=np.int32)
+    row_of = np.empty(T * K, np.int32)
+    src_of = np.empty(rows_cap, np.int32)
+    _check(lib().orc_row_maps(T, K, E, _p(idx), _p(pieces), pieces.shape[0], rows_cap,
+                              _p(row_of), _p(src_of)), "row_maps")
+    return row_of, src_of
+
+
+def dispatch(x: np.ndarray, src_of: np.ndarray, dtype: int, rows: int | None = None) -> np.ndarray:
+    x = np.ascontiguousarray(x)
+    src_of = np.ascontiguousarray(src_of, dtype=np.int32)
+    rows = src_of.shape[0] if rows is None else rows
+    d = x.shape[1]
+    xp = np.empty((rows, d), _elem_dtype(dtype))
+    _check(lib().orc_dispatch(rows, d, dtype, _p(x), _p(src_of), _p(xp)), "dispatch")
+    return xp
+
+
+def expert_ffn(xp, w_gu, w_down, blocks, tile: int, dtype: int, round_mode: int, rows: int):
+    xp = np.ascontiguousarray(xp)
+    w_gu = np.ascontiguousarray(w_gu)
+    w_down = np.ascontiguousarray(w_down)
+    blocks = np.ascontiguousarray(blocks, dtype=np.int32)
+    d = xp.shape[1]
+    F = w_down.shape[2]
+    h = np.zeros((rows, F), _elem_dtype(dtype))
+    yp = np.zeros((rows, d), _elem_dtype(dtype))
+    _check(lib().orc_expert_ffn(d, F, dtype, round_mode, tile, _p(blocks), blocks.shape[0],
+                                _p(xp), _p(w_gu), _p(w_down), _p(h), _p(yp)), "expert_ffn")
+    return h, yp
+
+
+def combine(yp, row_of, w, dtype: int, round_mode: int):
+    yp = np.ascontiguousarray(yp)
+    row_of = np.ascontiguousarray(row_of, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    T, K = w.shape
+    d = yp.shape[1]
+    out = np.empty((T, d), _elem_dtype(dtype))
+    _check(lib().orc_combine(T, K, d, dtype, round_mode, _p(yp), _p(row_of), _p(w), _p(out)),
+           "combine")
+    return out
+
+
+def token_out(tokens, x, idx, w, w_gu, w_down, dtype: int, round_mode: int) -> np.ndarray:
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    x = np.ascontiguousarray(x)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    w_gu = np.ascontiguousarray(w_gu)
+    w_down = np.ascontiguousarray(w_down)
+    K = idx.shape[1]
+    d = x.shape[1]
+    F = w_down.shape[2]
+    out = np.empty((tokens.shape[0], d), np.float64)
+    _check(lib().orc_token_out(d, F, K, dtype, round_mode, tokens.shape[0], _p(tokens), _p(x),
+                               _p(idx), _p(w), _p(w_gu), _p(w_down), _p(out)), "token_out")
+    return out
+
+
+def dense_layer(logits, x, w_gu, w_down, K: int, gating: int) -> np.ndarray:
+    logits = np.ascontiguousarray(logits, dtype=np.float64)
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    w_gu = np.ascontiguousarray(w_gu, dtype=np.float64)
+    w_down = np.ascontiguousarray(w_down, dtype=np.float64)
+    T, E = logits.shape
+    d = x.shape[1]
+    F = w_down.shape[2]
+    out = np.empty((T, d), np.float64)
+    _check(lib().orc_dense_layer(T, d, E, K, F, gating, _p(logits), _p(x), _p(w_gu),
+                                 _p(w_down), _p(out)), "dense_layer")
+    return out
+
+
+def double_to_bf16(v: float) -> int:
+    return int(lib().orc_double_to_bf16(float(v)))
+
+
+# ---------------------------------------------------------------- conversions
+
+def bf16_bits_to_f64(a: np.ndarray) -> np.ndarray:
+    return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def to_f64(a: np.ndarray, dtype: int) -> np.ndarray:
+    return bf16_bits_to_f64(a) if dtype == BF16 else a.astype(np.float64)
+
+
+# ---------------------------------------------------------------- the whole layer
+
+def default_round_mode(dtype: int) -> int:
+    return ROUND_BF16 if dtype == BF16 else ROUND_F32
+
+
+def layer(logits, x, w_gu, w_down, *, K, R, tile, budget, gating, dtype, round_mode=None,
+          ffn=True) -> dict:
+    """Every step of the layer on numpy inputs; returns each intermediate."""
+    rm = default_round_mode(dtype) if round_mode is None else round_mode
+    T, E = logits.shape
+    idx, w = topk_gate(logits, K, gating)
+    counts = histogram(idx, E)
+    pl = plan(T, E, K, R, tile, budget, counts)
+    cap = rows_capacity(T * K, E, R, budget, tile)
+    row_of, src_of = row_maps(idx, E, pl["pieces"], cap)
+    res = {"idx": idx, "w": w, "counts": counts, "plan": pl, "row_of": row_of,
+           "src_of": src_of, "rows_cap": cap}
+    if ffn:
+        xp = dispatch(x, src_of, dtype, rows=cap)
+        h, yp = expert_ffn(xp, w_gu, w_down, pl["blocks"], tile, dtype, rm, cap)
+        out = combine(yp, row_of, w, dtype, rm)
+        res.update(xp=xp, h=h, yp=yp, out=out)
+    return res
+
+
+def timed_sample(logits, x, w_gu, w_down, *, K, R, tile, budget, gating, dtype,
+                 n_tokens: int, seed: int = 0) -> dict:
+    """Time the oracle on a bounded sample of a layer.
+
+    Routing, planning and row maps run over all tokens; the FFN and combine
+    run on ``n_tokens`` evenly spaced tokens (their cost is per token), and
+    the whole-layer time is that routing time plus the per-token FFN time
+    times T. Single-threaded.
+    """
+    T = logits.shape[0]
+    t0 = time.perf_counter()
+    r = layer(logits, x, w_gu, w_down, K=K, R=R, tile=tile, budget=budget, gating=gating,
+              dtype=dtype, ffn=False)
+    t1 = time.perf_counter()
+    toks = np.linspace(0, T - 1, num=min(n_tokens, T)).astype(np.int64)
+    token_out(toks, x, r["idx"], r["w"], w_gu, w_down, dtype, default_round_mode(dtype))
+    t2 = time.perf_counter()
+    per_tok = (t2 - t1) / len(toks)
+    est = (t1 - t0) + per_tok * T
+    return {"routing_s": t1 - t0, "ffn_s_per_token": per_tok, "layer_s_est": est,
+            "sample_tokens": int(len(toks)), "measured_s": t2 - t0}
