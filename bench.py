@@ -1,0 +1,379 @@
+"""Benchmark of the routed-expert MoE layer on B200: tokens/s of one layer pass.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config olmoe] [--impl mine|reference]
+
+One step = one pass of the whole layer (top-k and gating, histogram, planner,
+row maps, dispatch, FC1 + SwiGLU, FC2, combine) over one batch of seeded
+synthetic inputs already resident in HBM, through the C ABI. Under torchrun
+every rank runs its own independent layer (its own tokens, replicated
+weights, no collective on the data path: weak scaling); the timed region is
+bracketed by a barrier and a device synchronisation, and the time is the
+maximum over ranks. Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (oracle/, plain fp64 C, one core) on a
+bounded sample of the same workload: routing, planning and row maps over
+every token, the expert FFN and combine over a few tokens, scaled to the
+whole layer.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from routed_experts_b200 import configs as C  # noqa: E402
+from routed_experts_b200 import inputs as I  # noqa: E402
+
+METRIC = "routed MoE layer tokens/s at 1 B200; % of bf16 tensor / HBM roofline"
+LAUNCHES_PER_STEP = 7   # topk_hist, plan, row_maps, gather, fc1, fc2, combine
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--config", default="olmoe", choices=sorted(C.NAMED))
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--impl", default="mine", choices=["mine", "reference"])
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-tokens", type=int, default=48, help="tokens of the oracle's FFN sample")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while running."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def source_sha(*rel):
+    h = hashlib.sha256()
+    for r in rel:
+        with open(os.path.join(ROOT, r), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+GEMM_SOURCES = ("routed_experts_b200/csrc/ffn_tc.cu", "routed_experts_b200/csrc/ptx.cuh",
+                "routed_experts_b200/csrc/common.cuh")
+
+
+def ncu_traffic(kernel_key: str):
+    """DRAM bytes per launch of a kernel from a committed ncu capture, or None
+    when the capture is missing or the kernel's sources changed since."""
+    path = os.path.join(ROOT, "profiles", "ncu_counters.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel_key)
+    if not e or e.get("source_sha") != source_sha(*GEMM_SOURCES):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------------ reference arm
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    from oracle import oracle as O
+    cfg = C.NAMED[args.config]
+    inp = I.make_inputs(cfg, args.seed, "cpu")
+    h = {k: I.to_numpy_bits(v) for k, v in inp.items()}
+    kw = dict(K=cfg.K, R=cfg.R, tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype)
+    n_tok = max(2, args.cpu_tokens // 4)
+    for _ in range(args.warmup):
+        O.timed_sample(h["logits"], h["x"], h["w_gate_up"], h["w_down"], n_tokens=2, **kw)
+    est = []
+    for _ in range(args.steps):
+        r = O.timed_sample(h["logits"], h["x"], h["w_gate_up"], h["w_down"], n_tokens=n_tok, **kw)
+        est.append(r["layer_s_est"])
+    total = sum(est)
+    value = cfg.T * len(est) / total
+    sample = (f"per step: top-k, gating, histogram, plan and row maps over all {cfg.T} tokens; expert FFN and "
+              f"combine over {n_tok} evenly spaced tokens, scaled by T/{n_tok}; single-threaded fp64 C oracle")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(est),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded; see DESIGN.md input recipe)",
+            "config": {"workload": cfg.name, **C.describe(cfg)},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ the CUDA path
+
+def cpu_baseline(cfg, inp, n_tokens):
+    from oracle import oracle as O
+    h = {k: I.to_numpy_bits(v) for k, v in inp.items()}
+    r = O.timed_sample(h["logits"], h["x"], h["w_gate_up"], h["w_down"], K=cfg.K, R=cfg.R, tile=cfg.tile,
+                       budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype, n_tokens=n_tokens)
+    return {"value": cfg.T / r["layer_s_est"], "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": (f"top-k, gating, histogram, plan and row maps over all {cfg.T} tokens "
+                       f"({r['routing_s']:.2f} s) plus expert FFN and combine over {r['sample_tokens']} evenly "
+                       f"spaced tokens ({r['ffn_s_per_token'] * 1e3:.1f} ms/token), scaled to {cfg.T} tokens; "
+                       f"{r['measured_s']:.1f} s of single-threaded fp64 C"),
+            "measured_s": r["measured_s"]}
+
+
+def run_mine(args, world, rank, local):
+    from routed_experts_b200 import moe as M
+    cfg = C.NAMED[args.config]
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=dev)
+        pg = torch.distributed.group.WORLD
+    inp = I.make_inputs(cfg, args.seed + rank, dev)
+    stream = torch.cuda.current_stream(dev)
+    T, K, E, d, F = cfg.T, cfg.K, cfg.E, cfg.d, cfg.F
+    dt = M.act_dtype(cfg)
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
+    cap = M.moe_rows_capacity(cfg)
+    xp = torch.empty(cap, d, dtype=dt, device=dev)
+    h = torch.empty(cap, F, dtype=dt, device=dev)
+    yp = torch.empty(cap, d, dtype=dt, device=dev)
+    out = torch.empty(T, d, dtype=dt, device=dev)
+    lg, x, wgu, wdn = inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"]
+
+    n_ev = 6
+    def step(evs=None):
+        if evs is not None: evs[0].record(stream)
+        M.moe_plan(cfg, lg, idx, w, counts, ws, stream)
+        if evs is not None: evs[1].record(stream)
+        M.moe_dispatch(cfg, x, xp, ws, stream)
+        if evs is not None: evs[2].record(stream)
+        M.moe_expert_fc1(cfg, xp, wgu, h, ws, stream)
+        if evs is not None: evs[3].record(stream)
+        M.moe_expert_fc2(cfg, h, wdn, yp, ws, stream)
+        if evs is not None: evs[4].record(stream)
+        M.moe_combine(cfg, yp, w, out, ws, stream)
+        if evs is not None: evs[5].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = M.moe_read_status(ws, stream)
+    if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
+        raise RuntimeError(f"device status {st} after warm-up")
+    plan = M.read_plan(cfg, ws)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    if pg is not None:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    smi_index = int(vis.split(",")[local]) if vis and vis.split(",")[local].strip().isdigit() else local
+    with ClockSampler(smi_index) as clk:
+        t0.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+    if pg is not None:
+        torch.distributed.barrier()
+    elapsed_ms = t0.elapsed_time(t1)
+    stage_ms = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n_ev - 1)] for e in evs])
+    st = M.moe_read_status(ws, stream)
+    if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
+        raise RuntimeError(f"device status {st} after the timed steps")
+
+    # end to end through the public API with host buffers: H2D of logits and x
+    # from pinned memory, the layer, D2H of the output, every step
+    layer_h = M.Layer(cfg, dev, host_io=True)
+    lg_h = lg.cpu().pin_memory()
+    x_h = x.cpu().pin_memory()
+    out_h = torch.empty(T, d, dtype=dt).pin_memory()
+    for _ in range(args.warmup):
+        layer_h.forward_host(lg_h, x_h, wgu, wdn, out_h, stream)
+    if pg is not None:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer_h.forward_host(lg_h, x_h, wgu, wdn, out_h, stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    if pg is not None:
+        torch.distributed.barrier()
+        tt = torch.tensor([elapsed_ms, e2e_ms], device=dev)
+        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms, e2e_ms = float(tt[0]), float(tt[1])
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, inp, args.cpu_tokens)
+
+    if pg is not None:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank != 0:
+        return
+
+    pk, pk_kind = peaks()
+    med = np.median(stage_ms, axis=0)
+    mean = stage_ms.mean(axis=0)
+    N = cfg.N
+    # algorithmic work, valid entries only (padding rows are not counted)
+    fc1_flop = 2.0 * N * d * (2 * F)
+    fc2_flop = 2.0 * N * F * d
+    fc1_s = mean[2] * 1e-3
+    fc2_s = mean[3] * 1e-3
+    tensor_peak = pk["bf16_tflops"]
+    eb = cfg.elem_bytes
+    active = int((np.bincount(plan["blocks"][:, 0].numpy(), minlength=E) > 0).sum()) if plan["n_blocks"] else 0
+    weight_bytes = active * 3 * F * d * eb
+    alg_bytes = 4 * T * E + T * d * eb + weight_bytes + T * d * eb
+    layer_flop = fc1_flop + fc2_flop
+    t_roof = max(layer_flop / (tensor_peak * 1e12), alg_bytes / (pk["hbm_gbs"] * 1e9))
+    ms_per_step = elapsed_ms / args.steps
+    value = world * T / (ms_per_step * 1e-3)
+    gather_bytes = T * d * eb + N * d * eb + 4 * N + (plan["total_rows"] - N) * d * eb
+    combine_bytes = N * d * eb + 8 * N + T * d * eb
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == C.BF16 else "fp32",
+        "data": "synthetic (seeded SplitMix64 + Box-Muller inputs; see DESIGN.md input recipe)",
+        "config": {"workload": cfg.name, **C.describe(cfg), "seed": args.seed,
+                   "l2": "no flush: one step touches ~%.1f GB (weights %.2f GB) >> 126 MB L2"
+                         % ((alg_bytes + 3 * cap * d * eb + cap * F * eb) / 1e9, weight_bytes / 1e9),
+                   "parallelism": f"replicas x{world} (independent layers, no collective)"},
+        "roofline": {"bound": "tensor", "kernel": "ffn_tc_kernel<FC1+SwiGLU>",
+                     "achieved": fc1_flop / fc1_s / 1e12, "peak": tensor_peak, "unit": "TFLOP/s",
+                     "frac": fc1_flop / fc1_s / 1e12 / tensor_peak,
+                     "traffic": ncu_traffic(f"fc1@{cfg.name}"),
+                     "peak_kind": f"{pk_kind} bf16 burst",
+                     "flop_per_launch": fc1_flop, "launch_ms": mean[2]},
+        "layer_roofline": {"frac": (t_roof * 1e3) / ms_per_step, "roofline_ms": t_roof * 1e3,
+                           "flop": layer_flop, "alg_bytes": alg_bytes,
+                           "peaks": {"bf16_tflops": tensor_peak, "hbm_gbs": pk["hbm_gbs"], "kind": pk_kind}},
+        "stages_ms": {"plan(topk+hist+plan+rowmaps)": med[0], "dispatch": med[1], "fc1": med[2], "fc2": med[3],
+                      "combine": med[4]},
+        "stage_rates": {"fc1_tflops": fc1_flop / fc1_s / 1e12, "fc2_tflops": fc2_flop / fc2_s / 1e12,
+                        "dispatch_gbs": gather_bytes / (mean[1] * 1e-3) / 1e9,
+                        "combine_gbs": combine_bytes / (mean[4] * 1e-3) / 1e9},
+        "plan": {"moves": plan["moves"], "replicas": plan["replicas"], "status": plan["status"],
+                 "padded_rows": plan["total_rows"] - N, "blocks": plan["n_blocks"]},
+        "e2e": {"value": world * T / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 4 * T * E + T * d * eb, "d2h_bytes_per_step": T * d * eb,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_mine(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

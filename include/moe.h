@@ -1,0 +1,229 @@
+/*
+ * moe.h - C ABI of the routed-expert MoE layer library (libmoe.so), sm_100a.
+ *
+ * The layer: router top-k and gating, an expert-load histogram, a greedy
+ * replication planner that gives each of R virtual expert-parallel ranks
+ * exactly S*K routed entries under a per-rank replica budget, a permute of
+ * token rows into an expert-major, tile-padded buffer, a grouped SwiGLU
+ * expert FFN on the tensor cores, and a weighted combine.
+ *
+ * Sources, cited by page title and section:
+ *   [MegaFlux] "MegaFlux: Skew-Resilient MoE Megakernels via Pipelined
+ *              Expert Replication"
+ *   [MoonEP]   "MoonEP routing flow - live" (an explainer of MoonEP's
+ *              planning kernel)
+ *
+ * Conventions for every call:
+ *  - Pointers named as device buffers are device pointers (cudaMalloc or
+ *    torch CUDA tensors), row-major and contiguous, 16-byte aligned. The
+ *    caller allocates and owns every buffer, the workspace included; the
+ *    library never allocates, frees or synchronises, except where a call
+ *    says so (moe_read_status, moe_layer_fwd_host).
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream). A return other than MOE_OK is synchronous and means
+ *    nothing was launched. Conditions found on the device go to a status
+ *    word in the workspace; moe_read_status returns them.
+ *  - cfg->dtype applies to x, the expert weights, xp, h, yp and out
+ *    (bf16 on the tensor-core path, fp32 on the CUDA-core path). Router
+ *    logits and gating weights are always fp32.
+ *  - The library keeps no state between calls: distinct workspaces may be
+ *    used from distinct host threads at once. A workspace holds one plan;
+ *    calls that read it must follow the moe_plan that wrote it, on the same
+ *    stream (or after it in stream order), with the same cfg.
+ *  - There is no CPU fallback: a cfg the kernels do not cover returns
+ *    MOE_ERR_UNSUPPORTED.
+ */
+#ifndef ROUTED_EXPERTS_MOE_H
+#define ROUTED_EXPERTS_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t; /* a cudaStream_t */
+
+/* Synchronous return codes (host-detected). */
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null or misaligned pointer, inconsistent sizes */
+    MOE_ERR_UNSUPPORTED = 2,   /* a valid cfg that no kernel here covers */
+    MOE_ERR_WORKSPACE = 3,     /* ws_bytes smaller than moe_workspace_size asks */
+    MOE_ERR_CUDA = 4           /* a CUDA runtime call failed (launch, copy, query) */
+} moe_status;
+
+/* Device status bits (read with moe_read_status). */
+enum {
+    MOE_DEV_PLAN_INEXACT = 1u, /* the planner could not give every rank exactly S*K
+                                  entries within the replica budget; the plan is still a
+                                  valid partition and the layer output is still correct */
+    MOE_DEV_TIMEOUT = 2u,      /* a bounded device-side wait gave up; outputs are invalid */
+    MOE_DEV_BAD_INDEX = 4u     /* a non-finite router logit or an out-of-range index */
+};
+
+typedef enum { MOE_BF16 = 0, MOE_FP32 = 1 } moe_dtype;
+typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_SIGMOID_TOPK = 1 } moe_gating;
+
+/* Workspace kinds for moe_workspace_size. */
+typedef enum {
+    MOE_WS_PLAN = 0,       /* plan, row maps and scratch: moe_plan .. moe_combine */
+    MOE_WS_LAYER = 1,      /* MOE_WS_PLAN plus top-k, xp, h and yp: moe_layer_fwd */
+    MOE_WS_LAYER_HOST = 2  /* MOE_WS_LAYER plus device copies of logits, x and out:
+                              moe_layer_fwd_host */
+} moe_ws_kind;
+
+/*
+ * Layer shape. T tokens, hidden size d, E experts, top-K, expert FFN width
+ * F, R virtual expert-parallel ranks, token-block rows `tile` (beta), and
+ * `budget` replicas a rank may host. S = T/R tokens per rank; every rank's
+ * capacity is C = S*K entries. Expert e is owned by rank e / (E/R).
+ * Requirements: T % R == 0, E % R == 0, 1 <= K <= min(E, 16), E <= 1024,
+ * R <= 256, 0 <= budget <= 32. bf16: tile == 128, F % 128 == 0,
+ * d % 256 == 0. fp32: tile in {16, 32, 64, 128}, d % 64 == 0, F % 64 == 0.
+ */
+typedef struct {
+    int32_t T, d, E, K, F, R, tile, budget;
+    int32_t dtype;   /* moe_dtype */
+    int32_t gating;  /* moe_gating */
+} moe_config;
+
+/*
+ * Where moe_plan leaves the plan inside the workspace (byte offsets from
+ * the workspace base) and the capacities those arrays are sized for.
+ * All arrays are int32.
+ *   header     [8]: device status bits, n_pieces, n_blocks, total_rows,
+ *                   moves, replicas in total, 0, 0
+ *   pieces     [max_pieces][5]: expert, rank, start, len, row0 - rank
+ *                   `rank` computes entries [start, start+len) of expert's
+ *                   (token, slot)-ordered list at padded rows row0..;
+ *                   ordered by (rank, expert)
+ *   blocks     [max_blocks][4]: expert, row0, valid rows, rank - one
+ *                   tile of one expert, in piece order
+ *   rank_load  [R]: valid entries per rank (exactly S*K when exact)
+ *   rank_replicas [R]: foreign experts hosted per rank (<= budget)
+ *   rank_row0  [R+1]: first padded row of each rank; [R] = total rows
+ *   row_of     [T*K]: padded row of entry (t, k)
+ *   src_of     [rows_cap]: token of each padded row, -1 for padding;
+ *                   defined for rows below total_rows
+ */
+typedef struct {
+    int64_t header, pieces, blocks, rank_load, rank_replicas, rank_row0, row_of, src_of;
+    int64_t max_pieces, max_blocks, rows_cap;
+} moe_plan_layout;
+
+/* Bytes of workspace a call sequence needs (see moe_ws_kind). */
+moe_status moe_workspace_size(const moe_config* cfg, int32_t kind, size_t* bytes);
+
+/* Rows of the padded expert-major buffers xp, h and yp:
+ * T*K + (E + R*budget)*tile (each of at most E + R*budget pieces pads
+ * fewer than tile rows). */
+moe_status moe_rows_capacity(const moe_config* cfg, int64_t* rows_cap);
+
+/* Offsets of the plan arrays inside a MOE_WS_PLAN workspace (host only). */
+moe_status moe_plan_view(const moe_config* cfg, moe_plan_layout* out);
+
+/*
+ * moe_plan - steps A1 to A5: top-k, gating, histogram, planner, row maps.
+ *   logits    fp32 [T, E] (device): router logits, any bias already added.
+ *   topk_idx  int32 [T, K] (device, out): the K largest logits of each
+ *             token, in descending order, ties to the lower expert id
+ *             ([MegaFlux] §1; §4.1: k distinct experts per token).
+ *   topk_w    fp32 [T, K] (device, out): softmax of the chosen logits
+ *             renormalised over them, or their sigmoids normalised over
+ *             them (cfg->gating).
+ *   counts    int32 [E] (device, out): routed entries per expert, the
+ *             routing profile the planner consumes ([MegaFlux] §3.1).
+ *   ws        device workspace of at least moe_workspace_size(MOE_WS_PLAN)
+ *             bytes; receives the plan (moe_plan_view) and scratch.
+ * The planner ([MoonEP] "The greedy balance, step by step"; [MegaFlux]
+ * §3.1, §4.1, App. A.1, A.2): starting from every expert on its owner,
+ * each move refills the rank with the fewest entries from the rank with
+ * the most, slicing the donor's largest experts (the tail of the entries
+ * it still holds) until the receiver holds S*K; a receiver takes at most
+ * `budget` foreign experts. Every piece is padded to whole tiles at a
+ * tile-aligned row; pieces are laid out in (rank, expert) order. Token
+ * counts, expert choices and routing weights are untouched.
+ */
+moe_status moe_plan(const moe_config* cfg, const float* logits, int32_t* topk_idx, float* topk_w,
+                    int32_t* counts, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_dispatch - step A6: xp[row] = x[src_of[row]] for every row below
+ * the plan's total rows, zero for padding rows ([MegaFlux] §1: routed
+ * activations go to the ranks that compute their experts).
+ *   x   [T, d] (device), xp [rows_cap, d] (device, out).
+ */
+moe_status moe_dispatch(const moe_config* cfg, const void* x, void* xp, const void* ws,
+                        size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_ffn - steps A7 and A8, the grouped SwiGLU expert FFN over the
+ * planned blocks ([MegaFlux] §2.1, §3.2 "Forward": FC1 then FC2 per token
+ * block; §4.1: SwiGLU experts).
+ *   xp         [rows_cap, d] (device)
+ *   w_gate_up  [E, 2F, d] (device): rows 0..F-1 of expert e are the gate
+ *              projection, rows F..2F-1 the up projection (K-major).
+ *   w_down     [E, d, F] (device, K-major).
+ *   h          [rows_cap, F] (device, out): silu(xp.gate) * (xp.up).
+ *   yp         [rows_cap, d] (device, out): h . w_down.
+ * fp32 accumulation; in bf16 mode h and yp are rounded to bf16 once.
+ */
+moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const void* w_gate_up,
+                          const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/*
+ * moe_expert_fc1 / moe_expert_fc2 - the two halves of moe_expert_ffn, for
+ * callers that schedule or time them apart: fc1 writes h from xp and
+ * w_gate_up (step A7), fc2 writes yp from h and w_down (step A8). Same
+ * arguments, layouts and rounding as moe_expert_ffn.
+ */
+moe_status moe_expert_fc1(const moe_config* cfg, const void* xp, const void* w_gate_up, void* h, void* ws,
+                          size_t ws_bytes, moe_stream_t stream);
+moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_down, void* yp, void* ws,
+                          size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_combine - step A9, the weighted top-k sum ([MegaFlux] §1, §2.1):
+ * out[t] = sum over k in order of topk_w[t,k] * yp[row_of(t,k)], in fp32,
+ * rounded once to cfg->dtype.
+ *   yp [rows_cap, d] (device), topk_w fp32 [T, K] (device),
+ *   out [T, d] (device, out).
+ */
+moe_status moe_combine(const moe_config* cfg, const void* yp, const float* topk_w, void* out,
+                       const void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_layer_fwd - the whole layer, A1 to A9, on device buffers, with
+ * top-k, xp, h and yp carved from a MOE_WS_LAYER workspace.
+ */
+moe_status moe_layer_fwd(const moe_config* cfg, const float* logits, const void* x,
+                         const void* w_gate_up, const void* w_down, void* out, void* ws,
+                         size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_layer_fwd_host - the whole layer with the activations in host
+ * memory: copies logits [T,E] and x [T,d] from host to the device copies
+ * in a MOE_WS_LAYER_HOST workspace, runs moe_layer_fwd, and copies out
+ * [T,d] back to host memory, all on `stream` with cudaMemcpyAsync (host
+ * buffers should be pinned for the copies to be asynchronous). Expert
+ * weights stay device-resident. Does not synchronise: out_host is valid
+ * once the stream has reached the end of this call.
+ */
+moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, const void* x_host,
+                              const void* w_gate_up, const void* w_down, void* out_host,
+                              void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Synchronises `stream`, then reads the device status bits of `ws`. */
+moe_status moe_read_status(const void* ws, moe_stream_t stream, uint32_t* dev_bits);
+
+/* A static string naming a moe_status. */
+const char* moe_status_string(moe_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ROUTED_EXPERTS_MOE_H */

@@ -453,6 +453,22 @@ int orc_token_out(int32_t d, int32_t F, int32_t K, int32_t dtype, int32_t round_
     return ORC_OK;
 }
 
+/* ------------------------------------------------- sampled entries
+ * h and y of single routed entries (token t, expert e), straight from x, in
+ * the same arithmetic as the expert FFN above. Used to check sampled rows of
+ * large layers.
+ */
+int orc_entry_ffn(int32_t d, int32_t F, int32_t dtype, int32_t round_mode, int64_t n,
+                  const int64_t* tokens, const int32_t* experts, const void* x,
+                  const void* w_gu, const void* w_down, double* h_out /*[n,F]*/,
+                  double* y_out /*[n,d]*/)
+{
+    for (int64_t i = 0; i < n; ++i)
+        ffn_row(d, F, dtype, round_mode, x, tokens[i] * d, w_gu, w_down, experts[i],
+                h_out + (size_t)i * F, y_out + (size_t)i * d);
+    return ORC_OK;
+}
+
 /* ------------------------------------------------- dense reference
  * The plain definition of the routed layer: run every expert on every
  * token in fp64 and add expert e's output with weight gate(t,e) when e is

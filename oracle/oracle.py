@@ -57,10 +57,11 @@ def lib():
         L.orc_combine.argtypes = [i64, i32, i32, i32, i32, P, P, P, P]
         L.orc_token_out.argtypes = [i32, i32, i32, i32, i32, i64, P, P, P, P, P, P, P]
         L.orc_dense_layer.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P]
+        L.orc_entry_ffn.argtypes = [i32, i32, i32, i32, i64, P, P, P, P, P, P, P]
         L.orc_double_to_bf16.argtypes = [ctypes.c_double]
         L.orc_double_to_bf16.restype = ctypes.c_uint16
         for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_row_maps", "orc_dispatch",
-                  "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer"):
+                  "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer", "orc_entry_ffn"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -195,6 +196,23 @@ def token_out(tokens, x, idx, w, w_gu, w_down, dtype: int, round_mode: int) -> n
     _check(lib().orc_token_out(d, F, K, dtype, round_mode, tokens.shape[0], _p(tokens), _p(x),
                                _p(idx), _p(w), _p(w_gu), _p(w_down), _p(out)), "token_out")
     return out
+
+
+def entry_ffn(tokens, experts, x, w_gu, w_down, dtype: int, round_mode: int):
+    """h [n,F] and y [n,d] (fp64 arrays holding the rounded values) of entries (tokens[i], experts[i])."""
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    x = np.ascontiguousarray(x)
+    w_gu = np.ascontiguousarray(w_gu)
+    w_down = np.ascontiguousarray(w_down)
+    d = x.shape[1]
+    F = w_down.shape[2]
+    n = tokens.shape[0]
+    h = np.empty((n, F), np.float64)
+    y = np.empty((n, d), np.float64)
+    _check(lib().orc_entry_ffn(d, F, dtype, round_mode, n, _p(tokens), _p(experts), _p(x), _p(w_gu),
+                               _p(w_down), _p(h), _p(y)), "entry_ffn")
+    return h, y
 
 
 def dense_layer(logits, x, w_gu, w_down, K: int, gating: int) -> np.ndarray:

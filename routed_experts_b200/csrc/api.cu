@@ -1,0 +1,303 @@
+// api.cu - the C ABI (include/moe.h): argument checks, the workspace layout and
+// the launch sequence of each call. Host code only; no allocation, no
+// synchronisation except in moe_read_status.
+#include <string.h>
+
+#include "common.cuh"
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Validates cfg and fills the derived shape. INVALID_ARG for an ill-formed
+// cfg, UNSUPPORTED for a well-formed one no kernel covers.
+moe_status make_shape(const moe_config* cfg, Shape* s) {
+    if (!cfg || !s) return MOE_ERR_INVALID_ARG;
+    const moe_config c = *cfg;
+    if (c.T <= 0 || c.d <= 0 || c.E <= 0 || c.K <= 0 || c.F <= 0 || c.R <= 0 || c.tile <= 0 || c.budget < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (c.K > c.E || c.T % c.R != 0 || c.E % c.R != 0) return MOE_ERR_INVALID_ARG;
+    if (c.dtype != MOE_BF16 && c.dtype != MOE_FP32) return MOE_ERR_INVALID_ARG;
+    if (c.gating != MOE_GATE_SOFTMAX_TOPK && c.gating != MOE_GATE_SIGMOID_TOPK) return MOE_ERR_INVALID_ARG;
+    if (c.K > kMaxK || c.E > kMaxE || c.R > kMaxR || c.budget > kMaxBudget || (int64_t)c.R * c.budget > 1024)
+        return MOE_ERR_UNSUPPORTED;
+    if (c.dtype == MOE_BF16) {
+        if (c.tile != 128 || c.F % 128 != 0 || c.d % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    } else {
+        if (!(c.tile == 16 || c.tile == 32 || c.tile == 64 || c.tile == 128) || c.d % 64 != 0 || c.F % 64 != 0)
+            return MOE_ERR_UNSUPPORTED;
+    }
+    s->T = c.T; s->d = c.d; s->E = c.E; s->K = c.K; s->F = c.F; s->R = c.R; s->tile = c.tile;
+    s->budget = c.budget; s->dtype = c.dtype; s->gating = c.gating;
+    s->N = (int64_t)c.T * c.K;
+    s->C = (int64_t)(c.T / c.R) * c.K;
+    s->per = c.E / c.R;
+    s->max_pieces = (int64_t)c.E + (int64_t)c.R * c.budget;
+    s->max_blocks = (s->N + c.tile - 1) / c.tile + s->max_pieces;
+    s->rows_cap = s->N + s->max_pieces * c.tile;
+    s->n_chunks = (c.T + kTokPerChunk - 1) / kTokPerChunk;
+    s->eb = c.dtype == MOE_BF16 ? 2 : 4;
+    if (s->rows_cap >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;   // int32 row indices
+    return MOE_OK;
+}
+
+WsLayout make_layout(const Shape& s) {
+    WsLayout L;
+    int64_t o = 0;
+    auto take = [&](int64_t bytes) { const int64_t at = o; o = align_up(o + bytes, 256); return at; };
+    L.header = take(sizeof(uint32_t) * H_WORDS);
+    L.chunk_counts = take(sizeof(int32_t) * (int64_t)s.n_chunks * s.E);
+    L.chunk_base = take(sizeof(int32_t) * (int64_t)s.n_chunks * s.E);
+    L.chunk_flags = take(sizeof(uint32_t) * (int64_t)s.n_chunks);
+    L.pieces = take(sizeof(int32_t) * kPieceInts * s.max_pieces);
+    L.exp_piece_off = take(sizeof(int32_t) * (s.E + 1));
+    L.exp_piece_idx = take(sizeof(int32_t) * s.max_pieces);
+    L.blocks = take(sizeof(int32_t) * kBlockInts * s.max_blocks);
+    L.sched_off = take(sizeof(int32_t) * (s.E + 1));
+    L.sched = take(sizeof(int32_t) * s.max_blocks);
+    L.rank_load = take(sizeof(int32_t) * s.R);
+    L.rank_replicas = take(sizeof(int32_t) * s.R);
+    L.rank_row0 = take(sizeof(int32_t) * (s.R + 1));
+    L.row_of = take(sizeof(int32_t) * s.N);
+    L.src_of = take(sizeof(int32_t) * s.rows_cap);
+    L.plan_end = o;
+    L.idx = take(sizeof(int32_t) * s.N);
+    L.w = take(sizeof(float) * s.N);
+    L.counts = take(sizeof(int32_t) * s.E);
+    L.xp = take((int64_t)s.eb * s.rows_cap * s.d);
+    L.h = take((int64_t)s.eb * s.rows_cap * s.F);
+    L.yp = take((int64_t)s.eb * s.rows_cap * s.d);
+    L.layer_end = o;
+    L.logits_dev = take(sizeof(float) * (int64_t)s.T * s.E);
+    L.x_dev = take((int64_t)s.eb * s.T * s.d);
+    L.out_dev = take((int64_t)s.eb * s.T * s.d);
+    L.host_end = o;
+    return L;
+}
+
+moe_status check_ws(const void* ws, size_t ws_bytes, int64_t need) {
+    if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;
+    if ((int64_t)ws_bytes < need) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+moe_status from_cuda(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+moe_status plan_impl(const Shape& s, const WsLayout& L, const float* logits, int32_t* idx, float* w,
+                     int32_t* counts, void* ws, cudaStream_t st) {
+    const WsPtrs P = ws_ptrs(ws, L);
+    cudaError_t e = launch_topk_hist(s, logits, idx, w, P, st);
+    if (e == cudaSuccess) e = launch_plan(s, counts, P, st);
+    if (e == cudaSuccess) e = launch_row_maps(s, idx, P, st);
+    return from_cuda(e);
+}
+
+moe_status fc_impl(const Shape& s, const WsLayout& L, int which, const void* a_mat, const void* w, void* out,
+                   void* ws, cudaStream_t st) {
+    const WsPtrs P = ws_ptrs(ws, L);
+    cudaError_t e = s.dtype == MOE_BF16 ? launch_ffn_tc(s, which, a_mat, w, out, P, st, kSpinBudget)
+                                        : launch_ffn_simt(s, which, a_mat, w, out, P, st);
+    return from_cuda(e);
+}
+
+moe_status ffn_impl(const Shape& s, const WsLayout& L, const void* xp, const void* wgu, const void* wdn,
+                    void* h, void* yp, void* ws, cudaStream_t st) {
+    moe_status r = fc_impl(s, L, 1, xp, wgu, h, ws, st);
+    if (r != MOE_OK) return r;
+    return fc_impl(s, L, 2, h, wdn, yp, ws, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_workspace_size(const moe_config* cfg, int32_t kind, size_t* bytes) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!bytes) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    switch (kind) {
+        case MOE_WS_PLAN: *bytes = (size_t)L.plan_end; return MOE_OK;
+        case MOE_WS_LAYER: *bytes = (size_t)L.layer_end; return MOE_OK;
+        case MOE_WS_LAYER_HOST: *bytes = (size_t)L.host_end; return MOE_OK;
+        default: return MOE_ERR_INVALID_ARG;
+    }
+}
+
+moe_status moe_rows_capacity(const moe_config* cfg, int64_t* rows_cap) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!rows_cap) return MOE_ERR_INVALID_ARG;
+    *rows_cap = s.rows_cap;
+    return MOE_OK;
+}
+
+moe_status moe_plan_view(const moe_config* cfg, moe_plan_layout* out) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!out) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    out->header = L.header;
+    out->pieces = L.pieces;
+    out->blocks = L.blocks;
+    out->rank_load = L.rank_load;
+    out->rank_replicas = L.rank_replicas;
+    out->rank_row0 = L.rank_row0;
+    out->row_of = L.row_of;
+    out->src_of = L.src_of;
+    out->max_pieces = s.max_pieces;
+    out->max_blocks = s.max_blocks;
+    out->rows_cap = s.rows_cap;
+    return MOE_OK;
+}
+
+moe_status moe_plan(const moe_config* cfg, const float* logits, int32_t* topk_idx, float* topk_w,
+                    int32_t* counts, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!logits || !topk_idx || !topk_w || !counts) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(topk_idx) || !aligned16(topk_w) || !aligned16(counts))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    return plan_impl(s, L, logits, topk_idx, topk_w, counts, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_dispatch(const moe_config* cfg, const void* x, void* xp, const void* ws, size_t ws_bytes,
+                        moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!x || !xp || !aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(const_cast<void*>(ws), L);
+    return from_cuda(launch_gather(s, x, xp, P, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const void* w_gate_up, const void* w_down,
+                          void* h, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!xp || !w_gate_up || !w_down || !h || !yp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(h) || !aligned16(yp))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    return ffn_impl(s, L, xp, w_gate_up, w_down, h, yp, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_fc1(const moe_config* cfg, const void* xp, const void* w_gate_up, void* h, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!xp || !w_gate_up || !h || !aligned16(xp) || !aligned16(w_gate_up) || !aligned16(h))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    return fc_impl(s, L, 1, xp, w_gate_up, h, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_down, void* yp, void* ws,
+                          size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!h || !w_down || !yp || !aligned16(h) || !aligned16(w_down) || !aligned16(yp))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    return fc_impl(s, L, 2, h, w_down, yp, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_combine(const moe_config* cfg, const void* yp, const float* topk_w, void* out, const void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!yp || !topk_w || !out || !aligned16(yp) || !aligned16(topk_w) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(const_cast<void*>(ws), L);
+    return from_cuda(launch_combine(s, yp, topk_w, out, P, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_layer_fwd(const moe_config* cfg, const float* logits, const void* x, const void* w_gate_up,
+                         const void* w_down, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!logits || !x || !w_gate_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.layer_end)) != MOE_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    int32_t* idx = reinterpret_cast<int32_t*>(b + L.idx);
+    float* w = reinterpret_cast<float*>(b + L.w);
+    int32_t* counts = reinterpret_cast<int32_t*>(b + L.counts);
+    void* xp = b + L.xp;
+    void* h = b + L.h;
+    void* yp = b + L.yp;
+    if ((r = plan_impl(s, L, logits, idx, w, counts, ws, st)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(ws, L);
+    if ((r = from_cuda(launch_gather(s, x, xp, P, st))) != MOE_OK) return r;
+    if ((r = ffn_impl(s, L, xp, w_gate_up, w_down, h, yp, ws, st)) != MOE_OK) return r;
+    return from_cuda(launch_combine(s, yp, w, out, P, st));
+}
+
+moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, const void* x_host,
+                              const void* w_gate_up, const void* w_down, void* out_host, void* ws,
+                              size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!logits_host || !x_host || !out_host) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.host_end)) != MOE_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    float* lg = reinterpret_cast<float*>(b + L.logits_dev);
+    void* x = b + L.x_dev;
+    void* out = b + L.out_dev;
+    const size_t lg_bytes = sizeof(float) * (size_t)s.T * s.E;
+    const size_t x_bytes = (size_t)s.eb * s.T * s.d;
+    if (cudaMemcpyAsync(lg, logits_host, lg_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpyAsync(x, x_host, x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess) return MOE_ERR_CUDA;
+    if ((r = moe_layer_fwd(cfg, lg, x, w_gate_up, w_down, out, ws, ws_bytes, stream)) != MOE_OK) return r;
+    if (cudaMemcpyAsync(out_host, out, x_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+moe_status moe_read_status(const void* ws, moe_stream_t stream, uint32_t* dev_bits) {
+    if (!ws || !dev_bits) return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return MOE_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, ws, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+    *dev_bits = v;
+    return MOE_OK;
+}
+
+const char* moe_status_string(moe_status s) {
+    switch (s) {
+        case MOE_OK: return "MOE_OK";
+        case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+        case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+        case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+        case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    }
+    return "MOE_ERR_UNKNOWN";
+}
+
+}  // extern "C"

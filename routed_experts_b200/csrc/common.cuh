@@ -1,0 +1,113 @@
+// common.cuh - shared definitions of the CUDA library: the workspace layout,
+// device status handling and small device helpers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kTokPerChunk = 32;          // tokens per top-k CTA-chunk (histogram granularity)
+constexpr int kMaxK = 16;
+constexpr int kMaxE = 1024;
+constexpr int kMaxR = 256;
+constexpr int kMaxBudget = 32;
+constexpr int kPieceInts = 5;             // expert, rank, start, len, row0
+constexpr int kBlockInts = 4;             // expert, row0, valid, rank
+
+// header words
+enum { H_STATUS = 0, H_NPIECES = 1, H_NBLOCKS = 2, H_TOTAL_ROWS = 3, H_MOVES = 4,
+       H_REPLICAS = 5, H_WORDS = 8 };
+
+// Default bound of a device-side spin (clock cycles, about 2 s at 1.9 GHz).
+constexpr long long kSpinBudget = 4000000000LL;
+
+struct Shape {
+    int32_t T, d, E, K, F, R, tile, budget, dtype, gating;
+    int64_t N;          // T*K
+    int64_t C;          // (T/R)*K
+    int32_t per;        // E/R
+    int64_t max_pieces, max_blocks, rows_cap;
+    int32_t n_chunks;
+    int32_t eb;         // element bytes of activations / weights
+};
+
+// Byte offsets of every array in a workspace.
+struct WsLayout {
+    int64_t header, chunk_counts, chunk_base, chunk_flags, pieces, exp_piece_off, exp_piece_idx,
+        blocks, sched_off, sched, rank_load, rank_replicas, rank_row0, row_of, src_of;
+    int64_t plan_end;
+    // MOE_WS_LAYER extras
+    int64_t idx, w, counts, xp, h, yp;
+    int64_t layer_end;
+    // MOE_WS_LAYER_HOST extras
+    int64_t logits_dev, x_dev, out_dev;
+    int64_t host_end;
+};
+
+__host__ __device__ inline int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+// Device pointers into a workspace, passed by value to kernels.
+struct WsPtrs {
+    uint32_t* header;
+    int32_t* chunk_counts;
+    int32_t* chunk_base;
+    uint32_t* chunk_flags;
+    int32_t* pieces;
+    int32_t* exp_piece_off;
+    int32_t* exp_piece_idx;
+    int32_t* blocks;
+    int32_t* sched_off;
+    int32_t* sched;
+    int32_t* rank_load;
+    int32_t* rank_replicas;
+    int32_t* rank_row0;
+    int32_t* row_of;
+    int32_t* src_of;
+};
+
+inline WsPtrs ws_ptrs(void* ws, const WsLayout& L) {
+    char* b = static_cast<char*>(ws);
+    WsPtrs p;
+    p.header = reinterpret_cast<uint32_t*>(b + L.header);
+    p.chunk_counts = reinterpret_cast<int32_t*>(b + L.chunk_counts);
+    p.chunk_base = reinterpret_cast<int32_t*>(b + L.chunk_base);
+    p.chunk_flags = reinterpret_cast<uint32_t*>(b + L.chunk_flags);
+    p.pieces = reinterpret_cast<int32_t*>(b + L.pieces);
+    p.exp_piece_off = reinterpret_cast<int32_t*>(b + L.exp_piece_off);
+    p.exp_piece_idx = reinterpret_cast<int32_t*>(b + L.exp_piece_idx);
+    p.blocks = reinterpret_cast<int32_t*>(b + L.blocks);
+    p.sched_off = reinterpret_cast<int32_t*>(b + L.sched_off);
+    p.sched = reinterpret_cast<int32_t*>(b + L.sched);
+    p.rank_load = reinterpret_cast<int32_t*>(b + L.rank_load);
+    p.rank_replicas = reinterpret_cast<int32_t*>(b + L.rank_replicas);
+    p.rank_row0 = reinterpret_cast<int32_t*>(b + L.rank_row0);
+    p.row_of = reinterpret_cast<int32_t*>(b + L.row_of);
+    p.src_of = reinterpret_cast<int32_t*>(b + L.src_of);
+    return p;
+}
+
+__device__ inline void set_status(uint32_t* header, uint32_t bits) {
+    atomicOr(header + H_STATUS, bits);
+}
+
+// ---- launchers (one per kernel family), defined in the kernel files ----
+cudaError_t launch_topk_hist(const Shape& s, const float* logits, int32_t* idx, float* w,
+                             const WsPtrs& ws, cudaStream_t st);
+cudaError_t launch_plan(const Shape& s, int32_t* counts_out, const WsPtrs& ws, cudaStream_t st);
+cudaError_t launch_row_maps(const Shape& s, const int32_t* idx, const WsPtrs& ws, cudaStream_t st);
+cudaError_t launch_gather(const Shape& s, const void* x, void* xp, const WsPtrs& ws,
+                          cudaStream_t st);
+cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void* out,
+                           const WsPtrs& ws, cudaStream_t st);
+// which = 1: FC1 + SwiGLU (a_mat = xp, w = w_gate_up, out = h);
+// which = 2: FC2 (a_mat = h, w = w_down, out = yp).
+cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const void* w, void* out,
+                            const WsPtrs& ws, cudaStream_t st);
+cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
+                          const WsPtrs& ws, cudaStream_t st, long long spin_budget);
+
+}  // namespace moe

@@ -1,0 +1,127 @@
+// permute.cu - row maps (step A5) and the dispatch gather into the expert-major,
+// tile-padded buffer (step A6).
+//
+// [MegaFlux] "MegaFlux: Skew-Resilient MoE Megakernels via Pipelined Expert
+// Replication", App. A.2 'Mapping blocks to routed assignments': within each
+// expert, routed assignments are ordered by source rank and then local
+// (token, top-k position) and cut into the planned blocks. With source rank
+// t / S this is plain (t, k) order, so pos(t,k) is the number of earlier
+// entries that chose the same expert, and the entry lands in the piece of its
+// expert whose [start, start+len) holds pos.
+//
+// Ranking is order-preserving and deterministic: one warp walks its
+// 32-token chunk in (t, k) order, 32 entries at a time; __match_any_sync
+// groups lanes that chose the same expert, a lane's rank inside its group is
+// the popcount of the group's lanes below it, and the group leader advances
+// the warp's per-expert counter, which starts at the chunk's exclusive offset
+// from the planner. No slot is claimed with atomics.
+//
+// [MegaFlux] §1: routed activations travel to the ranks computing their
+// experts. On one GPU that is a copy of token rows: one warp per destination
+// row, 16-byte vector loads and stores, padding rows written as zero.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kRmWarps = 4;
+
+__global__ void __launch_bounds__(kRmWarps * 32)
+row_maps_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int n_chunks, WsPtrs ws) {
+    extern __shared__ int32_t base_all[];   // [kRmWarps][E]
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int chunk = blockIdx.x * kRmWarps + warp;
+    if (chunk >= n_chunks) return;           // whole warp leaves; no CTA-wide barrier below
+    int32_t* base = base_all + warp * E;
+    for (int e = lane; e < E; e += 32) base[e] = ws.chunk_base[(int64_t)chunk * E + e];
+    __syncwarp();
+    const int64_t i0 = (int64_t)chunk * kTokPerChunk * K;
+    const int64_t t1 = min((int64_t)T, (int64_t)(chunk + 1) * kTokPerChunk);
+    const int64_t i1 = t1 * K;
+    uint32_t bad = 0;
+    for (int64_t ib = i0; ib < i1; ib += 32) {
+        const int64_t i = ib + lane;
+        const bool valid = i < i1;
+        int e = valid ? idx[i] : -1;
+        if (valid && (e < 0 || e >= E)) { bad = 1; e = -2; }
+        const bool ok = valid && e >= 0;
+        const unsigned m = __match_any_sync(0xffffffffu, e);
+        const int rank = __popc(m & ((1u << lane) - 1u));
+        const int pos = ok ? base[e] + rank : 0;
+        __syncwarp();
+        if (ok && lane == __ffs(m) - 1) base[e] += __popc(m);
+        __syncwarp();
+        if (ok) {
+            int row = -1;
+            const int p1 = ws.exp_piece_off[e + 1];
+            for (int p = ws.exp_piece_off[e]; p < p1; ++p) {
+                const int32_t* P = ws.pieces + (int64_t)kPieceInts * ws.exp_piece_idx[p];
+                if (pos < P[2] + P[3]) { row = P[4] + pos - P[2]; break; }
+            }
+            if (row < 0) {
+                bad = 1;
+            } else {
+                ws.row_of[i] = row;
+                ws.src_of[row] = (int32_t)(i / K);
+            }
+        }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(ws.header, MOE_DEV_BAD_INDEX);
+}
+
+constexpr int kGWarps = 8;
+constexpr int kUnroll = 8;
+
+__global__ void __launch_bounds__(kGWarps * 32)
+gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp, int nvec, WsPtrs ws) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int total = (int)ws.header[H_TOTAL_ROWS];
+    for (int row = blockIdx.x * kGWarps + warp; row < total; row += gridDim.x * kGWarps) {
+        const int s = ws.src_of[row];
+        uint4* dst = xp + (int64_t)row * nvec;
+        if (s >= 0) {
+            const uint4* src = x + (int64_t)s * nvec;
+            for (int v0 = 0; v0 < nvec; v0 += 32 * kUnroll) {
+                uint4 buf[kUnroll];
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) buf[u] = __ldg(src + v);
+                }
+#pragma unroll
+                for (int u = 0; u < kUnroll; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) dst[v] = buf[u];
+                }
+            }
+        } else {
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            for (int v = lane; v < nvec; v += 32) dst[v] = z;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_row_maps(const Shape& s, const int32_t* idx, const WsPtrs& ws, cudaStream_t st) {
+    const int grid = (s.n_chunks + kRmWarps - 1) / kRmWarps;
+    const size_t smem = sizeof(int32_t) * kRmWarps * s.E;
+    row_maps_kernel<<<grid, kRmWarps * 32, smem, st>>>(idx, s.T, s.K, s.E, s.n_chunks, ws);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const Shape& s, const void* x, void* xp, const WsPtrs& ws,
+                          cudaStream_t st) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int nvec = (int)((int64_t)s.d * s.eb / 16);
+    int64_t want = (s.rows_cap + kGWarps - 1) / kGWarps;
+    int64_t cap = (int64_t)sms * 8;
+    const int grid = (int)(want < cap ? want : cap);
+    gather_kernel<<<grid, kGWarps * 32, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(xp),
+                                                nvec, ws);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

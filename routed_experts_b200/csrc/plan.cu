@@ -1,0 +1,338 @@
+// plan.cu - the on-device greedy replication planner and tile layout (step A4),
+// one CTA of 1024 threads.
+//
+// [MoonEP] "MoonEP routing flow - live", 'Per-expert breakdown': every rank's
+// capacity is S*K entries. 'The greedy balance, step by step': each move
+// refills the currently hungriest rank in one shot from the currently biggest
+// donor; the donor may overshoot into deficit and is refilled by a later move;
+// a move slices off the donor's biggest experts; each foreign slice is one
+// weight copy.
+// [MegaFlux] "MegaFlux: Skew-Resilient MoE Megakernels via Pipelined Expert
+// Replication", §3.1 and App. A.1: planning starts from the no-replica
+// assignment under a per-GPU replica budget; §3.1 'Problem formulation':
+// token blocks of at most beta rows; §3.1 'On-device planning and route
+// construction' and App. A.2: a stable per-expert order maps every routed
+// assignment to its block.
+//
+// Readings (shared with the CPU oracle, which is written independently):
+// owner(e) = e / (E/R); every tie goes to the lowest index; a slice is the
+// tail of the rows the donor still holds of that expert; a receiver that has
+// used its budget takes nothing more, and when the hungriest rank can take
+// nothing the plan is flagged inexact; pieces are laid out in (rank, expert)
+// order, each padded to whole tiles at a tile-aligned row.
+//
+// Phases: (A) per-expert totals and per-chunk exclusive offsets from the
+// top-k kernel's chunk histograms (all threads); (B) the greedy moves (warp
+// 0, warp-shuffle arg-min/arg-max); (C) per-rank piece lists and block table
+// (one thread per rank, block scans for offsets); (D) per-expert piece index
+// in start order and the expert-major block schedule the GEMM walks.
+#include <limits.h>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 1024;
+
+// Exclusive scan of one int per thread over the whole CTA (1024 threads).
+// Returns the exclusive prefix; *total receives the sum. tmp: 32 ints.
+__device__ int block_excl_scan(int v, int* tmp, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) tmp[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = tmp[lane];
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, off);
+            if (lane >= off) w += y;
+        }
+        tmp[lane] = w;   // inclusive warp totals
+    }
+    __syncthreads();
+    const int base = warp > 0 ? tmp[warp - 1] : 0;
+    const int tot = tmp[31];
+    __syncthreads();
+    if (total) *total = tot;
+    return base + x - v;
+}
+
+struct PlanArgs {
+    int E, R, per, tile, budget, n_chunks, G;
+    int C;
+    int max_rep;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
+    extern __shared__ int32_t sm[];
+    const int E = a.E, R = a.R;
+    int32_t* part = sm;                              // [G*E]
+    int32_t* cnt = part + a.G * E;                   // [E]
+    int32_t* rem = cnt + E;                          // [E]
+    int32_t* own_pid = rem + E;                      // [E]
+    int32_t* L = own_pid + E;                        // [R]
+    int32_t* used = L + R;                           // [R]
+    int32_t* rep = used + R;                         // [max_rep][5]: rank, expert, start, len, pid
+    int32_t* pfb = rep + 5 * a.max_rep;              // [max_pieces]: first block of each piece
+    int32_t* tmp = pfb + (E + a.max_rep);            // [32]
+    __shared__ uint32_t s_status;
+    __shared__ int s_moves, s_nrep;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+    // ---------------- (A) totals and per-chunk offsets
+    if (tid == 0) s_status = 0;
+    __syncthreads();
+    {
+        uint32_t f = 0;
+        for (int c = tid; c < a.n_chunks; c += kThreads) f |= ws.chunk_flags[c];
+        if (f) atomicOr(&s_status, f);
+    }
+    const int g = tid / E, e0 = tid % E;
+    if (g < a.G) {
+        const int c0 = (int)((int64_t)g * a.n_chunks / a.G), c1 = (int)((int64_t)(g + 1) * a.n_chunks / a.G);
+        int s = 0;
+        for (int c = c0; c < c1; ++c) s += ws.chunk_counts[(int64_t)c * E + e0];
+        part[g * E + e0] = s;
+    }
+    __syncthreads();
+    if (tid < E) {
+        int run = 0;
+        for (int gg = 0; gg < a.G; ++gg) {
+            const int t = part[gg * E + tid];
+            part[gg * E + tid] = run;
+            run += t;
+        }
+        cnt[tid] = run;
+        rem[tid] = run;
+        own_pid[tid] = -1;
+        counts_out[tid] = run;
+    }
+    __syncthreads();
+    if (g < a.G) {
+        const int c0 = (int)((int64_t)g * a.n_chunks / a.G), c1 = (int)((int64_t)(g + 1) * a.n_chunks / a.G);
+        int run = part[g * E + e0];
+        for (int c = c0; c < c1; ++c) {
+            ws.chunk_base[(int64_t)c * E + e0] = run;
+            run += ws.chunk_counts[(int64_t)c * E + e0];
+        }
+    }
+    if (tid < R) {
+        int s = 0;
+        for (int e = tid * a.per; e < (tid + 1) * a.per; ++e) s += cnt[e];
+        L[tid] = s;
+        used[tid] = 0;
+    }
+    __syncthreads();
+
+    // ---------------- (B) greedy moves, warp 0
+    if (warp == 0) {
+        const int C = a.C;
+        const int cap = R * R + E;
+        int moves = 0, nrep = 0;
+        uint32_t st = 0;
+        for (;;) {
+            // hungriest rank: lowest load, lowest index on ties
+            int mv = INT_MAX, mr = INT_MAX;
+            int xv = INT_MIN, xr = INT_MAX;
+            for (int r = lane; r < R; r += 32) {
+                const int l = L[r];
+                if (l < mv) { mv = l; mr = r; }
+                if (l > xv) { xv = l; xr = r; }
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const int ov = __shfl_xor_sync(0xffffffffu, mv, off);
+                const int orr = __shfl_xor_sync(0xffffffffu, mr, off);
+                if (ov < mv || (ov == mv && orr < mr)) { mv = ov; mr = orr; }
+                const int pv = __shfl_xor_sync(0xffffffffu, xv, off);
+                const int pr = __shfl_xor_sync(0xffffffffu, xr, off);
+                if (pv > xv || (pv == xv && pr < xr)) { xv = pv; xr = pr; }
+            }
+            const int recv = mr, donor = xr;
+            if (mv >= C) break;
+            if (moves == cap) { st |= MOE_DEV_PLAN_INEXACT; break; }
+            int need = C - mv;
+            int gave = 0;
+            while (need > 0) {
+                // donor's biggest remaining expert, lowest id on ties
+                int bv = 0, be = INT_MAX;
+                for (int e = donor * a.per + lane; e < (donor + 1) * a.per; e += 32) {
+                    const int r_ = rem[e];
+                    if (r_ > bv) { bv = r_; be = e; }
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const int ov = __shfl_xor_sync(0xffffffffu, bv, off);
+                    const int oe = __shfl_xor_sync(0xffffffffu, be, off);
+                    if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+                }
+                if (bv <= 0) break;                       // donor holds nothing
+                if (used[recv] >= a.budget) break;        // no replica slot left
+                if (nrep >= a.max_rep) { st |= MOE_DEV_PLAN_INEXACT; break; }
+                const int x = bv < need ? bv : need;
+                if (lane == 0) {
+                    int32_t* q = rep + 5 * nrep;
+                    q[0] = recv; q[1] = be; q[2] = bv - x; q[3] = x; q[4] = -1;
+                    used[recv] += 1;
+                    rem[be] -= x;
+                    L[donor] -= x;
+                    L[recv] += x;
+                }
+                __syncwarp();
+                ++nrep;
+                need -= x;
+                gave += x;
+            }
+            if (gave == 0) { st |= MOE_DEV_PLAN_INEXACT; break; }
+            ++moves;
+        }
+        if (lane == 0) {
+            s_moves = moves;
+            s_nrep = nrep;
+            if (st) atomicOr(&s_status, st);
+        }
+    }
+    __syncthreads();
+    const int nrep = s_nrep;
+
+    // ---------------- (C) per-rank pieces and blocks
+    // pass 1: counts per rank (thread r); replica slices of r sorted by expert
+    int my_rep[kMaxBudget];
+    int nr = 0, np_r = 0, nb_r = 0, rows_r = 0;
+    if (tid < R) {
+        for (int i = 0; i < nrep; ++i) {
+            if (rep[5 * i] != tid) continue;
+            int j = nr++;
+            while (j > 0 && rep[5 * my_rep[j - 1] + 1] > rep[5 * i + 1]) { my_rep[j] = my_rep[j - 1]; --j; }
+            my_rep[j] = i;
+        }
+        for (int k = 0; k < nr; ++k) {
+            const int len = rep[5 * my_rep[k] + 3];
+            const int nt = (len + a.tile - 1) / a.tile;
+            np_r += 1; nb_r += nt; rows_r += nt * a.tile;
+        }
+        for (int e = tid * a.per; e < (tid + 1) * a.per; ++e) {
+            if (rem[e] > 0) {
+                const int nt = (rem[e] + a.tile - 1) / a.tile;
+                np_r += 1; nb_r += nt; rows_r += nt * a.tile;
+            }
+        }
+    }
+    int tot_p, tot_b, tot_rows;
+    const int p_off = block_excl_scan(tid < R ? np_r : 0, tmp, &tot_p);
+    const int b_off = block_excl_scan(tid < R ? nb_r : 0, tmp, &tot_b);
+    const int r_off = block_excl_scan(tid < R ? rows_r : 0, tmp, &tot_rows);
+    if (tid < R) {
+        // pass 2: merge owned experts (ascending) with replica slices (ascending)
+        int pid = p_off, bid = b_off, row = r_off, load = 0;
+        int k = 0;
+        int e = tid * a.per;
+        const int e_end = (tid + 1) * a.per;
+        for (;;) {
+            // next piece in expert order
+            int pe = INT_MAX, pstart = 0, plen = 0, rep_i = -1;
+            while (e < e_end && rem[e] <= 0) ++e;
+            if (e < e_end) { pe = e; pstart = 0; plen = rem[e]; }
+            if (k < nr && rep[5 * my_rep[k] + 1] < pe) {
+                rep_i = my_rep[k];
+                pe = rep[5 * rep_i + 1]; pstart = rep[5 * rep_i + 2]; plen = rep[5 * rep_i + 3];
+            }
+            if (pe == INT_MAX) break;
+            if (rep_i >= 0) { rep[5 * rep_i + 4] = pid; ++k; }
+            else { own_pid[e] = pid; ++e; }
+            int32_t* P = ws.pieces + (int64_t)kPieceInts * pid;
+            P[0] = pe; P[1] = tid; P[2] = pstart; P[3] = plen; P[4] = row;
+            pfb[pid] = bid;
+            const int nt = (plen + a.tile - 1) / a.tile;
+            for (int i = 0; i < nt; ++i) {
+                int32_t* B = ws.blocks + (int64_t)kBlockInts * (bid + i);
+                const int v = plen - i * a.tile;
+                B[0] = pe; B[1] = row + i * a.tile; B[2] = v < a.tile ? v : a.tile; B[3] = tid;
+            }
+            for (int r = row + plen; r < row + nt * a.tile; ++r) ws.src_of[r] = -1;
+            bid += nt;
+            row += nt * a.tile;
+            load += plen;
+            ++pid;
+        }
+        ws.rank_load[tid] = load;
+        ws.rank_replicas[tid] = used[tid];
+        ws.rank_row0[tid] = r_off;
+        if (tid == R - 1) ws.rank_row0[R] = row;
+    }
+    __syncthreads();
+
+    // ---------------- (D) per-expert piece index (start order) and block schedule
+    int np_e = 0, nb_e = 0;
+    if (tid < E) {
+        if (own_pid[tid] >= 0) { np_e = 1; nb_e = (rem[tid] + a.tile - 1) / a.tile; }
+        for (int i = 0; i < nrep; ++i) {
+            if (rep[5 * i + 1] != tid) continue;
+            np_e += 1;
+            nb_e += (rep[5 * i + 3] + a.tile - 1) / a.tile;
+        }
+    }
+    int dummy;
+    const int ep_off = block_excl_scan(tid < E ? np_e : 0, tmp, &dummy);
+    const int eb_off = block_excl_scan(tid < E ? nb_e : 0, tmp, &dummy);
+    if (tid < E) {
+        ws.exp_piece_off[tid] = ep_off;
+        ws.sched_off[tid] = eb_off;
+        if (tid == E - 1) { ws.exp_piece_off[E] = ep_off + np_e; ws.sched_off[E] = eb_off + nb_e; }
+        int pi = ep_off, bi = eb_off;
+        // the owner's prefix starts at 0; later slices were cut from the tail,
+        // so reverse creation order is ascending start order
+        if (own_pid[tid] >= 0) {
+            const int pid = own_pid[tid];
+            ws.exp_piece_idx[pi++] = pid;
+            const int nt = (rem[tid] + a.tile - 1) / a.tile;
+            for (int i = 0; i < nt; ++i) ws.sched[bi++] = pfb[pid] + i;
+        }
+        for (int i = nrep - 1; i >= 0; --i) {
+            if (rep[5 * i + 1] != tid) continue;
+            const int pid = rep[5 * i + 4];
+            ws.exp_piece_idx[pi++] = pid;
+            const int nt = (rep[5 * i + 3] + a.tile - 1) / a.tile;
+            for (int j = 0; j < nt; ++j) ws.sched[bi++] = pfb[pid] + j;
+        }
+    }
+    if (tid == 0) {
+        ws.header[H_STATUS] = s_status;
+        ws.header[H_NPIECES] = (uint32_t)tot_p;
+        ws.header[H_NBLOCKS] = (uint32_t)tot_b;
+        ws.header[H_TOTAL_ROWS] = (uint32_t)tot_rows;
+        ws.header[H_MOVES] = (uint32_t)s_moves;
+        ws.header[H_REPLICAS] = (uint32_t)nrep;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_plan(const Shape& s, int32_t* counts_out, const WsPtrs& ws, cudaStream_t st) {
+    PlanArgs a;
+    a.E = s.E; a.R = s.R; a.per = s.per; a.tile = s.tile; a.budget = s.budget;
+    a.n_chunks = s.n_chunks;
+    int G = kThreads / s.E;
+    if (G < 1) G = 1;
+    if (G > s.n_chunks) G = s.n_chunks;
+    a.G = G;
+    a.C = (int)s.C;
+    a.max_rep = s.R * s.budget;
+    const size_t smem = sizeof(int32_t) * ((size_t)G * s.E + 3 * s.E + 2 * s.R + 5 * a.max_rep +
+                                           (s.E + a.max_rep) + 32);
+    cudaError_t err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)smem);
+    if (err != cudaSuccess) return err;
+    plan_kernel<<<1, kThreads, smem, st>>>(a, counts_out, ws);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

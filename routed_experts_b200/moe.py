@@ -1,0 +1,236 @@
+"""ctypes binding of libmoe.so (include/moe.h), over torch CUDA tensors.
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels. There is no CPU fallback; if the library is missing or a call
+fails, this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import configs as _cfgs
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe.so")
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
+DEV_PLAN_INEXACT, DEV_TIMEOUT, DEV_BAD_INDEX = 1, 2, 4
+WS_PLAN, WS_LAYER, WS_LAYER_HOST = 0, 1, 2
+
+
+class MoeError(RuntimeError):
+    def __init__(self, what: str, code: int):
+        super().__init__(f"{what} failed: {status_string(code)}")
+        self.code = code
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("T", "d", "E", "K", "F", "R", "tile", "budget", "dtype",
+                                              "gating")]
+
+
+class PlanLayout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in ("header", "pieces", "blocks", "rank_load", "rank_replicas",
+                                              "rank_row0", "row_of", "src_of", "max_pieces", "max_blocks",
+                                              "rows_cap")]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m routed_experts_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, S = ctypes.c_void_p, ctypes.c_size_t
+        C = ctypes.POINTER(MoeConfig)
+        L.moe_workspace_size.argtypes = [C, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_rows_capacity.argtypes = [C, ctypes.POINTER(ctypes.c_int64)]
+        L.moe_plan_view.argtypes = [C, ctypes.POINTER(PlanLayout)]
+        L.moe_plan.argtypes = [C, P, P, P, P, P, S, P]
+        L.moe_dispatch.argtypes = [C, P, P, P, S, P]
+        L.moe_expert_ffn.argtypes = [C, P, P, P, P, P, P, S, P]
+        L.moe_expert_fc1.argtypes = [C, P, P, P, P, S, P]
+        L.moe_expert_fc2.argtypes = [C, P, P, P, P, S, P]
+        L.moe_combine.argtypes = [C, P, P, P, P, S, P]
+        L.moe_layer_fwd.argtypes = [C, P, P, P, P, P, P, S, P]
+        L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
+        L.moe_read_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_status_string.restype = ctypes.c_char_p
+        for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
+                  "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_combine", "moe_layer_fwd",
+                  "moe_layer_fwd_host", "moe_read_status"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().moe_status_string(code).decode()
+    except Exception:  # pragma: no cover
+        return f"status {code}"
+
+
+def _check(code: int, what: str):
+    if code != MOE_OK:
+        raise MoeError(what, code)
+
+
+def config(c: "_cfgs.LayerConfig") -> MoeConfig:
+    return MoeConfig(c.T, c.d, c.E, c.K, c.F, c.R, c.tile, c.budget, c.dtype, c.gating)
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ws(ws: torch.Tensor):
+    return _ptr(ws), ctypes.c_size_t(ws.numel() * ws.element_size())
+
+
+# ---------------------------------------------------------------- the C calls
+
+def moe_workspace_size(c, kind: int = WS_PLAN) -> int:
+    n = ctypes.c_size_t(0)
+    _check(lib().moe_workspace_size(ctypes.byref(config(c)), kind, ctypes.byref(n)), "moe_workspace_size")
+    return n.value
+
+
+def moe_rows_capacity(c) -> int:
+    n = ctypes.c_int64(0)
+    _check(lib().moe_rows_capacity(ctypes.byref(config(c)), ctypes.byref(n)), "moe_rows_capacity")
+    return n.value
+
+
+def moe_plan_view(c) -> dict:
+    v = PlanLayout()
+    _check(lib().moe_plan_view(ctypes.byref(config(c)), ctypes.byref(v)), "moe_plan_view")
+    return {f: getattr(v, f) for f, _ in PlanLayout._fields_}
+
+
+def moe_plan(c, logits, topk_idx, topk_w, counts, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_plan(ctypes.byref(config(c)), _ptr(logits), _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
+                          p, n, _stream(stream)), "moe_plan")
+
+
+def moe_dispatch(c, x, xp, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_dispatch(ctypes.byref(config(c)), _ptr(x), _ptr(xp), p, n, _stream(stream)), "moe_dispatch")
+
+
+def moe_expert_ffn(c, xp, w_gate_up, w_down, h, yp, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_expert_ffn(ctypes.byref(config(c)), _ptr(xp), _ptr(w_gate_up), _ptr(w_down), _ptr(h),
+                                _ptr(yp), p, n, _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_fc1(c, xp, w_gate_up, h, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_expert_fc1(ctypes.byref(config(c)), _ptr(xp), _ptr(w_gate_up), _ptr(h), p, n, _stream(stream)),
+           "moe_expert_fc1")
+
+
+def moe_expert_fc2(c, h, w_down, yp, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_expert_fc2(ctypes.byref(config(c)), _ptr(h), _ptr(w_down), _ptr(yp), p, n, _stream(stream)),
+           "moe_expert_fc2")
+
+
+def moe_combine(c, yp, topk_w, out, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_combine(ctypes.byref(config(c)), _ptr(yp), _ptr(topk_w), _ptr(out), p, n, _stream(stream)),
+           "moe_combine")
+
+
+def moe_layer_fwd(c, logits, x, w_gate_up, w_down, out, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_layer_fwd(ctypes.byref(config(c)), _ptr(logits), _ptr(x), _ptr(w_gate_up), _ptr(w_down),
+                               _ptr(out), p, n, _stream(stream)), "moe_layer_fwd")
+
+
+def moe_layer_fwd_host(c, logits_host, x_host, w_gate_up, w_down, out_host, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_layer_fwd_host(ctypes.byref(config(c)), _ptr(logits_host), _ptr(x_host), _ptr(w_gate_up),
+                                    _ptr(w_down), _ptr(out_host), p, n, _stream(stream)), "moe_layer_fwd_host")
+
+
+def moe_read_status(ws, stream=None) -> int:
+    v = ctypes.c_uint32(0)
+    _check(lib().moe_read_status(_ptr(ws), _stream(stream), ctypes.byref(v)), "moe_read_status")
+    return v.value
+
+
+# ---------------------------------------------------------------- conveniences
+
+def act_dtype(c) -> torch.dtype:
+    return torch.bfloat16 if c.dtype == _cfgs.BF16 else torch.float32
+
+
+def alloc_workspace(c, kind: int = WS_PLAN, device="cuda") -> torch.Tensor:
+    return torch.empty(moe_workspace_size(c, kind), dtype=torch.uint8, device=device)
+
+
+def read_plan(c, ws: torch.Tensor) -> dict:
+    """Copies the plan out of a workspace (after moe_plan) into host tensors."""
+    v = moe_plan_view(c)
+    raw = ws.cpu()
+
+    def arr(off, n, dt=torch.int32):
+        return raw[off: off + n * 4].view(dt).clone()
+
+    hdr = arr(v["header"], 8)
+    npc, nbl = int(hdr[1]), int(hdr[2])
+    total = int(hdr[3])
+    return {
+        "status": int(hdr[0]), "n_pieces": npc, "n_blocks": nbl, "total_rows": total, "moves": int(hdr[4]),
+        "replicas": int(hdr[5]),
+        "pieces": arr(v["pieces"], 5 * npc).view(npc, 5),
+        "blocks": arr(v["blocks"], 4 * nbl).view(nbl, 4),
+        "rank_load": arr(v["rank_load"], c.R),
+        "rank_replicas": arr(v["rank_replicas"], c.R),
+        "rank_row0": arr(v["rank_row0"], c.R + 1),
+        "row_of": arr(v["row_of"], c.T * c.K),
+        "src_of": arr(v["src_of"], total),
+    }
+
+
+class Layer:
+    """Owns a workspace for one layer shape and runs the whole layer on it."""
+
+    def __init__(self, c, device="cuda", host_io: bool = False):
+        self.cfg = c
+        self.kind = WS_LAYER_HOST if host_io else WS_LAYER
+        self.ws = alloc_workspace(c, self.kind, device)
+        self.out = torch.empty(c.T, c.d, dtype=act_dtype(c), device=device)
+
+    def forward(self, logits, x, w_gate_up, w_down, out=None, stream=None):
+        out = self.out if out is None else out
+        moe_layer_fwd(self.cfg, logits, x, w_gate_up, w_down, out, self.ws, stream)
+        return out
+
+    def forward_host(self, logits_host, x_host, w_gate_up, w_down, out_host, stream=None):
+        moe_layer_fwd_host(self.cfg, logits_host, x_host, w_gate_up, w_down, out_host, self.ws, stream)
+        return out_host
+
+    def status(self, stream=None) -> int:
+        return moe_read_status(self.ws, stream)

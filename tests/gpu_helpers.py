@@ -1,0 +1,178 @@
+"""Helpers for the GPU parity tests: run the layer through the C ABI stage by
+stage, and compare every stage with the CPU oracle on the same inputs."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from oracle import oracle as O
+from routed_experts_b200 import configs as C
+from routed_experts_b200 import inputs as I
+from routed_experts_b200 import moe as M
+
+# Output tolerances: bf16 |g - o| <= 2e-2 + 1e-2 |o| elementwise and a
+# normwise relative error <= 1e-2; fp32 |g - o| <= 1e-4 + 1e-4 |o| and
+# normwise <= 1e-5. Gating weights (fp32 on both sides, fp32 exp on the GPU,
+# fp64 in the oracle) within 1e-6.
+TOL = {C.BF16: (2e-2, 1e-2, 1e-2), C.FP32: (1e-4, 1e-4, 1e-5)}
+W_ATOL = 1e-6
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, dtype: int, what: str):
+    atol, rtol, nrm = TOL[dtype]
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    err = np.abs(got - ref)
+    bad = err > atol + rtol * np.abs(ref)
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements out of tolerance, max err {err.max():.3e}"
+    den = np.linalg.norm(ref)
+    if den > 0:
+        rel = np.linalg.norm(got - ref) / den
+        assert rel <= nrm, f"{what}: normwise error {rel:.3e} > {nrm}"
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def run_stages(cfg, inp: dict) -> dict:
+    """moe_plan, moe_dispatch, moe_expert_ffn, moe_combine on device inputs."""
+    dev = inp["x"].device
+    T, K, E, d, F = cfg.T, cfg.K, cfg.E, cfg.d, cfg.F
+    dt = M.act_dtype(cfg)
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
+    cap = M.moe_rows_capacity(cfg)
+    xp = torch.empty(cap, d, dtype=dt, device=dev)
+    h = torch.empty(cap, F, dtype=dt, device=dev)
+    yp = torch.empty(cap, d, dtype=dt, device=dev)
+    out = torch.empty(T, d, dtype=dt, device=dev)
+    M.moe_plan(cfg, inp["logits"], idx, w, counts, ws)
+    M.moe_dispatch(cfg, inp["x"], xp, ws)
+    M.moe_expert_ffn(cfg, xp, inp["w_gate_up"], inp["w_down"], h, yp, ws)
+    M.moe_combine(cfg, yp, w, out, ws)
+    status = M.moe_read_status(ws)
+    plan = M.read_plan(cfg, ws)
+    return {"idx": idx, "w": w, "counts": counts, "xp": xp, "h": h, "yp": yp, "out": out,
+            "status": status, "plan": plan, "ws": ws, "rows_cap": cap}
+
+
+def host_inputs(inp: dict, with_weights: bool = True) -> dict:
+    keys = ("logits", "x", "w_gate_up", "w_down") if with_weights else ("logits", "x")
+    return {k: I.to_numpy_bits(inp[k]) for k in keys}
+
+
+def check_routing_and_plan(cfg, g: dict, ref: dict):
+    """Bit-exact checks of top-k, counts, plan and row maps; weights within 1e-6."""
+    assert np.array_equal(g["idx"].cpu().numpy(), ref["idx"]), "top-k indices differ"
+    np.testing.assert_allclose(g["w"].cpu().numpy(), ref["w"], rtol=0, atol=W_ATOL)
+    assert np.array_equal(g["counts"].cpu().numpy(), ref["counts"]), "counts differ"
+    gp, rp = g["plan"], ref["plan"]
+    assert gp["moves"] == rp["moves"]
+    assert (gp["status"] & O.PLAN_INEXACT) == rp["status"]
+    assert gp["total_rows"] == rp["total_rows"]
+    assert np.array_equal(gp["pieces"].numpy(), rp["pieces"]), "pieces differ"
+    assert np.array_equal(gp["blocks"].numpy(), rp["blocks"]), "blocks differ"
+    assert np.array_equal(gp["rank_load"].numpy(), rp["rank_load"])
+    assert np.array_equal(gp["rank_replicas"].numpy(), rp["rank_replicas"])
+    assert np.array_equal(gp["rank_row0"].numpy(), rp["rank_row0"])
+    assert gp["replicas"] == int(rp["rank_replicas"].sum())
+    assert np.array_equal(gp["row_of"].numpy(), ref["row_of"]), "row_of differs"
+    total = rp["total_rows"]
+    assert np.array_equal(gp["src_of"].numpy(), ref["src_of"][:total]), "src_of differs"
+
+
+def oracle_routing(cfg, hin: dict) -> dict:
+    idx, w = O.topk_gate(hin["logits"], cfg.K, cfg.gating)
+    counts = O.histogram(idx, cfg.E)
+    pl = O.plan(cfg.T, cfg.E, cfg.K, cfg.R, cfg.tile, cfg.budget, counts)
+    cap = O.rows_capacity(cfg.N, cfg.E, cfg.R, cfg.budget, cfg.tile)
+    row_of, src_of = O.row_maps(idx, cfg.E, pl["pieces"], cap)
+    return {"idx": idx, "w": w, "counts": counts, "plan": pl, "row_of": row_of, "src_of": src_of,
+            "rows_cap": cap}
+
+
+def check_full_small(cfg, seed: int, device="cuda"):
+    """Every stage against the oracle, every element (sizes the oracle runs in seconds)."""
+    inp = I.make_inputs(cfg, seed, device)
+    g = run_stages(cfg, inp)
+    hin = host_inputs(inp)
+    ref = O.layer(hin["logits"], hin["x"], hin["w_gate_up"], hin["w_down"], K=cfg.K, R=cfg.R,
+                  tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype)
+    assert g["rows_cap"] == ref["rows_cap"]
+    check_routing_and_plan(cfg, g, ref)
+    assert (g["status"] & ~O.PLAN_INEXACT) == 0, f"device status {g['status']}"
+    total = ref["plan"]["total_rows"]
+    assert np.array_equal(I.to_numpy_bits(g["xp"][:total]), ref["xp"][:total]), "xp differs"
+    valid = ref["src_of"][:total] >= 0
+    gh, gy = to_f64(g["h"][:total]), to_f64(g["yp"][:total])
+    rh, ry = O.to_f64(ref["h"][:total], cfg.dtype), O.to_f64(ref["yp"][:total], cfg.dtype)
+    assert_close(gh[valid], rh[valid], cfg.dtype, "h")
+    assert_close(gy[valid], ry[valid], cfg.dtype, "yp")
+    assert not gh[~valid].any() and not gy[~valid].any(), "padding rows must be zero"
+    assert_close(to_f64(g["out"]), O.to_f64(ref["out"], cfg.dtype), cfg.dtype, "out")
+    return g, ref, inp
+
+
+class ExpertWeights:
+    """Host copies of single experts' weights, fetched on demand."""
+
+    def __init__(self, inp: dict):
+        self.wgu, self.wdn = inp["w_gate_up"], inp["w_down"]
+        self.cache = {}
+
+    def stack(self, experts):
+        es = list(experts)
+        for e in es:
+            if e not in self.cache:
+                self.cache[e] = (I.to_numpy_bits(self.wgu[e]), I.to_numpy_bits(self.wdn[e]))
+        return (np.stack([self.cache[e][0] for e in es]), np.stack([self.cache[e][1] for e in es]))
+
+
+def check_full_size(cfg, seed: int, n_tokens: int = 8, n_rows: int = 32, device="cuda"):
+    """Full-size layer: bit-exact routing, plan, row maps and dispatch; sampled
+    rows of h and yp and sampled tokens of out against the oracle."""
+    inp = I.make_inputs(cfg, seed, device)
+    g = run_stages(cfg, inp)
+    hin = host_inputs(inp, with_weights=False)
+    ref = oracle_routing(cfg, hin)
+    check_routing_and_plan(cfg, g, ref)
+    assert (g["status"] & ~O.PLAN_INEXACT) == 0, f"device status {g['status']}"
+    total = ref["plan"]["total_rows"]
+    src = ref["src_of"][:total]
+    # dispatch: every row is the token row it names (or zero), bit for bit
+    xp = I.to_numpy_bits(g["xp"][:total])
+    x = hin["x"]
+    valid = src >= 0
+    assert np.array_equal(xp[valid], x[src[valid]]), "xp rows differ from their token rows"
+    assert not xp[~valid].any(), "padding rows of xp must be zero"
+    del xp
+    rng = np.random.default_rng(seed + 17)
+    ew = ExpertWeights(inp)
+    # sampled rows of h and yp, from a few experts
+    blocks = ref["plan"]["blocks"]
+    experts = rng.choice(np.unique(blocks[:, 0]), size=min(4, len(np.unique(blocks[:, 0]))), replace=False)
+    rows, exps = [], []
+    for k, e in enumerate(experts):
+        eb = blocks[blocks[:, 0] == e]
+        cand = np.concatenate([np.arange(b[1], b[1] + b[2]) for b in eb])
+        pick = rng.choice(cand, size=min(n_rows // len(experts), len(cand)), replace=False)
+        rows += pick.tolist()
+        exps += [k] * len(pick)
+    rows = np.array(rows)
+    wgu, wdn = ew.stack(experts)
+    rh, ry = O.entry_ffn(src[rows], np.array(exps), x, wgu, wdn, cfg.dtype, O.default_round_mode(cfg.dtype))
+    assert_close(to_f64(g["h"][torch.as_tensor(rows, device=device)]), rh, cfg.dtype, "sampled h rows")
+    assert_close(to_f64(g["yp"][torch.as_tensor(rows, device=device)]), ry, cfg.dtype, "sampled yp rows")
+    # sampled tokens of the output
+    toks = rng.choice(cfg.T, size=n_tokens, replace=False)
+    gout = to_f64(g["out"][torch.as_tensor(toks, device=device)])
+    for i, t in enumerate(toks):
+        es = ref["idx"][t]
+        wgu, wdn = ew.stack(es)
+        o = O.token_out(np.array([0]), x[t:t + 1], np.arange(cfg.K, dtype=np.int32)[None, :],
+                        ref["w"][t:t + 1], wgu, wdn, cfg.dtype, O.default_round_mode(cfg.dtype))
+        assert_close(gout[i:i + 1], o, cfg.dtype, f"out[{t}]")
+    return g, ref, inp

@@ -1,0 +1,113 @@
+"""The C ABI library without a GPU: it builds, loads, exports every function
+include/moe.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from routed_experts_b200 import build
+from routed_experts_b200 import configs as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def M():
+    build.build()
+    from routed_experts_b200 import moe
+    moe.lib()
+    return moe
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_function(M):
+    names = declared_functions()
+    assert "moe_plan" in names and "moe_layer_fwd" in names and len(names) >= 13
+    lib = ctypes.CDLL(M.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(M):
+    assert M.status_string(0) == "MOE_OK"
+    assert M.status_string(3) == "MOE_ERR_WORKSPACE"
+
+
+@pytest.mark.parametrize("cfg", list(C.NAMED.values()), ids=lambda c: c.name)
+def test_sizes_of_named_configs(M, cfg):
+    from oracle import oracle as O
+    cap = M.moe_rows_capacity(cfg)
+    assert cap == O.rows_capacity(cfg.N, cfg.E, cfg.R, cfg.budget, cfg.tile)
+    plan_b = M.moe_workspace_size(cfg, M.WS_PLAN)
+    layer_b = M.moe_workspace_size(cfg, M.WS_LAYER)
+    host_b = M.moe_workspace_size(cfg, M.WS_LAYER_HOST)
+    eb = cfg.elem_bytes
+    assert plan_b < layer_b < host_b
+    assert layer_b - plan_b >= eb * cap * (2 * cfg.d + cfg.F)
+    v = M.moe_plan_view(cfg)
+    assert v["rows_cap"] == cap and v["max_pieces"] == cfg.E + cfg.R * cfg.budget
+    offs = [v[k] for k in ("header", "pieces", "blocks", "rank_load", "rank_replicas", "rank_row0",
+                           "row_of", "src_of")]
+    assert all(o % 16 == 0 for o in offs) and max(offs) < plan_b
+
+
+def _code(fn, *args):
+    return fn(*args)
+
+
+def test_invalid_configs(M):
+    L = M.lib()
+    n = ctypes.c_size_t()
+    bad = [
+        dict(T=0), dict(R=3), dict(K=9, E=8), dict(E=6, R=4), dict(budget=-1), dict(dtype=7),
+        dict(gating=5),
+    ]
+    for kw in bad:
+        cfg = C.TINY.replace(**kw)
+        assert L.moe_workspace_size(ctypes.byref(M.config(cfg)), 0, ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG, kw
+    unsupported = [
+        C.OLMOE.replace(tile=64), C.OLMOE.replace(F=1000), C.OLMOE.replace(d=2048 + 64),
+        C.TINY.replace(tile=8), C.TINY.replace(K=17, E=32), C.TINY.replace(E=2048, R=4),
+    ]
+    for cfg in unsupported:
+        assert L.moe_workspace_size(ctypes.byref(M.config(cfg)), 0, ctypes.byref(n)) == M.MOE_ERR_UNSUPPORTED, cfg
+    assert L.moe_workspace_size(None, 0, ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_workspace_size(ctypes.byref(M.config(C.TINY)), 9, ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
+
+
+def test_calls_reject_bad_pointers_and_small_workspace(M):
+    L = M.lib()
+    cfg = ctypes.byref(M.config(C.TINY))
+    fake = ctypes.c_void_p(1 << 20)      # never dereferenced: every check below fails first
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    need = M.moe_workspace_size(C.TINY, M.WS_PLAN)
+    s = ctypes.c_size_t
+    assert L.moe_plan(cfg, None, fake, fake, fake, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_plan(cfg, odd, fake, fake, fake, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_plan(cfg, fake, fake, fake, fake, fake, s(need - 1), None) == M.MOE_ERR_WORKSPACE
+    assert L.moe_plan(cfg, fake, fake, fake, fake, None, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_dispatch(cfg, fake, None, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_ffn(cfg, fake, fake, fake, fake, odd, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_combine(cfg, fake, fake, fake, fake, s(16), None) == M.MOE_ERR_WORKSPACE
+    layer_need = M.moe_workspace_size(C.TINY, M.WS_LAYER)
+    assert L.moe_layer_fwd(cfg, fake, fake, fake, fake, fake, fake, s(layer_need - 1), None) == M.MOE_ERR_WORKSPACE
+    host_need = M.moe_workspace_size(C.TINY, M.WS_LAYER_HOST)
+    assert L.moe_layer_fwd_host(cfg, fake, fake, fake, fake, fake, fake, s(host_need - 1), None) == \
+        M.MOE_ERR_WORKSPACE
+    v = ctypes.c_uint32()
+    assert L.moe_read_status(None, None, ctypes.byref(v)) == M.MOE_ERR_INVALID_ARG
+
+
+def test_binding_refuses_to_run_without_library(tmp_path, monkeypatch):
+    from routed_experts_b200 import moe
+    monkeypatch.setattr(moe, "_lib", None)
+    monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        moe.lib()
