@@ -22,7 +22,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -50,7 +49,7 @@ def parse():
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--impl", default="mine", choices=["mine", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-tokens", type=int, default=48, help="tokens of the oracle's FFN sample")
+    p.add_argument("--cpu-tokens", type=int, default=320, help="tokens of the oracle's FFN sample")
     return p.parse_args()
 
 
@@ -64,58 +63,70 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 100 ms while running."""
+    """SM clock, its maximum and the active clock-event (throttle) reasons of
+    one GPU, polled through NVML every 2 ms while the timed region runs (the
+    region can be only tens of milliseconds long). Reads settings only."""
 
-    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    def __init__(self, device: torch.device):
+        self.device = device
+        self.samples = []
+        self.sm_max = None
+        self.handle = None
+        self.stop = threading.Event()
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def _handle(self):
+        import pynvml as N
+        N.nvmlInit()
+        p = torch.cuda.get_device_properties(self.device)
+        try:
+            bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+            return N.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+            ids = [v for v in vis.split(",") if v.strip()]
+            idx = self.device.index or 0
+            return N.nvmlDeviceGetHandleByIndex(int(ids[idx]) if idx < len(ids) and ids[idx].isdigit() else idx)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml as N
+            self.N = N
+            self.handle = self._handle()
+            self.sm_max = N.nvmlDeviceGetMaxClockInfo(self.handle, N.NVML_CLOCK_SM)
+            self.t = threading.Thread(target=self._poll, daemon=True)
             self.t.start()
         except Exception:
-            self.proc = None
+            self.handle = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll(self):
+        N = self.N
+        while not self.stop.is_set():
+            try:
+                sm = N.nvmlDeviceGetClockInfo(self.handle, N.NVML_CLOCK_SM)
+                rs = N.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __exit__(self, *a):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self.stop.set()
+        if self.handle is not None:
             self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 7:
-                continue
-            try:
-                sm.append(float(f[0]))
-                mx = float(f[1])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[3:7]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [], "samples": 0}
+        N = self.N
+        names = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                 "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                 "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                 "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap,
+                 "hw_power_brake": N.nvmlClocksEventReasonHwPowerBrakeSlowdown}
+        reasons = sorted(n for n, bit in names.items() if any(r & bit for _, r in self.samples))
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.sm_max,
+                "reasons": reasons, "samples": len(self.samples), "source": "NVML, 2 ms polling"}
 
 
 def source_sha(*rel):
@@ -161,7 +172,7 @@ def run_reference(args, world, rank):
     inp = I.make_inputs(cfg, args.seed, "cpu")
     h = {k: I.to_numpy_bits(v) for k, v in inp.items()}
     kw = dict(K=cfg.K, R=cfg.R, tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype)
-    n_tok = max(2, args.cpu_tokens // 4)
+    n_tok = max(2, args.cpu_tokens // 16)
     for _ in range(args.warmup):
         O.timed_sample(h["logits"], h["x"], h["w_gate_up"], h["w_down"], n_tokens=2, **kw)
     est = []
@@ -251,9 +262,7 @@ def run_mine(args, world, rank, local):
     torch.cuda.synchronize(dev)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
-    smi_index = int(vis.split(",")[local]) if vis and vis.split(",")[local].strip().isdigit() else local
-    with ClockSampler(smi_index) as clk:
+    with ClockSampler(dev) as clk:
         t0.record(stream)
         for k in range(args.steps):
             step(evs[k])
