@@ -216,6 +216,35 @@ moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, c
                               const void* w_gate_up, const void* w_down, void* out_host,
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/*
+ * moe_plan_noalloc - moe_plan for callers that cannot allocate device
+ * memory. The papers have no counterpart: this is an interface for callers
+ * that are handed only their inputs and outputs (a plugin inside another
+ * framework's engine with no workspace to offer, or a serving loop whose
+ * device memory is reserved up front by its own pool allocator, where
+ * cudaMalloc can fail once the pool holds the free memory and can stall the
+ * device mid-step).
+ *   logits, topk_idx, topk_w, counts: as in moe_plan.
+ *   row_of  int32 [T*K] (device, out): padded row of entry (t, k), as in
+ *           moe_plan_layout.
+ *   header  uint32 [8] (device, out): device status bits, n_pieces,
+ *           n_blocks, total_rows, moves, replicas in total, 0, 0 - as the
+ *           header of moe_plan_layout.
+ * The planner's scratch lives in one static device array of
+ * MOE_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library keeps reserved until the process exits. A shape whose scratch
+ * exceeds it returns MOE_ERR_WORKSPACE (moe_workspace_size with MOE_WS_PLAN
+ * gives the bytes a shape needs). The call allocates and frees nothing.
+ * The first call on each device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Every call shares the one array and it keeps the last call's contents;
+ * calls that overlap on the GPU (for example on two streams at once) race
+ * on it, so order them on one stream or with events.
+ */
+#define MOE_NOALLOC_SCRATCH_BYTES ((size_t)4 << 20)
+moe_status moe_plan_noalloc(const moe_config* cfg, const float* logits, int32_t* topk_idx, float* topk_w,
+                            int32_t* counts, int32_t* row_of, uint32_t* header, moe_stream_t stream);
+
 /* Synchronises `stream`, then reads the device status bits of `ws`. */
 moe_status moe_read_status(const void* ws, moe_stream_t stream, uint32_t* dev_bits);
 

@@ -7,7 +7,7 @@
 
 using namespace moe;
 
-namespace {
+namespace moe {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -76,6 +76,10 @@ WsLayout make_layout(const Shape& s) {
     L.host_end = o;
     return L;
 }
+
+}  // namespace moe
+
+namespace {
 
 moe_status check_ws(const void* ws, size_t ws_bytes, int64_t need) {
     if (!ws || !aligned16(ws)) return MOE_ERR_INVALID_ARG;

@@ -94,6 +94,13 @@ __device__ inline void set_status(uint32_t* header, uint32_t bits) {
     atomicOr(header + H_STATUS, bits);
 }
 
+// ---- shape and workspace layout, defined in api.cu ----
+bool aligned16(const void* p);
+// Validates cfg and fills the derived shape: INVALID_ARG for an ill-formed
+// cfg, UNSUPPORTED for a well-formed one no kernel covers.
+moe_status make_shape(const moe_config* cfg, Shape* s);
+WsLayout make_layout(const Shape& s);
+
 // ---- launchers (one per kernel family), defined in the kernel files ----
 cudaError_t launch_topk_hist(const Shape& s, const float* logits, int32_t* idx, float* w,
                              const WsPtrs& ws, cudaStream_t st);

@@ -63,11 +63,12 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_fwd.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_read_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+        L.moe_plan_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_combine", "moe_layer_fwd",
-                  "moe_layer_fwd_host", "moe_read_status"):
+                  "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -172,6 +173,12 @@ def moe_layer_fwd_host(c, logits_host, x_host, w_gate_up, w_down, out_host, ws, 
     p, n = _ws(ws)
     _check(lib().moe_layer_fwd_host(ctypes.byref(config(c)), _ptr(logits_host), _ptr(x_host), _ptr(w_gate_up),
                                     _ptr(w_down), _ptr(out_host), p, n, _stream(stream)), "moe_layer_fwd_host")
+
+
+def moe_plan_noalloc(c, logits, topk_idx, topk_w, counts, row_of, header, stream=None):
+    """moe_plan with its scratch in the library's static device array (no workspace)."""
+    _check(lib().moe_plan_noalloc(ctypes.byref(config(c)), _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
+                                  _ptr(counts), _ptr(row_of), _ptr(header), _stream(stream)), "moe_plan_noalloc")
 
 
 def moe_read_status(ws, stream=None) -> int:
