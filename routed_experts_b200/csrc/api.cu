@@ -62,6 +62,7 @@ WsLayout make_layout(const Shape& s) {
     L.rank_row0 = take(sizeof(int32_t) * (s.R + 1));
     L.row_of = take(sizeof(int32_t) * s.N);
     L.src_of = take(sizeof(int32_t) * s.rows_cap);
+    L.gemm_q = take(sizeof(int32_t) * kGemmQWords);
     L.plan_end = o;
     L.idx = take(sizeof(int32_t) * s.N);
     L.w = take(sizeof(float) * s.N);

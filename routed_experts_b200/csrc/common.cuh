@@ -22,6 +22,10 @@ constexpr int kBlockInts = 4;             // expert, row0, valid, rank
 enum { H_STATUS = 0, H_NPIECES = 1, H_NBLOCKS = 2, H_TOTAL_ROWS = 3, H_MOVES = 4,
        H_REPLICAS = 5, H_WORDS = 8 };
 
+// Work-queue counters of the grouped GEMM: for FC1 then FC2, two queue
+// heads and a count of clusters that finished (all zero between launches).
+constexpr int kGemmQWords = 8;
+
 // Default bound of a device-side spin (clock cycles, about 2 s at 1.9 GHz).
 constexpr long long kSpinBudget = 4000000000LL;
 
@@ -38,7 +42,7 @@ struct Shape {
 // Byte offsets of every array in a workspace.
 struct WsLayout {
     int64_t header, chunk_counts, chunk_base, chunk_flags, pieces, exp_piece_off, exp_piece_idx,
-        blocks, sched_off, sched, rank_load, rank_replicas, rank_row0, row_of, src_of;
+        blocks, sched_off, sched, rank_load, rank_replicas, rank_row0, row_of, src_of, gemm_q;
     int64_t plan_end;
     // MOE_WS_LAYER extras
     int64_t idx, w, counts, xp, h, yp;
@@ -67,6 +71,7 @@ struct WsPtrs {
     int32_t* rank_row0;
     int32_t* row_of;
     int32_t* src_of;
+    int32_t* gemm_q;     // [kGemmQWords] work-queue counters of the two GEMM launches
 };
 
 inline WsPtrs ws_ptrs(void* ws, const WsLayout& L) {
@@ -87,6 +92,7 @@ inline WsPtrs ws_ptrs(void* ws, const WsLayout& L) {
     p.rank_row0 = reinterpret_cast<int32_t*>(b + L.rank_row0);
     p.row_of = reinterpret_cast<int32_t*>(b + L.row_of);
     p.src_of = reinterpret_cast<int32_t*>(b + L.src_of);
+    p.gemm_q = reinterpret_cast<int32_t*>(b + L.gemm_q);
     return p;
 }
 

@@ -1,30 +1,51 @@
 // ffn_tc.cu - the grouped SwiGLU expert FFN on the 5th-generation tensor cores
 // (steps A7, A8 for bf16 layers): a persistent, warp-specialised tcgen05 GEMM
-// over the planned token blocks, fed by TMA, accumulating in TMEM.
+// over the planned token blocks, run by CTA pairs, fed by TMA, accumulating
+// in TMEM.
 //
 // [MegaFlux] "MegaFlux: Skew-Resilient MoE Megakernels via Pipelined Expert
 // Replication", §2.1 'Persistent MoE execution': persistent CTAs with
 // warp-specialised workers (token movement, MMA, epilogue), tcgen05 MMA with
-// fp32 accumulation in TMEM, operands staged by TMA; §3.1 'Problem
-// formulation': the token blocks of the plan match the FC1/FC2 token tile
-// (128 rows here); §3.2 'Forward': FC1 needs W1 and an input block, FC2 needs
-// W2 and the finished activation block.
+// fp32 accumulation in TMEM, operands staged by TMA, and two-CTA MMA; §3.1
+// 'Problem formulation': the token blocks of the plan match the FC1/FC2 token
+// tile (128 rows here); §3.2 'Forward': FC1 needs W1 and an input block, FC2
+// needs W2 and the finished activation block.
 //
-// Work item = (planned block of one expert, column tile). FC1 tiles are 128
-// gate columns plus the matching 128 up columns, computed as one 128x256 MMA
-// tile so the SwiGLU epilogue has both halves in one TMEM accumulator
-// (gate+up fused in one pass over the A tile); FC2 tiles are 256 columns of
-// d. Items are ordered expert-major (then column tile, then block), so the
-// CTAs running at one time share a few experts' weight tiles in L2, and a
-// block's activation rows are reused across its expert's column tiles.
+// Work item = (two planned blocks of one expert, column tile), computed by a
+// cluster of two CTAs on neighbouring SMs as one 256 x 256 MMA tile
+// (tcgen05.mma.cta_group::2, M = 256, N = 256, K = 16): each CTA holds its own
+// block's 128 activation rows and half (128 rows) of the weight tile in its
+// shared memory, and receives its 128 rows of the accumulator in its own TMEM.
+// So every CTA loads 32 KB per 64-deep k-step instead of 48 KB for a 128 x 256
+// tile of its own. FC1 tiles are 128 gate columns (even CTA's weight half)
+// plus the matching 128 up columns (odd CTA's half), so both halves of SwiGLU
+// sit side by side in each CTA's accumulator; FC2 tiles are 256 columns of d.
+// An expert with an odd number of blocks gives its last pair one block: the
+// odd CTA then reloads the even CTA's rows and stores nothing.
 //
-// CTA = 6 warps: warp 0 issues TMA loads into a 4-stage ring (A 128x64 and
-// B 256x64 bf16 per stage, 128-byte swizzle); warp 1 allocates 512 TMEM
-// columns and one thread issues tcgen05.mma (M=128, N=256, K=16) into one of
-// two accumulators; warps 2-5 drain the other accumulator (tcgen05.ld), apply
-// the epilogue and store bf16 rows, so epilogue and MMA overlap. Every wait is
-// bounded: a wait that runs out sets MOE_DEV_TIMEOUT, raises a CTA-wide abort
-// flag, lets in-flight copies and MMAs finish, frees TMEM and returns.
+// Scheduling is dynamic. Items are listed expert-major (then column tile,
+// then block pair), so consecutive items share an expert's weight tiles and a
+// pair's activation rows. The list is cut at an expert boundary into two
+// halves with a queue each (global atomic counters in the workspace); a
+// cluster takes items from the queue of its half of the GPU (by the SM index
+// of its even CTA) and steals from the other queue once its own is empty. The
+// even CTA's TMA thread fetches each item and hands it to every consumer of
+// both CTAs through a small ring in shared memory (a remote store plus a
+// remote mbarrier arrive for the odd CTA). A scheduler warp of the even CTA
+// fetches and decodes items several ahead (expert, column tile, first rows of
+// both blocks), so no role waits on a global load at an item boundary. The
+// last cluster to finish resets the counters for the next launch.
+//
+// CTA = 7 warps: warp 0 issues TMA loads into a 6-stage ring of 32 KB stages
+// (128-byte swizzle), counted on the even CTA's "full" barrier; warp 6 of the
+// even CTA fetches and decodes work items; warp 1 of the
+// even CTA issues the pair MMAs into one of two 256-column accumulators and
+// commits to the "empty"/"full" barriers of both CTAs; warps 2-5 of each CTA
+// drain the other accumulator (tcgen05.ld), apply the epilogue and store bf16
+// rows, then arrive on the even CTA's "accumulator empty" barrier. Every wait
+// is bounded: a wait that runs out sets MOE_DEV_TIMEOUT, raises the CTA's
+// abort flag, lets its in-flight copies and MMAs finish and returns; both CTAs
+// then meet at the cluster barrier and free TMEM.
 #include <cudaTypedefs.h>
 #include <math.h>
 
@@ -36,12 +57,19 @@
 namespace moe {
 namespace {
 
-constexpr int kBM = 128, kBK = 64, kStages = 4, kThreads = 192;
-constexpr int kN = 256;                       // accumulator columns per item
-constexpr uint32_t kTmemCols = 2 * kN;        // two accumulators
-constexpr int kABytes = kBM * kBK * 2;        // 16 KB
-constexpr int kBBytes = kN * kBK * 2;         // 32 KB
+constexpr int kBM = 128, kBK = 64, kStages = 6, kThreads = 224;
+constexpr int kN = 256;                        // accumulator columns per item (pair MMA N)
+constexpr int kHalfN = 128;                    // weight rows each CTA of the pair holds
+constexpr uint32_t kTmemCols = 2 * kN;         // two accumulators
+constexpr int kABytes = kBM * kBK * 2;         // 16 KB
+constexpr int kBBytes = kHalfN * kBK * 2;      // 16 KB
+constexpr int kStageBytes = kABytes + kBBytes; // 32 KB
 constexpr long long kDrainBudget = 2000000000LL;
+constexpr int kItemSlots = 4;                  // ring of fetched, decoded work items (few: a short window keeps L2 reuse)
+// item-slot consumers: TMA thread, MMA thread and 4 epilogue warps of the even
+// CTA; TMA thread and 4 epilogue warps of the odd CTA
+constexpr uint32_t kItemConsumers = 11;
+constexpr int kSchedWarp = 6;
 
 struct TcArgs {
     __nv_bfloat16* out;       // h (FC1) or yp (FC2)
@@ -56,16 +84,19 @@ struct TcArgs {
     const int32_t* sched;
     const int32_t* sched_off;
     uint32_t* header;
+    int32_t* queue;           // [3]: head of queue 0, head of queue 1, clusters finished
 };
 
 struct Smem {
     uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
+    uint64_t item_full[kItemSlots], item_empty[kItemSlots];
+    int4 items[kItemSlots];   // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
     uint32_t tmem_base;
     int abort_flag;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * (kABytes + kBBytes) + sizeof(Smem) +
-                              sizeof(int32_t) * (kMaxE + 1);
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + sizeof(Smem) +
+                              2 * sizeof(int32_t) * (kMaxE + 1);
 
 __device__ __forceinline__ bool role_wait(uint64_t* bar, uint32_t parity, long long budget,
                                           volatile int* abort_flag, uint32_t* header) {
@@ -82,23 +113,53 @@ __device__ __forceinline__ bool role_wait(uint64_t* bar, uint32_t parity, long l
     }
 }
 
-// Work item -> (expert, first row, column tile). Items run expert-major:
-// expert e owns items [n_tiles*off[e], n_tiles*off[e+1]), column tile major,
-// then its blocks in schedule order.
-__device__ __forceinline__ void decode_item(long long it, int n_tiles, const int32_t* s_off, int E,
-                                            const int32_t* sched, const int32_t* blocks, int& expert,
-                                            int& row0, int& j) {
+// As role_wait, acquiring at cluster scope (the item ring of the odd CTA is
+// written by the even CTA).
+__device__ __forceinline__ bool role_wait_cluster(uint64_t* bar, uint32_t parity, long long budget,
+                                                  volatile int* abort_flag, uint32_t* header) {
+    if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (clock64() - t0 > budget) {
+            *abort_flag = 1;
+            atomicOr(header + H_STATUS, (uint32_t)MOE_DEV_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+// Next work item for a cluster of group g (0 or 1), or -1 when none is left:
+// its own half of the list first, then the other half.
+__device__ __forceinline__ int fetch_item(int32_t* queue, int g, int split, int n_items) {
+    const int lo = g ? split : 0, hi = g ? n_items : split;
+    const int i = atomicAdd(&queue[g], 1);
+    if (lo + i < hi) return lo + i;
+    const int lo2 = g ? 0 : split, hi2 = g ? split : n_items;
+    const int i2 = atomicAdd(&queue[1 - g], 1);
+    if (lo2 + i2 < hi2) return lo2 + i2;
+    return -1;
+}
+
+// Work item -> (expert, its two blocks, column tile). Expert e owns items
+// [n_tiles*p_off[e], n_tiles*p_off[e+1]), column tile major, then its block
+// pairs in schedule order; b1 = -1 when the pair has one block.
+__device__ __forceinline__ void decode_item(long long it, int n_tiles, const int32_t* s_off, const int32_t* p_off,
+                                            int E, const int32_t* sched, int& e, int& b0, int& b1, int& j) {
     int lo = 0, hi = E;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if ((long long)n_tiles * s_off[mid] <= it) lo = mid; else hi = mid;
+        if ((long long)n_tiles * p_off[mid] <= it) lo = mid; else hi = mid;
     }
+    const int np = p_off[lo + 1] - p_off[lo];
     const int nb = s_off[lo + 1] - s_off[lo];
-    const long long local = it - (long long)n_tiles * s_off[lo];
-    j = (int)(local / nb);
-    const int b = sched[s_off[lo] + (int)(local % nb)];
-    expert = blocks[kBlockInts * b];
-    row0 = blocks[kBlockInts * b + 1];
+    const long long local = it - (long long)n_tiles * p_off[lo];
+    j = (int)(local / np);
+    const int q = (int)(local % np);
+    e = lo;
+    b0 = sched[s_off[lo] + 2 * q];
+    b1 = 2 * q + 1 < nb ? sched[s_off[lo] + 2 * q + 1] : -1;
 }
 
 __device__ __forceinline__ float silu(float a) { return a / (1.f + __expf(-a)); }
@@ -110,159 +171,260 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 // MODE 0: FC1 + SwiGLU -> h; MODE 1: FC2 -> yp.
 template <int MODE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* sA = base;
-    uint8_t* sB = base + kStages * kABytes;
-    Smem* S = reinterpret_cast<Smem*>(sB + kStages * kBBytes);
+    Smem* S = reinterpret_cast<Smem*>(base + kStages * kStageBytes);
     int32_t* s_off = reinterpret_cast<int32_t*>(S + 1);
+    int32_t* p_off = s_off + (a.E + 1);
     volatile int* abort_flag = &S->abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = ptx::cluster_ctarank();
+    const bool even = rank == 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) { ptx::mbar_init(&S->full[s], 1); ptx::mbar_init(&S->empty[s], 1); }
-        for (int q = 0; q < 2; ++q) { ptx::mbar_init(&S->acc_full[q], 1); ptx::mbar_init(&S->acc_empty[q], 128); }
+        for (int q = 0; q < 2; ++q) { ptx::mbar_init(&S->acc_full[q], 1); ptx::mbar_init(&S->acc_empty[q], 8); }
+        for (int q = 0; q < kItemSlots; ++q) {
+            ptx::mbar_init(&S->item_full[q], 1);
+            ptx::mbar_init(&S->item_empty[q], kItemConsumers);
+        }
         ptx::mbar_init(&S->drain, 1);
         S->abort_flag = 0;
         ptx::fence_barrier_init();
     }
     for (int i = threadIdx.x; i <= a.E; i += kThreads) s_off[i] = a.sched_off[i];
+    __syncthreads();
+    if (warp == 0) {
+        // pair offsets: p_off[e] = sum over e' < e of ceil(blocks(e') / 2)
+        int carry = 0;
+        if (lane == 0) p_off[0] = 0;
+        for (int b = 0; b < a.E; b += 32) {
+            const int i = b + lane;
+            const int v = i < a.E ? (s_off[i + 1] - s_off[i] + 1) >> 1 : 0;
+            int x = v;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (i < a.E) p_off[i + 1] = carry + x;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+    }
     if (warp == 0 && lane == 0) { ptx::prefetch_tmap(&tmA); ptx::prefetch_tmap(&tmB); }
-    if (warp == 1) { ptx::tmem_alloc(&S->tmem_base, kTmemCols); ptx::tmem_relinquish(); }
+    __syncthreads();
+    ptx::cluster_sync();   // the peer's barriers exist before any remote arrive, store or copy
+    if (warp == 1) { ptx::tmem_alloc_pair(&S->tmem_base, kTmemCols); ptx::tmem_relinquish_pair(); }
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    const long long n_items = (long long)a.header[H_NBLOCKS] * a.n_tiles;
+    const int n_items = p_off[a.E] * a.n_tiles;
     const int kb_count = a.Kdim / kBK;
     constexpr int kColTile = MODE == 0 ? 128 : 256;
 
-    if (warp == 0) {
-        // ------------------------------------------------ TMA producer
+    // the ring slot of the k-th item, and the parity of its phase
+    auto slot_of = [](int k) { return k % kItemSlots; };
+    auto parity_of = [](int k) { return (uint32_t)((k / kItemSlots) & 1); };
+    // take item k from the ring (both CTAs; the slot barriers of "empty" live in
+    // the even CTA). Returns false when the wait gave up.
+    auto take_item = [&](int k, int4& item) -> bool {
+        if (!role_wait_cluster(&S->item_full[slot_of(k)], parity_of(k), a.spin, abort_flag, a.header)) return false;
+        item = S->items[slot_of(k)];
+        return true;
+    };
+    auto release_item = [&](int k) {
+        ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_empty[slot_of(k)]), 0));
+    };
+
+    if (warp == kSchedWarp) {
+        // ------------------------------------------------ scheduler (even CTA)
+        if (lane == 0 && even) {
+            // group of this cluster: the half of the GPU its even CTA runs on
+            const int g = ptx::smid() >= (ptx::nsmid() >> 1) ? 1 : 0;
+            int lo = 0, hi = a.E;   // first expert whose pairs start at or after half of all pairs
+            const int half = p_off[a.E] / 2;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (p_off[mid] < half) lo = mid + 1; else hi = mid;
+            }
+            const int split = p_off[lo] * a.n_tiles;
+            int next = fetch_item(a.queue, g, split, n_items);
+            for (int k = 0;; ++k) {
+                int4 item = make_int4(-1, 0, -1, -1);
+                bool ok = role_wait(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
+                if (ok && next >= 0) {
+                    int e, b0, b1, j;
+                    decode_item(next, a.n_tiles, s_off, p_off, a.E, a.sched, e, b0, b1, j);
+                    item = make_int4(e, j, a.blocks[kBlockInts * b0 + 1], b1 >= 0 ? a.blocks[kBlockInts * b1 + 1] : -1);
+                }
+                // publish to both CTAs
+                S->items[slot_of(k)] = item;
+                const uint32_t peer = ptx::map_to_rank(ptx::smem_addr(&S->items[slot_of(k)]), 1);
+                ptx::st_cluster_u32(peer, (uint32_t)item.x);
+                ptx::st_cluster_u32(peer + 4, (uint32_t)item.y);
+                ptx::st_cluster_u32(peer + 8, (uint32_t)item.z);
+                ptx::st_cluster_u32(peer + 12, (uint32_t)item.w);
+                ptx::mbar_arrive(&S->item_full[slot_of(k)]);
+                ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_full[slot_of(k)]), 1));
+                if (item.x < 0) break;
+                next = fetch_item(a.queue, g, split, n_items);   // its latency hides behind the ring
+            }
+            // the last cluster to finish resets the queues for the next launch
+            __threadfence();
+            const int done = atomicAdd(&a.queue[2], 1);
+            if (done == (int)ptx::cluster_count_x() - 1) {
+                a.queue[0] = 0;
+                a.queue[1] = 0;
+                __threadfence();
+                a.queue[2] = 0;
+            }
+        }
+    } else if (warp == 0) {
+        // ------------------------------------------------ TMA producer (both CTAs)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
             long long fills = 0;
             bool ok = true;
-            for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-                int e, row0, j;
-                decode_item(it, a.n_tiles, s_off, a.E, a.sched, a.blocks, e, row0, j);
-                const int brow = e * a.b_rows + j * kColTile;
+            for (int k = 0; ok; ++k) {
+                int4 item;
+                if (!take_item(k, item)) { ok = false; break; }
+                release_item(k);
+                if (item.x < 0) break;
+                const int e = item.x, j = item.y;
+                const int row0 = even ? item.z : (item.w >= 0 ? item.w : item.z);
+                const int brow = e * a.b_rows + j * kColTile + (even ? 0 : (MODE == 0 ? a.F : kHalfN));
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!role_wait(&S->empty[stage], phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
-                    ptx::mbar_arrive_expect_tx(&S->full[stage], kABytes + kBBytes);
-                    ptx::tma_load_2d(sA + stage * kABytes, &tmA, kb * kBK, row0, &S->full[stage]);
-                    if (MODE == 0) {
-                        ptx::tma_load_2d(sB + stage * kBBytes, &tmB, kb * kBK, brow, &S->full[stage]);
-                        ptx::tma_load_2d(sB + stage * kBBytes + kBBytes / 2, &tmB, kb * kBK, brow + a.F,
-                                         &S->full[stage]);
-                    } else {
-                        ptx::tma_load_2d(sB + stage * kBBytes, &tmB, kb * kBK, brow, &S->full[stage]);
-                    }
+                    if (even) ptx::mbar_arrive_expect_tx(&S->full[stage], 2 * kStageBytes);
+                    const uint32_t bar = ptx::map_to_rank(ptx::smem_addr(&S->full[stage]), 0);
+                    uint8_t* st = base + stage * kStageBytes;
+                    ptx::tma_load_2d_pair(st, &tmA, kb * kBK, row0, bar);
+                    ptx::tma_load_2d_pair(st + kABytes, &tmB, kb * kBK, brow, bar);
                     ++fills;
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
             }
-            if (!ok) {
-                // let every copy still in flight land before the CTA exits
+            if (!ok && even) {
+                // let the copies still in flight land before the CTA exits
                 const long long first = fills > kStages ? fills - kStages : 0;
                 for (long long f = first; f < fills; ++f)
                     ptx::mbar_wait(&S->full[f % kStages], (uint32_t)((f / kStages) & 1), kDrainBudget);
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = ptx::idesc_bf16_f32(kBM, kN);
+        // ------------------------------------------------ MMA issuer (even CTA)
+        if (lane == 0 && even) {
+            const uint32_t idesc = ptx::idesc_bf16_f32(2 * kBM, kN);
             int stage = 0;
             uint32_t phase = 0;
-            int local = 0;
             bool ok = true, issued = false;
-            for (long long it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++local) {
-                const int acc = local & 1;
-                const uint32_t acc_phase = (uint32_t)((local >> 1) & 1);
+            for (int k = 0; ok; ++k) {
+                int4 item;
+                if (!take_item(k, item)) { ok = false; break; }
+                release_item(k);
+                if (item.x < 0) break;
+                const int acc = k & 1;
+                const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
                 if (!role_wait(&S->acc_empty[acc], acc_phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * kN);
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!role_wait(&S->full[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    const uint32_t a_addr = ptx::smem_addr(sA + stage * kABytes);
-                    const uint32_t b_addr = ptx::smem_addr(sB + stage * kBBytes);
+                    const uint32_t a_addr = ptx::smem_addr(base + stage * kStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
 #pragma unroll
                     for (int ks = 0; ks < kBK / 16; ++ks) {
-                        ptx::mma_bf16(d_tmem, ptx::sdesc_k_sw128(a_addr + ks * 32), ptx::sdesc_k_sw128(b_addr + ks * 32),
-                                      idesc, (kb | ks) != 0 ? 1u : 0u);
+                        ptx::mma_bf16_pair(d_tmem, ptx::sdesc_k_sw128(a_addr + ks * 32),
+                                           ptx::sdesc_k_sw128(b_addr + ks * 32), idesc, (kb | ks) != 0 ? 1u : 0u);
                     }
                     issued = true;
-                    ptx::mma_commit(&S->empty[stage]);
+                    const uint32_t empty_addr = ptx::smem_addr(&S->empty[stage]);
+                    ptx::mma_commit_pair(empty_addr);
+                    ptx::mma_commit_pair(ptx::map_to_rank(empty_addr, 1));
                     if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
-                if (ok) ptx::mma_commit(&S->acc_full[acc]);
+                if (ok) {
+                    const uint32_t full_addr = ptx::smem_addr(&S->acc_full[acc]);
+                    ptx::mma_commit_pair(full_addr);
+                    ptx::mma_commit_pair(ptx::map_to_rank(full_addr, 1));
+                }
             }
             if (!ok && issued) {
                 // wait for every MMA issued so far before TMEM is freed
-                ptx::mma_commit(&S->drain);
+                ptx::mma_commit_pair(ptx::smem_addr(&S->drain));
                 ptx::mbar_wait(&S->drain, 0, kDrainBudget);
             }
         }
     } else {
-        // ------------------------------------------------ epilogue, warps 2..5
+        // ------------------------------------------------ epilogue, warps 2..5 of both CTAs
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
-        const int m = quad * 32 + lane;            // row inside the tile
-        int local = 0;
-        for (long long it = blockIdx.x; it < n_items; it += gridDim.x, ++local) {
-            int e, row0, j;
-            decode_item(it, a.n_tiles, s_off, a.E, a.sched, a.blocks, e, row0, j);
-            const int acc = local & 1;
-            const uint32_t acc_phase = (uint32_t)((local >> 1) & 1);
+        const int m = quad * 32 + lane;            // row inside this CTA's block
+        for (int k = 0;; ++k) {
+            int4 item;
+            if (!take_item(k, item)) break;
+            __syncwarp();
+            if (lane == 0) release_item(k);
+            if (item.x < 0) break;
+            const int j = item.y;
+            const int row0 = even ? item.z : item.w;   // -1: this CTA's half of the pair is empty
+            const int acc = k & 1;
+            const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
             if (!role_wait(&S->acc_full[acc], acc_phase, a.spin, abort_flag, a.header)) break;
             ptx::tc_fence_after();
-            const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN);
-            uint4* orow = reinterpret_cast<uint4*>(a.out + (int64_t)(row0 + m) * a.out_ld + (int64_t)j * kColTile);
-            if (MODE == 0) {
+            if (row0 >= 0) {
+                const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN);
+                uint4* orow =
+                    reinterpret_cast<uint4*>(a.out + (int64_t)(row0 + m) * a.out_ld + (int64_t)j * kColTile);
+                if (MODE == 0) {
 #pragma unroll 1
-                for (int c = 0; c < 128; c += 32) {
-                    uint32_t g[32], u[32];
-                    ptx::tmem_ld32(t_row + c, g);
-                    ptx::tmem_ld32(t_row + 128 + c, u);
-                    ptx::tmem_ld_wait();
-                    uint32_t pk[16];
+                    for (int c = 0; c < 128; c += 32) {
+                        uint32_t gt[32], up[32];
+                        ptx::tmem_ld32(t_row + c, gt);
+                        ptx::tmem_ld32(t_row + 128 + c, up);
+                        ptx::tmem_ld_wait();
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float h0 = silu(__uint_as_float(g[2 * i])) * __uint_as_float(u[2 * i]);
-                        const float h1 = silu(__uint_as_float(g[2 * i + 1])) * __uint_as_float(u[2 * i + 1]);
-                        pk[i] = pack_bf16(h0, h1);
+                        for (int i = 0; i < 16; ++i) {
+                            const float h0 = silu(__uint_as_float(gt[2 * i])) * __uint_as_float(up[2 * i]);
+                            const float h1 = silu(__uint_as_float(gt[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
+                            pk[i] = pack_bf16(h0, h1);
+                        }
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            orow[c / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     }
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        orow[c / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                }
-            } else {
+                } else {
 #pragma unroll 1
-                for (int c = 0; c < 256; c += 32) {
-                    uint32_t y[32];
-                    ptx::tmem_ld32(t_row + c, y);
-                    ptx::tmem_ld_wait();
-                    uint32_t pk[16];
+                    for (int c = 0; c < 256; c += 32) {
+                        uint32_t y[32];
+                        ptx::tmem_ld32(t_row + c, y);
+                        ptx::tmem_ld_wait();
+                        uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = pack_bf16(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
+                        for (int i = 0; i < 16; ++i)
+                            pk[i] = pack_bf16(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
 #pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        orow[c / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                        for (int v = 0; v < 4; ++v)
+                            orow[c / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    }
                 }
             }
             ptx::tc_fence_before();
-            ptx::mbar_arrive(&S->acc_empty[acc]);
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->acc_empty[acc]), 0));
         }
     }
     ptx::tc_fence_before();
     __syncthreads();
+    ptx::cluster_sync();   // no CTA leaves while its peer may still signal it
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem, kTmemCols);
+        ptx::tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
@@ -310,6 +472,7 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    sms &= ~1;   // whole CTA pairs
     TcArgs a;
     a.E = s.E;
     a.spin = spin_budget;
@@ -317,12 +480,13 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.sched = ws.sched;
     a.sched_off = ws.sched_off;
     a.header = ws.header;
+    a.queue = ws.gemm_q + (which == 1 ? 0 : 4);
     a.out = static_cast<__nv_bfloat16*>(out);
     CUtensorMap tA, tB;
     if (which == 1) {
         // FC1 + SwiGLU: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h [rows_cap, F]
         if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
-            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, 128))
+            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN))
             return cudaErrorInvalidValue;
         a.out_ld = s.F;
         a.Kdim = s.d;
@@ -333,7 +497,7 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     }
     // FC2: h [rows_cap, F] x w_down [E*d, F] -> yp [rows_cap, d]
     if (!make_tmap(&tA, a_mat, (uint64_t)s.F, (uint64_t)s.rows_cap, kBM) ||
-        !make_tmap(&tB, w, (uint64_t)s.F, (uint64_t)s.E * s.d, 256))
+        !make_tmap(&tB, w, (uint64_t)s.F, (uint64_t)s.E * s.d, kHalfN))
         return cudaErrorInvalidValue;
     a.out_ld = s.d;
     a.Kdim = s.F;

@@ -311,6 +311,7 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
         ws.header[H_TOTAL_ROWS] = (uint32_t)tot_rows;
         ws.header[H_MOVES] = (uint32_t)s_moves;
         ws.header[H_REPLICAS] = (uint32_t)nrep;
+        for (int q = 0; q < kGemmQWords; ++q) ws.gemm_q[q] = 0;   // fresh GEMM work queues
     }
 }
 
