@@ -237,6 +237,7 @@ def run_mine(args, world, rank, local):
 
     n_ev = 6
     def step(evs=None):
+        # the kernels moe_layer_fwd runs, one ABI call per stage so each stage can be timed
         if evs is not None: evs[0].record(stream)
         M.moe_plan(cfg, lg, idx, w, counts, ws, stream)
         if evs is not None: evs[1].record(stream)
@@ -329,7 +330,7 @@ def run_mine(args, world, rank, local):
     t_roof = max(layer_flop / (tensor_peak * 1e12), alg_bytes / (pk["hbm_gbs"] * 1e9))
     ms_per_step = elapsed_ms / args.steps
     value = world * T / (ms_per_step * 1e-3)
-    gather_bytes = T * d * eb + N * d * eb + 4 * N + (plan["total_rows"] - N) * d * eb
+    gather_bytes = T * d * eb + plan["total_rows"] * d * eb + 4 * plan["total_rows"]
     combine_bytes = N * d * eb + 8 * N + T * d * eb
     line = {
         "metric": METRIC,
@@ -346,7 +347,7 @@ def run_mine(args, world, rank, local):
         "data": "synthetic (seeded SplitMix64 + Box-Muller inputs; see DESIGN.md input recipe)",
         "config": {"workload": cfg.name, **C.describe(cfg), "seed": args.seed,
                    "l2": "no flush: one step touches ~%.1f GB (weights %.2f GB) >> 126 MB L2"
-                         % ((alg_bytes + 3 * cap * d * eb + cap * F * eb) / 1e9, weight_bytes / 1e9),
+                         % ((alg_bytes + 3 * cap * d * eb + 2 * cap * F * eb) / 1e9, weight_bytes / 1e9),
                    "parallelism": f"replicas x{world} (independent layers, no collective)"},
         "roofline": {"bound": "tensor", "kernel": "ffn_tc_kernel<FC1+SwiGLU>",
                      "achieved": fc1_flop / fc1_s / 1e12, "peak": tensor_peak, "unit": "TFLOP/s",
@@ -368,6 +369,7 @@ def run_mine(args, world, rank, local):
                 "h2d_bytes_per_step": 4 * T * E + T * d * eb, "d2h_bytes_per_step": T * d * eb,
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "layer_path": "moe_plan; moe_dispatch; moe_expert_fc1; moe_expert_fc2; moe_combine (the kernels of moe_layer_fwd)",
         "clocks": clk.summary(),
     }
     if cpu is not None:

@@ -186,6 +186,22 @@ moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_do
                           size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_expert_fc1_gather - steps A6 and A7 in one pass (bf16 layers only):
+ * FC1 + SwiGLU whose activation rows are gathered straight from x [T, d]
+ * (device) through the plan's row map, so no xp buffer is written or read
+ * ([MegaFlux] §2.1: token movement overlapped with the tiled FC1 work).
+ * h [rows_cap, F] (device, out) holds the same values as moe_dispatch +
+ * moe_expert_fc1 on every valid row; padding rows hold unspecified values
+ * (they repeat their block's first token) and are never read by
+ * moe_combine. It needs no xp buffer (rows_cap * d elements less memory)
+ * but runs FC1 at about half the speed of moe_expert_fc1: each 16 KB
+ * activation tile takes 32 four-row gathers instead of one tile copy.
+ * fp32 layers return MOE_ERR_UNSUPPORTED.
+ */
+moe_status moe_expert_fc1_gather(const moe_config* cfg, const void* x, const void* w_gate_up, void* h, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_combine - step A9, the weighted top-k sum ([MegaFlux] §1, §2.1):
  * out[t] = sum over k in order of topk_w[t,k] * yp[row_of(t,k)], in fp32,
  * rounded once to cfg->dtype.

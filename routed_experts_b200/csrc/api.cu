@@ -211,6 +211,19 @@ moe_status moe_expert_fc1(const moe_config* cfg, const void* xp, const void* w_g
     return fc_impl(s, L, 1, xp, w_gate_up, h, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
+moe_status moe_expert_fc1_gather(const moe_config* cfg, const void* x, const void* w_gate_up, void* h, void* ws,
+                                 size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!x || !w_gate_up || !h || !aligned16(x) || !aligned16(w_gate_up) || !aligned16(h))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    return fc_impl(s, L, 3, x, w_gate_up, h, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
 moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_down, void* yp, void* ws,
                           size_t ws_bytes, moe_stream_t stream) {
     Shape s;

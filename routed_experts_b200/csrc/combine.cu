@@ -14,7 +14,9 @@ namespace {
 
 constexpr int kCWarps = 8;
 
-template <bool BF16>
+// KMAX: a compile-time bound on K (K <= KMAX) so the K rows a lane reads stay in
+// registers without reserving room for the largest K.
+template <bool BF16, int KMAX>
 __global__ void __launch_bounds__(kCWarps * 32)
 combine_kernel(const uint4* __restrict__ yp, const float* __restrict__ w, uint4* __restrict__ out,
                int T, int K, int nvec, int64_t rows_cap, WsPtrs ws) {
@@ -28,24 +30,24 @@ combine_kernel(const uint4* __restrict__ yp, const float* __restrict__ w, uint4*
             my_w = w[(int64_t)t * K + lane];
             if (my_row < 0 || my_row >= rows_cap) { bad = 1; my_row = 0; my_w = 0.f; }
         }
-        int rows[kMaxK];
-        float ws_[kMaxK];
+        int rows[KMAX];
+        float ws_[KMAX];
 #pragma unroll
-        for (int k = 0; k < kMaxK; ++k) {
+        for (int k = 0; k < KMAX; ++k) {
             rows[k] = __shfl_sync(0xffffffffu, my_row, k);
             ws_[k] = __shfl_sync(0xffffffffu, my_w, k);
         }
         for (int v = lane; v < nvec; v += 32) {
-            uint4 val[kMaxK];
+            uint4 val[KMAX];
 #pragma unroll
-            for (int k = 0; k < kMaxK; ++k)
+            for (int k = 0; k < KMAX; ++k)
                 if (k < K) val[k] = __ldg(yp + (int64_t)rows[k] * nvec + v);
             if (BF16) {
                 float acc[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) acc[j] = 0.f;
 #pragma unroll
-                for (int k = 0; k < kMaxK; ++k) {
+                for (int k = 0; k < KMAX; ++k) {
                     if (k >= K) break;
                     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&val[k]);
 #pragma unroll
@@ -63,7 +65,7 @@ combine_kernel(const uint4* __restrict__ yp, const float* __restrict__ w, uint4*
             } else {
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int k = 0; k < kMaxK; ++k) {
+                for (int k = 0; k < KMAX; ++k) {
                     if (k >= K) break;
                     const float* f = reinterpret_cast<const float*>(&val[k]);
 #pragma unroll
@@ -86,14 +88,17 @@ cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void*
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int nvec = (int)((int64_t)s.d * s.eb / 16);
     int64_t want = (s.T + kCWarps - 1) / kCWarps;
-    int64_t cap = (int64_t)sms * 8;
+    int64_t cap = (int64_t)sms * 16;
     const int grid = (int)(want < cap ? want : cap);
-    if (s.dtype == MOE_BF16)
-        combine_kernel<true><<<grid, kCWarps * 32, 0, st>>>(
-            static_cast<const uint4*>(yp), w, static_cast<uint4*>(out), s.T, s.K, nvec, s.rows_cap, ws);
-    else
-        combine_kernel<false><<<grid, kCWarps * 32, 0, st>>>(
-            static_cast<const uint4*>(yp), w, static_cast<uint4*>(out), s.T, s.K, nvec, s.rows_cap, ws);
+    const uint4* y4 = static_cast<const uint4*>(yp);
+    uint4* o4 = static_cast<uint4*>(out);
+#define MOE_COMBINE(B, KM) combine_kernel<B, KM><<<grid, kCWarps * 32, 0, st>>>(y4, w, o4, s.T, s.K, nvec, s.rows_cap, ws)
+    const bool bf = s.dtype == MOE_BF16;
+    if (s.K <= 2) { if (bf) MOE_COMBINE(true, 2); else MOE_COMBINE(false, 2); }
+    else if (s.K <= 4) { if (bf) MOE_COMBINE(true, 4); else MOE_COMBINE(false, 4); }
+    else if (s.K <= 8) { if (bf) MOE_COMBINE(true, 8); else MOE_COMBINE(false, 8); }
+    else { if (bf) MOE_COMBINE(true, 16); else MOE_COMBINE(false, 16); }
+#undef MOE_COMBINE
     return cudaGetLastError();
 }
 

@@ -117,7 +117,8 @@ cudaError_t launch_gather(const Shape& s, const void* x, void* xp, const WsPtrs&
 cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void* out,
                            const WsPtrs& ws, cudaStream_t st);
 // which = 1: FC1 + SwiGLU (a_mat = xp, w = w_gate_up, out = h);
-// which = 2: FC2 (a_mat = h, w = w_down, out = yp).
+// which = 2: FC2 (a_mat = h, w = w_down, out = yp);
+// which = 3 (tensor cores only): FC1 + SwiGLU with a_mat = x, rows gathered by the row map.
 cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                             const WsPtrs& ws, cudaStream_t st);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,

@@ -23,6 +23,12 @@
 // An expert with an odd number of blocks gives its last pair one block: the
 // odd CTA then reloads the even CTA's rows and stores nothing.
 //
+// FC1 can also read its activation rows straight from x (dispatch fused into
+// FC1): each 128-row A tile is built by 32 four-row TMA gathers
+// (tile::gather4, one per lane of the TMA warp) of the token rows the plan's
+// row map names; padding rows repeat the block's first token and their h rows
+// are never read by the combine.
+//
 // Scheduling is dynamic. Items are listed expert-major (then column tile,
 // then block pair), so consecutive items share an expert's weight tiles and a
 // pair's activation rows. The list is cut at an expert boundary into two
@@ -72,6 +78,7 @@ constexpr uint32_t kItemConsumers = 11;
 constexpr int kSchedWarp = 6;
 
 struct TcArgs {
+    const int32_t* src_of;    // row -> token (gathered FC1 only)
     __nv_bfloat16* out;       // h (FC1) or yp (FC2)
     int out_ld;               // F or d
     int Kdim;                 // d or F
@@ -91,6 +98,7 @@ struct Smem {
     uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
     uint64_t item_full[kItemSlots], item_empty[kItemSlots];
     int4 items[kItemSlots];   // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
+    int32_t rows[kItemSlots][kBM];   // gathered FC1: token of each row of this CTA's block
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -169,7 +177,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// MODE 0: FC1 + SwiGLU -> h; MODE 1: FC2 -> yp.
+// MODE 0: FC1 + SwiGLU -> h (A = xp); MODE 1: FC2 -> yp (A = h);
+// MODE 2: FC1 + SwiGLU -> h with A gathered from x.
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcArgs a) {
@@ -223,7 +232,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const uint32_t tmem = S->tmem_base;
     const int n_items = p_off[a.E] * a.n_tiles;
     const int kb_count = a.Kdim / kBK;
-    constexpr int kColTile = MODE == 0 ? 128 : 256;
+    constexpr bool kFC1 = MODE != 1;
+    constexpr bool kGather = MODE == 2;
+    constexpr int kColTile = kFC1 ? 128 : 256;
 
     // the ring slot of the k-th item, and the parity of its phase
     auto slot_of = [](int k) { return k % kItemSlots; };
@@ -241,7 +252,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 
     if (warp == kSchedWarp) {
         // ------------------------------------------------ scheduler (even CTA)
-        if (lane == 0 && even) {
+        if (even) {
             // group of this cluster: the half of the GPU its even CTA runs on
             const int g = ptx::smid() >= (ptx::nsmid() >> 1) ? 1 : 0;
             int lo = 0, hi = a.E;   // first expert whose pairs start at or after half of all pairs
@@ -251,69 +262,96 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (p_off[mid] < half) lo = mid + 1; else hi = mid;
             }
             const int split = p_off[lo] * a.n_tiles;
-            int next = fetch_item(a.queue, g, split, n_items);
+            int next = lane == 0 ? fetch_item(a.queue, g, split, n_items) : 0;
             for (int k = 0;; ++k) {
+                const bool ok = role_wait(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
                 int4 item = make_int4(-1, 0, -1, -1);
-                bool ok = role_wait(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
-                if (ok && next >= 0) {
+                if (lane == 0 && ok && next >= 0) {
                     int e, b0, b1, j;
                     decode_item(next, a.n_tiles, s_off, p_off, a.E, a.sched, e, b0, b1, j);
                     item = make_int4(e, j, a.blocks[kBlockInts * b0 + 1], b1 >= 0 ? a.blocks[kBlockInts * b1 + 1] : -1);
                 }
-                // publish to both CTAs
-                S->items[slot_of(k)] = item;
-                const uint32_t peer = ptx::map_to_rank(ptx::smem_addr(&S->items[slot_of(k)]), 1);
-                ptx::st_cluster_u32(peer, (uint32_t)item.x);
-                ptx::st_cluster_u32(peer + 4, (uint32_t)item.y);
-                ptx::st_cluster_u32(peer + 8, (uint32_t)item.z);
-                ptx::st_cluster_u32(peer + 12, (uint32_t)item.w);
-                ptx::mbar_arrive(&S->item_full[slot_of(k)]);
-                ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_full[slot_of(k)]), 1));
+                item.x = __shfl_sync(0xffffffffu, item.x, 0);
+                item.y = __shfl_sync(0xffffffffu, item.y, 0);
+                item.z = __shfl_sync(0xffffffffu, item.z, 0);
+                item.w = __shfl_sync(0xffffffffu, item.w, 0);
+                if (kGather && item.x >= 0) {
+                    // tokens of the rows of both blocks; a padding row takes its block's first token
+                    const int r_even = item.z, r_odd = item.w >= 0 ? item.w : item.z;
+                    const int first_even = __ldg(a.src_of + r_even), first_odd = __ldg(a.src_of + r_odd);
+                    int4 ve, vo;
+                    ve.x = __ldg(a.src_of + r_even + 4 * lane + 0); vo.x = __ldg(a.src_of + r_odd + 4 * lane + 0);
+                    ve.y = __ldg(a.src_of + r_even + 4 * lane + 1); vo.y = __ldg(a.src_of + r_odd + 4 * lane + 1);
+                    ve.z = __ldg(a.src_of + r_even + 4 * lane + 2); vo.z = __ldg(a.src_of + r_odd + 4 * lane + 2);
+                    ve.w = __ldg(a.src_of + r_even + 4 * lane + 3); vo.w = __ldg(a.src_of + r_odd + 4 * lane + 3);
+                    ve.x = ve.x < 0 ? first_even : ve.x; vo.x = vo.x < 0 ? first_odd : vo.x;
+                    ve.y = ve.y < 0 ? first_even : ve.y; vo.y = vo.y < 0 ? first_odd : vo.y;
+                    ve.z = ve.z < 0 ? first_even : ve.z; vo.z = vo.z < 0 ? first_odd : vo.z;
+                    ve.w = ve.w < 0 ? first_even : ve.w; vo.w = vo.w < 0 ? first_odd : vo.w;
+                    *reinterpret_cast<int4*>(&S->rows[slot_of(k)][4 * lane]) = ve;
+                    ptx::st_cluster_v4(ptx::map_to_rank(ptx::smem_addr(&S->rows[slot_of(k)][4 * lane]), 1), vo);
+                    ptx::fence_acq_rel_cluster();
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    // publish to both CTAs
+                    S->items[slot_of(k)] = item;
+                    const uint32_t peer = ptx::map_to_rank(ptx::smem_addr(&S->items[slot_of(k)]), 1);
+                    ptx::st_cluster_v4(peer, item);
+                    ptx::mbar_arrive(&S->item_full[slot_of(k)]);
+                    ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_full[slot_of(k)]), 1));
+                }
                 if (item.x < 0) break;
-                next = fetch_item(a.queue, g, split, n_items);   // its latency hides behind the ring
+                if (lane == 0) next = fetch_item(a.queue, g, split, n_items);   // latency hides behind the ring
             }
-            // the last cluster to finish resets the queues for the next launch
-            __threadfence();
-            const int done = atomicAdd(&a.queue[2], 1);
-            if (done == (int)ptx::cluster_count_x() - 1) {
-                a.queue[0] = 0;
-                a.queue[1] = 0;
+            if (lane == 0) {
+                // the last cluster to finish resets the queues for the next launch
                 __threadfence();
-                a.queue[2] = 0;
+                const int done = atomicAdd(&a.queue[2], 1);
+                if (done == (int)ptx::cluster_count_x() - 1) {
+                    a.queue[0] = 0;
+                    a.queue[1] = 0;
+                    __threadfence();
+                    a.queue[2] = 0;
+                }
             }
         }
     } else if (warp == 0) {
-        // ------------------------------------------------ TMA producer (both CTAs)
-        if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            long long fills = 0;
-            bool ok = true;
-            for (int k = 0; ok; ++k) {
-                int4 item;
-                if (!take_item(k, item)) { ok = false; break; }
-                release_item(k);
-                if (item.x < 0) break;
-                const int e = item.x, j = item.y;
-                const int row0 = even ? item.z : (item.w >= 0 ? item.w : item.z);
-                const int brow = e * a.b_rows + j * kColTile + (even ? 0 : (MODE == 0 ? a.F : kHalfN));
-                for (int kb = 0; kb < kb_count; ++kb) {
-                    if (!role_wait(&S->empty[stage], phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
+        // ------------------------------------------------ TMA producer (both CTAs, whole warp)
+        int stage = 0;
+        uint32_t phase = 0;
+        long long fills = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            int4 item;
+            if (!take_item(k, item)) { ok = false; break; }
+            int4 tok = make_int4(0, 0, 0, 0);   // gathered FC1: tokens of this lane's four rows
+            if (kGather && item.x >= 0) tok = *reinterpret_cast<const int4*>(&S->rows[slot_of(k)][4 * lane]);
+            __syncwarp();
+            if (lane == 0) release_item(k);
+            if (item.x < 0) break;
+            const int e = item.x, j = item.y;
+            const int row0 = even ? item.z : (item.w >= 0 ? item.w : item.z);
+            const int brow = e * a.b_rows + j * kColTile + (even ? 0 : (kFC1 ? a.F : kHalfN));
+            for (int kb = 0; kb < kb_count; ++kb) {
+                if (!role_wait(&S->empty[stage], phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
+                const uint32_t bar = ptx::map_to_rank(ptx::smem_addr(&S->full[stage]), 0);
+                uint8_t* st = base + stage * kStageBytes;
+                if (lane == 0) {
                     if (even) ptx::mbar_arrive_expect_tx(&S->full[stage], 2 * kStageBytes);
-                    const uint32_t bar = ptx::map_to_rank(ptx::smem_addr(&S->full[stage]), 0);
-                    uint8_t* st = base + stage * kStageBytes;
-                    ptx::tma_load_2d_pair(st, &tmA, kb * kBK, row0, bar);
+                    if (!kGather) ptx::tma_load_2d_pair(st, &tmA, kb * kBK, row0, bar);
                     ptx::tma_load_2d_pair(st + kABytes, &tmB, kb * kBK, brow, bar);
-                    ++fills;
-                    if (++stage == kStages) { stage = 0; phase ^= 1; }
                 }
+                if (kGather) ptx::tma_gather4_pair(st + 4 * 128 * lane, &tmA, kb * kBK, tok.x, tok.y, tok.z, tok.w, bar);
+                ++fills;
+                if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
-            if (!ok && even) {
-                // let the copies still in flight land before the CTA exits
-                const long long first = fills > kStages ? fills - kStages : 0;
-                for (long long f = first; f < fills; ++f)
-                    ptx::mbar_wait(&S->full[f % kStages], (uint32_t)((f / kStages) & 1), kDrainBudget);
-            }
+        }
+        if (!ok && even && lane == 0) {
+            // let the copies still in flight land before the CTA exits
+            const long long first = fills > kStages ? fills - kStages : 0;
+            for (long long f = first; f < fills; ++f)
+                ptx::mbar_wait(&S->full[f % kStages], (uint32_t)((f / kStages) & 1), kDrainBudget);
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (even CTA)
@@ -380,7 +418,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN);
                 uint4* orow =
                     reinterpret_cast<uint4*>(a.out + (int64_t)(row0 + m) * a.out_ld + (int64_t)j * kColTile);
-                if (MODE == 0) {
+                if (kFC1) {
 #pragma unroll 1
                     for (int c = 0; c < 128; c += 32) {
                         uint32_t gt[32], up[32];
@@ -480,9 +518,22 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.sched = ws.sched;
     a.sched_off = ws.sched_off;
     a.header = ws.header;
-    a.queue = ws.gemm_q + (which == 1 ? 0 : 4);
+    a.queue = ws.gemm_q + (which == 2 ? 4 : 0);
+    a.src_of = ws.src_of;
     a.out = static_cast<__nv_bfloat16*>(out);
     CUtensorMap tA, tB;
+    if (which == 3) {
+        // FC1 + SwiGLU with A gathered from x [T, d] by the row map -> h [rows_cap, F]
+        if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.T, 1) ||
+            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN))
+            return cudaErrorInvalidValue;
+        a.out_ld = s.F;
+        a.Kdim = s.d;
+        a.n_tiles = s.F / 128;
+        a.F = s.F;
+        a.b_rows = 2 * s.F;
+        return launch_mode<2>(tA, tB, a, sms, st);
+    }
     if (which == 1) {
         // FC1 + SwiGLU: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h [rows_cap, F]
         if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||

@@ -27,9 +27,20 @@ namespace {
 constexpr int kRmWarps = 4;
 
 __global__ void __launch_bounds__(kRmWarps * 32)
-row_maps_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int n_chunks, WsPtrs ws) {
-    extern __shared__ int32_t base_all[];   // [kRmWarps][E]
+row_maps_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int n_chunks, int max_pieces, WsPtrs ws) {
+    extern __shared__ int32_t sm_rm[];
+    int32_t* s_poff = sm_rm;                       // [E+1] first piece of each expert (start order)
+    int4* s_piece = reinterpret_cast<int4*>(s_poff + ((E + 1 + 3) & ~3));   // [n_pieces]: start, len, row0
+    int32_t* base_all = reinterpret_cast<int32_t*>(s_piece + max_pieces);  // [kRmWarps][E]
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the piece tables, in expert/start order, staged once per CTA
+    const int n_pieces = (int)ws.header[H_NPIECES];
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) s_poff[e] = ws.exp_piece_off[e];
+    for (int p = threadIdx.x; p < n_pieces; p += blockDim.x) {
+        const int32_t* P = ws.pieces + (int64_t)kPieceInts * ws.exp_piece_idx[p];
+        s_piece[p] = make_int4(P[2], P[3], P[4], 0);
+    }
+    __syncthreads();
     const int chunk = blockIdx.x * kRmWarps + warp;
     if (chunk >= n_chunks) return;           // whole warp leaves; no CTA-wide barrier below
     int32_t* base = base_all + warp * E;
@@ -39,10 +50,19 @@ row_maps_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int n_chun
     const int64_t t1 = min((int64_t)T, (int64_t)(chunk + 1) * kTokPerChunk);
     const int64_t i1 = t1 * K;
     uint32_t bad = 0;
-    for (int64_t ib = i0; ib < i1; ib += 32) {
-        const int64_t i = ib + lane;
+    // the chunk's expert ids, loaded up front (a full chunk is K rounds of 32)
+    int ev[kMaxK];
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+        const int64_t i = i0 + (int64_t)r * 32 + lane;
+        ev[r] = (r < K && i < i1) ? __ldg(idx + i) : -1;
+    }
+#pragma unroll
+    for (int r = 0; r < kMaxK; ++r) {
+        if (r >= K) break;
+        const int64_t i = i0 + (int64_t)r * 32 + lane;
         const bool valid = i < i1;
-        int e = valid ? idx[i] : -1;
+        int e = valid ? ev[r] : -1;
         if (valid && (e < 0 || e >= E)) { bad = 1; e = -2; }
         const bool ok = valid && e >= 0;
         const unsigned m = __match_any_sync(0xffffffffu, e);
@@ -53,10 +73,10 @@ row_maps_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int n_chun
         __syncwarp();
         if (ok) {
             int row = -1;
-            const int p1 = ws.exp_piece_off[e + 1];
-            for (int p = ws.exp_piece_off[e]; p < p1; ++p) {
-                const int32_t* P = ws.pieces + (int64_t)kPieceInts * ws.exp_piece_idx[p];
-                if (pos < P[2] + P[3]) { row = P[4] + pos - P[2]; break; }
+            const int p1 = s_poff[e + 1];
+            for (int p = s_poff[e]; p < p1; ++p) {
+                const int4 P = s_piece[p];
+                if (pos < P.x + P.y) { row = P.z + pos - P.x; break; }
             }
             if (row < 0) {
                 bad = 1;
@@ -105,8 +125,12 @@ gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp, int nvec, WsP
 
 cudaError_t launch_row_maps(const Shape& s, const int32_t* idx, const WsPtrs& ws, cudaStream_t st) {
     const int grid = (s.n_chunks + kRmWarps - 1) / kRmWarps;
-    const size_t smem = sizeof(int32_t) * kRmWarps * s.E;
-    row_maps_kernel<<<grid, kRmWarps * 32, smem, st>>>(idx, s.T, s.K, s.E, s.n_chunks, ws);
+    const size_t smem = sizeof(int32_t) * (((s.E + 1 + 3) & ~3) + kRmWarps * s.E) + sizeof(int4) * s.max_pieces;
+    if (smem > 48 * 1024) {
+        cudaError_t err = cudaFuncSetAttribute(row_maps_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (err != cudaSuccess) return err;
+    }
+    row_maps_kernel<<<grid, kRmWarps * 32, smem, st>>>(idx, s.T, s.K, s.E, s.n_chunks, (int)s.max_pieces, ws);
     return cudaGetLastError();
 }
 

@@ -81,8 +81,9 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
     int32_t* L = own_pid + E;                        // [R]
     int32_t* used = L + R;                           // [R]
     int32_t* rep = used + R;                         // [max_rep][5]: rank, expert, start, len, pid
-    int32_t* pfb = rep + 5 * a.max_rep;              // [max_pieces]: first block of each piece
-    int32_t* tmp = pfb + (E + a.max_rep);            // [32]
+    int32_t* pfb = rep + 5 * a.max_rep;              // [max_pieces+1]: first block of each piece
+    int32_t* pq = pfb + (E + a.max_rep + 1);         // [max_pieces][4]: expert, rank, len, row0
+    int32_t* tmp = pq + 4 * (E + a.max_rep);         // [32]
     __shared__ uint32_t s_status;
     __shared__ int s_moves, s_nrep;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -99,7 +100,8 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
     if (g < a.G) {
         const int c0 = (int)((int64_t)g * a.n_chunks / a.G), c1 = (int)((int64_t)(g + 1) * a.n_chunks / a.G);
         int s = 0;
-        for (int c = c0; c < c1; ++c) s += ws.chunk_counts[(int64_t)c * E + e0];
+#pragma unroll 8
+        for (int c = c0; c < c1; ++c) s += __ldg(ws.chunk_counts + (int64_t)c * E + e0);
         part[g * E + e0] = s;
     }
     __syncthreads();
@@ -119,9 +121,10 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
     if (g < a.G) {
         const int c0 = (int)((int64_t)g * a.n_chunks / a.G), c1 = (int)((int64_t)(g + 1) * a.n_chunks / a.G);
         int run = part[g * E + e0];
+#pragma unroll 8
         for (int c = c0; c < c1; ++c) {
             ws.chunk_base[(int64_t)c * E + e0] = run;
-            run += ws.chunk_counts[(int64_t)c * E + e0];
+            run += __ldg(ws.chunk_counts + (int64_t)c * E + e0);
         }
     }
     if (tid < R) {
@@ -251,13 +254,8 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
             int32_t* P = ws.pieces + (int64_t)kPieceInts * pid;
             P[0] = pe; P[1] = tid; P[2] = pstart; P[3] = plen; P[4] = row;
             pfb[pid] = bid;
+            pq[4 * pid] = pe; pq[4 * pid + 1] = tid; pq[4 * pid + 2] = plen; pq[4 * pid + 3] = row;
             const int nt = (plen + a.tile - 1) / a.tile;
-            for (int i = 0; i < nt; ++i) {
-                int32_t* B = ws.blocks + (int64_t)kBlockInts * (bid + i);
-                const int v = plen - i * a.tile;
-                B[0] = pe; B[1] = row + i * a.tile; B[2] = v < a.tile ? v : a.tile; B[3] = tid;
-            }
-            for (int r = row + plen; r < row + nt * a.tile; ++r) ws.src_of[r] = -1;
             bid += nt;
             row += nt * a.tile;
             load += plen;
@@ -268,7 +266,27 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
         ws.rank_row0[tid] = r_off;
         if (tid == R - 1) ws.rank_row0[R] = row;
     }
+    if (tid == 0) pfb[tot_p] = tot_b;
     __syncthreads();
+    // blocks of every piece, written by the whole CTA: block b belongs to the
+    // last piece whose first block is <= b
+    for (int b = tid; b < tot_b; b += kThreads) {
+        int lo = 0, hi = tot_p - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (pfb[mid] <= b) lo = mid; else hi = mid - 1;
+        }
+        const int i = b - pfb[lo];
+        const int v = pq[4 * lo + 2] - i * a.tile;
+        int32_t* B = ws.blocks + (int64_t)kBlockInts * b;
+        B[0] = pq[4 * lo]; B[1] = pq[4 * lo + 3] + i * a.tile; B[2] = v < a.tile ? v : a.tile; B[3] = pq[4 * lo + 1];
+    }
+    // padding rows (the tail of each piece's last tile) map to no token
+    for (int p = warp; p < tot_p; p += kThreads / 32) {
+        const int len = pq[4 * p + 2], row0 = pq[4 * p + 3];
+        const int padded = (len + a.tile - 1) / a.tile * a.tile;
+        for (int r = row0 + len + lane; r < row0 + padded; r += 32) ws.src_of[r] = -1;
+    }
 
     // ---------------- (D) per-expert piece index (start order) and block schedule
     int np_e = 0, nb_e = 0;
@@ -328,7 +346,7 @@ cudaError_t launch_plan(const Shape& s, int32_t* counts_out, const WsPtrs& ws, c
     a.C = (int)s.C;
     a.max_rep = s.R * s.budget;
     const size_t smem = sizeof(int32_t) * ((size_t)G * s.E + 3 * s.E + 2 * s.R + 5 * a.max_rep +
-                                           (s.E + a.max_rep) + 32);
+                                           5 * (s.E + a.max_rep) + 1 + 32);
     cudaError_t err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;

@@ -209,6 +209,29 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* t
         : "memory");
 }
 
+// Four rows (row coordinates r0..r3, one-row box of the tensor map) of the
+// columns starting at x, gathered into this CTA's shared memory as a 4-row
+// tile; completed bytes are counted on an mbarrier of either CTA of the pair.
+__device__ __forceinline__ void tma_gather4_pair(void* dst, const CUtensorMap* tm, int x, int r0, int r1, int r2,
+                                                 int r3, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        ::"r"(smem_addr(dst)), "l"(tm), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(bar)
+        : "memory");
+}
+
+// Store four 32-bit values to shared memory given by its shared::cluster address.
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, int4 v) {
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
+                 "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel_cluster() {
+    asm volatile("fence.acq_rel.cluster;" ::: "memory");
+}
+
 // TMEM allocation shared by a CTA pair (one warp of each CTA, same warp index).
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(dst_smem)),

@@ -7,7 +7,7 @@
 // construction": k distinct experts per token; §3.1: the planner starts from
 // the routing profile (per-expert load).
 //
-// One warp per token. Lane l holds logits of experts l, l+32, l+64, ...
+// One warp per token (a CTA per 32-token chunk). Lane l holds logits of experts l, l+32, l+64, ...
 // (coalesced 128-byte rows). K rounds of a warp arg-max pick the experts in
 // descending logit order, ties to the lower expert id. Gating: softmax over
 // the chosen logits (equal to the full softmax renormalised over them), or
@@ -22,14 +22,14 @@
 namespace moe {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = kTokPerChunk;   // one warp per token
 
 __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
     return va > vb || (va == vb && ea < eb);
 }
 
 template <int EPT>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 1)
 topk_hist_kernel(const float* __restrict__ logits, int32_t* __restrict__ idx,
                  float* __restrict__ wout, int T, int E, int K, int gating,
                  int32_t* __restrict__ chunk_counts, uint32_t* __restrict__ chunk_flags) {

@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_ffn.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_expert_fc1.argtypes = [C, P, P, P, P, S, P]
         L.moe_expert_fc2.argtypes = [C, P, P, P, P, S, P]
+        L.moe_expert_fc1_gather.argtypes = [C, P, P, P, P, S, P]
         L.moe_combine.argtypes = [C, P, P, P, P, S, P]
         L.moe_layer_fwd.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
@@ -67,7 +68,8 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
-                  "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_combine", "moe_layer_fwd",
+                  "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
+                  "moe_layer_fwd",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -149,6 +151,12 @@ def moe_expert_fc1(c, xp, w_gate_up, h, ws, stream=None):
     p, n = _ws(ws)
     _check(lib().moe_expert_fc1(ctypes.byref(config(c)), _ptr(xp), _ptr(w_gate_up), _ptr(h), p, n, _stream(stream)),
            "moe_expert_fc1")
+
+
+def moe_expert_fc1_gather(c, x, w_gate_up, h, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_expert_fc1_gather(ctypes.byref(config(c)), _ptr(x), _ptr(w_gate_up), _ptr(h), p, n,
+                                       _stream(stream)), "moe_expert_fc1_gather")
 
 
 def moe_expert_fc2(c, h, w_down, yp, ws, stream=None):
