@@ -155,6 +155,17 @@ def ncu_traffic(kernel_key: str):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise maximum of per-rank floats over all ranks (a no-op without a
+    process group). The tensor lives on `device` (the rank's GPU under NCCL,
+    the CPU under gloo)."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
 def dist_setup(args):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -298,9 +309,7 @@ def run_mine(args, world, rank, local):
     e2e_ms = e0.elapsed_time(e1)
     if pg is not None:
         torch.distributed.barrier()
-        tt = torch.tensor([elapsed_ms, e2e_ms], device=dev)
-        torch.distributed.all_reduce(tt, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms, e2e_ms = float(tt[0]), float(tt[1])
+        elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -264,6 +264,17 @@ moe_status moe_plan_noalloc(const moe_config* cfg, const float* logits, int32_t*
 /* Synchronises `stream`, then reads the device status bits of `ws`. */
 moe_status moe_read_status(const void* ws, moe_stream_t stream, uint32_t* dev_bits);
 
+/*
+ * moe_probe_bounded_wait - a check of the device-side failure detection:
+ * one CTA waits, through the same bounded wait the expert-FFN kernels use,
+ * on an mbarrier that nothing ever arrives on. After budget_cycles clock
+ * cycles (at most 2^34) the wait gives up, ORs MOE_DEV_TIMEOUT into
+ * *status_word (a device uint32) and the kernel returns; the context stays
+ * usable. No papers' counterpart: it exists so the timeout path can be
+ * exercised without hanging or faulting a GPU.
+ */
+moe_status moe_probe_bounded_wait(uint32_t* status_word, int64_t budget_cycles, moe_stream_t stream);
+
 /* A static string naming a moe_status. */
 const char* moe_status_string(moe_status s);
 

@@ -307,6 +307,12 @@ moe_status moe_read_status(const void* ws, moe_stream_t stream, uint32_t* dev_bi
     return MOE_OK;
 }
 
+moe_status moe_probe_bounded_wait(uint32_t* status_word, int64_t budget_cycles, moe_stream_t stream) {
+    if (!status_word || budget_cycles < 0 || budget_cycles > ((int64_t)1 << 34)) return MOE_ERR_INVALID_ARG;
+    return from_cuda(launch_bounded_wait_probe(status_word, (long long)budget_cycles,
+                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char* moe_status_string(moe_status s) {
     switch (s) {
         case MOE_OK: return "MOE_OK";

@@ -121,6 +121,7 @@ cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void*
 // which = 3 (tensor cores only): FC1 + SwiGLU with a_mat = x, rows gathered by the row map.
 cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                             const WsPtrs& ws, cudaStream_t st);
+cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget);
 

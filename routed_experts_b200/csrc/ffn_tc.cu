@@ -466,6 +466,21 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     }
 }
 
+// One CTA waits, through the same bounded wait as the GEMM's roles, on an
+// mbarrier no thread ever arrives on; when the wait runs out it reports
+// MOE_DEV_TIMEOUT in *status and returns.
+__global__ void bounded_wait_probe_kernel(uint32_t* status, long long budget) {
+    __shared__ uint64_t never;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(&never, 1);
+        abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) role_wait(&never, 0, budget, &abort_flag, status);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -504,6 +519,11 @@ cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const TcAr
 }
 
 }  // namespace
+
+cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st) {
+    bounded_wait_probe_kernel<<<1, 32, 0, st>>>(status, budget);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget) {

@@ -65,12 +65,13 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_read_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_plan_noalloc.argtypes = [C, P, P, P, P, P, P, P]
+        L.moe_probe_bounded_wait.argtypes = [P, ctypes.c_int64, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
                   "moe_layer_fwd",
-                  "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc"):
+                  "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -187,6 +188,12 @@ def moe_plan_noalloc(c, logits, topk_idx, topk_w, counts, row_of, header, stream
     """moe_plan with its scratch in the library's static device array (no workspace)."""
     _check(lib().moe_plan_noalloc(ctypes.byref(config(c)), _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
                                   _ptr(counts), _ptr(row_of), _ptr(header), _stream(stream)), "moe_plan_noalloc")
+
+
+def moe_probe_bounded_wait(status_word, budget_cycles: int, stream=None):
+    """Runs the device timeout check: a wait on an mbarrier nothing arrives on."""
+    _check(lib().moe_probe_bounded_wait(_ptr(status_word), int(budget_cycles), _stream(stream)),
+           "moe_probe_bounded_wait")
 
 
 def moe_read_status(ws, stream=None) -> int:

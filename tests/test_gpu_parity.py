@@ -56,6 +56,27 @@ def test_medium_bf16_layers(cfg):
     check_full_small(cfg, 0)
 
 
+# Degenerate and edge shapes: ragged chunks and tiles (T not a multiple of
+# 32, S*K not a multiple of 128), every expert chosen by every token (K = E),
+# one expert per rank, one token per rank, one hot expert in every token,
+# the widest top-k path (E = 1024, K = 16) with most experts nearly empty.
+EDGE = [
+    C.LayerConfig("ragged", T=500, d=256, E=8, K=2, F=256, R=4, tile=128, budget=2, zipf_s=1.0),
+    C.LayerConfig("k_eq_e", T=256, d=256, E=4, K=4, F=128, R=2, tile=128, budget=1),
+    C.LayerConfig("e_eq_r", T=512, d=256, E=4, K=2, F=128, R=4, tile=128, budget=2, zipf_s=2.0),
+    C.LayerConfig("s_eq_1", T=8, d=256, E=8, K=2, F=128, R=8, tile=128, budget=1),
+    C.LayerConfig("hot", T=512, d=256, E=16, K=2, F=128, R=4, tile=128, budget=2, hot_bias=30.0),
+    C.LayerConfig("wide_e", T=256, d=256, E=1024, K=16, F=128, R=8, tile=128, budget=4, zipf_s=1.0,
+                  gating=C.GATE_SIGMOID_TOPK),
+    C.TINY.replace(name="tiny_fp32_ragged", T=100, R=4, tile=16),
+]
+
+
+@pytest.mark.parametrize("cfg", EDGE, ids=lambda c: c.name)
+def test_edge_shapes(cfg):
+    check_full_small(cfg, 1)
+
+
 def test_budget_zero_is_flagged_and_still_correct():
     cfg = SMALL_BF16.replace(name="nobudget", budget=0, zipf_s=2.0)
     g, ref, _ = check_full_small(cfg, 1)
