@@ -207,6 +207,40 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ the CUDA path
 
+def plan_comparison(cfg, lg, dev, reps=20):
+    """The planners side by side on the step's routing: exact S*K (the layer's
+    planner), MegaFlux's block-granular search, and fixed placement (no
+    replica budget). Per mode: moe_plan time (top-k, histogram, planner, row
+    maps; CUDA events), the busiest rank's tiles against the mean (the
+    straggler an expert-parallel layer would wait for), valid entries on the
+    busiest rank, padded rows, replicas, moves."""
+    from routed_experts_b200 import moe as M
+    out = {}
+    T, K, E = cfg.T, cfg.K, cfg.E
+    for name, c in (("exact_SK", cfg), ("blocks", cfg.replace(plan_mode=C.PLAN_BLOCKS)),
+                    ("fixed_placement", cfg.replace(budget=0))):
+        idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+        w = torch.empty(T, K, dtype=torch.float32, device=dev)
+        counts = torch.empty(E, dtype=torch.int32, device=dev)
+        ws = M.alloc_workspace(c, M.WS_PLAN, dev)
+        for _ in range(3):
+            M.moe_plan(c, lg, idx, w, counts, ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            M.moe_plan(c, lg, idx, w, counts, ws)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        pl = M.read_plan(c, ws)
+        tiles = np.diff(pl["rank_row0"].numpy()) // c.tile
+        out[name] = {"moe_plan_us": 1e3 * e0.elapsed_time(e1) / reps,
+                     "max_tiles_per_rank": int(tiles.max()), "mean_tiles_per_rank": float(tiles.mean()),
+                     "max_entries_per_rank": int(pl["rank_load"].max()), "entries_per_rank_mean": T * K / c.R,
+                     "padded_rows": pl["total_rows"] - T * K, "replicas": pl["replicas"], "moves": pl["moves"],
+                     "inexact": bool(pl["status"] & 1)}
+    return out
+
+
 def cpu_baseline(cfg, inp, n_tokens):
     from oracle import oracle as O
     h = {k: I.to_numpy_bits(v) for k, v in inp.items()}
@@ -311,6 +345,7 @@ def run_mine(args, world, rank, local):
         torch.distributed.barrier()
         elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dev)
 
+    plans = plan_comparison(cfg, lg, dev) if rank == 0 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(cfg, inp, args.cpu_tokens)
@@ -374,6 +409,7 @@ def run_mine(args, world, rank, local):
                         "combine_gbs": combine_bytes / (mean[4] * 1e-3) / 1e9},
         "plan": {"moves": plan["moves"], "replicas": plan["replicas"], "status": plan["status"],
                  "padded_rows": plan["total_rows"] - N, "blocks": plan["n_blocks"]},
+        "planners": plans,
         "e2e": {"value": world * T / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * T * E + T * d * eb, "d2h_bytes_per_step": T * d * eb,
                 "ms_per_step": e2e_ms / args.steps},

@@ -66,6 +66,21 @@ enum {
 typedef enum { MOE_BF16 = 0, MOE_FP32 = 1 } moe_dtype;
 typedef enum { MOE_GATE_SOFTMAX_TOPK = 0, MOE_GATE_SIGMOID_TOPK = 1 } moe_gating;
 
+/* Planner modes.
+ * MOE_PLAN_EXACT: [MoonEP] "The greedy balance, step by step" - every rank
+ *   gets exactly S*K entries; each piece is padded to whole tiles.
+ * MOE_PLAN_BLOCKS: [MegaFlux] §3.1 "Bounded greedy search", App. A.1, A.2 -
+ *   load counted in token blocks of `tile` rows, tau = ceil(sum_e b_e / R);
+ *   four greedy candidates (donor priority: overload or largest home
+ *   expert; fan-out: one new copy per expert per round or many), at most
+ *   budget+2 rounds each; the one with the smallest maximum load wins (then
+ *   fewer replicas); replicas whose blocks fit on another copy within that
+ *   maximum are pruned, then single blocks move from the most- to the
+ *   least-loaded rank while they share an expert. Blocks are cut from each
+ *   expert's list owner first, then by rank, so only an expert's last block
+ *   is partial. Requires E*R <= 16384 and T <= 32767*tile. */
+typedef enum { MOE_PLAN_EXACT = 0, MOE_PLAN_BLOCKS = 1 } moe_plan_mode;
+
 /* Workspace kinds for moe_workspace_size. */
 typedef enum {
     MOE_WS_PLAN = 0,       /* plan, row maps and scratch: moe_plan .. moe_combine */
@@ -85,8 +100,9 @@ typedef enum {
  */
 typedef struct {
     int32_t T, d, E, K, F, R, tile, budget;
-    int32_t dtype;   /* moe_dtype */
-    int32_t gating;  /* moe_gating */
+    int32_t dtype;      /* moe_dtype */
+    int32_t gating;     /* moe_gating */
+    int32_t plan_mode;  /* moe_plan_mode */
 } moe_config;
 
 /*
@@ -94,7 +110,8 @@ typedef struct {
  * the workspace base) and the capacities those arrays are sized for.
  * All arrays are int32.
  *   header     [8]: device status bits, n_pieces, n_blocks, total_rows,
- *                   moves, replicas in total, 0, 0
+ *                   moves, replicas in total, then for MOE_PLAN_BLOCKS tau
+ *                   and the winning candidate (2*priority + fan-out), else 0, 0
  *   pieces     [max_pieces][5]: expert, rank, start, len, row0 - rank
  *                   `rank` computes entries [start, start+len) of expert's
  *                   (token, slot)-ordered list at padded rows row0..;

@@ -167,6 +167,48 @@ int orc_histogram(int64_t n_entries, int32_t E, const int32_t* idx, int32_t* cou
  *    plan is exact); each piece is then padded to whole beta-row tiles at a
  *    beta-aligned row, pieces laid out in (rank, expert) order.
  */
+/* Tile layout of a plan given as a table of pieces (rank r computes entries
+ * [start, start+len) of expert e's list): pieces in (rank, expert) order,
+ * each padded to whole tiles at a tile-aligned row, and one block per tile.
+ * [MegaFlux] §3.1 'Problem formulation': blocks of at most beta rows match
+ * the FC1/FC2 token tile. */
+static void layout_pieces(int32_t E, int32_t R, int32_t tile, const int64_t* p_start,
+                          const int64_t* p_len, const int32_t* used, orc_piece* pieces,
+                          int32_t* n_pieces, orc_block* blocks, int32_t* n_blocks,
+                          int64_t* rank_load, int32_t* rank_replicas, int64_t* rank_row0)
+{
+    int32_t np = 0, nb = 0;
+    int64_t row = 0;
+    for (int r = 0; r < R; ++r) {
+        rank_row0[r] = row;
+        rank_load[r] = 0;
+        rank_replicas[r] = used[r];
+        for (int e = 0; e < E; ++e) {
+            int64_t len = p_len[(size_t)r * E + e];
+            if (len == 0) continue;
+            orc_piece* p = &pieces[np++];
+            p->expert = e;
+            p->rank = r;
+            p->start = (int32_t)p_start[(size_t)r * E + e];
+            p->len = (int32_t)len;
+            p->row0 = (int32_t)row;
+            int64_t ntiles = (len + tile - 1) / tile;
+            for (int64_t i = 0; i < ntiles; ++i) {
+                orc_block* b = &blocks[nb++];
+                b->expert = e;
+                b->row0 = (int32_t)(row + i * tile);
+                b->valid = (int32_t)((len - i * tile) < tile ? (len - i * tile) : tile);
+                b->rank = r;
+            }
+            row += ntiles * tile;
+            rank_load[r] += len;
+        }
+    }
+    rank_row0[R] = row;
+    *n_pieces = np;
+    *n_blocks = nb;
+}
+
 int orc_plan(int64_t T, int32_t E, int32_t K, int32_t R, int32_t tile, int32_t budget,
              const int32_t* counts,
              orc_piece* pieces, int32_t* n_pieces,
@@ -248,44 +290,278 @@ int orc_plan(int64_t T, int32_t E, int32_t K, int32_t R, int32_t tile, int32_t b
         }
     }
 
-    /* tile layout: pieces in (rank, expert) order, each padded to whole tiles */
-    {
-        int32_t np = 0, nb = 0;
-        int64_t row = 0;
-        for (int r = 0; r < R; ++r) {
-            rank_row0[r] = row;
-            rank_load[r] = 0;
-            rank_replicas[r] = used[r];
-            for (int e = 0; e < E; ++e) {
-                int64_t len = p_len[(size_t)r * E + e];
-                if (len == 0) continue;
-                orc_piece* p = &pieces[np++];
-                p->expert = e;
-                p->rank = r;
-                p->start = (int32_t)p_start[(size_t)r * E + e];
-                p->len = (int32_t)len;
-                p->row0 = (int32_t)row;
-                int64_t ntiles = (len + tile - 1) / tile;
-                for (int64_t i = 0; i < ntiles; ++i) {
-                    orc_block* b = &blocks[nb++];
-                    b->expert = e;
-                    b->row0 = (int32_t)(row + i * tile);
-                    b->valid = (int32_t)((len - i * tile) < tile ? (len - i * tile) : tile);
-                    b->rank = r;
-                }
-                row += ntiles * tile;
-                rank_load[r] += len;
-            }
-        }
-        rank_row0[R] = row;
-        *n_pieces = np;
-        *n_blocks = nb;
-    }
+    layout_pieces(E, R, tile, p_start, p_len, used, pieces, n_pieces, blocks, n_blocks,
+                  rank_load, rank_replicas, rank_row0);
     *moves_out = moves;
     *status = st;
 done:
     free(rem); free(L); free(used); free(p_start); free(p_len);
     return rc;
+}
+
+/* ------------------------------------------------- block-granular planner
+ * [MegaFlux] §3.1 'Bounded greedy search', App. A.1 'Candidate construction'
+ * and 'Refinement', App. A.2 'Mapping blocks to routed assignments', §4.1
+ * (s replica slots per GPU).
+ *
+ * Load is counted in token blocks: b_e = ceil(c_e / beta), tau =
+ * ceil(sum_e b_e / R). Each of four candidates starts from the no-replica
+ * assignment q[e][owner(e)] = b_e and runs at most s+2 rounds; a round with
+ * no movement ends it. A round visits the over-loaded owners once, in the
+ * candidate's donor priority (decreasing overload load-tau, or decreasing
+ * largest remaining home-expert block count). A visit scans the donor's home
+ * experts by decreasing remaining blocks and moves blocks of each to ranks
+ * below tau: first to ranks already holding a copy of the expert, then by
+ * opening a new copy on the least-loaded rank with a free replica slot; the
+ * visit ends when the donor reaches tau or its scan finishes, an expert's
+ * fan-out ends when the donor has no block of it left or no eligible
+ * receiver remains. The SINGLE fan-out opens at most one new copy per expert
+ * per round, MULTI any number. The candidate with the smallest maximum load
+ * wins (ties: fewer replicas, then candidate order). Pruning visits the
+ * replicas in increasing block count and moves a replica's whole allocation
+ * to the owner, else to the least-loaded other copy, when that copy stays
+ * within the winner's maximum load. A bounded pass then moves single blocks
+ * from the most- to the least-loaded rank while they share an expert and
+ * their loads differ by more than one.
+ *
+ * READINGS: ties go to the lowest index everywhere; a move carries
+ * min(donor blocks of e, donor load - tau, tau - receiver load) blocks (no
+ * donor drops below tau, no receiver rises above it); a rank shares an
+ * expert when it owns it or holds blocks of it; materialisation cuts each
+ * expert's (token, slot)-ordered list into blocks of beta and gives the
+ * owner the first q blocks, then the other ranks in increasing index, so only
+ * the expert's last block is partial. moves counts greedy transfers, pruning
+ * relocations and refinement moves. The plan is never flagged inexact.
+ * info: [0] tau, [1] winning candidate (2*priority + fan-out), [2] its
+ * maximum load in blocks, [3] replicas in total after refinement.
+ */
+static void run_candidate(int32_t E, int32_t R, int32_t per, int32_t budget, int64_t tau,
+                          const int64_t* b, int prio, int fan, int64_t* q, int64_t* load,
+                          int32_t* nrep, int32_t* moves_out, char* newcopy, int32_t* order,
+                          int32_t* donors)
+{
+    int32_t moves = 0;
+    for (int e = 0; e < E; ++e)
+        for (int r = 0; r < R; ++r) q[(size_t)e * R + r] = (r == e / per) ? b[e] : 0;
+    for (int r = 0; r < R; ++r) { load[r] = 0; nrep[r] = 0; }
+    for (int e = 0; e < E; ++e) load[e / per] += b[e];
+
+    for (int round = 0; round < budget + 2; ++round) {
+        int64_t moved = 0;
+        memset(newcopy, 0, (size_t)E);
+        /* donors of this round, in priority order (selection sort, stable by index) */
+        int nd = 0;
+        for (int r = 0; r < R; ++r) if (load[r] > tau) donors[nd++] = r;
+        int64_t* key = (int64_t*)malloc(sizeof(int64_t) * (size_t)(nd ? nd : 1));
+        for (int i = 0; i < nd; ++i) {
+            int r = donors[i];
+            if (prio == 0) key[i] = load[r] - tau;
+            else {
+                int64_t m = 0;
+                for (int e = r * per; e < (r + 1) * per; ++e)
+                    if (q[(size_t)e * R + r] > m) m = q[(size_t)e * R + r];
+                key[i] = m;
+            }
+        }
+        for (int i = 0; i < nd; ++i) {
+            int best = i;
+            for (int j = i + 1; j < nd; ++j)
+                if (key[j] > key[best] || (key[j] == key[best] && donors[j] < donors[best])) best = j;
+            int tr = donors[i]; donors[i] = donors[best]; donors[best] = tr;
+            int64_t tk = key[i]; key[i] = key[best]; key[best] = tk;
+        }
+        free(key);
+        for (int di = 0; di < nd; ++di) {
+            const int d = donors[di];
+            if (load[d] <= tau) continue;
+            /* home experts by decreasing remaining blocks, at visit start */
+            int no = 0;
+            for (int e = d * per; e < (d + 1) * per; ++e) order[no++] = e;
+            for (int i = 0; i < no; ++i) {
+                int best = i;
+                for (int j = i + 1; j < no; ++j) {
+                    int64_t qj = q[(size_t)order[j] * R + d], qb = q[(size_t)order[best] * R + d];
+                    if (qj > qb || (qj == qb && order[j] < order[best])) best = j;
+                }
+                int t = order[i]; order[i] = order[best]; order[best] = t;
+            }
+            for (int i = 0; i < no && load[d] > tau; ++i) {
+                const int e = order[i];
+                while (load[d] > tau && q[(size_t)e * R + d] > 0) {
+                    int rcv = -1;
+                    for (int r = 0; r < R; ++r) {           /* an existing copy first */
+                        if (r == d || q[(size_t)e * R + r] == 0 || load[r] >= tau) continue;
+                        if (rcv < 0 || load[r] < load[rcv]) rcv = r;
+                    }
+                    if (rcv < 0) {
+                        if (fan == 0 && newcopy[e]) break;
+                        for (int r = 0; r < R; ++r) {       /* a new copy */
+                            if (r == d || q[(size_t)e * R + r] > 0 || load[r] >= tau || nrep[r] >= budget)
+                                continue;
+                            if (rcv < 0 || load[r] < load[rcv]) rcv = r;
+                        }
+                        if (rcv < 0) break;
+                        nrep[rcv] += 1;
+                        newcopy[e] = 1;
+                    }
+                    int64_t x = q[(size_t)e * R + d];
+                    if (load[d] - tau < x) x = load[d] - tau;
+                    if (tau - load[rcv] < x) x = tau - load[rcv];
+                    q[(size_t)e * R + d] -= x;
+                    q[(size_t)e * R + rcv] += x;
+                    load[d] -= x;
+                    load[rcv] += x;
+                    moved += x;
+                    moves += 1;
+                }
+            }
+        }
+        if (moved == 0) break;
+    }
+    *moves_out = moves;
+}
+
+int orc_plan_blocks(int64_t T, int32_t E, int32_t K, int32_t R, int32_t tile, int32_t budget,
+                    const int32_t* counts,
+                    orc_piece* pieces, int32_t* n_pieces,
+                    orc_block* blocks, int32_t* n_blocks,
+                    int64_t* rank_load, int32_t* rank_replicas, int64_t* rank_row0,
+                    int32_t* moves_out, uint32_t* status, int32_t* info)
+{
+    if (R <= 0 || E <= 0 || E % R != 0 || T % R != 0 || tile <= 0 || budget < 0)
+        return ORC_ERR_ARG;
+    (void)K;
+    const int32_t per = E / R;
+    int64_t* b = (int64_t*)malloc(sizeof(int64_t) * (size_t)E);
+    int64_t* qbest = (int64_t*)malloc(sizeof(int64_t) * (size_t)E * R);
+    int64_t* q = (int64_t*)malloc(sizeof(int64_t) * (size_t)E * R);
+    int64_t* load = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
+    int64_t* lbest = (int64_t*)malloc(sizeof(int64_t) * (size_t)R);
+    int32_t* nrep = (int32_t*)malloc(sizeof(int32_t) * (size_t)R);
+    int32_t* nbest = (int32_t*)malloc(sizeof(int32_t) * (size_t)R);
+    char* newcopy = (char*)malloc((size_t)E);
+    int32_t* order = (int32_t*)malloc(sizeof(int32_t) * (size_t)(per + E * R + 1));
+    int32_t* donors = (int32_t*)malloc(sizeof(int32_t) * (size_t)R);
+    int64_t* p_start = (int64_t*)calloc((size_t)R * E, sizeof(int64_t));
+    int64_t* p_len = (int64_t*)calloc((size_t)R * E, sizeof(int64_t));
+    if (!b || !qbest || !q || !load || !lbest || !nrep || !nbest || !newcopy || !order || !donors ||
+        !p_start || !p_len) {
+        free(b); free(qbest); free(q); free(load); free(lbest); free(nrep); free(nbest); free(newcopy);
+        free(order); free(donors); free(p_start); free(p_len);
+        return ORC_ERR_INTERNAL;
+    }
+    int64_t total = 0;
+    for (int e = 0; e < E; ++e) { b[e] = (counts[e] + tile - 1) / tile; total += b[e]; }
+    const int64_t tau = (total + R - 1) / R;
+
+    /* four candidates: (donor priority, fan-out) = (0,0), (0,1), (1,0), (1,1) */
+    int best_c = -1, moves = 0;
+    int64_t best_max = 0, best_reps = 0;
+    for (int c = 0; c < 4; ++c) {
+        int32_t mv = 0;
+        run_candidate(E, R, per, budget, tau, b, c / 2, c % 2, q, load, nrep, &mv, newcopy, order, donors);
+        int64_t mx = 0, reps = 0;
+        for (int r = 0; r < R; ++r) { if (load[r] > mx) mx = load[r]; reps += nrep[r]; }
+        if (best_c < 0 || mx < best_max || (mx == best_max && reps < best_reps)) {
+            best_c = c; best_max = mx; best_reps = reps; moves = mv;
+            memcpy(qbest, q, sizeof(int64_t) * (size_t)E * R);
+            memcpy(lbest, load, sizeof(int64_t) * (size_t)R);
+            memcpy(nbest, nrep, sizeof(int32_t) * (size_t)R);
+        }
+    }
+    q = (int64_t*)memcpy(q, qbest, sizeof(int64_t) * (size_t)E * R);
+    memcpy(load, lbest, sizeof(int64_t) * (size_t)R);
+    memcpy(nrep, nbest, sizeof(int32_t) * (size_t)R);
+
+    /* pruning: replicas in increasing allocation size (at pass entry) */
+    {
+        int nr = 0;
+        int32_t* rl = order;   /* pairs (e, r) packed as e*R + r */
+        for (int e = 0; e < E; ++e)
+            for (int r = 0; r < R; ++r)
+                if (r != e / per && q[(size_t)e * R + r] > 0) rl[nr++] = e * R + r;
+        for (int i = 0; i < nr; ++i) {   /* stable selection sort by (blocks, e, r) */
+            int best = i;
+            for (int j = i + 1; j < nr; ++j) {
+                int64_t qj = q[rl[j]], qb = q[rl[best]];
+                if (qj < qb || (qj == qb && rl[j] < rl[best])) best = j;
+            }
+            int t = rl[i]; rl[i] = rl[best]; rl[best] = t;
+        }
+        for (int i = 0; i < nr; ++i) {
+            const int e = rl[i] / R, r = rl[i] % R, o = e / per;
+            const int64_t x = q[(size_t)e * R + r];
+            if (x == 0) continue;
+            int tgt = -1;
+            if (load[o] + x <= best_max) tgt = o;
+            else {
+                for (int c2 = 0; c2 < R; ++c2) {
+                    if (c2 == r || c2 == o || q[(size_t)e * R + c2] == 0 || load[c2] + x > best_max) continue;
+                    if (tgt < 0 || load[c2] < load[tgt]) tgt = c2;
+                }
+            }
+            if (tgt < 0) continue;
+            q[(size_t)e * R + r] = 0;
+            q[(size_t)e * R + tgt] += x;
+            load[r] -= x;
+            load[tgt] += x;
+            nrep[r] -= 1;
+            moves += 1;
+        }
+    }
+    /* refinement: single blocks from the most- to the least-loaded rank */
+    for (int64_t it = 0; it < total; ++it) {
+        int hi = 0, lo = 0;
+        for (int r = 1; r < R; ++r) {
+            if (load[r] > load[hi]) hi = r;
+            if (load[r] < load[lo]) lo = r;
+        }
+        if (load[hi] - load[lo] <= 1) break;
+        int e_sh = -1;
+        for (int e = 0; e < E && e_sh < 0; ++e)
+            if (q[(size_t)e * R + hi] > 0 && (lo == e / per || q[(size_t)e * R + lo] > 0)) e_sh = e;
+        if (e_sh < 0) break;
+        q[(size_t)e_sh * R + hi] -= 1;
+        q[(size_t)e_sh * R + lo] += 1;
+        load[hi] -= 1;
+        load[lo] += 1;
+        moves += 1;
+    }
+    /* materialise: owner first, then the other ranks in increasing index */
+    int32_t* used = nrep;
+    for (int r = 0; r < R; ++r) used[r] = 0;
+    int64_t mx = 0;
+    for (int r = 0; r < R; ++r) if (load[r] > mx) mx = load[r];
+    for (int e = 0; e < E; ++e) {
+        const int o = e / per;
+        int64_t off = 0;
+        for (int k = -1; k < R; ++k) {
+            const int r = k < 0 ? o : k;
+            if (k >= 0 && r == o) continue;
+            const int64_t n = q[(size_t)e * R + r];
+            if (n == 0) continue;
+            const int64_t start = off * tile;
+            int64_t end = (off + n) * tile;
+            if (end > counts[e]) end = counts[e];
+            p_start[(size_t)r * E + e] = start;
+            p_len[(size_t)r * E + e] = end - start;
+            if (r != o) used[r] += 1;
+            off += n;
+        }
+    }
+    layout_pieces(E, R, tile, p_start, p_len, used, pieces, n_pieces, blocks, n_blocks, rank_load,
+                  rank_replicas, rank_row0);
+    int64_t reps = 0;
+    for (int r = 0; r < R; ++r) reps += used[r];
+    *moves_out = moves;
+    *status = 0;
+    info[0] = (int32_t)tau;
+    info[1] = best_c;
+    info[2] = (int32_t)mx;
+    info[3] = (int32_t)reps;
+    free(b); free(qbest); free(q); free(load); free(lbest); free(nrep); free(nbest); free(newcopy);
+    free(order); free(donors); free(p_start); free(p_len);
+    return ORC_OK;
 }
 
 /* ------------------------------------------------- row maps (A5)

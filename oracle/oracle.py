@@ -51,6 +51,7 @@ def lib():
         L.orc_topk_gate.argtypes = [i64, i32, i32, i32, P, P, P]
         L.orc_histogram.argtypes = [i64, i32, P, P]
         L.orc_plan.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P]
+        L.orc_plan_blocks.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P, P]
         L.orc_row_maps.argtypes = [i64, i32, i32, P, P, i32, i64, P, P]
         L.orc_dispatch.argtypes = [i64, i32, i32, P, P, P]
         L.orc_expert_ffn.argtypes = [i32, i32, i32, i32, i32, P, i32, P, P, P, P, P]
@@ -60,7 +61,7 @@ def lib():
         L.orc_entry_ffn.argtypes = [i32, i32, i32, i32, i64, P, P, P, P, P, P, P]
         L.orc_double_to_bf16.argtypes = [ctypes.c_double]
         L.orc_double_to_bf16.restype = ctypes.c_uint16
-        for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_row_maps", "orc_dispatch",
+        for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_plan_blocks", "orc_row_maps", "orc_dispatch",
                   "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer", "orc_entry_ffn"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -114,7 +115,14 @@ def histogram(idx: np.ndarray, E: int) -> np.ndarray:
     return counts
 
 
-def plan(T: int, E: int, K: int, R: int, tile: int, budget: int, counts: np.ndarray) -> dict:
+PLAN_EXACT, PLAN_BLOCKS = 0, 1
+
+
+def plan(T: int, E: int, K: int, R: int, tile: int, budget: int, counts: np.ndarray,
+         mode: int = PLAN_EXACT) -> dict:
+    """The replication plan. mode PLAN_EXACT: the MoonEP-style greedy to exactly
+    S*K entries per rank; PLAN_BLOCKS: MegaFlux's block-granular four-candidate
+    search, pruning and refinement."""
     counts = np.ascontiguousarray(counts, dtype=np.int32)
     N = T * K
     pieces = np.zeros((max_pieces(E, R, budget), 5), np.int32)
@@ -126,13 +134,19 @@ def plan(T: int, E: int, K: int, R: int, tile: int, budget: int, counts: np.ndar
     rank_row0 = np.zeros(R + 1, np.int64)
     moves = np.zeros(1, np.int32)
     status = np.zeros(1, np.uint32)
-    _check(lib().orc_plan(T, E, K, R, tile, budget, _p(counts), _p(pieces), _p(npc), _p(blocks),
-                          _p(nbl), _p(rank_load), _p(rank_rep), _p(rank_row0), _p(moves),
-                          _p(status)), "plan")
+    info = np.zeros(4, np.int32)
+    if mode == PLAN_EXACT:
+        _check(lib().orc_plan(T, E, K, R, tile, budget, _p(counts), _p(pieces), _p(npc), _p(blocks),
+                              _p(nbl), _p(rank_load), _p(rank_rep), _p(rank_row0), _p(moves),
+                              _p(status)), "plan")
+    else:
+        _check(lib().orc_plan_blocks(T, E, K, R, tile, budget, _p(counts), _p(pieces), _p(npc), _p(blocks),
+                                     _p(nbl), _p(rank_load), _p(rank_rep), _p(rank_row0), _p(moves),
+                                     _p(status), _p(info)), "plan_blocks")
     return {"pieces": pieces[:npc[0]].copy(), "blocks": blocks[:nbl[0]].copy(),
             "rank_load": rank_load, "rank_replicas": rank_rep, "rank_row0": rank_row0,
             "moves": int(moves[0]), "status": int(status[0]),
-            "total_rows": int(rank_row0[R])}
+            "total_rows": int(rank_row0[R]), "info": info}
 
 
 def row_maps(idx: np.ndarray, E: int, pieces: np.ndarray, rows_cap: int):
@@ -250,13 +264,13 @@ def default_round_mode(dtype: int) -> int:
 
 
 def layer(logits, x, w_gu, w_down, *, K, R, tile, budget, gating, dtype, round_mode=None,
-          ffn=True) -> dict:
+          ffn=True, plan_mode: int = PLAN_EXACT) -> dict:
     """Every step of the layer on numpy inputs; returns each intermediate."""
     rm = default_round_mode(dtype) if round_mode is None else round_mode
     T, E = logits.shape
     idx, w = topk_gate(logits, K, gating)
     counts = histogram(idx, E)
-    pl = plan(T, E, K, R, tile, budget, counts)
+    pl = plan(T, E, K, R, tile, budget, counts, plan_mode)
     cap = rows_capacity(T * K, E, R, budget, tile)
     row_of, src_of = row_maps(idx, E, pl["pieces"], cap)
     res = {"idx": idx, "w": w, "counts": counts, "plan": pl, "row_of": row_of,

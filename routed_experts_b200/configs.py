@@ -18,6 +18,8 @@ BF16 = 0
 FP32 = 1
 GATE_SOFTMAX_TOPK = 0
 GATE_SIGMOID_TOPK = 1
+PLAN_EXACT = 0    # exactly S*K entries per rank (greedy refill from the biggest donor)
+PLAN_BLOCKS = 1   # block-granular four-candidate search, pruning and refinement
 
 
 @dataclasses.dataclass(frozen=True)
@@ -33,6 +35,7 @@ class LayerConfig:
     budget: int     # replicas a rank may host
     dtype: int = BF16
     gating: int = GATE_SOFTMAX_TOPK
+    plan_mode: int = PLAN_EXACT
     # input recipe
     logits: str = "xwr"      # "xwr": x @ Wr + bias; "normal": N(0,1) + bias
     zipf_s: float = 0.0      # bias_e = -s * ln(rank_e) over a seeded expert permutation
@@ -78,5 +81,6 @@ def describe(c: LayerConfig) -> dict:
             "R": c.R, "tile": c.tile, "budget": c.budget,
             "dtype": "bf16" if c.dtype == BF16 else "fp32",
             "gating": "softmax_topk" if c.gating == GATE_SOFTMAX_TOPK else "sigmoid_topk",
+            "planner": "exact_SK" if c.plan_mode == PLAN_EXACT else "blocks",
             "router": c.logits, "zipf_s": c.zipf_s, "hot_bias": c.hot_bias,
             "hot_frac": c.hot_frac}

@@ -21,6 +21,10 @@ moe_status make_shape(const moe_config* cfg, Shape* s) {
     if (c.K > c.E || c.T % c.R != 0 || c.E % c.R != 0) return MOE_ERR_INVALID_ARG;
     if (c.dtype != MOE_BF16 && c.dtype != MOE_FP32) return MOE_ERR_INVALID_ARG;
     if (c.gating != MOE_GATE_SOFTMAX_TOPK && c.gating != MOE_GATE_SIGMOID_TOPK) return MOE_ERR_INVALID_ARG;
+    if (c.plan_mode != MOE_PLAN_EXACT && c.plan_mode != MOE_PLAN_BLOCKS) return MOE_ERR_INVALID_ARG;
+    if (c.plan_mode == MOE_PLAN_BLOCKS &&
+        ((int64_t)c.E * c.R > 16384 || (int64_t)c.T > (int64_t)32767 * c.tile))
+        return MOE_ERR_UNSUPPORTED;
     if (c.K > kMaxK || c.E > kMaxE || c.R > kMaxR || c.budget > kMaxBudget || (int64_t)c.R * c.budget > 1024)
         return MOE_ERR_UNSUPPORTED;
     if (c.dtype == MOE_BF16) {
@@ -30,7 +34,7 @@ moe_status make_shape(const moe_config* cfg, Shape* s) {
             return MOE_ERR_UNSUPPORTED;
     }
     s->T = c.T; s->d = c.d; s->E = c.E; s->K = c.K; s->F = c.F; s->R = c.R; s->tile = c.tile;
-    s->budget = c.budget; s->dtype = c.dtype; s->gating = c.gating;
+    s->budget = c.budget; s->dtype = c.dtype; s->gating = c.gating; s->plan_mode = c.plan_mode;
     s->N = (int64_t)c.T * c.K;
     s->C = (int64_t)(c.T / c.R) * c.K;
     s->per = c.E / c.R;

@@ -20,7 +20,7 @@ constexpr int kBlockInts = 4;             // expert, row0, valid, rank
 
 // header words
 enum { H_STATUS = 0, H_NPIECES = 1, H_NBLOCKS = 2, H_TOTAL_ROWS = 3, H_MOVES = 4,
-       H_REPLICAS = 5, H_WORDS = 8 };
+       H_REPLICAS = 5, H_TAU = 6, H_CANDIDATE = 7, H_WORDS = 8 };
 
 // Work-queue counters of the grouped GEMM: for FC1 then FC2, two queue
 // heads and a count of clusters that finished (all zero between launches).
@@ -30,7 +30,7 @@ constexpr int kGemmQWords = 8;
 constexpr long long kSpinBudget = 4000000000LL;
 
 struct Shape {
-    int32_t T, d, E, K, F, R, tile, budget, dtype, gating;
+    int32_t T, d, E, K, F, R, tile, budget, dtype, gating, plan_mode;
     int64_t N;          // T*K
     int64_t C;          // (T/R)*K
     int32_t per;        // E/R

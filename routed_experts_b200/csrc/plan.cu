@@ -68,7 +68,126 @@ struct PlanArgs {
     int E, R, per, tile, budget, n_chunks, G;
     int C;
     int max_rep;
+    int plan_mode;
 };
+
+// ---------------------------------------------------------------- warp helpers
+// Minimum of (v, i) over the warp, lowest i on ties.
+__device__ __forceinline__ void warp_min_vi(int& v, int& i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const int ov = __shfl_xor_sync(0xffffffffu, v, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, off);
+        if (ov < v || (ov == v && oi < i)) { v = ov; i = oi; }
+    }
+}
+
+// Maximum of v over the warp, lowest i on ties.
+__device__ __forceinline__ void warp_max_vi(int& v, int& i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const int ov = __shfl_xor_sync(0xffffffffu, v, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, off);
+        if (ov > v || (ov == v && oi < i)) { v = ov; i = oi; }
+    }
+}
+
+// One greedy candidate of the block-granular planner ([MegaFlux] §3.1
+// 'Bounded greedy search', App. A.1), run by one warp on its own copy of the
+// assignment q[e*R + r] (blocks of expert e on rank r). prio 0: donors by
+// decreasing overload; prio 1: by largest remaining home-expert blocks.
+// fan 0: at most one new copy per expert per round; fan 1: any number.
+__device__ void block_candidate(int prio, int fan, const int32_t* b, int E, int R, int per, int budget, int tau,
+                                int16_t* q, int32_t* load, int32_t* nrep, uint8_t* newcopy, int32_t* dkey,
+                                int32_t* ekey, int32_t* moves_out) {
+    const int lane = threadIdx.x & 31;
+    for (int i = lane; i < E * R; i += 32) q[i] = 0;
+    __syncwarp();
+    for (int e = lane; e < E; e += 32) q[e * R + e / per] = (int16_t)b[e];
+    for (int r = lane; r < R; r += 32) {
+        int sum = 0;
+        for (int e = r * per; e < (r + 1) * per; ++e) sum += b[e];
+        load[r] = sum;
+        nrep[r] = 0;
+    }
+    __syncwarp();
+    int moves = 0;
+    for (int round = 0; round < budget + 2; ++round) {
+        int moved = 0;
+        for (int e = lane; e < E; e += 32) newcopy[e] = 0;
+        for (int r = lane; r < R; r += 32) {
+            int key = -1;
+            if (load[r] > tau) {
+                if (prio == 0) key = load[r] - tau;
+                else {
+                    key = 0;
+                    for (int e = r * per; e < (r + 1) * per; ++e) key = max(key, (int)q[e * R + r]);
+                }
+            }
+            dkey[r] = key;
+        }
+        __syncwarp();
+        for (;;) {
+            // next donor of this round: largest key, lowest rank on ties
+            int bk = -1, br = INT_MAX;
+            for (int r = lane; r < R; r += 32) if (dkey[r] > bk) { bk = dkey[r]; br = r; }
+            warp_max_vi(bk, br);
+            if (bk < 0) break;
+            const int d = br;
+            __syncwarp();
+            if (lane == 0) dkey[d] = -1;
+            for (int i = lane; i < per; i += 32) ekey[i] = q[(d * per + i) * R + d];
+            __syncwarp();
+            for (;;) {
+                if (load[d] <= tau) break;
+                // the donor's next home expert: most remaining blocks, lowest id on ties
+                int bv = -1, bi = INT_MAX;
+                for (int i = lane; i < per; i += 32) if (ekey[i] > bv) { bv = ekey[i]; bi = i; }
+                warp_max_vi(bv, bi);
+                if (bv < 0) break;
+                __syncwarp();
+                if (lane == 0) ekey[bi] = -1;
+                __syncwarp();
+                const int e = d * per + bi;
+                while (load[d] > tau && q[e * R + d] > 0) {
+                    // an existing copy below tau, least loaded first
+                    int lv = INT_MAX, lr = INT_MAX;
+                    for (int r = lane; r < R; r += 32)
+                        if (r != d && q[e * R + r] > 0 && load[r] < tau && load[r] < lv) { lv = load[r]; lr = r; }
+                    warp_min_vi(lv, lr);
+                    if (lv == INT_MAX) {
+                        if (fan == 0 && newcopy[e]) break;
+                        for (int r = lane; r < R; r += 32)
+                            if (r != d && q[e * R + r] == 0 && load[r] < tau && nrep[r] < budget && load[r] < lv) {
+                                lv = load[r];
+                                lr = r;
+                            }
+                        warp_min_vi(lv, lr);
+                        if (lv == INT_MAX) break;
+                        __syncwarp();
+                        if (lane == 0) { nrep[lr] += 1; newcopy[e] = 1; }
+                    }
+                    const int rcv = lr;
+                    int x = q[e * R + d];
+                    x = min(x, load[d] - tau);
+                    x = min(x, tau - load[rcv]);
+                    __syncwarp();
+                    if (lane == 0) {
+                        q[e * R + d] = (int16_t)(q[e * R + d] - x);
+                        q[e * R + rcv] = (int16_t)(q[e * R + rcv] + x);
+                        load[d] -= x;
+                        load[rcv] += x;
+                    }
+                    __syncwarp();
+                    moved += x;
+                    moves += 1;
+                }
+            }
+        }
+        if (moved == 0) break;
+    }
+    if (lane == 0) *moves_out = moves;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
@@ -84,8 +203,19 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
     int32_t* pfb = rep + 5 * a.max_rep;              // [max_pieces+1]: first block of each piece
     int32_t* pq = pfb + (E + a.max_rep + 1);         // [max_pieces][4]: expert, rank, len, row0
     int32_t* tmp = pq + 4 * (E + a.max_rep);         // [32]
+    // block-granular planner (plan_mode 1) state
+    int32_t* bl = tmp + 32;                           // [E] blocks per expert
+    int32_t* cload = bl + E;                          // [4][R]
+    int32_t* cnrep = cload + 4 * R;                   // [4][R]
+    int32_t* cdkey = cnrep + 4 * R;                   // [4][R]
+    int32_t* cekey = cdkey + 4 * R;                   // [4][per]
+    int32_t* cmoves = cekey + 4 * a.per;              // [4]
+    int32_t* plist = cmoves + 4;                      // [max_rep][2]: (e*R + r, blocks at pass entry)
+    uint8_t* cnew = reinterpret_cast<uint8_t*>(plist + 2 * a.max_rep);        // [4][E]
+    int16_t* cq = reinterpret_cast<int16_t*>(cnew + ((4 * E + 15) & ~15));   // [4][E*R]
     __shared__ uint32_t s_status;
     __shared__ int s_moves, s_nrep;
+    __shared__ int s_tot_blocks, s_tau, s_best;   // block-granular planner
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
     // ---------------- (A) totals and per-chunk offsets
@@ -136,7 +266,7 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
     __syncthreads();
 
     // ---------------- (B) greedy moves, warp 0
-    if (warp == 0) {
+    if (a.plan_mode == MOE_PLAN_EXACT && warp == 0) {
         const int C = a.C;
         const int cap = R * R + E;
         int moves = 0, nrep = 0;
@@ -202,6 +332,159 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
             s_nrep = nrep;
             if (st) atomicOr(&s_status, st);
         }
+    }
+    if (a.plan_mode == MOE_PLAN_BLOCKS) {
+        // ---------------- (B') block-granular planner ([MegaFlux] §3.1, App. A.1, A.2)
+        int tot_blocks = 0;
+        for (int e = tid; e < E; e += kThreads) bl[e] = (cnt[e] + a.tile - 1) / a.tile;
+        __syncthreads();
+        if (warp == 0) {
+            int sum = 0;
+            for (int e = lane; e < E; e += 32) sum += bl[e];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+            if (lane == 0) s_tot_blocks = sum;
+        }
+        __syncthreads();
+        tot_blocks = s_tot_blocks;
+        const int tau = (tot_blocks + R - 1) / R;
+        if (warp < 4) {
+            block_candidate(warp / 2, warp % 2, bl, E, R, a.per, a.budget, tau, cq + (size_t)warp * E * R,
+                            cload + warp * R, cnrep + warp * R, cnew + warp * E, cdkey + warp * R,
+                            cekey + warp * a.per, cmoves + warp);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // the winner: smallest maximum load, then fewest replicas, then candidate order
+            int best = 0, best_max = INT_MAX, best_reps = INT_MAX;
+            for (int c = 0; c < 4; ++c) {
+                int mx = 0, reps = 0;
+                for (int r = lane; r < R; r += 32) { mx = max(mx, cload[c * R + r]); reps += cnrep[c * R + r]; }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+                    reps += __shfl_xor_sync(0xffffffffu, reps, off);
+                }
+                if (mx < best_max || (mx == best_max && reps < best_reps)) { best = c; best_max = mx; best_reps = reps; }
+            }
+            int16_t* q = cq + (size_t)best * E * R;
+            int32_t* load = cload + best * R;
+            int32_t* nr = cnrep + best * R;
+            int moves = cmoves[best];
+            // pruning: replicas in increasing blocks at pass entry (then e, r)
+            int np = 0;
+            for (int base = 0; base < E * R; base += 32) {
+                const int i = base + lane;
+                const bool is_rep = i < E * R && (i % R) != (i / R) / a.per && q[i] > 0;
+                const unsigned m = __ballot_sync(0xffffffffu, is_rep);
+                if (is_rep) {
+                    const int at = np + __popc(m & ((1u << lane) - 1u));
+                    plist[2 * at] = i;
+                    plist[2 * at + 1] = q[i];
+                }
+                np += __popc(m);
+            }
+            __syncwarp();
+            for (int k = 0; k < np; ++k) {
+                // next replica: smallest (blocks at entry, e*R + r) among the unvisited
+                int kv = INT_MAX, ki = INT_MAX;
+                for (int j = lane; j < np; j += 32) {
+                    const int v = plist[2 * j + 1], id = plist[2 * j];
+                    if (v >= 0 && (v < kv || (v == kv && id < ki))) { kv = v; ki = id; }
+                }
+                warp_min_vi(kv, ki);
+                for (int j = lane; j < np; j += 32) if (plist[2 * j] == ki) plist[2 * j + 1] = -1;
+                __syncwarp();
+                const int e = ki / R, r = ki % R, o = e / a.per;
+                const int x = q[ki];
+                if (x == 0) continue;
+                int tgt = -1;
+                if (load[o] + x <= best_max) {
+                    tgt = o;
+                } else {
+                    int lv = INT_MAX, lr = INT_MAX;
+                    for (int c2 = lane; c2 < R; c2 += 32)
+                        if (c2 != r && c2 != o && q[e * R + c2] > 0 && load[c2] + x <= best_max && load[c2] < lv) {
+                            lv = load[c2];
+                            lr = c2;
+                        }
+                    warp_min_vi(lv, lr);
+                    if (lv != INT_MAX) tgt = lr;
+                }
+                if (tgt < 0) continue;
+                __syncwarp();
+                if (lane == 0) {
+                    q[ki] = 0;
+                    q[e * R + tgt] = (int16_t)(q[e * R + tgt] + x);
+                    load[r] -= x;
+                    load[tgt] += x;
+                    nr[r] -= 1;
+                }
+                __syncwarp();
+                moves += 1;
+            }
+            // refinement: single blocks from the most- to the least-loaded rank
+            for (int it = 0; it < tot_blocks; ++it) {
+                int hv = INT_MIN, hr = INT_MAX, lv = INT_MAX, lr = INT_MAX;
+                for (int r = lane; r < R; r += 32) {
+                    if (load[r] > hv) { hv = load[r]; hr = r; }
+                    if (load[r] < lv) { lv = load[r]; lr = r; }
+                }
+                warp_max_vi(hv, hr);
+                warp_min_vi(lv, lr);
+                if (hv - lv <= 1) break;
+                int es = INT_MAX;
+                for (int e = lane; e < E; e += 32)
+                    if (q[e * R + hr] > 0 && (e / a.per == lr || q[e * R + lr] > 0)) { es = e; break; }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) es = min(es, __shfl_xor_sync(0xffffffffu, es, off));
+                if (es == INT_MAX) break;
+                __syncwarp();
+                if (lane == 0) {
+                    q[es * R + hr] = (int16_t)(q[es * R + hr] - 1);
+                    q[es * R + lr] = (int16_t)(q[es * R + lr] + 1);
+                    load[hr] -= 1;
+                    load[lr] += 1;
+                }
+                __syncwarp();
+                moves += 1;
+            }
+            if (lane == 0) {
+                s_moves = moves;
+                s_best = best;
+                s_tau = tau;
+            }
+        }
+        __syncthreads();
+        const int best = s_best;
+        const int16_t* q = cq + (size_t)best * E * R;
+        // materialise: the owner takes the first blocks of each expert's list,
+        // then the other ranks in increasing index; replica slices are listed
+        // per expert in decreasing start (the order the layout phase expects)
+        int nrep_e = 0;
+        if (tid < E) for (int r = 0; r < R; ++r) nrep_e += (r != tid / a.per && q[tid * R + r] > 0);
+        int tot_rep;
+        const int rep_off = block_excl_scan(tid < E ? nrep_e : 0, tmp, &tot_rep);
+        if (tid < R) used[tid] = 0;
+        __syncthreads();
+        if (tid < E) {
+            const int e = tid, o = e / a.per, ce = cnt[e];
+            const int owner_blocks = q[e * R + o];
+            rem[e] = min(owner_blocks * a.tile, ce);
+            int off = owner_blocks;
+            int k = rep_off + nrep_e;   // fill from the end: decreasing start
+            for (int r = 0; r < R; ++r) {
+                if (r == o || q[e * R + r] == 0) continue;
+                const int n = q[e * R + r];
+                const int start = off * a.tile;
+                const int end = min((off + n) * a.tile, ce);
+                int32_t* Q = rep + 5 * (--k);
+                Q[0] = r; Q[1] = e; Q[2] = start; Q[3] = end - start; Q[4] = -1;
+                atomicAdd(&used[r], 1);
+                off += n;
+            }
+        }
+        if (tid == 0) s_nrep = tot_rep;
     }
     __syncthreads();
     const int nrep = s_nrep;
@@ -329,6 +612,8 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
         ws.header[H_TOTAL_ROWS] = (uint32_t)tot_rows;
         ws.header[H_MOVES] = (uint32_t)s_moves;
         ws.header[H_REPLICAS] = (uint32_t)nrep;
+        ws.header[H_TAU] = a.plan_mode == MOE_PLAN_BLOCKS ? (uint32_t)s_tau : 0u;
+        ws.header[H_CANDIDATE] = a.plan_mode == MOE_PLAN_BLOCKS ? (uint32_t)s_best : 0u;
         for (int q = 0; q < kGemmQWords; ++q) ws.gemm_q[q] = 0;   // fresh GEMM work queues
     }
 }
@@ -345,8 +630,12 @@ cudaError_t launch_plan(const Shape& s, int32_t* counts_out, const WsPtrs& ws, c
     a.G = G;
     a.C = (int)s.C;
     a.max_rep = s.R * s.budget;
-    const size_t smem = sizeof(int32_t) * ((size_t)G * s.E + 3 * s.E + 2 * s.R + 5 * a.max_rep +
-                                           5 * (s.E + a.max_rep) + 1 + 32);
+    a.plan_mode = s.plan_mode;
+    size_t smem = sizeof(int32_t) * ((size_t)G * s.E + 3 * s.E + 2 * s.R + 5 * a.max_rep +
+                                     5 * (s.E + a.max_rep) + 1 + 32);
+    if (s.plan_mode == MOE_PLAN_BLOCKS)
+        smem += sizeof(int32_t) * ((size_t)s.E + 12 * s.R + 4 * s.per + 4 + 2 * a.max_rep) +
+                (((size_t)4 * s.E + 15) & ~(size_t)15) + sizeof(int16_t) * 4 * (size_t)s.E * s.R;
     cudaError_t err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;

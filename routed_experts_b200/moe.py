@@ -29,7 +29,7 @@ class MoeError(RuntimeError):
 
 class MoeConfig(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in ("T", "d", "E", "K", "F", "R", "tile", "budget", "dtype",
-                                              "gating")]
+                                              "gating", "plan_mode")]
 
 
 class PlanLayout(ctypes.Structure):
@@ -90,7 +90,8 @@ def _check(code: int, what: str):
 
 
 def config(c: "_cfgs.LayerConfig") -> MoeConfig:
-    return MoeConfig(c.T, c.d, c.E, c.K, c.F, c.R, c.tile, c.budget, c.dtype, c.gating)
+    return MoeConfig(c.T, c.d, c.E, c.K, c.F, c.R, c.tile, c.budget, c.dtype, c.gating,
+                     getattr(c, "plan_mode", 0))
 
 
 def _ptr(t: torch.Tensor | None):
@@ -225,7 +226,7 @@ def read_plan(c, ws: torch.Tensor) -> dict:
     total = int(hdr[3])
     return {
         "status": int(hdr[0]), "n_pieces": npc, "n_blocks": nbl, "total_rows": total, "moves": int(hdr[4]),
-        "replicas": int(hdr[5]),
+        "replicas": int(hdr[5]), "tau": int(hdr[6]), "candidate": int(hdr[7]),
         "pieces": arr(v["pieces"], 5 * npc).view(npc, 5),
         "blocks": arr(v["blocks"], 4 * nbl).view(nbl, 4),
         "rank_load": arr(v["rank_load"], c.R),

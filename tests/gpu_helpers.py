@@ -79,6 +79,8 @@ def check_routing_and_plan(cfg, g: dict, ref: dict):
     assert np.array_equal(gp["rank_replicas"].numpy(), rp["rank_replicas"])
     assert np.array_equal(gp["rank_row0"].numpy(), rp["rank_row0"])
     assert gp["replicas"] == int(rp["rank_replicas"].sum())
+    if getattr(cfg, "plan_mode", 0) == O.PLAN_BLOCKS:
+        assert gp["tau"] == rp["info"][0] and gp["candidate"] == rp["info"][1]
     assert np.array_equal(gp["row_of"].numpy(), ref["row_of"]), "row_of differs"
     total = rp["total_rows"]
     assert np.array_equal(gp["src_of"].numpy(), ref["src_of"][:total]), "src_of differs"
@@ -87,7 +89,7 @@ def check_routing_and_plan(cfg, g: dict, ref: dict):
 def oracle_routing(cfg, hin: dict) -> dict:
     idx, w = O.topk_gate(hin["logits"], cfg.K, cfg.gating)
     counts = O.histogram(idx, cfg.E)
-    pl = O.plan(cfg.T, cfg.E, cfg.K, cfg.R, cfg.tile, cfg.budget, counts)
+    pl = O.plan(cfg.T, cfg.E, cfg.K, cfg.R, cfg.tile, cfg.budget, counts, getattr(cfg, "plan_mode", 0))
     cap = O.rows_capacity(cfg.N, cfg.E, cfg.R, cfg.budget, cfg.tile)
     row_of, src_of = O.row_maps(idx, cfg.E, pl["pieces"], cap)
     return {"idx": idx, "w": w, "counts": counts, "plan": pl, "row_of": row_of, "src_of": src_of,
@@ -100,7 +102,8 @@ def check_full_small(cfg, seed: int, device="cuda"):
     g = run_stages(cfg, inp)
     hin = host_inputs(inp)
     ref = O.layer(hin["logits"], hin["x"], hin["w_gate_up"], hin["w_down"], K=cfg.K, R=cfg.R,
-                  tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype)
+                  tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype,
+                  plan_mode=getattr(cfg, "plan_mode", 0))
     assert g["rows_cap"] == ref["rows_cap"]
     check_routing_and_plan(cfg, g, ref)
     assert (g["status"] & ~O.PLAN_INEXACT) == 0, f"device status {g['status']}"

@@ -67,7 +67,7 @@ def test_invalid_configs(M):
     n = ctypes.c_size_t()
     bad = [
         dict(T=0), dict(R=3), dict(K=9, E=8), dict(E=6, R=4), dict(budget=-1), dict(dtype=7),
-        dict(gating=5),
+        dict(gating=5), dict(plan_mode=2),
     ]
     for kw in bad:
         cfg = C.TINY.replace(**kw)
@@ -75,6 +75,8 @@ def test_invalid_configs(M):
     unsupported = [
         C.OLMOE.replace(tile=64), C.OLMOE.replace(F=1000), C.OLMOE.replace(d=2048 + 64),
         C.TINY.replace(tile=8), C.TINY.replace(K=17, E=32), C.TINY.replace(E=2048, R=4),
+        C.TINY.replace(E=1024, R=32, T=256, plan_mode=C.PLAN_BLOCKS),
+        C.TINY.replace(T=32768 * 16, R=4, plan_mode=C.PLAN_BLOCKS),
     ]
     for cfg in unsupported:
         assert L.moe_workspace_size(ctypes.byref(M.config(cfg)), 0, ctypes.byref(n)) == M.MOE_ERR_UNSUPPORTED, cfg

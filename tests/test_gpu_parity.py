@@ -159,6 +159,24 @@ def test_repeated_calls_are_deterministic():
         assert torch.equal(a, b)
 
 
+# MegaFlux's block-granular planner (plan mode 1): the same downstream
+# kernels, a different plan; bit-exact against the oracle's planner.
+BLOCK_SMALL = [c.replace(name=c.name + "_blocks", plan_mode=C.PLAN_BLOCKS)
+               for c in (C.TINY, SMALL_BF16, MED_BF16, WIDE_BF16)] + \
+              [c.replace(name=c.name + "_blocks", plan_mode=C.PLAN_BLOCKS) for c in EDGE if c.E * c.R <= 16384]
+
+
+@pytest.mark.parametrize("cfg", BLOCK_SMALL, ids=lambda c: c.name)
+def test_block_planner_small_layers(cfg):
+    check_full_small(cfg, 0)
+
+
+@pytest.mark.parametrize("cfg", [C.OLMOE, C.QWEN3, C.EXTREME, C.DSV3], ids=lambda c: c.name)
+def test_block_planner_full_size(cfg):
+    check_full_size(cfg.replace(name=cfg.name + "_blocks", plan_mode=C.PLAN_BLOCKS), 0, n_tokens=4, n_rows=16)
+    torch.cuda.empty_cache()
+
+
 FULL = [C.OLMOE, C.QWEN3, C.EXTREME, C.DSV3]
 
 
