@@ -44,7 +44,8 @@
 //
 // CTA = 7 warps: warp 0 issues TMA loads into a 6-stage ring of 32 KB stages
 // (128-byte swizzle), counted on the even CTA's "full" barrier; warp 6 of the
-// even CTA fetches and decodes work items; warp 1 of the
+// even CTA fetches and decodes work items, warp 6 of the odd CTA hands its
+// CTA's releases of item slots back to it; warp 1 of the
 // even CTA issues the pair MMAs into one of two 256-column accumulators and
 // commits to the "empty"/"full" barriers of both CTAs; warps 2-5 of each CTA
 // drain the other accumulator (tcgen05.ld), apply the epilogue and store bf16
@@ -72,10 +73,16 @@ constexpr int kBBytes = kHalfN * kBK * 2;      // 16 KB
 constexpr int kStageBytes = kABytes + kBBytes; // 32 KB
 constexpr long long kDrainBudget = 2000000000LL;
 constexpr int kItemSlots = 4;                  // ring of fetched, decoded work items (few: a short window keeps L2 reuse)
-// item-slot consumers: TMA thread, MMA thread and 4 epilogue warps of the even
-// CTA; TMA thread and 4 epilogue warps of the odd CTA
-constexpr uint32_t kItemConsumers = 11;
-constexpr int kSchedWarp = 6;
+// Releases of an item slot. Even CTA: its TMA thread, MMA thread and 4
+// epilogue warps arrive locally, and the odd CTA's forwarder arrives once for
+// its CTA; odd CTA: its TMA thread and 4 epilogue warps arrive locally on the
+// forwarder's barrier. Only the forwarder, which holds nothing in flight,
+// makes the cluster-scope release: that release waits for the releasing
+// thread's outstanding copies and MMAs, which costs the TMA and MMA threads
+// about a microsecond per item when they make it themselves.
+constexpr uint32_t kItemConsumers = 7;
+constexpr uint32_t kOddConsumers = 5;
+constexpr int kSchedWarp = 6;                  // scheduler (even CTA), forwarder (odd CTA)
 
 struct TcArgs {
     const int32_t* src_of;    // row -> token (gathered FC1 only)
@@ -96,7 +103,7 @@ struct TcArgs {
 
 struct Smem {
     uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
-    uint64_t item_full[kItemSlots], item_empty[kItemSlots];
+    uint64_t item_full[kItemSlots], item_empty[kItemSlots], fwd_empty[kItemSlots];
     int4 items[kItemSlots];   // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
     int32_t rows[kItemSlots][kBM];   // gathered FC1: token of each row of this CTA's block
     uint32_t tmem_base;
@@ -170,7 +177,10 @@ __device__ __forceinline__ void decode_item(long long it, int n_tiles, const int
     b1 = 2 * q + 1 < nb ? sched[s_off[lo] + 2 * q + 1] : -1;
 }
 
-__device__ __forceinline__ float silu(float a) { return a / (1.f + __expf(-a)); }
+// silu(a) = a / (1 + e^-a) with the fast reciprocal-based divide (the IEEE
+// divide's range checks made the FC1 epilogue slower than the main loop it
+// must hide behind); the result is rounded to bf16 right after.
+__device__ __forceinline__ float silu(float a) { return __fdividef(a, 1.f + __expf(-a)); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -198,6 +208,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         for (int q = 0; q < kItemSlots; ++q) {
             ptx::mbar_init(&S->item_full[q], 1);
             ptx::mbar_init(&S->item_empty[q], kItemConsumers);
+            ptx::mbar_init(&S->fwd_empty[q], kOddConsumers);
         }
         ptx::mbar_init(&S->drain, 1);
         S->abort_flag = 0;
@@ -239,16 +250,17 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     // the ring slot of the k-th item, and the parity of its phase
     auto slot_of = [](int k) { return k % kItemSlots; };
     auto parity_of = [](int k) { return (uint32_t)((k / kItemSlots) & 1); };
-    // take item k from the ring (both CTAs; the slot barriers of "empty" live in
-    // the even CTA). Returns false when the wait gave up.
+    // take item k from the ring (both CTAs; the odd CTA's copy is written by
+    // the even CTA's scheduler). Returns false when the wait gave up.
     auto take_item = [&](int k, int4& item) -> bool {
-        if (!role_wait_cluster(&S->item_full[slot_of(k)], parity_of(k), a.spin, abort_flag, a.header)) return false;
+        const bool ok = even ? role_wait(&S->item_full[slot_of(k)], parity_of(k), a.spin, abort_flag, a.header)
+                             : role_wait_cluster(&S->item_full[slot_of(k)], parity_of(k), a.spin, abort_flag, a.header);
+        if (!ok) return false;
         item = S->items[slot_of(k)];
         return true;
     };
-    auto release_item = [&](int k) {
-        ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_empty[slot_of(k)]), 0));
-    };
+    // a local arrive (release at CTA scope) on this CTA's "slot empty" barrier
+    auto release_item = [&](int k) { ptx::mbar_arrive(even ? &S->item_empty[slot_of(k)] : &S->fwd_empty[slot_of(k)]); };
 
     if (warp == kSchedWarp) {
         // ------------------------------------------------ scheduler (even CTA)
@@ -264,7 +276,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const int split = p_off[lo] * a.n_tiles;
             int next = lane == 0 ? fetch_item(a.queue, g, split, n_items) : 0;
             for (int k = 0;; ++k) {
-                const bool ok = role_wait(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
+                const bool ok = role_wait_cluster(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
                 int4 item = make_int4(-1, 0, -1, -1);
                 if (lane == 0 && ok && next >= 0) {
                     int e, b0, b1, j;
@@ -314,6 +326,16 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     __threadfence();
                     a.queue[2] = 0;
                 }
+            }
+        } else if (lane == 0) {
+            // forwarder (odd CTA): once this CTA's consumers have all released a
+            // slot, release it to the even CTA's scheduler at cluster scope
+            for (int k = 0;; ++k) {
+                int4 item;
+                if (!take_item(k, item)) break;
+                if (!role_wait(&S->fwd_empty[slot_of(k)], parity_of(k), a.spin, abort_flag, a.header)) break;
+                ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_empty[slot_of(k)]), 0));
+                if (item.x < 0) break;
             }
         }
     } else if (warp == 0) {
@@ -367,7 +389,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (item.x < 0) break;
                 const int acc = k & 1;
                 const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
-                if (!role_wait(&S->acc_empty[acc], acc_phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
+                if (!role_wait_cluster(&S->acc_empty[acc], acc_phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * kN);
                 for (int kb = 0; kb < kb_count; ++kb) {
@@ -454,7 +476,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             }
             ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->acc_empty[acc]), 0));
+            if (lane == 0) {
+                if (even) ptx::mbar_arrive(&S->acc_empty[acc]);
+                else ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->acc_empty[acc]), 0));
+            }
         }
     }
     ptx::tc_fence_before();
