@@ -167,9 +167,11 @@ moe_status moe_plan(const moe_config* cfg, const float* logits, int32_t* topk_id
                     int32_t* counts, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
- * moe_dispatch - step A6: xp[row] = x[src_of[row]] for every row below
- * the plan's total rows, zero for padding rows ([MegaFlux] §1: routed
- * activations go to the ranks that compute their experts).
+ * moe_dispatch - step A6: xp[row] = x[src_of[row]] for every valid row
+ * ([MegaFlux] §1: routed activations go to the ranks that compute their
+ * experts). Padding rows of xp are not written: moe_expert_ffn and
+ * moe_expert_fc1/fc2 store zero h and yp rows for them whatever xp holds
+ * there, so their contents never reach the output.
  *   x   [T, d] (device), xp [rows_cap, d] (device, out).
  */
 moe_status moe_dispatch(const moe_config* cfg, const void* x, void* xp, const void* ws,
@@ -183,8 +185,10 @@ moe_status moe_dispatch(const moe_config* cfg, const void* x, void* xp, const vo
  *   w_gate_up  [E, 2F, d] (device): rows 0..F-1 of expert e are the gate
  *              projection, rows F..2F-1 the up projection (K-major).
  *   w_down     [E, d, F] (device, K-major).
- *   h          [rows_cap, F] (device, out): silu(xp.gate) * (xp.up).
- *   yp         [rows_cap, d] (device, out): h . w_down.
+ *   h          [rows_cap, F] (device, out): silu(xp.gate) * (xp.up) on
+ *              valid rows, zero on padding rows.
+ *   yp         [rows_cap, d] (device, out): h . w_down on valid rows, zero
+ *              on padding rows.
  * fp32 accumulation; in bf16 mode h and yp are rounded to bf16 once.
  */
 moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const void* w_gate_up,
@@ -208,9 +212,7 @@ moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_do
  * (device) through the plan's row map, so no xp buffer is written or read
  * ([MegaFlux] §2.1: token movement overlapped with the tiled FC1 work).
  * h [rows_cap, F] (device, out) holds the same values as moe_dispatch +
- * moe_expert_fc1 on every valid row; padding rows hold unspecified values
- * (they repeat their block's first token) and are never read by
- * moe_combine. It needs no xp buffer (rows_cap * d elements less memory)
+ * moe_expert_fc1 on every row (padding rows zero). It needs no xp buffer (rows_cap * d elements less memory)
  * but runs FC1 at about half the speed of moe_expert_fc1: each 16 KB
  * activation tile takes 32 four-row gathers instead of one tile copy.
  * fp32 layers return MOE_ERR_UNSUPPORTED.

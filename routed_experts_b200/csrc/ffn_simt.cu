@@ -8,7 +8,8 @@
 // 10 mantissa bits), so they run here: each CTA takes (block, column tile)
 // work items of the planned block table, stages a BK-deep slice of the block's
 // rows and of the expert's weight rows in shared memory, and accumulates in
-// registers. h = silu(gate) * up with silu(a) = a / (1 + exp(-a)).
+// registers. h = silu(gate) * up with silu(a) = a / (1 + exp(-a)). Rows of
+// a block past its valid ones (padding) are stored as zero.
 #include <math.h>
 
 #include "common.cuh"
@@ -34,7 +35,7 @@ ffn_simt_kernel(const float* __restrict__ a_mat, const float* __restrict__ w, fl
     for (int64_t it = blockIdx.x; it < n_items; it += gridDim.x) {
         const int b = (int)(it / n_tiles), j = (int)(it % n_tiles);
         const int32_t* B = ws.blocks + (int64_t)kBlockInts * b;
-        const int e = B[0], row0 = B[1];
+        const int e = B[0], row0 = B[1], valid = B[2];
         const int n0 = j * kBN;
         float acc_g[MR], acc_u[MR];
 #pragma unroll
@@ -71,7 +72,7 @@ ffn_simt_kernel(const float* __restrict__ a_mat, const float* __restrict__ w, fl
             float v;
             if (MODE == 0) v = acc_g[i] / (1.f + expf(-acc_g[i])) * acc_u[i];
             else v = acc_g[i];
-            out[(int64_t)(row0 + m) * Nout + n0 + tx] = v;
+            out[(int64_t)(row0 + m) * Nout + n0 + tx] = m < valid ? v : 0.f;   // padding rows: zero
         }
     }
 }

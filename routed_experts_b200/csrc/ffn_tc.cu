@@ -21,13 +21,14 @@
 // plus the matching 128 up columns (odd CTA's half), so both halves of SwiGLU
 // sit side by side in each CTA's accumulator; FC2 tiles are 256 columns of d.
 // An expert with an odd number of blocks gives its last pair one block: the
-// odd CTA then reloads the even CTA's rows and stores nothing.
+// odd CTA then reloads the even CTA's rows and stores nothing. Rows of a
+// block past its valid ones (padding) are stored as zero, whatever the
+// activation rows held there.
 //
 // FC1 can also read its activation rows straight from x (dispatch fused into
 // FC1): each 128-row A tile is built by 32 four-row TMA gathers
 // (tile::gather4, one per lane of the TMA warp) of the token rows the plan's
-// row map names; padding rows repeat the block's first token and their h rows
-// are never read by the combine.
+// row map names; padding rows repeat the block's first token.
 //
 // Scheduling is dynamic. Items are listed expert-major (then column tile,
 // then block pair), so consecutive items share an expert's weight tiles and a
@@ -105,6 +106,7 @@ struct Smem {
     uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
     uint64_t item_full[kItemSlots], item_empty[kItemSlots], fwd_empty[kItemSlots];
     int4 items[kItemSlots];   // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
+    uint32_t valid[kItemSlots];   // valid rows of the even CTA's block (low 16 bits) and the odd CTA's (high)
     int32_t rows[kItemSlots][kBM];   // gathered FC1: token of each row of this CTA's block
     uint32_t tmem_base;
     int abort_flag;
@@ -278,10 +280,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             for (int k = 0;; ++k) {
                 const bool ok = role_wait_cluster(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
                 int4 item = make_int4(-1, 0, -1, -1);
+                uint32_t valid = 0;
                 if (lane == 0 && ok && next >= 0) {
                     int e, b0, b1, j;
                     decode_item(next, a.n_tiles, s_off, p_off, a.E, a.sched, e, b0, b1, j);
                     item = make_int4(e, j, a.blocks[kBlockInts * b0 + 1], b1 >= 0 ? a.blocks[kBlockInts * b1 + 1] : -1);
+                    valid = (uint32_t)a.blocks[kBlockInts * b0 + 2] |
+                            (b1 >= 0 ? (uint32_t)a.blocks[kBlockInts * b1 + 2] << 16 : 0u);
                 }
                 item.x = __shfl_sync(0xffffffffu, item.x, 0);
                 item.y = __shfl_sync(0xffffffffu, item.y, 0);
@@ -308,8 +313,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (lane == 0) {
                     // publish to both CTAs
                     S->items[slot_of(k)] = item;
+                    S->valid[slot_of(k)] = valid;
                     const uint32_t peer = ptx::map_to_rank(ptx::smem_addr(&S->items[slot_of(k)]), 1);
                     ptx::st_cluster_v4(peer, item);
+                    ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_addr(&S->valid[slot_of(k)]), 1), valid);
                     ptx::mbar_arrive(&S->item_full[slot_of(k)]);
                     ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_full[slot_of(k)]), 1));
                 }
@@ -427,10 +434,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         for (int k = 0;; ++k) {
             int4 item;
             if (!take_item(k, item)) break;
+            const uint32_t vv = S->valid[slot_of(k)];
             __syncwarp();
             if (lane == 0) release_item(k);
             if (item.x < 0) break;
             const int j = item.y;
+            // rows of the block past its valid ones are padding: written as zero
+            const bool pad = m >= (int)(even ? (vv & 0xffffu) : (vv >> 16));
             const int row0 = even ? item.z : item.w;   // -1: this CTA's half of the pair is empty
             const int acc = k & 1;
             const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
@@ -452,7 +462,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                         for (int i = 0; i < 16; ++i) {
                             const float h0 = silu(__uint_as_float(gt[2 * i])) * __uint_as_float(up[2 * i]);
                             const float h1 = silu(__uint_as_float(gt[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
-                            pk[i] = pack_bf16(h0, h1);
+                            pk[i] = pad ? 0u : pack_bf16(h0, h1);
                         }
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
@@ -467,7 +477,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                         uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
-                            pk[i] = pack_bf16(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
+                            pk[i] = pad ? 0u : pack_bf16(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
 #pragma unroll
                         for (int v = 0; v < 4; ++v)
                             orow[c / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);

@@ -17,8 +17,12 @@
 // from the planner. No slot is claimed with atomics.
 //
 // [MegaFlux] §1: routed activations travel to the ranks computing their
-// experts. On one GPU that is a copy of token rows: one warp per destination
-// row, 16-byte vector loads and stores, padding rows written as zero.
+// experts. On one GPU that is a copy of token rows, done as a scatter: one
+// warp per token reads its row of x once (16-byte vectors) and stores it to
+// the K rows the row map names, so x is read from memory once even when it
+// does not fit in L2. Padding rows of xp are not written: the FFN writes
+// zero h and yp rows for them whatever xp holds there, and nothing reads
+// them after that.
 #include "common.cuh"
 
 namespace moe {
@@ -93,32 +97,37 @@ constexpr int kGWarps = 8;
 constexpr int kUnroll = 8;
 
 __global__ void __launch_bounds__(kGWarps * 32)
-gather_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp, int nvec, WsPtrs ws) {
+dispatch_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp, int T, int K, int nvec, int64_t rows_cap,
+                WsPtrs ws) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int total = (int)ws.header[H_TOTAL_ROWS];
-    for (int row = blockIdx.x * kGWarps + warp; row < total; row += gridDim.x * kGWarps) {
-        const int s = ws.src_of[row];
-        uint4* dst = xp + (int64_t)row * nvec;
-        if (s >= 0) {
-            const uint4* src = x + (int64_t)s * nvec;
-            for (int v0 = 0; v0 < nvec; v0 += 32 * kUnroll) {
-                uint4 buf[kUnroll];
+    uint32_t bad = 0;
+    for (int t = blockIdx.x * kGWarps + warp; t < T; t += gridDim.x * kGWarps) {
+        int my_row = -1;
+        if (lane < K) {
+            my_row = ws.row_of[(int64_t)t * K + lane];
+            if (my_row < 0 || my_row >= rows_cap) { bad = 1; my_row = -1; }
+        }
+        const uint4* src = x + (int64_t)t * nvec;
+        for (int v0 = 0; v0 < nvec; v0 += 32 * kUnroll) {
+            uint4 buf[kUnroll];
 #pragma unroll
-                for (int u = 0; u < kUnroll; ++u) {
-                    const int v = v0 + u * 32 + lane;
-                    if (v < nvec) buf[u] = __ldg(src + v);
-                }
+            for (int u = 0; u < kUnroll; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec) buf[u] = __ldg(src + v);
+            }
+            for (int k = 0; k < K; ++k) {
+                const int row = __shfl_sync(0xffffffffu, my_row, k);
+                if (row < 0) continue;
+                uint4* dst = xp + (int64_t)row * nvec;
 #pragma unroll
                 for (int u = 0; u < kUnroll; ++u) {
                     const int v = v0 + u * 32 + lane;
                     if (v < nvec) dst[v] = buf[u];
                 }
             }
-        } else {
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            for (int v = lane; v < nvec; v += 32) dst[v] = z;
         }
     }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(ws.header, MOE_DEV_BAD_INDEX);
 }
 
 }  // namespace
@@ -140,11 +149,12 @@ cudaError_t launch_gather(const Shape& s, const void* x, void* xp, const WsPtrs&
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int nvec = (int)((int64_t)s.d * s.eb / 16);
-    int64_t want = (s.rows_cap + kGWarps - 1) / kGWarps;
+    int64_t want = (s.T + kGWarps - 1) / kGWarps;
     int64_t cap = (int64_t)sms * 8;
     const int grid = (int)(want < cap ? want : cap);
-    gather_kernel<<<grid, kGWarps * 32, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(xp),
-                                                nvec, ws);
+    if (grid == 0) return cudaSuccess;
+    dispatch_kernel<<<grid, kGWarps * 32, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(xp), s.T,
+                                                  s.K, nvec, s.rows_cap, ws);
     return cudaGetLastError();
 }
 
