@@ -112,8 +112,13 @@ struct Smem {
     int abort_flag;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + sizeof(Smem) +
+// epilogue staging: two 32 x 32 bf16 tiles (2 KB) per epilogue warp, each
+// written to global memory by one TMA store
+constexpr int kEpiBuf = 32 * 32 * 2;
+constexpr int kEpiBytes = 4 * 2 * kEpiBuf;
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + sizeof(Smem) +
                               2 * sizeof(int32_t) * (kMaxE + 1);
+static_assert(kSmemBytes <= 232448, "shared memory per CTA");
 
 __device__ __forceinline__ bool role_wait(uint64_t* bar, uint32_t parity, long long budget,
                                           volatile int* abort_flag, uint32_t* header) {
@@ -193,10 +198,12 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // MODE 2: FC1 + SwiGLU -> h with A gathered from x.
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, TcArgs a) {
+ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmO, TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    Smem* S = reinterpret_cast<Smem*>(base + kStages * kStageBytes);
+    uint8_t* epi_base = base + kStages * kStageBytes;
+    Smem* S = reinterpret_cast<Smem*>(epi_base + kEpiBytes);
     int32_t* s_off = reinterpret_cast<int32_t*>(S + 1);
     int32_t* p_off = s_off + (a.E + 1);
     volatile int* abort_flag = &S->abort_flag;
@@ -235,7 +242,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             carry += __shfl_sync(0xffffffffu, x, 31);
         }
     }
-    if (warp == 0 && lane == 0) { ptx::prefetch_tmap(&tmA); ptx::prefetch_tmap(&tmB); }
+    if (warp == 0 && lane == 0) { ptx::prefetch_tmap(&tmA); ptx::prefetch_tmap(&tmB); ptx::prefetch_tmap(&tmO); }
     __syncthreads();
     ptx::cluster_sync();   // the peer's barriers exist before any remote arrive, store or copy
     if (warp == 1) { ptx::tmem_alloc_pair(&S->tmem_base, kTmemCols); ptx::tmem_relinquish_pair(); }
@@ -431,6 +438,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         // ------------------------------------------------ epilogue, warps 2..5 of both CTAs
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
         const int m = quad * 32 + lane;            // row inside this CTA's block
+        uint8_t* stg = epi_base + quad * 2 * kEpiBuf;
+        int buf = 0;
         for (int k = 0;; ++k) {
             int4 item;
             if (!take_item(k, item)) break;
@@ -448,40 +457,42 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             ptx::tc_fence_after();
             if (row0 >= 0) {
                 const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN);
-                uint4* orow =
-                    reinterpret_cast<uint4*>(a.out + (int64_t)(row0 + m) * a.out_ld + (int64_t)j * kColTile);
-                if (kFC1) {
 #pragma unroll 1
-                    for (int c = 0; c < 128; c += 32) {
+                for (int c = 0; c < kColTile; c += 32) {
+                    uint32_t pk[16];
+                    if (kFC1) {
                         uint32_t gt[32], up[32];
                         ptx::tmem_ld32(t_row + c, gt);
                         ptx::tmem_ld32(t_row + 128 + c, up);
                         ptx::tmem_ld_wait();
-                        uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float h0 = silu(__uint_as_float(gt[2 * i])) * __uint_as_float(up[2 * i]);
                             const float h1 = silu(__uint_as_float(gt[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
                             pk[i] = pad ? 0u : pack_bf16(h0, h1);
                         }
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            orow[c / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                    }
-                } else {
-#pragma unroll 1
-                    for (int c = 0; c < 256; c += 32) {
+                    } else {
                         uint32_t y[32];
                         ptx::tmem_ld32(t_row + c, y);
                         ptx::tmem_ld_wait();
-                        uint32_t pk[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i)
                             pk[i] = pad ? 0u : pack_bf16(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
-#pragma unroll
-                        for (int v = 0; v < 4; ++v)
-                            orow[c / 8 + v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
                     }
+                    // this staging tile's previous store has finished reading it
+                    if (lane == 0) ptx::bulk_wait_group_read<1>();
+                    __syncwarp();
+                    uint8_t* tile = stg + buf * kEpiBuf;
+                    uint4* srow = reinterpret_cast<uint4*>(tile + lane * 64);   // row m: 32 bf16
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) srow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                    ptx::fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) {
+                        ptx::tma_store_2d(&tmO, tile, j * kColTile + c, row0 + quad * 32);
+                        ptx::bulk_commit_group();
+                    }
+                    buf ^= 1;
                 }
             }
             ptx::tc_fence_before();
@@ -491,6 +502,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 else ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->acc_empty[acc]), 0));
             }
         }
+        if (lane == 0) ptx::bulk_wait_group<0>();   // the stores are done before the CTA exits
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -543,13 +555,27 @@ bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t rows, 
     return r == CUDA_SUCCESS;
 }
 
+// The output (h or yp) as 32 x 32 tiles, unswizzled, for the epilogue's stores.
+bool make_tmap_out(CUtensorMap* tm, void* ptr, uint64_t cols, uint64_t rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {32, 32};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const TcArgs& a, int grid,
-                        cudaStream_t st) {
+cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const TcArgs& a,
+                        int grid, cudaStream_t st) {
     cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)kSmemBytes);
     if (err != cudaSuccess) return err;
-    ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, a);
+    ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, a);
     return cudaGetLastError();
 }
 
@@ -576,41 +602,44 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.queue = ws.gemm_q + (which == 2 ? 4 : 0);
     a.src_of = ws.src_of;
     a.out = static_cast<__nv_bfloat16*>(out);
-    CUtensorMap tA, tB;
+    CUtensorMap tA, tB, tO;
     if (which == 3) {
         // FC1 + SwiGLU with A gathered from x [T, d] by the row map -> h [rows_cap, F]
         if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.T, 1) ||
-            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN))
+            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
+            !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap))
             return cudaErrorInvalidValue;
         a.out_ld = s.F;
         a.Kdim = s.d;
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<2>(tA, tB, a, sms, st);
+        return launch_mode<2>(tA, tB, tO, a, sms, st);
     }
     if (which == 1) {
         // FC1 + SwiGLU: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h [rows_cap, F]
         if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
-            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN))
+            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
+            !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap))
             return cudaErrorInvalidValue;
         a.out_ld = s.F;
         a.Kdim = s.d;
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<0>(tA, tB, a, sms, st);
+        return launch_mode<0>(tA, tB, tO, a, sms, st);
     }
     // FC2: h [rows_cap, F] x w_down [E*d, F] -> yp [rows_cap, d]
     if (!make_tmap(&tA, a_mat, (uint64_t)s.F, (uint64_t)s.rows_cap, kBM) ||
-        !make_tmap(&tB, w, (uint64_t)s.F, (uint64_t)s.E * s.d, kHalfN))
+        !make_tmap(&tB, w, (uint64_t)s.F, (uint64_t)s.E * s.d, kHalfN) ||
+        !make_tmap_out(&tO, out, (uint64_t)s.d, (uint64_t)s.rows_cap))
         return cudaErrorInvalidValue;
     a.out_ld = s.d;
     a.Kdim = s.F;
     a.n_tiles = s.d / 256;
     a.F = 0;
     a.b_rows = s.d;
-    return launch_mode<1>(tA, tB, a, sms, st);
+    return launch_mode<1>(tA, tB, tO, a, sms, st);
 }
 
 }  // namespace moe
