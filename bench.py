@@ -374,7 +374,8 @@ def run_mine(args, world, rank, local):
     t_roof = max(layer_flop / (tensor_peak * 1e12), alg_bytes / (pk["hbm_gbs"] * 1e9))
     ms_per_step = elapsed_ms / args.steps
     value = world * T / (ms_per_step * 1e-3)
-    gather_bytes = T * d * eb + plan["total_rows"] * d * eb + 4 * plan["total_rows"]
+    # dispatch: x read once, N valid rows written, the row map read (padding rows are not written)
+    gather_bytes = T * d * eb + N * d * eb + 4 * N
     combine_bytes = N * d * eb + 8 * N + T * d * eb
     line = {
         "metric": METRIC,

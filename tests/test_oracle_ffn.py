@@ -117,6 +117,20 @@ def test_output_is_invariant_to_plan_parameters(orc):
         assert np.array_equal(r["out"], base["out"]), (R, tile, budget)
 
 
+def test_output_is_the_same_under_both_planners(orc):
+    """The exact-S*K greedy and the block-granular search place entries
+    differently ([MoonEP] "The greedy balance, step by step"; [MegaFlux] §3.1
+    "Bounded greedy search"), but every entry goes through the same arithmetic
+    wherever it lands, so the layer output must not change a bit."""
+    for cfg, seed in ((C.TINY, 2), (C.TINY.replace(dtype=C.BF16, tile=32, budget=2), 3)):
+        inp = _np_inputs(cfg, seed)
+        outs = [orc.layer(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"], K=cfg.K, R=cfg.R,
+                          tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype,
+                          plan_mode=mode) for mode in (orc.PLAN_EXACT, orc.PLAN_BLOCKS)]
+        assert outs[0]["plan"]["pieces"].tolist() != outs[1]["plan"]["pieces"].tolist(), "plans should differ"
+        assert np.array_equal(outs[0]["out"], outs[1]["out"])
+
+
 def test_combine_weights_select_rows(orc):
     yp = np.arange(12, dtype=np.float32).reshape(4, 3)
     row_of = np.array([2, 0, 3, 1], np.int32)
