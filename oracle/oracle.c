@@ -805,5 +805,205 @@ int orc_dense_layer(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32
     return ORC_OK;
 }
 
+/* ------------------------------------------------- backward (NEXT: training)
+ * [MegaFlux] §3.2 "Backward": DGrad runs through W2 then W1, WGrad forms
+ * each expert's weight gradients from the routed blocks, and replica
+ * partials of one expert are reduced into one gradient.
+ *
+ * Given dOut = dL/dout [T, d], for every routed entry (t, k) of expert e:
+ *   dY      = w[t,k] * dOut[t]                           (the combine's input gradient)
+ *   dw[t,k] = dOut[t] . y_(t,k)                         (the routing weight's gradient)
+ *   dH      = dY . W2_e            (DGrad through W2: sum over d)
+ *   dA      = dH * g * silu'(a),  dG = dH * silu(a)      (SwiGLU, silu' = s (1 + a (1 - s)), s = sigmoid(a))
+ *   dXp     = dA . W_gate_e + dG . W_up_e                (DGrad through W1: sum over F)
+ *   dx[t]   = sum over k, in k order, of dXp_(t,k)
+ *   dW2_e      += dY^T h,  dW_gate_e += dA^T x_t,  dW_up_e += dG^T x_t   (WGrad)
+ * and the router logits' gradient through the gating (zero off the top-k):
+ *   softmax over the chosen: dl[t, idx[t,m]] = w_m (dw_m - sum_k w_k dw_k)
+ *   sigmoid normalised:      dl[t, idx[t,m]] = w_m (1 - s_m) (dw_m - sum_k w_k dw_k), s_m = sigmoid(l).
+ * READING (rounding points, mirroring a bf16 GPU path; ORC_ROUND_NONE keeps
+ * everything in fp64): dY is the fp32 product w * dOut rounded to bf16; the
+ * pre-activations a and g are recomputed and rounded to bf16, and the
+ * SwiGLU derivative reads the rounded values; h and y are the forward's
+ * (rounded) values; dA, dG and dXp are rounded to bf16 once each; dx is
+ * rounded once after its k-ordered sum. Weight gradients, dw and the logits'
+ * gradient are returned in fp64 (the GPU path stores them as fp32).
+ * x, d_out, weights: arrays of `dtype`; logits and w: fp32.
+ */
+static double sigmoid_d(double v) { return 1.0 / (1.0 + exp(-v)); }
+
+typedef struct {
+    double *a, *g, *h, *y, *dy, *dh, *da, *dg, *dxp;
+} bwd_scratch;
+
+static int bwd_scratch_alloc(bwd_scratch* s, int32_t d, int32_t F)
+{
+    s->a = (double*)malloc(sizeof(double) * F);   s->g = (double*)malloc(sizeof(double) * F);
+    s->h = (double*)malloc(sizeof(double) * F);   s->y = (double*)malloc(sizeof(double) * d);
+    s->dy = (double*)malloc(sizeof(double) * d);  s->dh = (double*)malloc(sizeof(double) * F);
+    s->da = (double*)malloc(sizeof(double) * F);  s->dg = (double*)malloc(sizeof(double) * F);
+    s->dxp = (double*)malloc(sizeof(double) * d);
+    return s->a && s->g && s->h && s->y && s->dy && s->dh && s->da && s->dg && s->dxp;
+}
+
+static void bwd_scratch_free(bwd_scratch* s)
+{
+    free(s->a); free(s->g); free(s->h); free(s->y); free(s->dy); free(s->dh);
+    free(s->da); free(s->dg); free(s->dxp);
+}
+
+/* Every backward quantity of one routed entry (token t, expert e, weight wt).
+ * Returns dw for the entry. */
+static double bwd_entry(int32_t d, int32_t F, int32_t dtype, int32_t round_mode,
+                        const void* x, int64_t t, const void* w_gu, const void* w_down, int32_t e,
+                        float wt, const void* d_out, bwd_scratch* s)
+{
+    const int64_t gu_base = (int64_t)e * 2 * F * d;
+    const int64_t dn_base = (int64_t)e * d * F;
+    /* forward: pre-activations, h (from the unrounded pre-activations), y */
+    for (int32_t j = 0; j < F; ++j) {
+        double a = 0.0, g = 0.0;
+        for (int32_t i = 0; i < d; ++i) {
+            double xv = load_elem(x, t * d + i, dtype);
+            a += xv * load_elem(w_gu, gu_base + (int64_t)j * d + i, dtype);
+            g += xv * load_elem(w_gu, gu_base + (int64_t)(F + j) * d + i, dtype);
+        }
+        s->h[j] = round_as(a / (1.0 + exp(-a)) * g, round_mode);
+        s->a[j] = round_as(a, round_mode);
+        s->g[j] = round_as(g, round_mode);
+    }
+    double dw = 0.0;
+    for (int32_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int32_t j = 0; j < F; ++j) acc += s->h[j] * load_elem(w_down, dn_base + (int64_t)i * F + j, dtype);
+        s->y[i] = round_as(acc, round_mode);
+        const double go = load_elem(d_out, t * d + i, dtype);
+        dw += go * s->y[i];
+        /* dY: the product formed in fp32 before its bf16 rounding */
+        s->dy[i] = round_mode == ORC_ROUND_NONE ? (double)wt * go
+                                                : round_as((double)(float)((float)wt * (float)go), round_mode);
+    }
+    /* DGrad through W2, then the SwiGLU derivative */
+    for (int32_t j = 0; j < F; ++j) {
+        double acc = 0.0;
+        for (int32_t i = 0; i < d; ++i) acc += s->dy[i] * load_elem(w_down, dn_base + (int64_t)i * F + j, dtype);
+        s->dh[j] = acc;
+        const double a = s->a[j], sg = sigmoid_d(a);
+        s->da[j] = round_as(acc * s->g[j] * (sg * (1.0 + a * (1.0 - sg))), round_mode);
+        s->dg[j] = round_as(acc * (a * sg), round_mode);
+    }
+    /* DGrad through W1 */
+    for (int32_t i = 0; i < d; ++i) {
+        double acc = 0.0;
+        for (int32_t j = 0; j < F; ++j)
+            acc += s->da[j] * load_elem(w_gu, gu_base + (int64_t)j * d + i, dtype) +
+                   s->dg[j] * load_elem(w_gu, gu_base + (int64_t)(F + j) * d + i, dtype);
+        s->dxp[i] = round_as(acc, round_mode);
+    }
+    return dw;
+}
+
+/* The logits' gradient of one token from its routing weights' gradients. */
+static void bwd_gating(int32_t E, int32_t K, int32_t gating, const float* l, const int32_t* idx,
+                       const float* w, const double* dw, double* dl /*[E]*/)
+{
+    for (int32_t e = 0; e < E; ++e) dl[e] = 0.0;
+    double dot = 0.0;
+    for (int32_t k = 0; k < K; ++k) dot += (double)w[k] * dw[k];
+    for (int32_t m = 0; m < K; ++m) {
+        double v = (double)w[m] * (dw[m] - dot);
+        if (gating == ORC_GATE_SIGMOID_TOPK) v *= 1.0 - sigmoid_d((double)l[idx[m]]);
+        dl[idx[m]] = v;
+    }
+}
+
+int orc_layer_bwd(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32_t gating,
+                  int32_t dtype, int32_t round_mode,
+                  const float* logits, const int32_t* idx, const float* w,
+                  const void* x, const void* w_gu, const void* w_down, const void* d_out,
+                  void* dx /*[T,d] dtype*/, double* dw_gu /*[E,2F,d]*/, double* dw_down /*[E,d,F]*/,
+                  double* dw_topk /*[T,K]*/, double* dlogits /*[T,E]*/)
+{
+    bwd_scratch s;
+    double* dxs = (double*)malloc(sizeof(double) * (size_t)d);
+    if (!bwd_scratch_alloc(&s, d, F) || !dxs) { bwd_scratch_free(&s); free(dxs); return ORC_ERR_INTERNAL; }
+    memset(dw_gu, 0, sizeof(double) * (size_t)E * 2 * F * d);
+    memset(dw_down, 0, sizeof(double) * (size_t)E * d * F);
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t i = 0; i < d; ++i) dxs[i] = 0.0;
+        for (int32_t k = 0; k < K; ++k) {
+            const int32_t e = idx[t * K + k];
+            dw_topk[t * K + k] = bwd_entry(d, F, dtype, round_mode, x, t, w_gu, w_down, e, w[t * K + k],
+                                           d_out, &s);
+            for (int32_t i = 0; i < d; ++i) dxs[i] += s.dxp[i];
+            double* wd = dw_down + (int64_t)e * d * F;
+            for (int32_t i = 0; i < d; ++i)
+                for (int32_t j = 0; j < F; ++j) wd[(int64_t)i * F + j] += s.dy[i] * s.h[j];
+            double* wg = dw_gu + (int64_t)e * 2 * F * d;
+            for (int32_t j = 0; j < F; ++j)
+                for (int32_t i = 0; i < d; ++i) {
+                    const double xv = load_elem(x, t * d + i, dtype);
+                    wg[(int64_t)j * d + i] += s.da[j] * xv;
+                    wg[(int64_t)(F + j) * d + i] += s.dg[j] * xv;
+                }
+        }
+        for (int32_t i = 0; i < d; ++i) store_elem(dx, t * d + i, dtype, round_as(dxs[i], round_mode));
+        if (dlogits)
+            bwd_gating(E, K, gating, logits + t * E, idx + t * K, w + t * K, dw_topk + t * K, dlogits + t * E);
+    }
+    bwd_scratch_free(&s);
+    free(dxs);
+    return ORC_OK;
+}
+
+/* dx rows, dw and the logits' gradient of selected tokens (for large layers). */
+int orc_bwd_tokens(int32_t d, int32_t E, int32_t K, int32_t F, int32_t gating, int32_t dtype,
+                   int32_t round_mode, int64_t n_tok, const int64_t* tokens,
+                   const float* logits, const int32_t* idx, const float* w,
+                   const void* x, const void* w_gu, const void* w_down, const void* d_out,
+                   double* dx /*[n,d]*/, double* dw_topk /*[n,K]*/, double* dlogits /*[n,E]*/)
+{
+    bwd_scratch s;
+    if (!bwd_scratch_alloc(&s, d, F)) { bwd_scratch_free(&s); return ORC_ERR_INTERNAL; }
+    for (int64_t n = 0; n < n_tok; ++n) {
+        const int64_t t = tokens[n];
+        double* dxs = dx + n * d;
+        for (int32_t i = 0; i < d; ++i) dxs[i] = 0.0;
+        for (int32_t k = 0; k < K; ++k) {
+            dw_topk[n * K + k] = bwd_entry(d, F, dtype, round_mode, x, t, w_gu, w_down, idx[t * K + k],
+                                           w[t * K + k], d_out, &s);
+            for (int32_t i = 0; i < d; ++i) dxs[i] += s.dxp[i];
+        }
+        for (int32_t i = 0; i < d; ++i) dxs[i] = round_as(dxs[i], round_mode);
+        bwd_gating(E, K, gating, logits + t * E, idx + t * K, w + t * K, dw_topk + n * K, dlogits + n * E);
+    }
+    bwd_scratch_free(&s);
+    return ORC_OK;
+}
+
+/* Single elements of the weight gradients of one expert: which = 0 for
+ * dW_gate[e][r][c] and 1 for dW_up[e][r][c] (r < F, c < d), 2 for
+ * dW2[e][r][c] (r < d, c < F). Sums over every entry routed to e. */
+int orc_bwd_wgrad_elems(int64_t T, int32_t d, int32_t K, int32_t F, int32_t dtype, int32_t round_mode,
+                        const int32_t* idx, const float* w, const void* x, const void* w_gu,
+                        const void* w_down, const void* d_out, int32_t e, int64_t n,
+                        const int32_t* which, const int32_t* r, const int32_t* c, double* out)
+{
+    bwd_scratch s;
+    if (!bwd_scratch_alloc(&s, d, F)) { bwd_scratch_free(&s); return ORC_ERR_INTERNAL; }
+    for (int64_t q = 0; q < n; ++q) out[q] = 0.0;
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t k = 0; k < K; ++k) {
+            if (idx[t * K + k] != e) continue;
+            bwd_entry(d, F, dtype, round_mode, x, t, w_gu, w_down, e, w[t * K + k], d_out, &s);
+            for (int64_t q = 0; q < n; ++q) {
+                if (which[q] == 2) out[q] += s.dy[r[q]] * s.h[c[q]];
+                else out[q] += (which[q] == 0 ? s.da[r[q]] : s.dg[r[q]]) * load_elem(x, t * d + c[q], dtype);
+            }
+        }
+    bwd_scratch_free(&s);
+    return ORC_OK;
+}
+
 /* bf16 rounding exposed for pins of the rounding helper itself */
 uint16_t orc_double_to_bf16(double v) { return double_to_bf16(v); }

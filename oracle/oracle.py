@@ -60,6 +60,9 @@ def lib():
         L.orc_dense_layer.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P]
         L.orc_entry_ffn.argtypes = [i32, i32, i32, i32, i64, P, P, P, P, P, P, P]
         L.orc_double_to_bf16.argtypes = [ctypes.c_double]
+        L.orc_layer_bwd.argtypes = [i64, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.orc_bwd_tokens.argtypes = [i32, i32, i32, i32, i32, i32, i32, i64, P, P, P, P, P, P, P, P, P, P, P]
+        L.orc_bwd_wgrad_elems.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, i32, i64, P, P, P, P]
         L.orc_double_to_bf16.restype = ctypes.c_uint16
         for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_plan_blocks", "orc_row_maps", "orc_dispatch",
                   "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer", "orc_entry_ffn"):
@@ -240,6 +243,68 @@ def dense_layer(logits, x, w_gu, w_down, K: int, gating: int) -> np.ndarray:
     out = np.empty((T, d), np.float64)
     _check(lib().orc_dense_layer(T, d, E, K, F, gating, _p(logits), _p(x), _p(w_gu),
                                  _p(w_down), _p(out)), "dense_layer")
+    return out
+
+
+def layer_bwd(logits, idx, w, x, w_gu, w_down, d_out, *, gating: int, dtype: int, round_mode: int) -> dict:
+    """The backward of the routed layer for every token ([MegaFlux] §3.2
+    "Backward"): dx (dtype), weight gradients, routing-weight and logit
+    gradients (fp64)."""
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    x, w_gu, w_down, d_out = (np.ascontiguousarray(a) for a in (x, w_gu, w_down, d_out))
+    T, E = logits.shape
+    K = idx.shape[1]
+    d = x.shape[1]
+    F = w_down.shape[2]
+    dx = np.empty((T, d), _elem_dtype(dtype))
+    dw_gu = np.empty((E, 2 * F, d), np.float64)
+    dw_down = np.empty((E, d, F), np.float64)
+    dw = np.empty((T, K), np.float64)
+    dl = np.empty((T, E), np.float64)
+    _check(lib().orc_layer_bwd(T, d, E, K, F, gating, dtype, round_mode, _p(logits), _p(idx), _p(w), _p(x),
+                               _p(w_gu), _p(w_down), _p(d_out), _p(dx), _p(dw_gu), _p(dw_down), _p(dw),
+                               _p(dl)), "layer_bwd")
+    return {"dx": dx, "dw_gate_up": dw_gu, "dw_down": dw_down, "dw": dw, "dlogits": dl}
+
+
+def bwd_tokens(tokens, logits, idx, w, x, w_gu, w_down, d_out, *, gating: int, dtype: int, round_mode: int):
+    """dx rows (rounded values, fp64 array), dw and logit-gradient rows of selected tokens."""
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    x, w_gu, w_down, d_out = (np.ascontiguousarray(a) for a in (x, w_gu, w_down, d_out))
+    E = logits.shape[1]
+    K = idx.shape[1]
+    d = x.shape[1]
+    F = w_down.shape[2]
+    n = tokens.shape[0]
+    dx = np.empty((n, d), np.float64)
+    dw = np.empty((n, K), np.float64)
+    dl = np.empty((n, E), np.float64)
+    _check(lib().orc_bwd_tokens(d, E, K, F, gating, dtype, round_mode, n, _p(tokens), _p(logits), _p(idx),
+                                _p(w), _p(x), _p(w_gu), _p(w_down), _p(d_out), _p(dx), _p(dw), _p(dl)),
+           "bwd_tokens")
+    return dx, dw, dl
+
+
+def bwd_wgrad_elems(e: int, which, r, c, idx, w, x, w_gu, w_down, d_out, *, dtype: int, round_mode: int):
+    """Single weight-gradient elements of expert e (which: 0 gate [f][i], 1 up [f][i], 2 down [i][f])."""
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    x, w_gu, w_down, d_out = (np.ascontiguousarray(a) for a in (x, w_gu, w_down, d_out))
+    which = np.ascontiguousarray(which, dtype=np.int32)
+    r = np.ascontiguousarray(r, dtype=np.int32)
+    c = np.ascontiguousarray(c, dtype=np.int32)
+    T, K = idx.shape
+    d = x.shape[1]
+    F = w_down.shape[2]
+    out = np.empty(which.shape[0], np.float64)
+    _check(lib().orc_bwd_wgrad_elems(T, d, K, F, dtype, round_mode, _p(idx), _p(w), _p(x), _p(w_gu),
+                                     _p(w_down), _p(d_out), e, which.shape[0], _p(which), _p(r), _p(c),
+                                     _p(out)), "bwd_wgrad_elems")
     return out
 
 
