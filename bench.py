@@ -50,6 +50,7 @@ def parse():
     p.add_argument("--impl", default="mine", choices=["mine", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-tokens", type=int, default=320, help="tokens of the oracle's FFN sample")
+    p.add_argument("--no-backward", action="store_true", help="skip timing the layer's backward")
     return p.parse_args()
 
 
@@ -254,6 +255,57 @@ def cpu_baseline(cfg, inp, n_tokens):
             "measured_s": r["measured_s"]}
 
 
+def time_backward(cfg, inp, args, world, dev, stream, pg):
+    """moe_layer_bwd after one forward on a training workspace: W untimed and
+    K timed backward passes (CUDA events on the launching stream), max over
+    ranks. The forward state does not change between passes."""
+    from routed_experts_b200 import moe as M
+    lg, x, wgu, wdn = inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"]
+    layer = M.Layer(cfg, dev, train=True)
+    layer.forward(lg, x, wgu, wdn, stream=stream)
+    d_out = I.make_grad_out(cfg, args.seed, dev)
+    T, d, E, F = cfg.T, cfg.d, cfg.E, cfg.F
+    dx = torch.empty(T, d, dtype=M.act_dtype(cfg), device=dev)
+    dwgu = torch.empty(E, 2 * F, d, dtype=torch.float32, device=dev)
+    dwdn = torch.empty(E, d, F, dtype=torch.float32, device=dev)
+    dl = torch.empty(T, E, dtype=torch.float32, device=dev)
+
+    def bwd():
+        M.moe_layer_bwd(cfg, lg, wgu, wdn, d_out, dx, dwgu, dwdn, dl, layer.ws, stream)
+
+    for _ in range(args.warmup):
+        bwd()
+    st = M.moe_read_status(layer.ws, stream)
+    if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
+        raise RuntimeError(f"device status {st} after the backward warm-up")
+    if pg is not None:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    b0 = torch.cuda.Event(enable_timing=True)
+    b1 = torch.cuda.Event(enable_timing=True)
+    b0.record(stream)
+    for _ in range(args.steps):
+        bwd()
+    b1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = b0.elapsed_time(b1)
+    if pg is not None:
+        ms = max_over_ranks([ms], dev)[0]
+    ms /= args.steps
+    N = cfg.N
+    alg = 12.0 * N * d * F        # DGrad W2 2NdF + WGrad W2 2NdF + DGrad W1 4NdF + WGrad W1 4NdF
+    executed = alg + 4.0 * N * d * F   # + FC1 recomputed for the pre-activations
+    pk, _ = peaks()
+    del layer, dwgu, dwdn
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tokens_per_s": world * T / (ms * 1e-3),
+            "tflops": alg / (ms * 1e-3) / 1e12, "frac": alg / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+            "flop_algorithmic": alg, "flop_executed": executed,
+            "note": "moe_layer_bwd: dY and dw, FC1 pre-activations recomputed, DGrad W2 with the SwiGLU "
+                    "derivative, WGrad W2, DGrad W1, WGrad W1, dx, logits' gradient (9 launches); frac of "
+                    "the measured bf16 peak counts algorithmic FLOP only"}
+
+
 def run_mine(args, world, rank, local):
     from routed_experts_b200 import moe as M
     cfg = C.NAMED[args.config]
@@ -345,6 +397,12 @@ def run_mine(args, world, rank, local):
         torch.distributed.barrier()
         elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dev)
 
+    bwd = None
+    if not args.no_backward and cfg.dtype == C.BF16 and cfg.F % 256 == 0:
+        del layer_h
+        torch.cuda.empty_cache()
+        bwd = time_backward(cfg, inp, args, world, dev, stream, pg)
+
     plans = plan_comparison(cfg, lg, dev) if rank == 0 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -416,6 +474,7 @@ def run_mine(args, world, rank, local):
                 "ms_per_step": e2e_ms / args.steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "layer_path": "moe_plan; moe_dispatch; moe_expert_fc1; moe_expert_fc2; moe_combine (the kernels of moe_layer_fwd)",
+        "backward": bwd,
         "clocks": clk.summary(),
     }
     if cpu is not None:

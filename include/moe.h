@@ -85,8 +85,11 @@ typedef enum { MOE_PLAN_EXACT = 0, MOE_PLAN_BLOCKS = 1 } moe_plan_mode;
 typedef enum {
     MOE_WS_PLAN = 0,       /* plan, row maps and scratch: moe_plan .. moe_combine */
     MOE_WS_LAYER = 1,      /* MOE_WS_PLAN plus top-k, xp, h and yp: moe_layer_fwd */
-    MOE_WS_LAYER_HOST = 2  /* MOE_WS_LAYER plus device copies of logits, x and out:
+    MOE_WS_LAYER_HOST = 2, /* MOE_WS_LAYER plus device copies of logits, x and out:
                               moe_layer_fwd_host */
+    MOE_WS_LAYER_TRAIN = 3 /* MOE_WS_LAYER_HOST plus the backward's buffers (dY, the
+                              pre-activations, dA | dG, dw): moe_layer_fwd then
+                              moe_layer_bwd */
 } moe_ws_kind;
 
 /*
@@ -250,6 +253,33 @@ moe_status moe_layer_fwd(const moe_config* cfg, const float* logits, const void*
 moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, const void* x_host,
                               const void* w_gate_up, const void* w_down, void* out_host,
                               void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_layer_bwd - the layer's backward on one GPU ([MegaFlux] §3.2
+ * "Backward": DGrad through W2 then W1, WGrad per expert with the partial
+ * gradients of an expert's replicas reduced into one). bf16 layers with
+ * F % 256 == 0; others return MOE_ERR_UNSUPPORTED.
+ *   ws         a MOE_WS_LAYER_TRAIN workspace on which moe_layer_fwd last ran
+ *              with the same logits, x and weights (its top-k, plan, xp, h
+ *              and yp are read; xp's padding rows are zeroed).
+ *   logits     fp32 [T, E] (device), as given to moe_layer_fwd.
+ *   w_gate_up  [E, 2F, d], w_down [E, d, F] (device), as given to moe_layer_fwd.
+ *   d_out      [T, d] (device): the gradient of the loss with respect to out.
+ *   dx         [T, d] (device, out): sum over k, in k order, of each entry's
+ *              input gradient, in fp32, rounded once.
+ *   dw_gate_up fp32 [E, 2F, d], dw_down fp32 [E, d, F] (device, out): every
+ *              expert's weight gradients, zero for an expert no token chose.
+ *   dlogits    fp32 [T, E] (device, out) or NULL: the gradient through the
+ *              gating (softmax or sigmoid over the chosen logits); zero off
+ *              each token's top-k (selection itself has no gradient).
+ * Rounding points: each entry's dY = w * dOut is formed in fp32 and rounded
+ * to bf16; FC1's pre-activations are recomputed and rounded to bf16;
+ * dA | dG and each entry's dx row are rounded to bf16 once each; products
+ * accumulate in fp32. Asynchronous on `stream`; 9 kernel launches.
+ */
+moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void* w_gate_up, const void* w_down,
+                         const void* d_out, void* dx, float* dw_gate_up, float* dw_down, float* dlogits, void* ws,
+                         size_t ws_bytes, moe_stream_t stream);
 
 /*
  * moe_plan_noalloc - moe_plan for callers that cannot allocate device

@@ -821,6 +821,9 @@ int orc_dense_layer(int64_t T, int32_t d, int32_t E, int32_t K, int32_t F, int32
  * and the router logits' gradient through the gating (zero off the top-k):
  *   softmax over the chosen: dl[t, idx[t,m]] = w_m (dw_m - sum_k w_k dw_k)
  *   sigmoid normalised:      dl[t, idx[t,m]] = w_m (1 - s_m) (dw_m - sum_k w_k dw_k), s_m = sigmoid(l).
+ * READING: the weights of both gatings sum to one, so the inner term is
+ * taken as sum_k w_k (dw_m - dw_k): the same value, without the cancellation
+ * that the first form suffers when one weight is close to one.
  * READING (rounding points, mirroring a bf16 GPU path; ORC_ROUND_NONE keeps
  * everything in fp64): dY is the fp32 product w * dOut rounded to bf16; the
  * pre-activations a and g are recomputed and rounded to bf16, and the
@@ -908,10 +911,10 @@ static void bwd_gating(int32_t E, int32_t K, int32_t gating, const float* l, con
                        const float* w, const double* dw, double* dl /*[E]*/)
 {
     for (int32_t e = 0; e < E; ++e) dl[e] = 0.0;
-    double dot = 0.0;
-    for (int32_t k = 0; k < K; ++k) dot += (double)w[k] * dw[k];
     for (int32_t m = 0; m < K; ++m) {
-        double v = (double)w[m] * (dw[m] - dot);
+        double inner = 0.0;
+        for (int32_t k = 0; k < K; ++k) inner += (double)w[k] * (dw[m] - dw[k]);
+        double v = (double)w[m] * inner;
         if (gating == ORC_GATE_SIGMOID_TOPK) v *= 1.0 - sigmoid_d((double)l[idx[m]]);
         dl[idx[m]] = v;
     }

@@ -79,6 +79,11 @@ WsLayout make_layout(const Shape& s) {
     L.x_dev = take((int64_t)s.eb * s.T * s.d);
     L.out_dev = take((int64_t)s.eb * s.T * s.d);
     L.host_end = o;
+    L.dy = take((int64_t)s.eb * s.rows_cap * s.d);
+    L.ag = take((int64_t)s.eb * s.rows_cap * 2 * s.F);
+    L.dag = take((int64_t)s.eb * s.rows_cap * 2 * s.F);
+    L.dw = take(sizeof(float) * s.N);
+    L.train_end = o;
     return L;
 }
 
@@ -132,6 +137,7 @@ moe_status moe_workspace_size(const moe_config* cfg, int32_t kind, size_t* bytes
         case MOE_WS_PLAN: *bytes = (size_t)L.plan_end; return MOE_OK;
         case MOE_WS_LAYER: *bytes = (size_t)L.layer_end; return MOE_OK;
         case MOE_WS_LAYER_HOST: *bytes = (size_t)L.host_end; return MOE_OK;
+        case MOE_WS_LAYER_TRAIN: *bytes = (size_t)L.train_end; return MOE_OK;
         default: return MOE_ERR_INVALID_ARG;
     }
 }
@@ -299,6 +305,43 @@ moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, c
     if ((r = moe_layer_fwd(cfg, lg, x, w_gate_up, w_down, out, ws, ws_bytes, stream)) != MOE_OK) return r;
     if (cudaMemcpyAsync(out_host, out, x_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
+}
+
+moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void* w_gate_up, const void* w_down,
+                         const void* d_out, void* dx, float* dw_gate_up, float* dw_down, float* dlogits, void* ws,
+                         size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (s.dtype != MOE_BF16 || s.F % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    if (!logits || !w_gate_up || !w_down || !d_out || !dx || !dw_gate_up || !dw_down) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(d_out) || !aligned16(dx) ||
+        !aligned16(dw_gate_up) || !aligned16(dw_down) || (dlogits && !aligned16(dlogits)))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.train_end)) != MOE_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    const int32_t* idx = reinterpret_cast<const int32_t*>(b + L.idx);
+    const float* w = reinterpret_cast<const float*>(b + L.w);
+    void* xp = b + L.xp;
+    const void* h = b + L.h;
+    const void* yp = b + L.yp;
+    void* dy = b + L.dy;   // dY, then dXp once WGrad of W2 has read dY
+    void* ag = b + L.ag;
+    void* dag = b + L.dag;
+    float* dw = reinterpret_cast<float*>(b + L.dw);
+    const WsPtrs P = ws_ptrs(ws, L);
+    cudaError_t e = launch_bwd_scatter(s, d_out, yp, w, dy, dw, P, st);
+    if (e == cudaSuccess) e = launch_zero_padding(s, xp, dy, (int64_t)s.eb * s.d, P, st);
+    if (e == cudaSuccess) e = launch_ffn_tc(s, 4, xp, w_gate_up, ag, P, st, kSpinBudget);
+    if (e == cudaSuccess) e = launch_bwd_tc(s, 0, dy, w_down, dag, ag, P, st, kSpinBudget);
+    if (e == cudaSuccess) e = launch_bwd_tc(s, 2, dy, h, dw_down, nullptr, P, st, kSpinBudget);
+    if (e == cudaSuccess) e = launch_bwd_tc(s, 1, dag, w_gate_up, dy, nullptr, P, st, kSpinBudget);
+    if (e == cudaSuccess) e = launch_bwd_tc(s, 3, dag, xp, dw_gate_up, nullptr, P, st, kSpinBudget);
+    if (e == cudaSuccess) e = launch_combine(s, dy, nullptr, dx, P, st);
+    if (e == cudaSuccess && dlogits) e = launch_dlogits(s, logits, idx, w, dw, dlogits, st);
+    return from_cuda(e);
 }
 
 moe_status moe_read_status(const void* ws, moe_stream_t stream, uint32_t* dev_bits) {

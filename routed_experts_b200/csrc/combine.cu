@@ -27,7 +27,7 @@ combine_kernel(const uint4* __restrict__ yp, const float* __restrict__ w, uint4*
         float my_w = 0.f;
         if (lane < K) {
             my_row = ws.row_of[(int64_t)t * K + lane];
-            my_w = w[(int64_t)t * K + lane];
+            my_w = w ? w[(int64_t)t * K + lane] : 1.f;   // no weights: a plain sum (the backward's dx)
             if (my_row < 0 || my_row >= rows_cap) { bad = 1; my_row = 0; my_w = 0.f; }
         }
         int rows[KMAX];

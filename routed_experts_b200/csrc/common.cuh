@@ -50,6 +50,9 @@ struct WsLayout {
     // MOE_WS_LAYER_HOST extras
     int64_t logits_dev, x_dev, out_dev;
     int64_t host_end;
+    // MOE_WS_LAYER_TRAIN extras: dY (later dXp), the pre-activations, dA | dG, dw
+    int64_t dy, ag, dag, dw;
+    int64_t train_end;
 };
 
 __host__ __device__ inline int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
@@ -118,11 +121,23 @@ cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void*
                            const WsPtrs& ws, cudaStream_t st);
 // which = 1: FC1 + SwiGLU (a_mat = xp, w = w_gate_up, out = h);
 // which = 2: FC2 (a_mat = h, w = w_down, out = yp);
-// which = 3 (tensor cores only): FC1 + SwiGLU with a_mat = x, rows gathered by the row map.
+// which = 3 (tensor cores only): FC1 + SwiGLU with a_mat = x, rows gathered by the row map;
+// which = 4 (tensor cores only): FC1 pre-activations [gate | up] (a_mat = xp, out [rows_cap, 2F]).
 cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                             const WsPtrs& ws, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget);
+// backward (bf16): mode 0 DGrad W2 + SwiGLU derivative (a_mat = dY, b_mat = w_down, ag, out = dAG),
+// 1 DGrad W1 (a_mat = dAG, b_mat = w_gate_up, out = dXp), 2 WGrad W2 (a_mat = dY, b_mat = h,
+// out = dW2 fp32), 3 WGrad W1 (a_mat = dAG, b_mat = xp, out = dW1 fp32)
+cudaError_t launch_bwd_tc(const Shape& s, int mode, const void* a_mat, const void* b_mat, void* out,
+                          const void* ag, const WsPtrs& ws, cudaStream_t st, long long spin_budget);
+cudaError_t launch_bwd_scatter(const Shape& s, const void* d_out, const void* yp, const float* w, void* dy,
+                               float* dw, const WsPtrs& ws, cudaStream_t st);
+cudaError_t launch_zero_padding(const Shape& s, void* a, void* b, int64_t row_bytes, const WsPtrs& ws,
+                                cudaStream_t st);
+cudaError_t launch_dlogits(const Shape& s, const float* logits, const int32_t* idx, const float* w, const float* dw,
+                           float* dl, cudaStream_t st);
 
 }  // namespace moe

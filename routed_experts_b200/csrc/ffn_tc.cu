@@ -61,29 +61,12 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "tc_common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kBM = 128, kBK = 64, kStages = 6, kThreads = 224;
-constexpr int kN = 256;                        // accumulator columns per item (pair MMA N)
-constexpr int kHalfN = 128;                    // weight rows each CTA of the pair holds
-constexpr uint32_t kTmemCols = 2 * kN;         // two accumulators
-constexpr int kABytes = kBM * kBK * 2;         // 16 KB
-constexpr int kBBytes = kHalfN * kBK * 2;      // 16 KB
-constexpr int kStageBytes = kABytes + kBBytes; // 32 KB
-constexpr long long kDrainBudget = 2000000000LL;
-constexpr int kItemSlots = 4;                  // ring of fetched, decoded work items (few: a short window keeps L2 reuse)
-// Releases of an item slot. Even CTA: its TMA thread, MMA thread and 4
-// epilogue warps arrive locally, and the odd CTA's forwarder arrives once for
-// its CTA; odd CTA: its TMA thread and 4 epilogue warps arrive locally on the
-// forwarder's barrier. Only the forwarder, which holds nothing in flight,
-// makes the cluster-scope release: that release waits for the releasing
-// thread's outstanding copies and MMAs, which costs the TMA and MMA threads
-// about a microsecond per item when they make it themselves.
-constexpr uint32_t kItemConsumers = 7;
-constexpr uint32_t kOddConsumers = 5;
-constexpr int kSchedWarp = 6;                  // scheduler (even CTA), forwarder (odd CTA)
+using namespace tc;
 
 struct TcArgs {
     const int32_t* src_of;    // row -> token (gathered FC1 only)
@@ -102,100 +85,10 @@ struct TcArgs {
     int32_t* queue;           // [3]: head of queue 0, head of queue 1, clusters finished
 };
 
-struct Smem {
-    uint64_t full[kStages], empty[kStages], acc_full[2], acc_empty[2], drain;
-    uint64_t item_full[kItemSlots], item_empty[kItemSlots], fwd_empty[kItemSlots];
-    int4 items[kItemSlots];   // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
-    uint32_t valid[kItemSlots];   // valid rows of the even CTA's block (low 16 bits) and the odd CTA's (high)
-    int32_t rows[kItemSlots][kBM];   // gathered FC1: token of each row of this CTA's block
-    uint32_t tmem_base;
-    int abort_flag;
-};
-
-// epilogue staging: two 32 x 32 bf16 tiles (2 KB) per epilogue warp, each
-// written to global memory by one TMA store
-constexpr int kEpiBuf = 32 * 32 * 2;
-constexpr int kEpiBytes = 4 * 2 * kEpiBuf;
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + kStages * kStageBytes + kEpiBytes + sizeof(Smem) +
-                              2 * sizeof(int32_t) * (kMaxE + 1);
-static_assert(kSmemBytes <= 232448, "shared memory per CTA");
-
-__device__ __forceinline__ bool role_wait(uint64_t* bar, uint32_t parity, long long budget,
-                                          volatile int* abort_flag, uint32_t* header) {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
-    const long long t0 = clock64();
-    for (;;) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > budget) {
-            *abort_flag = 1;
-            atomicOr(header + H_STATUS, (uint32_t)MOE_DEV_TIMEOUT);
-            return false;
-        }
-    }
-}
-
-// As role_wait, acquiring at cluster scope (the item ring of the odd CTA is
-// written by the even CTA).
-__device__ __forceinline__ bool role_wait_cluster(uint64_t* bar, uint32_t parity, long long budget,
-                                                  volatile int* abort_flag, uint32_t* header) {
-    if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
-    const long long t0 = clock64();
-    for (;;) {
-        if (ptx::mbar_try_wait_cluster(bar, parity)) return true;
-        if (*abort_flag) return false;
-        if (clock64() - t0 > budget) {
-            *abort_flag = 1;
-            atomicOr(header + H_STATUS, (uint32_t)MOE_DEV_TIMEOUT);
-            return false;
-        }
-    }
-}
-
-// Next work item for a cluster of group g (0 or 1), or -1 when none is left:
-// its own half of the list first, then the other half.
-__device__ __forceinline__ int fetch_item(int32_t* queue, int g, int split, int n_items) {
-    const int lo = g ? split : 0, hi = g ? n_items : split;
-    const int i = atomicAdd(&queue[g], 1);
-    if (lo + i < hi) return lo + i;
-    const int lo2 = g ? 0 : split, hi2 = g ? split : n_items;
-    const int i2 = atomicAdd(&queue[1 - g], 1);
-    if (lo2 + i2 < hi2) return lo2 + i2;
-    return -1;
-}
-
-// Work item -> (expert, its two blocks, column tile). Expert e owns items
-// [n_tiles*p_off[e], n_tiles*p_off[e+1]), column tile major, then its block
-// pairs in schedule order; b1 = -1 when the pair has one block.
-__device__ __forceinline__ void decode_item(long long it, int n_tiles, const int32_t* s_off, const int32_t* p_off,
-                                            int E, const int32_t* sched, int& e, int& b0, int& b1, int& j) {
-    int lo = 0, hi = E;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if ((long long)n_tiles * p_off[mid] <= it) lo = mid; else hi = mid;
-    }
-    const int np = p_off[lo + 1] - p_off[lo];
-    const int nb = s_off[lo + 1] - s_off[lo];
-    const long long local = it - (long long)n_tiles * p_off[lo];
-    j = (int)(local / np);
-    const int q = (int)(local % np);
-    e = lo;
-    b0 = sched[s_off[lo] + 2 * q];
-    b1 = 2 * q + 1 < nb ? sched[s_off[lo] + 2 * q + 1] : -1;
-}
-
-// silu(a) = a / (1 + e^-a) with the fast reciprocal-based divide (the IEEE
-// divide's range checks made the FC1 epilogue slower than the main loop it
-// must hide behind); the result is rounded to bf16 right after.
-__device__ __forceinline__ float silu(float a) { return __fdividef(a, 1.f + __expf(-a)); }
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
 // MODE 0: FC1 + SwiGLU -> h (A = xp); MODE 1: FC2 -> yp (A = h);
-// MODE 2: FC1 + SwiGLU -> h with A gathered from x.
+// MODE 2: FC1 + SwiGLU -> h with A gathered from x;
+// MODE 3: FC1 pre-activations -> [gate | up] (A = xp), rounded to bf16, for
+// the backward's SwiGLU derivative.
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -254,6 +147,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const int kb_count = a.Kdim / kBK;
     constexpr bool kFC1 = MODE != 1;
     constexpr bool kGather = MODE == 2;
+    constexpr bool kPreact = MODE == 3;
     constexpr int kColTile = kFC1 ? 128 : 256;
 
     // the ring slot of the k-th item, and the parity of its phase
@@ -460,6 +354,36 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 #pragma unroll 1
                 for (int c = 0; c < kColTile; c += 32) {
                     uint32_t pk[16];
+                    if (kPreact) {
+                        uint32_t gt[32], up[32];
+                        ptx::tmem_ld32(t_row + c, gt);
+                        ptx::tmem_ld32(t_row + 128 + c, up);
+                        ptx::tmem_ld_wait();
+                        uint32_t pu[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            pk[i] = pad ? 0u : pack_bf16(__uint_as_float(gt[2 * i]), __uint_as_float(gt[2 * i + 1]));
+                            pu[i] = pad ? 0u : pack_bf16(__uint_as_float(up[2 * i]), __uint_as_float(up[2 * i + 1]));
+                        }
+                        // both staging tiles: gate at column j*128 + c, up at F + j*128 + c
+                        if (lane == 0) ptx::bulk_wait_group_read<0>();
+                        __syncwarp();
+                        uint4* sg = reinterpret_cast<uint4*>(stg + lane * 64);
+                        uint4* su = reinterpret_cast<uint4*>(stg + kEpiBuf + lane * 64);
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            sg[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+                            su[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+                        }
+                        ptx::fence_proxy_async_shared();
+                        __syncwarp();
+                        if (lane == 0) {
+                            ptx::tma_store_2d(&tmO, stg, j * kColTile + c, row0 + quad * 32);
+                            ptx::tma_store_2d(&tmO, stg + kEpiBuf, a.F + j * kColTile + c, row0 + quad * 32);
+                            ptx::bulk_commit_group();
+                        }
+                        continue;
+                    }
                     if (kFC1) {
                         uint32_t gt[32], up[32];
                         ptx::tmem_ld32(t_row + c, gt);
@@ -528,47 +452,6 @@ __global__ void bounded_wait_probe_kernel(uint32_t* status, long long budget) {
     if (threadIdx.x == 0) role_wait(&never, 0, budget, &abort_flag, status);
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    });
-    return fn;
-}
-
-// 2D bf16 tensor map of a row-major [rows, inner] matrix, box [box_rows, 64].
-bool make_tmap(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner * 2};
-    cuuint32_t box[2] = {(cuuint32_t)kBK, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-// The output (h or yp) as 32 x 32 tiles, unswizzled, for the epilogue's stores.
-bool make_tmap_out(CUtensorMap* tm, void* ptr, uint64_t cols, uint64_t rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * 2};
-    cuuint32_t box[2] = {32, 32};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ptr, dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                    CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const TcArgs& a,
                         int grid, cudaStream_t st) {
@@ -615,6 +498,19 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
         a.F = s.F;
         a.b_rows = 2 * s.F;
         return launch_mode<2>(tA, tB, tO, a, sms, st);
+    }
+    if (which == 4) {
+        // FC1 pre-activations: xp [rows_cap, d] x w_gate_up [E*2F, d] -> [gate | up] [rows_cap, 2F]
+        if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
+            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
+            !make_tmap_out(&tO, out, (uint64_t)2 * s.F, (uint64_t)s.rows_cap))
+            return cudaErrorInvalidValue;
+        a.out_ld = 2 * s.F;
+        a.Kdim = s.d;
+        a.n_tiles = s.F / 128;
+        a.F = s.F;
+        a.b_rows = 2 * s.F;
+        return launch_mode<3>(tA, tB, tO, a, sms, st);
     }
     if (which == 1) {
         // FC1 + SwiGLU: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h [rows_cap, F]

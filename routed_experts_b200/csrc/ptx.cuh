@@ -304,6 +304,20 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
     return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major operand tile in 128-byte
+// swizzle: the tile is cut into slabs of 64 elements (128 bytes) along M or
+// N, `slab_bytes` apart; a slab holds its K rows of 128 bytes, 8-row groups
+// 1024 bytes apart. Advancing K by 16 moves the start by 16 rows (2048 B).
+__device__ __forceinline__ uint64_t sdesc_mn_sw128(uint32_t saddr, uint32_t slab_bytes) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFF) >> 4);   // start address, 16-byte units
+    d |= (uint64_t)(slab_bytes >> 4) << 16;    // leading byte offset: next 64-element slab along M/N
+    d |= (uint64_t)(1024 >> 4) << 32;          // stride byte offset: next group of 8 K rows
+    d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;                    // 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor, kind::f16: bf16 A and B (both K-major), fp32 D,
 // M x N tile.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
@@ -312,6 +326,11 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            | (1u << 10)                        // B format: bf16
            | ((uint32_t)(N >> 3) << 17)        // N / 8
            | ((uint32_t)(M >> 4) << 24);       // M / 16
+}
+
+// As idesc_bf16_f32, with A and/or B stored MN-major (M or N contiguous).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
 }
 
 }  // namespace ptx

@@ -52,7 +52,7 @@ _M1 = 0xBF58476D1CE4E5B9
 _M2 = 0x94D049BB133111EB
 _MASK64 = (1 << 64) - 1
 
-TID_X, TID_WR, TID_WGU, TID_WDOWN, TID_LOGITS, TID_PERM, TID_HOT, TID_HOTTOK = 1, 2, 3, 4, 5, 6, 7, 8
+TID_X, TID_WR, TID_WGU, TID_WDOWN, TID_LOGITS, TID_PERM, TID_HOT, TID_HOTTOK, TID_DOUT = 1, 2, 3, 4, 5, 6, 7, 8, 9
 
 _CHUNK = 1 << 24
 
@@ -182,6 +182,13 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, device="cpu", weights: bool = T
     out["logits"] = lg.to(torch.float32).contiguous()
     out["x"] = x.contiguous()
     return out
+
+
+def make_grad_out(cfg: LayerConfig, seed: int = 0, device="cpu") -> torch.Tensor:
+    """A seeded upstream gradient dL/dout [T, d] for the backward, N(0, 1) in
+    the layer's activation type."""
+    dt = torch.bfloat16 if cfg.dtype == BF16 else torch.float32
+    return normal(stream_key(seed, TID_DOUT), cfg.T * cfg.d, device, dt).view(cfg.T, cfg.d).contiguous()
 
 
 def to_numpy_bits(t: torch.Tensor) -> np.ndarray:

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
 DEV_PLAN_INEXACT, DEV_TIMEOUT, DEV_BAD_INDEX = 1, 2, 4
-WS_PLAN, WS_LAYER, WS_LAYER_HOST = 0, 1, 2
+WS_PLAN, WS_LAYER, WS_LAYER_HOST, WS_LAYER_TRAIN = 0, 1, 2, 3
 
 
 class MoeError(RuntimeError):
@@ -63,6 +63,7 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [C, P, P, P, P, S, P]
         L.moe_layer_fwd.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
+        L.moe_layer_bwd.argtypes = [C, P, P, P, P, P, P, P, P, P, S, P]
         L.moe_read_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_plan_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         L.moe_probe_bounded_wait.argtypes = [P, ctypes.c_int64, P]
@@ -70,7 +71,7 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
-                  "moe_layer_fwd",
+                  "moe_layer_fwd", "moe_layer_bwd",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -185,6 +186,14 @@ def moe_layer_fwd_host(c, logits_host, x_host, w_gate_up, w_down, out_host, ws, 
                                     _ptr(w_down), _ptr(out_host), p, n, _stream(stream)), "moe_layer_fwd_host")
 
 
+def moe_layer_bwd(c, logits, w_gate_up, w_down, d_out, dx, dw_gate_up, dw_down, dlogits, ws, stream=None):
+    """The layer's backward on a MOE_WS_LAYER_TRAIN workspace that moe_layer_fwd last ran on."""
+    p, n = _ws(ws)
+    _check(lib().moe_layer_bwd(ctypes.byref(config(c)), _ptr(logits), _ptr(w_gate_up), _ptr(w_down), _ptr(d_out),
+                               _ptr(dx), _ptr(dw_gate_up), _ptr(dw_down), _ptr(dlogits), p, n, _stream(stream)),
+           "moe_layer_bwd")
+
+
 def moe_plan_noalloc(c, logits, topk_idx, topk_w, counts, row_of, header, stream=None):
     """moe_plan with its scratch in the library's static device array (no workspace)."""
     _check(lib().moe_plan_noalloc(ctypes.byref(config(c)), _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
@@ -240,9 +249,9 @@ def read_plan(c, ws: torch.Tensor) -> dict:
 class Layer:
     """Owns a workspace for one layer shape and runs the whole layer on it."""
 
-    def __init__(self, c, device="cuda", host_io: bool = False):
+    def __init__(self, c, device="cuda", host_io: bool = False, train: bool = False):
         self.cfg = c
-        self.kind = WS_LAYER_HOST if host_io else WS_LAYER
+        self.kind = WS_LAYER_TRAIN if train else (WS_LAYER_HOST if host_io else WS_LAYER)
         self.ws = alloc_workspace(c, self.kind, device)
         self.out = torch.empty(c.T, c.d, dtype=act_dtype(c), device=device)
 
@@ -254,6 +263,17 @@ class Layer:
     def forward_host(self, logits_host, x_host, w_gate_up, w_down, out_host, stream=None):
         moe_layer_fwd_host(self.cfg, logits_host, x_host, w_gate_up, w_down, out_host, self.ws, stream)
         return out_host
+
+    def backward(self, logits, w_gate_up, w_down, d_out, stream=None, dlogits: bool = True):
+        """Gradients after forward() on the same inputs (a `train=True` layer):
+        dx, dw_gate_up, dw_down (fp32) and the logits' gradient (or None)."""
+        c, dev = self.cfg, d_out.device
+        dx = torch.empty(c.T, c.d, dtype=act_dtype(c), device=dev)
+        dwgu = torch.empty(c.E, 2 * c.F, c.d, dtype=torch.float32, device=dev)
+        dwdn = torch.empty(c.E, c.d, c.F, dtype=torch.float32, device=dev)
+        dl = torch.empty(c.T, c.E, dtype=torch.float32, device=dev) if dlogits else None
+        moe_layer_bwd(c, logits, w_gate_up, w_down, d_out, dx, dwgu, dwdn, dl, self.ws, stream)
+        return dx, dwgu, dwdn, dl
 
     def status(self, stream=None) -> int:
         return moe_read_status(self.ws, stream)

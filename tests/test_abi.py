@@ -107,6 +107,25 @@ def test_calls_reject_bad_pointers_and_small_workspace(M):
     assert L.moe_read_status(None, None, ctypes.byref(v)) == M.MOE_ERR_INVALID_ARG
 
 
+def test_backward_rejects_unsupported_shapes_bad_pointers_and_small_workspace(M):
+    L = M.lib()
+    fake = ctypes.c_void_p(1 << 20)      # never dereferenced: every check below fails first
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    s = ctypes.c_size_t
+    bf = C.TINY.replace(dtype=C.BF16, tile=128, d=256, F=256)
+    cfg = ctypes.byref(M.config(bf))
+    need = M.moe_workspace_size(bf, M.WS_LAYER_TRAIN)
+    assert need > M.moe_workspace_size(bf, M.WS_LAYER_HOST)
+    args = [fake] * 8
+    assert L.moe_layer_bwd(cfg, *args, fake, s(need - 1), None) == M.MOE_ERR_WORKSPACE
+    assert L.moe_layer_bwd(cfg, None, *args[1:], fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_bwd(cfg, *args[:4], odd, *args[5:], fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    # fp32 layers and F not a multiple of 256 have no backward kernels
+    for c in (C.TINY, bf.replace(F=384)):
+        n = M.moe_workspace_size(c, M.WS_LAYER_TRAIN)
+        assert L.moe_layer_bwd(ctypes.byref(M.config(c)), *args, fake, s(n), None) == M.MOE_ERR_UNSUPPORTED
+
+
 def test_binding_refuses_to_run_without_library(tmp_path, monkeypatch):
     from routed_experts_b200 import moe
     monkeypatch.setattr(moe, "_lib", None)
