@@ -139,7 +139,7 @@ def source_sha(*rel):
 
 
 GEMM_SOURCES = ("routed_experts_b200/csrc/ffn_tc.cu", "routed_experts_b200/csrc/ptx.cuh",
-                "routed_experts_b200/csrc/common.cuh")
+                "routed_experts_b200/csrc/common.cuh", "routed_experts_b200/csrc/tc_common.cuh")
 
 
 def ncu_traffic(kernel_key: str):
@@ -256,9 +256,10 @@ def cpu_baseline(cfg, inp, n_tokens):
 
 
 def time_backward(cfg, inp, args, world, dev, stream, pg):
-    """moe_layer_bwd after one forward on a training workspace: W untimed and
-    K timed backward passes (CUDA events on the launching stream), max over
-    ranks. The forward state does not change between passes."""
+    """The training forward (moe_layer_fwd_train) and the backward
+    (moe_layer_bwd) on a training workspace, each W untimed and K timed
+    passes (CUDA events on the launching stream), max over ranks. The
+    forward state does not change between backward passes."""
     from routed_experts_b200 import moe as M
     lg, x, wgu, wdn = inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"]
     layer = M.Layer(cfg, dev, train=True)
@@ -273,37 +274,41 @@ def time_backward(cfg, inp, args, world, dev, stream, pg):
     def bwd():
         M.moe_layer_bwd(cfg, lg, wgu, wdn, d_out, dx, dwgu, dwdn, dl, layer.ws, stream)
 
-    for _ in range(args.warmup):
-        bwd()
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        if pg is not None:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1)
+        if pg is not None:
+            ms = max_over_ranks([ms], dev)[0]
+        return ms / args.steps
+
+    fwd_ms = timed(lambda: layer.forward(lg, x, wgu, wdn, stream=stream))
+    ms = timed(bwd)
     st = M.moe_read_status(layer.ws, stream)
     if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
-        raise RuntimeError(f"device status {st} after the backward warm-up")
-    if pg is not None:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    b0 = torch.cuda.Event(enable_timing=True)
-    b1 = torch.cuda.Event(enable_timing=True)
-    b0.record(stream)
-    for _ in range(args.steps):
-        bwd()
-    b1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms = b0.elapsed_time(b1)
-    if pg is not None:
-        ms = max_over_ranks([ms], dev)[0]
-    ms /= args.steps
+        raise RuntimeError(f"device status {st} after the backward passes")
     N = cfg.N
     alg = 12.0 * N * d * F        # DGrad W2 2NdF + WGrad W2 2NdF + DGrad W1 4NdF + WGrad W1 4NdF
-    executed = alg + 4.0 * N * d * F   # + FC1 recomputed for the pre-activations
     pk, _ = peaks()
     del layer, dwgu, dwdn
     torch.cuda.empty_cache()
-    return {"ms_per_step": ms, "tokens_per_s": world * T / (ms * 1e-3),
+    return {"ms_per_step": ms, "tokens_per_s": world * T / (ms * 1e-3), "forward_train_ms": fwd_ms,
+            "train_step_tokens_per_s": world * T / ((ms + fwd_ms) * 1e-3),
             "tflops": alg / (ms * 1e-3) / 1e12, "frac": alg / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
-            "flop_algorithmic": alg, "flop_executed": executed,
-            "note": "moe_layer_bwd: dY and dw, FC1 pre-activations recomputed, DGrad W2 with the SwiGLU "
-                    "derivative, WGrad W2, DGrad W1, WGrad W1, dx, logits' gradient (9 launches); frac of "
-                    "the measured bf16 peak counts algorithmic FLOP only"}
+            "flop_algorithmic": alg,
+            "note": "moe_layer_bwd: dY and dw, zeroed padding rows, DGrad W2 with the SwiGLU derivative "
+                    "(pre-activations kept by moe_layer_fwd_train), WGrad W2, DGrad W1, WGrad W1, dx, logits' "
+                    "gradient (8 launches); frac of the measured bf16 peak counts algorithmic FLOP"}
 
 
 def run_mine(args, world, rank, local):

@@ -88,7 +88,7 @@ typedef enum {
     MOE_WS_LAYER_HOST = 2, /* MOE_WS_LAYER plus device copies of logits, x and out:
                               moe_layer_fwd_host */
     MOE_WS_LAYER_TRAIN = 3 /* MOE_WS_LAYER_HOST plus the backward's buffers (dY, the
-                              pre-activations, dA | dG, dw): moe_layer_fwd then
+                              pre-activations, dA | dG, dw): moe_layer_fwd_train then
                               moe_layer_bwd */
 } moe_ws_kind;
 
@@ -255,15 +255,26 @@ moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, c
                               void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_layer_fwd_train - moe_layer_fwd on a MOE_WS_LAYER_TRAIN workspace
+ * that also keeps what the backward needs: FC1's epilogue stores the gate
+ * and up pre-activations, rounded to bf16, next to h. Same output bits as
+ * moe_layer_fwd. bf16 layers with F % 256 == 0; others return
+ * MOE_ERR_UNSUPPORTED.
+ */
+moe_status moe_layer_fwd_train(const moe_config* cfg, const float* logits, const void* x, const void* w_gate_up,
+                               const void* w_down, void* out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_layer_bwd - the layer's backward on one GPU ([MegaFlux] §3.2
  * "Backward": DGrad through W2 then W1, WGrad per expert with the partial
  * gradients of an expert's replicas reduced into one). bf16 layers with
  * F % 256 == 0; others return MOE_ERR_UNSUPPORTED.
- *   ws         a MOE_WS_LAYER_TRAIN workspace on which moe_layer_fwd last ran
- *              with the same logits, x and weights (its top-k, plan, xp, h
- *              and yp are read; xp's padding rows are zeroed).
- *   logits     fp32 [T, E] (device), as given to moe_layer_fwd.
- *   w_gate_up  [E, 2F, d], w_down [E, d, F] (device), as given to moe_layer_fwd.
+ *   ws         a MOE_WS_LAYER_TRAIN workspace on which moe_layer_fwd_train
+ *              last ran with the same logits, x and weights (its top-k,
+ *              plan, xp, h, yp and pre-activations are read; xp's padding
+ *              rows are zeroed).
+ *   logits     fp32 [T, E] (device), as given to moe_layer_fwd_train.
+ *   w_gate_up  [E, 2F, d], w_down [E, d, F] (device), as given to moe_layer_fwd_train.
  *   d_out      [T, d] (device): the gradient of the loss with respect to out.
  *   dx         [T, d] (device, out): sum over k, in k order, of each entry's
  *              input gradient, in fp32, rounded once.
@@ -273,9 +284,9 @@ moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, c
  *              gating (softmax or sigmoid over the chosen logits); zero off
  *              each token's top-k (selection itself has no gradient).
  * Rounding points: each entry's dY = w * dOut is formed in fp32 and rounded
- * to bf16; FC1's pre-activations are recomputed and rounded to bf16;
+ * to bf16; FC1's pre-activations are the forward's, rounded to bf16;
  * dA | dG and each entry's dx row are rounded to bf16 once each; products
- * accumulate in fp32. Asynchronous on `stream`; 9 kernel launches.
+ * accumulate in fp32. Asynchronous on `stream`; 8 kernel launches.
  */
 moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void* w_gate_up, const void* w_down,
                          const void* d_out, void* dx, float* dw_gate_up, float* dw_down, float* dlogits, void* ws,

@@ -284,6 +284,31 @@ moe_status moe_layer_fwd(const moe_config* cfg, const float* logits, const void*
     return from_cuda(launch_combine(s, yp, w, out, P, st));
 }
 
+moe_status moe_layer_fwd_train(const moe_config* cfg, const float* logits, const void* x, const void* w_gate_up,
+                               const void* w_down, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (s.dtype != MOE_BF16 || s.F % 256 != 0) return MOE_ERR_UNSUPPORTED;
+    if (!logits || !x || !w_gate_up || !w_down || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.train_end)) != MOE_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    int32_t* idx = reinterpret_cast<int32_t*>(b + L.idx);
+    float* w = reinterpret_cast<float*>(b + L.w);
+    int32_t* counts = reinterpret_cast<int32_t*>(b + L.counts);
+    if ((r = plan_impl(s, L, logits, idx, w, counts, ws, st)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(ws, L);
+    cudaError_t e = launch_gather(s, x, b + L.xp, P, st);
+    if (e == cudaSuccess) e = launch_ffn_tc(s, 4, b + L.xp, w_gate_up, b + L.h, P, st, kSpinBudget, b + L.ag);
+    if (e == cudaSuccess) e = launch_ffn_tc(s, 2, b + L.h, w_down, b + L.yp, P, st, kSpinBudget);
+    if (e == cudaSuccess) e = launch_combine(s, b + L.yp, w, out, P, st);
+    return from_cuda(e);
+}
+
 moe_status moe_layer_fwd_host(const moe_config* cfg, const float* logits_host, const void* x_host,
                               const void* w_gate_up, const void* w_down, void* out_host, void* ws,
                               size_t ws_bytes, moe_stream_t stream) {
@@ -328,13 +353,12 @@ moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void*
     const void* h = b + L.h;
     const void* yp = b + L.yp;
     void* dy = b + L.dy;   // dY, then dXp once WGrad of W2 has read dY
-    void* ag = b + L.ag;
+    const void* ag = b + L.ag;   // the pre-activations moe_layer_fwd_train stored
     void* dag = b + L.dag;
     float* dw = reinterpret_cast<float*>(b + L.dw);
     const WsPtrs P = ws_ptrs(ws, L);
     cudaError_t e = launch_bwd_scatter(s, d_out, yp, w, dy, dw, P, st);
     if (e == cudaSuccess) e = launch_zero_padding(s, xp, dy, (int64_t)s.eb * s.d, P, st);
-    if (e == cudaSuccess) e = launch_ffn_tc(s, 4, xp, w_gate_up, ag, P, st, kSpinBudget);
     if (e == cudaSuccess) e = launch_bwd_tc(s, 0, dy, w_down, dag, ag, P, st, kSpinBudget);
     if (e == cudaSuccess) e = launch_bwd_tc(s, 2, dy, h, dw_down, nullptr, P, st, kSpinBudget);
     if (e == cudaSuccess) e = launch_bwd_tc(s, 1, dag, w_gate_up, dy, nullptr, P, st, kSpinBudget);

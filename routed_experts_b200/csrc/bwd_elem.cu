@@ -45,6 +45,11 @@ bwd_scatter_kernel(const uint4* __restrict__ d_out, const uint4* __restrict__ yp
         }
         for (int v = lane; v < nvec; v += 32) {
             const uint4 go = __ldg(d_out + (int64_t)t * nvec + v);
+            // the K rows' vectors are all requested before any is used
+            uint4 yv[KMAX];
+#pragma unroll
+            for (int k = 0; k < KMAX; ++k)
+                if (k < K && rows[k] >= 0) yv[k] = __ldg(yp + (int64_t)rows[k] * nvec + v);
             const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&go);
             float gf[8];
 #pragma unroll
@@ -56,8 +61,7 @@ bwd_scatter_kernel(const uint4* __restrict__ d_out, const uint4* __restrict__ yp
 #pragma unroll
             for (int k = 0; k < KMAX; ++k) {
                 if (k >= K || rows[k] < 0) continue;
-                const uint4 yv = __ldg(yp + (int64_t)rows[k] * nvec + v);
-                const __nv_bfloat162* y2 = reinterpret_cast<const __nv_bfloat162*>(&yv);
+                const __nv_bfloat162* y2 = reinterpret_cast<const __nv_bfloat162*>(&yv[k]);
                 uint4 o;
                 __nv_bfloat162* o2 = reinterpret_cast<__nv_bfloat162*>(&o);
 #pragma unroll

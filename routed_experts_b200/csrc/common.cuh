@@ -122,12 +122,13 @@ cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void*
 // which = 1: FC1 + SwiGLU (a_mat = xp, w = w_gate_up, out = h);
 // which = 2: FC2 (a_mat = h, w = w_down, out = yp);
 // which = 3 (tensor cores only): FC1 + SwiGLU with a_mat = x, rows gathered by the row map;
-// which = 4 (tensor cores only): FC1 pre-activations [gate | up] (a_mat = xp, out [rows_cap, 2F]).
+// which = 4 (tensor cores only): FC1 + SwiGLU as which = 1, also storing the pre-activations
+// [gate | up] into preact [rows_cap, 2F] (the training forward).
 cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                             const WsPtrs& ws, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
-                          const WsPtrs& ws, cudaStream_t st, long long spin_budget);
+                          const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact = nullptr);
 // backward (bf16): mode 0 DGrad W2 + SwiGLU derivative (a_mat = dY, b_mat = w_down, ag, out = dAG),
 // 1 DGrad W1 (a_mat = dAG, b_mat = w_gate_up, out = dXp), 2 WGrad W2 (a_mat = dY, b_mat = h,
 // out = dW2 fp32), 3 WGrad W1 (a_mat = dAG, b_mat = xp, out = dW1 fp32)

@@ -87,12 +87,12 @@ struct TcArgs {
 
 // MODE 0: FC1 + SwiGLU -> h (A = xp); MODE 1: FC2 -> yp (A = h);
 // MODE 2: FC1 + SwiGLU -> h with A gathered from x;
-// MODE 3: FC1 pre-activations -> [gate | up] (A = xp), rounded to bf16, for
-// the backward's SwiGLU derivative.
+// MODE 3: FC1 + SwiGLU -> h, also storing the pre-activations [gate | up]
+// (rounded to bf16) for the backward's SwiGLU derivative (training forward).
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmO, TcArgs a) {
+              const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmP, TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_base = base + kStages * kStageBytes;
@@ -135,7 +135,12 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             carry += __shfl_sync(0xffffffffu, x, 31);
         }
     }
-    if (warp == 0 && lane == 0) { ptx::prefetch_tmap(&tmA); ptx::prefetch_tmap(&tmB); ptx::prefetch_tmap(&tmO); }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        ptx::prefetch_tmap(&tmO);
+        if (MODE == 3) ptx::prefetch_tmap(&tmP);
+    }
     __syncthreads();
     ptx::cluster_sync();   // the peer's barriers exist before any remote arrive, store or copy
     if (warp == 1) { ptx::tmem_alloc_pair(&S->tmem_base, kTmemCols); ptx::tmem_relinquish_pair(); }
@@ -147,7 +152,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const int kb_count = a.Kdim / kBK;
     constexpr bool kFC1 = MODE != 1;
     constexpr bool kGather = MODE == 2;
-    constexpr bool kPreact = MODE == 3;
+    constexpr bool kPreact = MODE == 3;   // also store the pre-activations through tmP
     constexpr int kColTile = kFC1 ? 128 : 256;
 
     // the ring slot of the k-th item, and the parity of its phase
@@ -354,41 +359,39 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
 #pragma unroll 1
                 for (int c = 0; c < kColTile; c += 32) {
                     uint32_t pk[16];
-                    if (kPreact) {
-                        uint32_t gt[32], up[32];
-                        ptx::tmem_ld32(t_row + c, gt);
-                        ptx::tmem_ld32(t_row + 128 + c, up);
-                        ptx::tmem_ld_wait();
-                        uint32_t pu[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            pk[i] = pad ? 0u : pack_bf16(__uint_as_float(gt[2 * i]), __uint_as_float(gt[2 * i + 1]));
-                            pu[i] = pad ? 0u : pack_bf16(__uint_as_float(up[2 * i]), __uint_as_float(up[2 * i + 1]));
-                        }
-                        // both staging tiles: gate at column j*128 + c, up at F + j*128 + c
-                        if (lane == 0) ptx::bulk_wait_group_read<0>();
-                        __syncwarp();
-                        uint4* sg = reinterpret_cast<uint4*>(stg + lane * 64);
-                        uint4* su = reinterpret_cast<uint4*>(stg + kEpiBuf + lane * 64);
-#pragma unroll
-                        for (int v = 0; v < 4; ++v) {
-                            sg[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                            su[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
-                        }
-                        ptx::fence_proxy_async_shared();
-                        __syncwarp();
-                        if (lane == 0) {
-                            ptx::tma_store_2d(&tmO, stg, j * kColTile + c, row0 + quad * 32);
-                            ptx::tma_store_2d(&tmO, stg + kEpiBuf, a.F + j * kColTile + c, row0 + quad * 32);
-                            ptx::bulk_commit_group();
-                        }
-                        continue;
-                    }
                     if (kFC1) {
                         uint32_t gt[32], up[32];
                         ptx::tmem_ld32(t_row + c, gt);
                         ptx::tmem_ld32(t_row + 128 + c, up);
                         ptx::tmem_ld_wait();
+                        if (kPreact) {
+                            // the pre-activations first: gate at column j*128 + c, up at F + j*128 + c,
+                            // through both staging tiles
+                            uint32_t pg[16], pu[16];
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                pg[i] = pad ? 0u : pack_bf16(__uint_as_float(gt[2 * i]), __uint_as_float(gt[2 * i + 1]));
+                                pu[i] = pad ? 0u : pack_bf16(__uint_as_float(up[2 * i]), __uint_as_float(up[2 * i + 1]));
+                            }
+                            if (lane == 0) ptx::bulk_wait_group_read<0>();
+                            __syncwarp();
+                            uint4* sg = reinterpret_cast<uint4*>(stg + lane * 64);
+                            uint4* su = reinterpret_cast<uint4*>(stg + kEpiBuf + lane * 64);
+#pragma unroll
+                            for (int v = 0; v < 4; ++v) {
+                                sg[v] = make_uint4(pg[4 * v], pg[4 * v + 1], pg[4 * v + 2], pg[4 * v + 3]);
+                                su[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+                            }
+                            ptx::fence_proxy_async_shared();
+                            __syncwarp();
+                            if (lane == 0) {
+                                ptx::tma_store_2d(&tmP, stg, j * kColTile + c, row0 + quad * 32);
+                                ptx::tma_store_2d(&tmP, stg + kEpiBuf, a.F + j * kColTile + c, row0 + quad * 32);
+                                ptx::bulk_commit_group();
+                                ptx::bulk_wait_group_read<0>();   // both tiles free again for h below
+                            }
+                            __syncwarp();
+                        }
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
                             const float h0 = silu(__uint_as_float(gt[2 * i])) * __uint_as_float(up[2 * i]);
@@ -453,12 +456,12 @@ __global__ void bounded_wait_probe_kernel(uint32_t* status, long long budget) {
 }
 
 template <int MODE>
-cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const TcArgs& a,
-                        int grid, cudaStream_t st) {
+cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const CUtensorMap& tP,
+                        const TcArgs& a, int grid, cudaStream_t st) {
     cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)kSmemBytes);
     if (err != cudaSuccess) return err;
-    ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, a);
+    ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, tP, a);
     return cudaGetLastError();
 }
 
@@ -470,7 +473,7 @@ cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaSt
 }
 
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
-                          const WsPtrs& ws, cudaStream_t st, long long spin_budget) {
+                          const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -485,7 +488,7 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.queue = ws.gemm_q + (which == 2 ? 4 : 0);
     a.src_of = ws.src_of;
     a.out = static_cast<__nv_bfloat16*>(out);
-    CUtensorMap tA, tB, tO;
+    CUtensorMap tA, tB, tO, tP;
     if (which == 3) {
         // FC1 + SwiGLU with A gathered from x [T, d] by the row map -> h [rows_cap, F]
         if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.T, 1) ||
@@ -497,20 +500,21 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<2>(tA, tB, tO, a, sms, st);
+        return launch_mode<2>(tA, tB, tO, tO, a, sms, st);
     }
     if (which == 4) {
-        // FC1 pre-activations: xp [rows_cap, d] x w_gate_up [E*2F, d] -> [gate | up] [rows_cap, 2F]
-        if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
+        // FC1 + SwiGLU -> h [rows_cap, F], and the pre-activations -> preact [rows_cap, 2F]
+        if (!preact || !make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
             !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
-            !make_tmap_out(&tO, out, (uint64_t)2 * s.F, (uint64_t)s.rows_cap))
+            !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap) ||
+            !make_tmap_out(&tP, preact, (uint64_t)2 * s.F, (uint64_t)s.rows_cap))
             return cudaErrorInvalidValue;
-        a.out_ld = 2 * s.F;
+        a.out_ld = s.F;
         a.Kdim = s.d;
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<3>(tA, tB, tO, a, sms, st);
+        return launch_mode<3>(tA, tB, tO, tP, a, sms, st);
     }
     if (which == 1) {
         // FC1 + SwiGLU: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h [rows_cap, F]
@@ -523,7 +527,7 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<0>(tA, tB, tO, a, sms, st);
+        return launch_mode<0>(tA, tB, tO, tO, a, sms, st);
     }
     // FC2: h [rows_cap, F] x w_down [E*d, F] -> yp [rows_cap, d]
     if (!make_tmap(&tA, a_mat, (uint64_t)s.F, (uint64_t)s.rows_cap, kBM) ||
@@ -535,7 +539,7 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.n_tiles = s.d / 256;
     a.F = 0;
     a.b_rows = s.d;
-    return launch_mode<1>(tA, tB, tO, a, sms, st);
+    return launch_mode<1>(tA, tB, tO, tO, a, sms, st);
 }
 
 }  // namespace moe

@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_fwd.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_bwd.argtypes = [C, P, P, P, P, P, P, P, P, P, S, P]
+        L.moe_layer_fwd_train.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_read_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
         L.moe_plan_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         L.moe_probe_bounded_wait.argtypes = [P, ctypes.c_int64, P]
@@ -71,7 +72,7 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
-                  "moe_layer_fwd", "moe_layer_bwd",
+                  "moe_layer_fwd", "moe_layer_bwd", "moe_layer_fwd_train",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -186,8 +187,15 @@ def moe_layer_fwd_host(c, logits_host, x_host, w_gate_up, w_down, out_host, ws, 
                                     _ptr(w_down), _ptr(out_host), p, n, _stream(stream)), "moe_layer_fwd_host")
 
 
+def moe_layer_fwd_train(c, logits, x, w_gate_up, w_down, out, ws, stream=None):
+    """moe_layer_fwd that also keeps FC1's pre-activations for moe_layer_bwd (MOE_WS_LAYER_TRAIN)."""
+    p, n = _ws(ws)
+    _check(lib().moe_layer_fwd_train(ctypes.byref(config(c)), _ptr(logits), _ptr(x), _ptr(w_gate_up),
+                                     _ptr(w_down), _ptr(out), p, n, _stream(stream)), "moe_layer_fwd_train")
+
+
 def moe_layer_bwd(c, logits, w_gate_up, w_down, d_out, dx, dw_gate_up, dw_down, dlogits, ws, stream=None):
-    """The layer's backward on a MOE_WS_LAYER_TRAIN workspace that moe_layer_fwd last ran on."""
+    """The layer's backward on a MOE_WS_LAYER_TRAIN workspace that moe_layer_fwd_train last ran on."""
     p, n = _ws(ws)
     _check(lib().moe_layer_bwd(ctypes.byref(config(c)), _ptr(logits), _ptr(w_gate_up), _ptr(w_down), _ptr(d_out),
                                _ptr(dx), _ptr(dw_gate_up), _ptr(dw_down), _ptr(dlogits), p, n, _stream(stream)),
@@ -256,8 +264,10 @@ class Layer:
         self.out = torch.empty(c.T, c.d, dtype=act_dtype(c), device=device)
 
     def forward(self, logits, x, w_gate_up, w_down, out=None, stream=None):
+        """The layer; a `train=True` layer also keeps what backward() needs."""
         out = self.out if out is None else out
-        moe_layer_fwd(self.cfg, logits, x, w_gate_up, w_down, out, self.ws, stream)
+        fwd = moe_layer_fwd_train if self.kind == WS_LAYER_TRAIN else moe_layer_fwd
+        fwd(self.cfg, logits, x, w_gate_up, w_down, out, self.ws, stream)
         return out
 
     def forward_host(self, logits_host, x_host, w_gate_up, w_down, out_host, stream=None):

@@ -120,10 +120,14 @@ def test_backward_rejects_unsupported_shapes_bad_pointers_and_small_workspace(M)
     assert L.moe_layer_bwd(cfg, *args, fake, s(need - 1), None) == M.MOE_ERR_WORKSPACE
     assert L.moe_layer_bwd(cfg, None, *args[1:], fake, s(need), None) == M.MOE_ERR_INVALID_ARG
     assert L.moe_layer_bwd(cfg, *args[:4], odd, *args[5:], fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_fwd_train(cfg, *args[:5], fake, s(need - 1), None) == M.MOE_ERR_WORKSPACE
+    assert L.moe_layer_fwd_train(cfg, *args[:4], None, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
     # fp32 layers and F not a multiple of 256 have no backward kernels
     for c in (C.TINY, bf.replace(F=384)):
         n = M.moe_workspace_size(c, M.WS_LAYER_TRAIN)
         assert L.moe_layer_bwd(ctypes.byref(M.config(c)), *args, fake, s(n), None) == M.MOE_ERR_UNSUPPORTED
+        assert L.moe_layer_fwd_train(ctypes.byref(M.config(c)), *args[:5], fake, s(n), None) == \
+            M.MOE_ERR_UNSUPPORTED
 
 
 def test_binding_refuses_to_run_without_library(tmp_path, monkeypatch):

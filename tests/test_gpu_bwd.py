@@ -106,6 +106,15 @@ def test_backward_is_deterministic_and_plan_invariant():
         assert_grad_close(b.cpu().numpy(), a.cpu().numpy(), n, rel=1e-5)
 
 
+def test_training_forward_gives_the_inference_output():
+    for cfg in (SMALL, WIDE):
+        inp = I.make_inputs(cfg, 6, "cuda")
+        train, infer = M.Layer(cfg, train=True), M.Layer(cfg)
+        a = train.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"])
+        b = infer.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"])
+        assert torch.equal(a, b)
+
+
 def test_backward_leaves_the_forward_output_alone():
     inp, d_out, layer, _ = run_bwd(SMALL, 4)
     before = layer.out.clone()
