@@ -183,3 +183,51 @@ def check_full_size(cfg, seed: int, n_tokens: int = 8, n_rows: int = 32, device=
                         ref["w"][t:t + 1], wgu, wdn, cfg.dtype, O.default_round_mode(cfg.dtype))
         assert_close(gout[i:i + 1], o, cfg.dtype, f"out[{t}]")
     return g, ref, inp
+
+
+def assert_grad_close(got: np.ndarray, ref: np.ndarray, what: str, rel: float = 1e-2):
+    """The bf16 output bound (2e-2 absolute + 1e-2 relative) with its absolute
+    part taken at the gradient's scale: |g - o| <= 2 rel rms(o) + rel |o|
+    elementwise, and ||g - o|| <= rel ||o||. Each weight-gradient element is
+    a sum of products of bf16 values that the GPU and the oracle round from
+    fp32 and fp64 sums, so single terms may differ by one bf16 ulp."""
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = np.sqrt(np.mean(ref ** 2)) if ref.size else 0.0
+    err = np.abs(got - ref)
+    bad = err > rel * (2 * scale + np.abs(ref))
+    assert not bad.any(), f"{what}: {int(bad.sum())} of {bad.size} out of tolerance, max err {err.max():.3e}"
+    den = np.linalg.norm(ref)
+    if den > 0:
+        assert np.linalg.norm(got - ref) / den <= rel, f"{what}: normwise {np.linalg.norm(got - ref) / den:.3e}"
+
+
+def run_bwd(cfg, seed, device="cuda"):
+    """The training forward then the backward of one seeded layer through the C ABI."""
+    inp = I.make_inputs(cfg, seed, device)
+    d_out = I.make_grad_out(cfg, seed, device)
+    layer = M.Layer(cfg, device, train=True)
+    layer.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"])
+    dx, dwgu, dwdn, dl = layer.backward(inp["logits"], inp["w_gate_up"], inp["w_down"], d_out)
+    assert layer.status() & ~M.DEV_PLAN_INEXACT == 0
+    return inp, d_out, layer, (dx, dwgu, dwdn, dl)
+
+
+def check_bwd_small(cfg, seed, device="cuda"):
+    """The backward against the oracle's, every element (sizes the oracle runs in seconds)."""
+    inp, d_out, _, (dx, dwgu, dwdn, dl) = run_bwd(cfg, seed, device)
+    hin = {k: I.to_numpy_bits(v) for k, v in inp.items()}
+    idx, w = O.topk_gate(hin["logits"], cfg.K, cfg.gating)
+    ref = O.layer_bwd(hin["logits"], idx, w, hin["x"], hin["w_gate_up"], hin["w_down"], I.to_numpy_bits(d_out),
+                      gating=cfg.gating, dtype=cfg.dtype, round_mode=O.ROUND_BF16)
+    assert_close(to_f64(dx), O.to_f64(ref["dx"], cfg.dtype), cfg.dtype, "dx")
+    assert_grad_close(dwgu.cpu().numpy(), ref["dw_gate_up"], "dw_gate_up")
+    assert_grad_close(dwdn.cpu().numpy(), ref["dw_down"], "dw_down")
+    assert_grad_close(dl.cpu().numpy(), ref["dlogits"], "dlogits")
+    # experts no token chose have exactly zero gradients; so do unchosen logits
+    counts = np.bincount(idx.ravel(), minlength=cfg.E)
+    for e in np.nonzero(counts == 0)[0]:
+        assert not dwgu[e].any() and not dwdn[e].any()
+    chosen = np.zeros((cfg.T, cfg.E), bool)
+    np.put_along_axis(chosen, idx, True, axis=1)
+    assert not dl.cpu().numpy()[~chosen].any()
