@@ -24,7 +24,7 @@ enum { H_STATUS = 0, H_NPIECES = 1, H_NBLOCKS = 2, H_TOTAL_ROWS = 3, H_MOVES = 4
 
 // Work-queue counters of the grouped GEMM: for FC1 then FC2, two queue
 // heads and a count of clusters that finished (all zero between launches).
-constexpr int kGemmQWords = 8;
+constexpr int kGemmQWords = 12;
 
 // Default bound of a device-side spin (clock cycles, about 2 s at 1.9 GHz).
 constexpr long long kSpinBudget = 4000000000LL;

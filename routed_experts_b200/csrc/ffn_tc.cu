@@ -70,8 +70,6 @@ using namespace tc;
 
 struct TcArgs {
     const int32_t* src_of;    // row -> token (gathered FC1 only)
-    __nv_bfloat16* out;       // h (FC1) or yp (FC2)
-    int out_ld;               // F or d
     int Kdim;                 // d or F
     int n_tiles;              // F/128 (FC1) or d/256 (FC2)
     int F;                    // FC1: row offset of the up projection inside an expert
@@ -83,7 +81,87 @@ struct TcArgs {
     const int32_t* sched_off;
     uint32_t* header;
     int32_t* queue;           // [3]: head of queue 0, head of queue 1, clusters finished
+    int lone_apart;           // 1: experts with a single block are left to the single-CTA kernel
 };
+
+// The epilogue of one work item for one warp (rows 32*quad .. 32*quad+31 of
+// the CTA's block): drain the accumulator at t_row 32 columns at a time,
+// apply FC1's SwiGLU (MODE 0, 2, 3) or nothing (FC2), and store bf16 tiles
+// through the warp's two staging tiles with TMA. MODE 3 first stores the
+// pre-activations through tmP. Rows past the block's valid ones are zero.
+template <int MODE>
+__device__ __forceinline__ void epilogue_item(uint32_t t_row, int lane, int quad, uint8_t* stg, int& buf,
+                                              const CUtensorMap* tmO, const CUtensorMap* tmP, int F, int j,
+                                              int row0, bool pad) {
+    constexpr bool kFC1 = MODE != 1;
+    constexpr bool kPreact = MODE == 3;
+    constexpr int kColTile = kFC1 ? 128 : 256;
+#pragma unroll 1
+    for (int c = 0; c < kColTile; c += 32) {
+        uint32_t pk[16];
+        if (kFC1) {
+            uint32_t gt[32], up[32];
+            ptx::tmem_ld32(t_row + c, gt);
+            ptx::tmem_ld32(t_row + 128 + c, up);
+            ptx::tmem_ld_wait();
+            if (kPreact) {
+                // the pre-activations first: gate at column j*128 + c, up at F + j*128 + c,
+                // through both staging tiles
+                uint32_t pg[16], pu[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    pg[i] = pad ? 0u : pack_bf16(__uint_as_float(gt[2 * i]), __uint_as_float(gt[2 * i + 1]));
+                    pu[i] = pad ? 0u : pack_bf16(__uint_as_float(up[2 * i]), __uint_as_float(up[2 * i + 1]));
+                }
+                if (lane == 0) ptx::bulk_wait_group_read<0>();
+                __syncwarp();
+                uint4* sg = reinterpret_cast<uint4*>(stg + lane * 64);
+                uint4* su = reinterpret_cast<uint4*>(stg + kEpiBuf + lane * 64);
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    sg[v] = make_uint4(pg[4 * v], pg[4 * v + 1], pg[4 * v + 2], pg[4 * v + 3]);
+                    su[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
+                }
+                ptx::fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    ptx::tma_store_2d(tmP, stg, j * kColTile + c, row0 + quad * 32);
+                    ptx::tma_store_2d(tmP, stg + kEpiBuf, F + j * kColTile + c, row0 + quad * 32);
+                    ptx::bulk_commit_group();
+                    ptx::bulk_wait_group_read<0>();   // both tiles free again for h below
+                }
+                __syncwarp();
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float h0 = silu(__uint_as_float(gt[2 * i])) * __uint_as_float(up[2 * i]);
+                const float h1 = silu(__uint_as_float(gt[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
+                pk[i] = pad ? 0u : pack_bf16(h0, h1);
+            }
+        } else {
+            uint32_t y[32];
+            ptx::tmem_ld32(t_row + c, y);
+            ptx::tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                pk[i] = pad ? 0u : pack_bf16(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
+        }
+        // this staging tile's previous store has finished reading it
+        if (lane == 0) ptx::bulk_wait_group_read<1>();
+        __syncwarp();
+        uint8_t* tile = stg + buf * kEpiBuf;
+        uint4* srow = reinterpret_cast<uint4*>(tile + lane * 64);   // row m: 32 bf16
+#pragma unroll
+        for (int v = 0; v < 4; ++v) srow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        ptx::fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+            ptx::tma_store_2d(tmO, tile, j * kColTile + c, row0 + quad * 32);
+            ptx::bulk_commit_group();
+        }
+        buf ^= 1;
+    }
+}
 
 // MODE 0: FC1 + SwiGLU -> h (A = xp); MODE 1: FC2 -> yp (A = h);
 // MODE 2: FC1 + SwiGLU -> h with A gathered from x;
@@ -117,14 +195,18 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::fence_barrier_init();
     }
     for (int i = threadIdx.x; i <= a.E; i += kThreads) s_off[i] = a.sched_off[i];
+    // the single-CTA kernel that follows may take SMs as this kernel's CTAs leave
+    if (threadIdx.x == 0) ptx::griddep_launch_dependents();
     __syncthreads();
     if (warp == 0) {
-        // pair offsets: p_off[e] = sum over e' < e of ceil(blocks(e') / 2)
+        // pair offsets: p_off[e] = sum over e' < e of the pairs of e' (ceil(blocks / 2);
+        // none for a one-block expert left to the single-CTA kernel)
         int carry = 0;
         if (lane == 0) p_off[0] = 0;
         for (int b = 0; b < a.E; b += 32) {
             const int i = b + lane;
-            const int v = i < a.E ? (s_off[i + 1] - s_off[i] + 1) >> 1 : 0;
+            const int nb = i < a.E ? s_off[i + 1] - s_off[i] : 0;
+            const int v = (a.lone_apart && nb == 1) ? 0 : (nb + 1) >> 1;
             int x = v;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -152,7 +234,6 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const int kb_count = a.Kdim / kBK;
     constexpr bool kFC1 = MODE != 1;
     constexpr bool kGather = MODE == 2;
-    constexpr bool kPreact = MODE == 3;   // also store the pre-activations through tmP
     constexpr int kColTile = kFC1 ? 128 : 256;
 
     // the ring slot of the k-th item, and the parity of its phase
@@ -354,74 +435,9 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
             if (!role_wait(&S->acc_full[acc], acc_phase, a.spin, abort_flag, a.header)) break;
             ptx::tc_fence_after();
-            if (row0 >= 0) {
-                const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN);
-#pragma unroll 1
-                for (int c = 0; c < kColTile; c += 32) {
-                    uint32_t pk[16];
-                    if (kFC1) {
-                        uint32_t gt[32], up[32];
-                        ptx::tmem_ld32(t_row + c, gt);
-                        ptx::tmem_ld32(t_row + 128 + c, up);
-                        ptx::tmem_ld_wait();
-                        if (kPreact) {
-                            // the pre-activations first: gate at column j*128 + c, up at F + j*128 + c,
-                            // through both staging tiles
-                            uint32_t pg[16], pu[16];
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) {
-                                pg[i] = pad ? 0u : pack_bf16(__uint_as_float(gt[2 * i]), __uint_as_float(gt[2 * i + 1]));
-                                pu[i] = pad ? 0u : pack_bf16(__uint_as_float(up[2 * i]), __uint_as_float(up[2 * i + 1]));
-                            }
-                            if (lane == 0) ptx::bulk_wait_group_read<0>();
-                            __syncwarp();
-                            uint4* sg = reinterpret_cast<uint4*>(stg + lane * 64);
-                            uint4* su = reinterpret_cast<uint4*>(stg + kEpiBuf + lane * 64);
-#pragma unroll
-                            for (int v = 0; v < 4; ++v) {
-                                sg[v] = make_uint4(pg[4 * v], pg[4 * v + 1], pg[4 * v + 2], pg[4 * v + 3]);
-                                su[v] = make_uint4(pu[4 * v], pu[4 * v + 1], pu[4 * v + 2], pu[4 * v + 3]);
-                            }
-                            ptx::fence_proxy_async_shared();
-                            __syncwarp();
-                            if (lane == 0) {
-                                ptx::tma_store_2d(&tmP, stg, j * kColTile + c, row0 + quad * 32);
-                                ptx::tma_store_2d(&tmP, stg + kEpiBuf, a.F + j * kColTile + c, row0 + quad * 32);
-                                ptx::bulk_commit_group();
-                                ptx::bulk_wait_group_read<0>();   // both tiles free again for h below
-                            }
-                            __syncwarp();
-                        }
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float h0 = silu(__uint_as_float(gt[2 * i])) * __uint_as_float(up[2 * i]);
-                            const float h1 = silu(__uint_as_float(gt[2 * i + 1])) * __uint_as_float(up[2 * i + 1]);
-                            pk[i] = pad ? 0u : pack_bf16(h0, h1);
-                        }
-                    } else {
-                        uint32_t y[32];
-                        ptx::tmem_ld32(t_row + c, y);
-                        ptx::tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            pk[i] = pad ? 0u : pack_bf16(__uint_as_float(y[2 * i]), __uint_as_float(y[2 * i + 1]));
-                    }
-                    // this staging tile's previous store has finished reading it
-                    if (lane == 0) ptx::bulk_wait_group_read<1>();
-                    __syncwarp();
-                    uint8_t* tile = stg + buf * kEpiBuf;
-                    uint4* srow = reinterpret_cast<uint4*>(tile + lane * 64);   // row m: 32 bf16
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) srow[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
-                    ptx::fence_proxy_async_shared();
-                    __syncwarp();
-                    if (lane == 0) {
-                        ptx::tma_store_2d(&tmO, tile, j * kColTile + c, row0 + quad * 32);
-                        ptx::bulk_commit_group();
-                    }
-                    buf ^= 1;
-                }
-            }
+            if (row0 >= 0)
+                epilogue_item<MODE>(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN), lane, quad, stg, buf,
+                                    &tmO, &tmP, a.F, j, row0, pad);
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -440,6 +456,238 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     }
 }
 
+// ---------------------------------------------------------------- lone blocks
+// An expert with a single planned block would run on a CTA pair beside an
+// empty half. Those blocks run here instead, one CTA per item with
+// tcgen05.mma.cta_group::1 (M = 128, N = 256; a kernel keeps to one
+// CTA-group size): the CTA loads the block's 128 rows and both halves of the
+// weight tile (256 rows), 48 KB per k-step, into a 4-stage ring, and the
+// same epilogue stores the result. Warp roles as in the pair kernel (TMA,
+// MMA, 4 epilogue warps, scheduler); items (lone block, column tile) come
+// from one atomic queue. The odd last block of an expert with three or more
+// blocks stays in the pair kernel: its weight tiles are in L2 while the
+// expert's pairs run there, and a later launch would read them again from
+// memory.
+constexpr int kSStages = 4;
+constexpr int kSStageBytes = kABytes + 2 * kBBytes;   // 48 KB
+constexpr uint32_t kSItemConsumers = 6;               // TMA thread, MMA thread, 4 epilogue warps
+
+struct SSmem {
+    uint64_t full[kSStages], empty[kSStages], acc_full[2], acc_empty[2], drain;
+    uint64_t item_full[kItemSlots], item_empty[kItemSlots];
+    int4 items[kItemSlots];   // expert (-1: no more work), column tile, first row of the block, valid rows
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr size_t kSSmemBytes = 1024 /*align slack*/ + kSStages * kSStageBytes + kEpiBytes + sizeof(SSmem) +
+                               2 * sizeof(int32_t) * (kMaxE + 1);
+static_assert(kSSmemBytes <= 232448, "shared memory per CTA");
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreads, 1)
+ffn_tc_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmP, TcArgs a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* epi_base = base + kSStages * kSStageBytes;
+    SSmem* S = reinterpret_cast<SSmem*>(epi_base + kEpiBytes);
+    int32_t* s_off = reinterpret_cast<int32_t*>(S + 1);
+    int32_t* q_off = s_off + (a.E + 1);
+    volatile int* abort_flag = &S->abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kSStages; ++s) { ptx::mbar_init(&S->full[s], 1); ptx::mbar_init(&S->empty[s], 1); }
+        for (int q = 0; q < 2; ++q) { ptx::mbar_init(&S->acc_full[q], 1); ptx::mbar_init(&S->acc_empty[q], 4); }
+        for (int q = 0; q < kItemSlots; ++q) {
+            ptx::mbar_init(&S->item_full[q], 1);
+            ptx::mbar_init(&S->item_empty[q], kSItemConsumers);
+        }
+        ptx::mbar_init(&S->drain, 1);
+        S->abort_flag = 0;
+        ptx::fence_barrier_init();
+    }
+    for (int i = threadIdx.x; i <= a.E; i += kThreads) s_off[i] = a.sched_off[i];
+    __syncthreads();
+    if (warp == 0) {
+        // q_off[e]: one-block experts before e
+        int carry = 0;
+        if (lane == 0) q_off[0] = 0;
+        for (int b = 0; b < a.E; b += 32) {
+            const int i = b + lane;
+            int x = i < a.E && s_off[i + 1] - s_off[i] == 1 ? 1 : 0;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, off);
+                if (lane >= off) x += y;
+            }
+            if (i < a.E) q_off[i + 1] = carry + x;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+    }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmA);
+        ptx::prefetch_tmap(&tmB);
+        ptx::prefetch_tmap(&tmO);
+        if (MODE == 3) ptx::prefetch_tmap(&tmP);
+    }
+    __syncthreads();
+    if (warp == 1) { ptx::tmem_alloc(&S->tmem_base, kTmemCols); ptx::tmem_relinquish(); }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = S->tmem_base;
+    const int n_items = q_off[a.E] * a.n_tiles;
+    const int kb_count = a.Kdim / kBK;
+    constexpr bool kFC1 = MODE != 1;
+    constexpr int kColTile = kFC1 ? 128 : 256;
+
+    auto slot_of = [](int k) { return k % kItemSlots; };
+    auto parity_of = [](int k) { return (uint32_t)((k / kItemSlots) & 1); };
+    auto take_item = [&](int k, int4& item) -> bool {
+        if (!role_wait(&S->item_full[slot_of(k)], parity_of(k), a.spin, abort_flag, a.header)) return false;
+        item = S->items[slot_of(k)];
+        return true;
+    };
+    auto release_item = [&](int k) { ptx::mbar_arrive(&S->item_empty[slot_of(k)]); };
+
+    if (warp == kSchedWarp) {
+        // ------------------------------------------------ scheduler
+        if (lane == 0) {
+            for (int k = 0;; ++k) {
+                const bool ok = role_wait(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
+                const int it = ok ? atomicAdd(&a.queue[0], 1) : n_items;
+                int4 item = make_int4(-1, 0, 0, 0);
+                if (it < n_items) {
+                    const int q = it / a.n_tiles, j = it % a.n_tiles;
+                    int lo = 0, hi = a.E;   // the expert of lone block q: q_off[lo] <= q < q_off[lo + 1]
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if (q_off[mid] <= q) lo = mid; else hi = mid;
+                    }
+                    const int b = a.sched[s_off[lo]];   // the expert's only block
+                    item = make_int4(lo, j, a.blocks[kBlockInts * b + 1], a.blocks[kBlockInts * b + 2]);
+                }
+                S->items[slot_of(k)] = item;
+                ptx::mbar_arrive(&S->item_full[slot_of(k)]);
+                if (item.x < 0) break;
+            }
+            // the last CTA to finish resets the queue for the next launch
+            __threadfence();
+            if (atomicAdd(&a.queue[1], 1) == (int)gridDim.x - 1) {
+                a.queue[0] = 0;
+                __threadfence();
+                a.queue[1] = 0;
+            }
+        }
+    } else if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        int stage = 0;
+        uint32_t phase = 0;
+        long long fills = 0;
+        bool ok = true;
+        for (int k = 0; ok; ++k) {
+            int4 item;
+            if (!take_item(k, item)) { ok = false; break; }
+            __syncwarp();
+            if (lane == 0) release_item(k);
+            if (item.x < 0) break;
+            const int e = item.x, j = item.y, row0 = item.z;
+            // both halves of the weight tile: FC1 gate rows j*128.. and up rows F + j*128..,
+            // FC2 rows j*256 .. j*256 + 255
+            const int brow0 = e * a.b_rows + j * kColTile;
+            const int brow1 = brow0 + (kFC1 ? a.F : kHalfN);
+            for (int kb = 0; kb < kb_count; ++kb) {
+                if (!role_wait(&S->empty[stage], phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
+                uint8_t* st = base + stage * kSStageBytes;
+                if (lane == 0) {
+                    ptx::mbar_arrive_expect_tx(&S->full[stage], kSStageBytes);
+                    ptx::tma_load_2d(st, &tmA, kb * kBK, row0, &S->full[stage]);
+                    ptx::tma_load_2d(st + kABytes, &tmB, kb * kBK, brow0, &S->full[stage]);
+                    ptx::tma_load_2d(st + kABytes + kBBytes, &tmB, kb * kBK, brow1, &S->full[stage]);
+                }
+                ++fills;
+                if (++stage == kSStages) { stage = 0; phase ^= 1; }
+            }
+        }
+        if (!ok && lane == 0) {
+            const long long first = fills > kSStages ? fills - kSStages : 0;
+            for (long long f = first; f < fills; ++f)
+                ptx::mbar_wait(&S->full[f % kSStages], (uint32_t)((f / kSStages) & 1), kDrainBudget);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc = ptx::idesc_bf16_f32(kBM, kN);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true, issued = false;
+            for (int k = 0; ok; ++k) {
+                int4 item;
+                if (!take_item(k, item)) { ok = false; break; }
+                release_item(k);
+                if (item.x < 0) break;
+                const int acc = k & 1;
+                const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
+                if (!role_wait(&S->acc_empty[acc], acc_phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(acc * kN);
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!role_wait(&S->full[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t a_addr = ptx::smem_addr(base + stage * kSStageBytes);
+                    const uint32_t b_addr = a_addr + kABytes;
+#pragma unroll
+                    for (int ks = 0; ks < kBK / 16; ++ks)
+                        ptx::mma_bf16(d_tmem, ptx::sdesc_k_sw128(a_addr + ks * 32), ptx::sdesc_k_sw128(b_addr + ks * 32),
+                                      idesc, (kb | ks) != 0 ? 1u : 0u);
+                    issued = true;
+                    ptx::mma_commit(&S->empty[stage]);
+                    if (++stage == kSStages) { stage = 0; phase ^= 1; }
+                }
+                if (ok) ptx::mma_commit(&S->acc_full[acc]);
+            }
+            if (!ok && issued) {
+                ptx::mma_commit(&S->drain);
+                ptx::mbar_wait(&S->drain, 0, kDrainBudget);
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue, warps 2..5
+        const int quad = warp & 3;
+        const int m = quad * 32 + lane;
+        uint8_t* stg = epi_base + quad * 2 * kEpiBuf;
+        int buf = 0;
+        for (int k = 0;; ++k) {
+            int4 item;
+            if (!take_item(k, item)) break;
+            __syncwarp();
+            if (lane == 0) release_item(k);
+            if (item.x < 0) break;
+            const int acc = k & 1;
+            const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
+            if (!role_wait(&S->acc_full[acc], acc_phase, a.spin, abort_flag, a.header)) break;
+            ptx::tc_fence_after();
+            epilogue_item<MODE>(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN), lane, quad, stg, buf,
+                                &tmO, &tmP, a.F, item.y, item.z, m >= item.w);
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&S->acc_empty[acc]);
+        }
+        if (lane == 0) ptx::bulk_wait_group<0>();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        ptx::tc_fence_after();
+        ptx::tmem_dealloc(tmem, kTmemCols);
+    }
+    // this kernel may start while the pair kernel before it still runs (it only
+    // fills SMs that kernel has left); it completes after that kernel, so the
+    // launches after both see every row of the output
+    ptx::griddep_wait();
+}
+
 // One CTA waits, through the same bounded wait as the GEMM's roles, on an
 // mbarrier no thread ever arrives on; when the wait runs out it reports
 // MOE_DEV_TIMEOUT in *status and returns.
@@ -455,14 +703,37 @@ __global__ void bounded_wait_probe_kernel(uint32_t* status, long long budget) {
     if (threadIdx.x == 0) role_wait(&never, 0, budget, &abort_flag, status);
 }
 
+// The pair kernel, then (except for the gathered FC1, whose pairs keep every
+// block) the single-CTA kernel over the one-block experts, with its own
+// queue words, launched to take SMs as the pair kernel's CTAs finish.
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const CUtensorMap& tP,
-                        const TcArgs& a, int grid, cudaStream_t st) {
+                        TcArgs a, int grid, cudaStream_t st, int32_t* single_queue) {
+    constexpr bool kSingles = MODE != 2;
+    a.lone_apart = kSingles ? 1 : 0;
     cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)kSmemBytes);
     if (err != cudaSuccess) return err;
     ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, tP, a);
-    return cudaGetLastError();
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if constexpr (kSingles) {
+        err = cudaFuncSetAttribute(ffn_tc_single_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)kSSmemBytes);
+        if (err != cudaSuccess) return err;
+        a.queue = single_queue;
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(grid);
+        lc.blockDim = dim3(kThreads);
+        lc.dynamicSmemBytes = kSSmemBytes;
+        lc.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+        err = cudaLaunchKernelEx(&lc, ffn_tc_single_kernel<MODE>, tA, tB, tO, tP, a);
+    }
+    return err;
 }
 
 }  // namespace
@@ -487,7 +758,6 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.header = ws.header;
     a.queue = ws.gemm_q + (which == 2 ? 4 : 0);
     a.src_of = ws.src_of;
-    a.out = static_cast<__nv_bfloat16*>(out);
     CUtensorMap tA, tB, tO, tP;
     if (which == 3) {
         // FC1 + SwiGLU with A gathered from x [T, d] by the row map -> h [rows_cap, F]
@@ -495,12 +765,11 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
             !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
             !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap))
             return cudaErrorInvalidValue;
-        a.out_ld = s.F;
         a.Kdim = s.d;
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<2>(tA, tB, tO, tO, a, sms, st);
+        return launch_mode<2>(tA, tB, tO, tO, a, sms, st, nullptr);
     }
     if (which == 4) {
         // FC1 + SwiGLU -> h [rows_cap, F], and the pre-activations -> preact [rows_cap, 2F]
@@ -509,12 +778,11 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
             !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap) ||
             !make_tmap_out(&tP, preact, (uint64_t)2 * s.F, (uint64_t)s.rows_cap))
             return cudaErrorInvalidValue;
-        a.out_ld = s.F;
         a.Kdim = s.d;
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<3>(tA, tB, tO, tP, a, sms, st);
+        return launch_mode<3>(tA, tB, tO, tP, a, sms, st, ws.gemm_q + 8);
     }
     if (which == 1) {
         // FC1 + SwiGLU: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h [rows_cap, F]
@@ -522,24 +790,22 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
             !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
             !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap))
             return cudaErrorInvalidValue;
-        a.out_ld = s.F;
         a.Kdim = s.d;
         a.n_tiles = s.F / 128;
         a.F = s.F;
         a.b_rows = 2 * s.F;
-        return launch_mode<0>(tA, tB, tO, tO, a, sms, st);
+        return launch_mode<0>(tA, tB, tO, tO, a, sms, st, ws.gemm_q + 8);
     }
     // FC2: h [rows_cap, F] x w_down [E*d, F] -> yp [rows_cap, d]
     if (!make_tmap(&tA, a_mat, (uint64_t)s.F, (uint64_t)s.rows_cap, kBM) ||
         !make_tmap(&tB, w, (uint64_t)s.F, (uint64_t)s.E * s.d, kHalfN) ||
         !make_tmap_out(&tO, out, (uint64_t)s.d, (uint64_t)s.rows_cap))
         return cudaErrorInvalidValue;
-    a.out_ld = s.d;
     a.Kdim = s.F;
     a.n_tiles = s.d / 256;
     a.F = 0;
     a.b_rows = s.d;
-    return launch_mode<1>(tA, tB, tO, tO, a, sms, st);
+    return launch_mode<1>(tA, tB, tO, tO, a, sms, st, ws.gemm_q + 8);
 }
 
 }  // namespace moe
