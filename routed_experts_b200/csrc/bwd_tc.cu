@@ -315,10 +315,25 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             if (item.x < 0) break;
             const int acc = k & 1;
             const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
+            const int j = item.y;
+            // MODE 0: this row's pre-activations (gate at column f, up at F + f) are loaded a
+            // chunk ahead of their use, the first chunk before the accumulator is ready
+            uint4 av[4], gv[4];
+            const __nv_bfloat16* ag_row = nullptr;
+            if (MODE == 0) {
+                const int row0 = even ? item.z : item.w;
+                if (row0 >= 0) {
+                    ag_row = a.ag + (int64_t)(row0 + m) * 2 * a.F + j * kN;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        av[q] = __ldg(reinterpret_cast<const uint4*>(ag_row) + q);
+                        gv[q] = __ldg(reinterpret_cast<const uint4*>(ag_row + a.F) + q);
+                    }
+                }
+            }
             if (!role_wait(&S->acc_full[acc], acc_phase, a.spin, abort_flag, a.header)) break;
             ptx::tc_fence_after();
             const uint32_t t_row = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN);
-            const int j = item.y;
             if (kWgrad) {
                 // fp32 gradient rows: expert e's row block of this CTA, 16-column stores
                 const bool empty = item.w == 0;   // no rows routed to the expert: zero gradient
@@ -364,11 +379,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                         if (MODE == 0) {
                             // SwiGLU derivative with this row's pre-activations a (gate) and g (up)
                             const int f0 = j * kN + c;
-                            const uint4* ap = reinterpret_cast<const uint4*>(a.ag + (int64_t)(row0 + m) * 2 * a.F + f0);
-                            const uint4* gp = reinterpret_cast<const uint4*>(a.ag + (int64_t)(row0 + m) * 2 * a.F + a.F + f0);
-                            uint4 av[4], gv[4];
+                            uint4 an[4], gn[4];
+                            if (c + 32 < kN) {
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) { av[q] = __ldg(ap + q); gv[q] = __ldg(gp + q); }
+                                for (int q = 0; q < 4; ++q) {
+                                    an[q] = __ldg(reinterpret_cast<const uint4*>(ag_row + c + 32) + q);
+                                    gn[q] = __ldg(reinterpret_cast<const uint4*>(ag_row + a.F + c + 32) + q);
+                                }
+                            }
                             const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(av);
                             const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(gv);
                             uint32_t pa[16], pg[16];
@@ -399,6 +417,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                                 ptx::tma_store_2d(&tmO, stg + kEpiBuf, a.F + f0, row0 + quad * 32);
                                 ptx::bulk_commit_group();
                             }
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) { av[q] = an[q]; gv[q] = gn[q]; }
                         } else {
                             uint32_t pk[16];
 #pragma unroll
