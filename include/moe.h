@@ -210,6 +210,21 @@ moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_do
                           size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_expert_ffn_fused - moe_expert_ffn in one persistent launch (bf16
+ * layers; fp32 returns MOE_ERR_UNSUPPORTED): the work list holds all FC1
+ * tiles, then all FC2 tiles, and an FC2 tile of a block pair starts once
+ * every FC1 tile of that pair is in memory ([MegaFlux] §2.1 and §3.2
+ * "Forward": FC2 waits only for the activation block it needs). The pair's
+ * readiness is a count in the workspace, raised with a release by each
+ * epilogue warp after its stores and read with an acquire by the scheduler;
+ * the wait is bounded and reports MOE_DEV_TIMEOUT. Same arguments, outputs
+ * and rounding as moe_expert_ffn (one-block experts run on a CTA pair beside
+ * an empty half here).
+ */
+moe_status moe_expert_ffn_fused(const moe_config* cfg, const void* xp, const void* w_gate_up, const void* w_down,
+                                void* h, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_expert_fc1_gather - steps A6 and A7 in one pass (bf16 layers only):
  * FC1 + SwiGLU whose activation rows are gathered straight from x [T, d]
  * (device) through the plan's row map, so no xp buffer is written or read

@@ -42,7 +42,7 @@ struct Shape {
 // Byte offsets of every array in a workspace.
 struct WsLayout {
     int64_t header, chunk_counts, chunk_base, chunk_flags, pieces, exp_piece_off, exp_piece_idx,
-        blocks, sched_off, sched, rank_load, rank_replicas, rank_row0, row_of, src_of, gemm_q;
+        blocks, sched_off, sched, rank_load, rank_replicas, rank_row0, row_of, src_of, gemm_q, pair_ready;
     int64_t plan_end;
     // MOE_WS_LAYER extras
     int64_t idx, w, counts, xp, h, yp;
@@ -56,6 +56,9 @@ struct WsLayout {
 };
 
 __host__ __device__ inline int64_t align_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+// Upper bound on block pairs: every expert's pairs are ceil(blocks / 2).
+inline int64_t max_pairs(const Shape& s) { return (s.max_blocks + s.E) / 2 + 1; }
 
 // Device pointers into a workspace, passed by value to kernels.
 struct WsPtrs {
@@ -75,6 +78,7 @@ struct WsPtrs {
     int32_t* row_of;
     int32_t* src_of;
     int32_t* gemm_q;     // [kGemmQWords] work-queue counters of the two GEMM launches
+    int32_t* pair_ready; // [max_pairs] fused FFN: FC1 tiles stored per block pair
 };
 
 inline WsPtrs ws_ptrs(void* ws, const WsLayout& L) {
@@ -96,6 +100,7 @@ inline WsPtrs ws_ptrs(void* ws, const WsLayout& L) {
     p.row_of = reinterpret_cast<int32_t*>(b + L.row_of);
     p.src_of = reinterpret_cast<int32_t*>(b + L.src_of);
     p.gemm_q = reinterpret_cast<int32_t*>(b + L.gemm_q);
+    p.pair_ready = reinterpret_cast<int32_t*>(b + L.pair_ready);
     return p;
 }
 
@@ -129,6 +134,9 @@ cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const 
 cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact = nullptr);
+// FC1 then FC2 in one launch (bf16): h and yp as launch_ffn_tc's which = 1 and 2
+cudaError_t launch_ffn_fused(const Shape& s, const void* xp, const void* w_gate_up, const void* w_down, void* h,
+                             void* yp, const WsPtrs& ws, cudaStream_t st, long long spin_budget);
 // backward (bf16): mode 0 DGrad W2 + SwiGLU derivative (a_mat = dY, b_mat = w_down, ag, out = dAG),
 // 1 DGrad W1 (a_mat = dAG, b_mat = w_gate_up, out = dXp), 2 WGrad W2 (a_mat = dY, b_mat = h,
 // out = dW2 fp32), 3 WGrad W1 (a_mat = dAG, b_mat = xp, out = dW1 fp32)

@@ -82,6 +82,10 @@ struct TcArgs {
     uint32_t* header;
     int32_t* queue;           // [3]: head of queue 0, head of queue 1, clusters finished
     int lone_apart;           // 1: experts with a single block are left to the single-CTA kernel
+    // fused FFN (MODE 4): FC2's contraction length, column tiles and weight rows per expert, and
+    // the per-pair counts of FC1 tiles stored
+    int Kdim2, n_tiles2, b_rows2;
+    int32_t* ready;
 };
 
 // The epilogue of one work item for one warp (rows 32*quad .. 32*quad+31 of
@@ -166,11 +170,19 @@ __device__ __forceinline__ void epilogue_item(uint32_t t_row, int lane, int quad
 // MODE 0: FC1 + SwiGLU -> h (A = xp); MODE 1: FC2 -> yp (A = h);
 // MODE 2: FC1 + SwiGLU -> h with A gathered from x;
 // MODE 3: FC1 + SwiGLU -> h, also storing the pre-activations [gate | up]
-// (rounded to bf16) for the backward's SwiGLU derivative (training forward).
+// (rounded to bf16) for the backward's SwiGLU derivative (training forward);
+// MODE 4: FC1 and FC2 in one launch (fused FFN): the work list holds every
+// FC1 item, then every FC2 item (per half of the GPU); the scheduler hands
+// out an FC2 item of a block pair only once all FC1 column tiles of that pair
+// are stored (a per-pair count each epilogue warp raises with a release add
+// after its TMA stores complete; bounded wait, acquire), so FC2 reads h while
+// it is still in L2. tmA2 / tmB2 / tmO2 are FC2's operands and output.
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-              const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmP, TcArgs a) {
+              const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmP,
+              const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
+              const __grid_constant__ CUtensorMap tmO2, TcArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_base = base + kStages * kStageBytes;
@@ -222,6 +234,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::prefetch_tmap(&tmB);
         ptx::prefetch_tmap(&tmO);
         if (MODE == 3) ptx::prefetch_tmap(&tmP);
+        if (MODE == 4) { ptx::prefetch_tmap(&tmA2); ptx::prefetch_tmap(&tmB2); ptx::prefetch_tmap(&tmO2); }
     }
     __syncthreads();
     ptx::cluster_sync();   // the peer's barriers exist before any remote arrive, store or copy
@@ -230,11 +243,12 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    const int n_items = p_off[a.E] * a.n_tiles;
+    constexpr bool kFused = MODE == 4;
+    const int n_items = p_off[a.E] * (a.n_tiles + (kFused ? a.n_tiles2 : 0));
     const int kb_count = a.Kdim / kBK;
-    constexpr bool kFC1 = MODE != 1;
     constexpr bool kGather = MODE == 2;
-    constexpr int kColTile = kFC1 ? 128 : 256;
+    // an item's phase (fused FFN: FC2 items carry it in the column field's bit 16)
+    auto is_fc2 = [&](const int4& item) { return kFused ? (item.y >> 16) != 0 : MODE == 1; };
 
     // the ring slot of the k-th item, and the parity of its phase
     auto slot_of = [](int k) { return k % kItemSlots; };
@@ -262,18 +276,50 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const int mid = (lo + hi) >> 1;
                 if (p_off[mid] < half) lo = mid + 1; else hi = mid;
             }
-            const int split = p_off[lo] * a.n_tiles;
+            const int n_t = a.n_tiles + (kFused ? a.n_tiles2 : 0);   // items per block pair
+            const int split = p_off[lo] * n_t;
             int next = lane == 0 ? fetch_item(a.queue, g, split, n_items) : 0;
             for (int k = 0;; ++k) {
-                const bool ok = role_wait_cluster(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
+                bool ok = role_wait_cluster(&S->item_empty[slot_of(k)], parity_of(k) ^ 1, a.spin, abort_flag, a.header);
                 int4 item = make_int4(-1, 0, -1, -1);
                 uint32_t valid = 0;
+                int pair = 0;
                 if (lane == 0 && ok && next >= 0) {
                     int e, b0, b1, j;
-                    decode_item(next, a.n_tiles, s_off, p_off, a.E, a.sched, e, b0, b1, j);
-                    item = make_int4(e, j, a.blocks[kBlockInts * b0 + 1], b1 >= 0 ? a.blocks[kBlockInts * b1 + 1] : -1);
-                    valid = (uint32_t)a.blocks[kBlockInts * b0 + 2] |
-                            (b1 >= 0 ? (uint32_t)a.blocks[kBlockInts * b1 + 2] << 16 : 0u);
+                    bool fc2 = false;
+                    if (kFused) {
+                        // this half's FC1 items, then its FC2 items
+                        const int pb = next < split ? 0 : p_off[lo];              // first pair of the half
+                        const int np = next < split ? p_off[lo] : p_off[a.E] - p_off[lo];
+                        const int local = next < split ? next : next - split;
+                        fc2 = local >= np * a.n_tiles;
+                        const int idx = fc2 ? pb * a.n_tiles2 + (local - np * a.n_tiles) : pb * a.n_tiles + local;
+                        decode_item(idx, fc2 ? a.n_tiles2 : a.n_tiles, s_off, p_off, a.E, a.sched, e, b0, b1, j, &pair);
+                        if (fc2) {
+                            // every FC1 tile of this pair stored (8 epilogue warps per FC1 item)
+                            const int target = 8 * a.n_tiles;
+                            const long long t0 = clock64();
+                            while (ptx::ld_acquire_gpu(a.ready + pair) < target) {
+                                if (*abort_flag) { ok = false; break; }
+                                if (clock64() - t0 > a.spin) {
+                                    *abort_flag = 1;
+                                    atomicOr(a.header + H_STATUS, (uint32_t)MOE_DEV_TIMEOUT);
+                                    ok = false;
+                                    break;
+                                }
+                                __nanosleep(128);
+                            }
+                            ptx::fence_proxy_async_global();
+                        }
+                    } else {
+                        decode_item(next, a.n_tiles, s_off, p_off, a.E, a.sched, e, b0, b1, j);
+                    }
+                    if (ok) {
+                        item = make_int4(e, j | (fc2 ? 0x10000 : 0), a.blocks[kBlockInts * b0 + 1],
+                                         b1 >= 0 ? a.blocks[kBlockInts * b1 + 1] : -1);
+                        valid = (uint32_t)a.blocks[kBlockInts * b0 + 2] |
+                                (b1 >= 0 ? (uint32_t)a.blocks[kBlockInts * b1 + 2] << 16 : 0u);
+                    }
                 }
                 item.x = __shfl_sync(0xffffffffu, item.x, 0);
                 item.y = __shfl_sync(0xffffffffu, item.y, 0);
@@ -301,9 +347,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     // publish to both CTAs
                     S->items[slot_of(k)] = item;
                     S->valid[slot_of(k)] = valid;
+                    S->pair_idx[slot_of(k)] = pair;
                     const uint32_t peer = ptx::map_to_rank(ptx::smem_addr(&S->items[slot_of(k)]), 1);
                     ptx::st_cluster_v4(peer, item);
                     ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_addr(&S->valid[slot_of(k)]), 1), valid);
+                    if (kFused)
+                        ptx::st_cluster_u32(ptx::map_to_rank(ptx::smem_addr(&S->pair_idx[slot_of(k)]), 1),
+                                            (uint32_t)pair);
                     ptx::mbar_arrive(&S->item_full[slot_of(k)]);
                     ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->item_full[slot_of(k)]), 1));
                 }
@@ -317,6 +367,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (done == (int)ptx::cluster_count_x() - 1) {
                     a.queue[0] = 0;
                     a.queue[1] = 0;
+                    if (kFused)   // every FC2 item was handed out, so every count is final
+                        for (int q = 0; q < p_off[a.E]; ++q) a.ready[q] = 0;
                     __threadfence();
                     a.queue[2] = 0;
                 }
@@ -346,17 +398,23 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             __syncwarp();
             if (lane == 0) release_item(k);
             if (item.x < 0) break;
-            const int e = item.x, j = item.y;
+            const int e = item.x, j = item.y & 0xffff;
+            const bool fc2 = is_fc2(item);
             const int row0 = even ? item.z : (item.w >= 0 ? item.w : item.z);
-            const int brow = e * a.b_rows + j * kColTile + (even ? 0 : (kFC1 ? a.F : kHalfN));
-            for (int kb = 0; kb < kb_count; ++kb) {
+            const int brow = fc2 ? e * (kFused ? a.b_rows2 : a.b_rows) + j * kN + (even ? 0 : kHalfN)
+                                 : e * a.b_rows + j * 128 + (even ? 0 : a.F);
+            const CUtensorMap* mA = (kFused && fc2) ? &tmA2 : &tmA;
+            const CUtensorMap* mB = (kFused && fc2) ? &tmB2 : &tmB;
+            const int kbc = (kFused && fc2) ? a.Kdim2 / kBK : kb_count;
+            if (kFused && fc2) ptx::fence_proxy_async_global();   // h was stored by other CTAs' TMA
+            for (int kb = 0; kb < kbc; ++kb) {
                 if (!role_wait(&S->empty[stage], phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
                 const uint32_t bar = ptx::map_to_rank(ptx::smem_addr(&S->full[stage]), 0);
                 uint8_t* st = base + stage * kStageBytes;
                 if (lane == 0) {
                     if (even) ptx::mbar_arrive_expect_tx(&S->full[stage], 2 * kStageBytes);
-                    if (!kGather) ptx::tma_load_2d_pair(st, &tmA, kb * kBK, row0, bar);
-                    ptx::tma_load_2d_pair(st + kABytes, &tmB, kb * kBK, brow, bar);
+                    if (!kGather) ptx::tma_load_2d_pair(st, mA, kb * kBK, row0, bar);
+                    ptx::tma_load_2d_pair(st + kABytes, mB, kb * kBK, brow, bar);
                 }
                 if (kGather) ptx::tma_gather4_pair(st + 4 * 128 * lane, &tmA, kb * kBK, tok.x, tok.y, tok.z, tok.w, bar);
                 ++fills;
@@ -381,12 +439,13 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (!take_item(k, item)) { ok = false; break; }
                 release_item(k);
                 if (item.x < 0) break;
+                const int kbc = (kFused && is_fc2(item)) ? a.Kdim2 / kBK : kb_count;
                 const int acc = k & 1;
                 const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
                 if (!role_wait_cluster(&S->acc_empty[acc], acc_phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * kN);
-                for (int kb = 0; kb < kb_count; ++kb) {
+                for (int kb = 0; kb < kbc; ++kb) {
                     if (!role_wait(&S->full[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t a_addr = ptx::smem_addr(base + stage * kStageBytes);
@@ -424,10 +483,12 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             int4 item;
             if (!take_item(k, item)) break;
             const uint32_t vv = S->valid[slot_of(k)];
+            const int pidx = S->pair_idx[slot_of(k)];
             __syncwarp();
             if (lane == 0) release_item(k);
             if (item.x < 0) break;
-            const int j = item.y;
+            const int j = item.y & 0xffff;
+            const bool fc2 = is_fc2(item);
             // rows of the block past its valid ones are padding: written as zero
             const bool pad = m >= (int)(even ? (vv & 0xffffu) : (vv >> 16));
             const int row0 = even ? item.z : item.w;   // -1: this CTA's half of the pair is empty
@@ -435,9 +496,20 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
             if (!role_wait(&S->acc_full[acc], acc_phase, a.spin, abort_flag, a.header)) break;
             ptx::tc_fence_after();
-            if (row0 >= 0)
-                epilogue_item<MODE>(tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN), lane, quad, stg, buf,
-                                    &tmO, &tmP, a.F, j, row0, pad);
+            const uint32_t t_acc = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kN);
+            if (!kFused) {
+                if (row0 >= 0) epilogue_item<MODE>(t_acc, lane, quad, stg, buf, &tmO, &tmP, a.F, j, row0, pad);
+            } else if (fc2) {
+                if (row0 >= 0) epilogue_item<1>(t_acc, lane, quad, stg, buf, &tmO2, &tmO2, a.F, j, row0, pad);
+            } else {
+                if (row0 >= 0) epilogue_item<0>(t_acc, lane, quad, stg, buf, &tmO, &tmO, a.F, j, row0, pad);
+                // this warp's rows of the FC1 tile are in memory: count them for the pair
+                if (lane == 0) {
+                    ptx::bulk_wait_group<0>();
+                    ptx::fence_proxy_async_global();
+                    ptx::red_release_gpu_add(a.ready + pidx, 1);
+                }
+            }
             ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -708,13 +780,17 @@ __global__ void bounded_wait_probe_kernel(uint32_t* status, long long budget) {
 // queue words, launched to take SMs as the pair kernel's CTAs finish.
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const CUtensorMap& tP,
-                        TcArgs a, int grid, cudaStream_t st, int32_t* single_queue) {
-    constexpr bool kSingles = MODE != 2;
+                        TcArgs a, int grid, cudaStream_t st, int32_t* single_queue,
+                        const CUtensorMap* t2 = nullptr) {
+    constexpr bool kSingles = MODE != 2 && MODE != 4;
     a.lone_apart = kSingles ? 1 : 0;
     cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)kSmemBytes);
     if (err != cudaSuccess) return err;
-    ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, tP, a);
+    const CUtensorMap& tA2 = t2 ? t2[0] : tA;
+    const CUtensorMap& tB2 = t2 ? t2[1] : tB;
+    const CUtensorMap& tO2 = t2 ? t2[2] : tO;
+    ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, tP, tA2, tB2, tO2, a);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     if constexpr (kSingles) {
         err = cudaFuncSetAttribute(ffn_tc_single_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -806,6 +882,41 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.F = 0;
     a.b_rows = s.d;
     return launch_mode<1>(tA, tB, tO, tO, a, sms, st, ws.gemm_q + 8);
+}
+
+cudaError_t launch_ffn_fused(const Shape& s, const void* xp, const void* w_gate_up, const void* w_down, void* h,
+                             void* yp, const WsPtrs& ws, cudaStream_t st, long long spin_budget) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    sms &= ~1;
+    TcArgs a{};
+    a.E = s.E;
+    a.spin = spin_budget;
+    a.blocks = ws.blocks;
+    a.sched = ws.sched;
+    a.sched_off = ws.sched_off;
+    a.header = ws.header;
+    a.queue = ws.gemm_q;
+    a.src_of = ws.src_of;
+    a.ready = ws.pair_ready;
+    // FC1: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h; FC2: h [rows_cap, F] x w_down [E*d, F] -> yp
+    CUtensorMap tA, tB, tO, t2[3];
+    if (!make_tmap(&tA, xp, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
+        !make_tmap(&tB, w_gate_up, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
+        !make_tmap_out(&tO, h, (uint64_t)s.F, (uint64_t)s.rows_cap) ||
+        !make_tmap(&t2[0], h, (uint64_t)s.F, (uint64_t)s.rows_cap, kBM) ||
+        !make_tmap(&t2[1], w_down, (uint64_t)s.F, (uint64_t)s.E * s.d, kHalfN) ||
+        !make_tmap_out(&t2[2], yp, (uint64_t)s.d, (uint64_t)s.rows_cap))
+        return cudaErrorInvalidValue;
+    a.Kdim = s.d;
+    a.n_tiles = s.F / 128;
+    a.F = s.F;
+    a.b_rows = 2 * s.F;
+    a.Kdim2 = s.F;
+    a.n_tiles2 = s.d / kN;
+    a.b_rows2 = s.d;
+    return launch_mode<4>(tA, tB, tO, tO, a, sms, st, nullptr, t2);
 }
 
 }  // namespace moe

@@ -69,6 +69,7 @@ struct PlanArgs {
     int C;
     int max_rep;
     int plan_mode;
+    int max_pairs;   // length of the fused FFN's readiness counters
 };
 
 // ---------------------------------------------------------------- warp helpers
@@ -616,6 +617,7 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
         ws.header[H_CANDIDATE] = a.plan_mode == MOE_PLAN_BLOCKS ? (uint32_t)s_best : 0u;
         for (int q = 0; q < kGemmQWords; ++q) ws.gemm_q[q] = 0;   // fresh GEMM work queues
     }
+    for (int q = tid; q < a.max_pairs; q += blockDim.x) ws.pair_ready[q] = 0;   // and readiness counters
 }
 
 }  // namespace
@@ -631,6 +633,7 @@ cudaError_t launch_plan(const Shape& s, int32_t* counts_out, const WsPtrs& ws, c
     a.C = (int)s.C;
     a.max_rep = s.R * s.budget;
     a.plan_mode = s.plan_mode;
+    a.max_pairs = (int)max_pairs(s);
     size_t smem = sizeof(int32_t) * ((size_t)G * s.E + 3 * s.E + 2 * s.R + 5 * a.max_rep +
                                      5 * (s.E + a.max_rep) + 1 + 32);
     if (s.plan_mode == MOE_PLAN_BLOCKS)

@@ -107,6 +107,21 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Cross-CTA readiness counters in global memory: an add with release and a
+// load with acquire at GPU scope, and the proxy fence that orders the async
+// proxy's global accesses (TMA) against them.
+__device__ __forceinline__ void red_release_gpu_add(int32_t* p, int32_t v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Programmatic dependent launch: let the next kernel of the stream (launched
 // with programmatic stream serialization) start its CTAs as SMs free up, and
 // wait for the kernels before this one to complete with their memory visible.

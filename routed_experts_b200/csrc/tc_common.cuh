@@ -40,6 +40,7 @@ struct Smem {
     uint64_t item_full[kItemSlots], item_empty[kItemSlots], fwd_empty[kItemSlots];
     int4 items[kItemSlots];   // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
     uint32_t valid[kItemSlots];   // valid rows of the even CTA's block (low 16 bits) and the odd CTA's (high)
+    int32_t pair_idx[kItemSlots];  // fused FFN: the item's block pair, counting over all experts
     int32_t rows[kItemSlots][kBM];   // gathered FC1: token of each row of this CTA's block
     uint32_t tmem_base;
     int abort_flag;
@@ -101,7 +102,8 @@ __device__ __forceinline__ int fetch_item(int32_t* queue, int g, int split, int 
 // [n_tiles*p_off[e], n_tiles*p_off[e+1]), column tile major, then its block
 // pairs in schedule order; b1 = -1 when the pair has one block.
 __device__ __forceinline__ void decode_item(long long it, int n_tiles, const int32_t* s_off, const int32_t* p_off,
-                                            int E, const int32_t* sched, int& e, int& b0, int& b1, int& j) {
+                                            int E, const int32_t* sched, int& e, int& b0, int& b1, int& j,
+                                            int* pair = nullptr) {
     int lo = 0, hi = E;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
@@ -115,6 +117,7 @@ __device__ __forceinline__ void decode_item(long long it, int n_tiles, const int
     e = lo;
     b0 = sched[s_off[lo] + 2 * q];
     b1 = 2 * q + 1 < nb ? sched[s_off[lo] + 2 * q + 1] : -1;
+    if (pair) *pair = p_off[lo] + q;
 }
 
 // silu(a) = a / (1 + e^-a) with the fast reciprocal-based divide (the IEEE

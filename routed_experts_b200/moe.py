@@ -58,6 +58,7 @@ def lib() -> ctypes.CDLL:
         L.moe_dispatch.argtypes = [C, P, P, P, S, P]
         L.moe_expert_ffn.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_expert_fc1.argtypes = [C, P, P, P, P, S, P]
+        L.moe_expert_ffn_fused.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_expert_fc2.argtypes = [C, P, P, P, P, S, P]
         L.moe_expert_fc1_gather.argtypes = [C, P, P, P, P, S, P]
         L.moe_combine.argtypes = [C, P, P, P, P, S, P]
@@ -71,7 +72,7 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.argtypes = [ctypes.c_int]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
-                  "moe_expert_ffn", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
+                  "moe_expert_ffn", "moe_expert_ffn_fused", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
                   "moe_layer_fwd", "moe_layer_bwd", "moe_layer_fwd_train",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait"):
             getattr(L, f).restype = ctypes.c_int
@@ -149,6 +150,13 @@ def moe_expert_ffn(c, xp, w_gate_up, w_down, h, yp, ws, stream=None):
     p, n = _ws(ws)
     _check(lib().moe_expert_ffn(ctypes.byref(config(c)), _ptr(xp), _ptr(w_gate_up), _ptr(w_down), _ptr(h),
                                 _ptr(yp), p, n, _stream(stream)), "moe_expert_ffn")
+
+
+def moe_expert_ffn_fused(c, xp, w_gate_up, w_down, h, yp, ws, stream=None):
+    """FC1 and FC2 in one persistent launch (FC2 tiles wait on per-pair readiness counts)."""
+    p, n = _ws(ws)
+    _check(lib().moe_expert_ffn_fused(ctypes.byref(config(c)), _ptr(xp), _ptr(w_gate_up), _ptr(w_down), _ptr(h),
+                                      _ptr(yp), p, n, _stream(stream)), "moe_expert_ffn_fused")
 
 
 def moe_expert_fc1(c, xp, w_gate_up, h, ws, stream=None):
