@@ -207,8 +207,6 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::fence_barrier_init();
     }
     for (int i = threadIdx.x; i <= a.E; i += kThreads) s_off[i] = a.sched_off[i];
-    // the single-CTA kernel that follows may take SMs as this kernel's CTAs leave
-    if (threadIdx.x == 0) ptx::griddep_launch_dependents();
     __syncthreads();
     if (warp == 0) {
         // pair offsets: p_off[e] = sum over e' < e of the pairs of e' (ceil(blocks / 2);
@@ -526,6 +524,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::tc_fence_after();
         ptx::tmem_dealloc_pair(tmem, kTmemCols);
     }
+    // launched as a dependent of the lone-block kernel before it, this kernel may
+    // start while that one runs; it completes only after it, so the launches
+    // that follow see every row of the output (a no-op for a plain launch)
+    ptx::griddep_wait();
 }
 
 // ---------------------------------------------------------------- lone blocks
@@ -580,6 +582,8 @@ ffn_tc_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         ptx::fence_barrier_init();
     }
     for (int i = threadIdx.x; i <= a.E; i += kThreads) s_off[i] = a.sched_off[i];
+    // the pair kernel launched after this one may take every SM this one does not hold
+    if (threadIdx.x == 0) ptx::griddep_launch_dependents();
     __syncthreads();
     if (warp == 0) {
         // q_off[e]: one-block experts before e
@@ -754,10 +758,6 @@ ffn_tc_single_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
-    // this kernel may start while the pair kernel before it still runs (it only
-    // fills SMs that kernel has left); it completes after that kernel, so the
-    // launches after both see every row of the output
-    ptx::griddep_wait();
 }
 
 // One CTA waits, through the same bounded wait as the GEMM's roles, on an
@@ -775,9 +775,11 @@ __global__ void bounded_wait_probe_kernel(uint32_t* status, long long budget) {
     if (threadIdx.x == 0) role_wait(&never, 0, budget, &abort_flag, status);
 }
 
-// The pair kernel, then (except for the gathered FC1, whose pairs keep every
-// block) the single-CTA kernel over the one-block experts, with its own
-// queue words, launched to take SMs as the pair kernel's CTAs finish.
+// The single-CTA kernel over the one-block experts (with its own queue
+// words), then the pair kernel as its programmatic dependent: the lone
+// kernel's CTAs that find no work leave at once and the pair kernel's
+// clusters take their SMs, so the two run side by side. The gathered FC1 and
+// the fused FFN keep every block in pairs and launch the pair kernel alone.
 template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const CUtensorMap& tP,
                         TcArgs a, int grid, cudaStream_t st, int32_t* single_queue,
@@ -790,26 +792,29 @@ cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUte
     const CUtensorMap& tA2 = t2 ? t2[0] : tA;
     const CUtensorMap& tB2 = t2 ? t2[1] : tB;
     const CUtensorMap& tO2 = t2 ? t2[2] : tO;
-    ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, tP, tA2, tB2, tO2, a);
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
-    if constexpr (kSingles) {
+    if constexpr (!kSingles) {
+        ffn_tc_kernel<MODE><<<grid, kThreads, kSmemBytes, st>>>(tA, tB, tO, tP, tA2, tB2, tO2, a);
+        return cudaGetLastError();
+    } else {
         err = cudaFuncSetAttribute(ffn_tc_single_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    (int)kSSmemBytes);
         if (err != cudaSuccess) return err;
-        a.queue = single_queue;
+        TcArgs lone = a;
+        lone.queue = single_queue;
+        ffn_tc_single_kernel<MODE><<<grid, kThreads, kSSmemBytes, st>>>(tA, tB, tO, tP, lone);
+        if ((err = cudaGetLastError()) != cudaSuccess) return err;
         cudaLaunchConfig_t lc = {};
         lc.gridDim = dim3(grid);
         lc.blockDim = dim3(kThreads);
-        lc.dynamicSmemBytes = kSSmemBytes;
+        lc.dynamicSmemBytes = kSmemBytes;
         lc.stream = st;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         lc.attrs = attr;
         lc.numAttrs = 1;
-        err = cudaLaunchKernelEx(&lc, ffn_tc_single_kernel<MODE>, tA, tB, tO, tP, a);
+        return cudaLaunchKernelEx(&lc, ffn_tc_kernel<MODE>, tA, tB, tO, tP, tA2, tB2, tO2, a);
     }
-    return err;
 }
 
 }  // namespace
