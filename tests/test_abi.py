@@ -130,6 +130,20 @@ def test_backward_rejects_unsupported_shapes_bad_pointers_and_small_workspace(M)
             M.MOE_ERR_UNSUPPORTED
 
 
+def test_fused_ffn_checks_its_arguments(M):
+    L = M.lib()
+    fake = ctypes.c_void_p(1 << 20)      # never dereferenced: every check below fails first
+    s = ctypes.c_size_t
+    bf = C.TINY.replace(dtype=C.BF16, tile=128, d=256, F=256)
+    need = M.moe_workspace_size(bf, M.WS_PLAN)
+    cfg = ctypes.byref(M.config(bf))
+    assert L.moe_expert_ffn_fused(cfg, fake, fake, fake, fake, fake, fake, s(need - 1), None) == M.MOE_ERR_WORKSPACE
+    assert L.moe_expert_ffn_fused(cfg, fake, fake, None, fake, fake, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    n = M.moe_workspace_size(C.TINY, M.WS_PLAN)
+    assert L.moe_expert_ffn_fused(ctypes.byref(M.config(C.TINY)), fake, fake, fake, fake, fake, fake, s(n),
+                                  None) == M.MOE_ERR_UNSUPPORTED
+
+
 def test_binding_refuses_to_run_without_library(tmp_path, monkeypatch):
     from routed_experts_b200 import moe
     monkeypatch.setattr(moe, "_lib", None)
