@@ -208,13 +208,15 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ the CUDA path
 
-def plan_comparison(cfg, lg, dev, reps=20):
+def plan_comparison(cfg, inp, dev, reps=20):
     """The planners side by side on the step's routing: exact S*K (the layer's
     planner), MegaFlux's block-granular search, and fixed placement (no
     replica budget). Per mode: moe_plan time (top-k, histogram, planner, row
-    maps; CUDA events), the busiest rank's tiles against the mean (the
-    straggler an expert-parallel layer would wait for), valid entries on the
-    busiest rank, padded rows, replicas, moves."""
+    maps; CUDA events), the whole layer's time with that plan (moe_layer_fwd),
+    the busiest rank's tiles against the mean (the straggler an
+    expert-parallel layer would wait for), valid entries on the busiest rank,
+    padded rows, replicas, moves."""
+    lg = inp["logits"]
     from routed_experts_b200 import moe as M
     out = {}
     T, K, E = cfg.T, cfg.K, cfg.E
@@ -234,7 +236,20 @@ def plan_comparison(cfg, lg, dev, reps=20):
         torch.cuda.synchronize(dev)
         pl = M.read_plan(c, ws)
         tiles = np.diff(pl["rank_row0"].numpy()) // c.tile
+        del ws
+        layer = M.Layer(c, dev)
+        for _ in range(3):
+            layer.forward(lg, inp["x"], inp["w_gate_up"], inp["w_down"])
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        l0.record()
+        for _ in range(reps // 2):
+            layer.forward(lg, inp["x"], inp["w_gate_up"], inp["w_down"])
+        l1.record()
+        torch.cuda.synchronize(dev)
+        del layer
+        torch.cuda.empty_cache()
         out[name] = {"moe_plan_us": 1e3 * e0.elapsed_time(e1) / reps,
+                     "layer_ms": l0.elapsed_time(l1) / (reps // 2),
                      "max_tiles_per_rank": int(tiles.max()), "mean_tiles_per_rank": float(tiles.mean()),
                      "max_entries_per_rank": int(pl["rank_load"].max()), "entries_per_rank_mean": T * K / c.R,
                      "padded_rows": pl["total_rows"] - T * K, "replicas": pl["replicas"], "moves": pl["moves"],
@@ -375,6 +390,7 @@ def run_mine(args, world, rank, local):
         torch.distributed.barrier()
     elapsed_ms = t0.elapsed_time(t1)
     stage_ms = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n_ev - 1)] for e in evs])
+    step_ms = np.array([e[0].elapsed_time(e[n_ev - 1]) for e in evs])   # each step, launch to last stage
     st = M.moe_read_status(ws, stream)
     if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
         raise RuntimeError(f"device status {st} after the timed steps")
@@ -417,18 +433,44 @@ def run_mine(args, world, rank, local):
         layer_h.forward_host(lg_h, x_h, wgu, wdn, out_h, stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1)
+    e2e_serial_ms = e0.elapsed_time(e1)
+
+    # the same calls as a serving loop issues them: two workspaces on two
+    # streams, steps alternating, so one step's copies overlap the other's kernels
+    layers = [layer_h, M.Layer(cfg, dev, host_io=True)]
+    streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
+    outs = [out_h, torch.empty(T, d, dtype=dt).pin_memory()]
+    for k in range(args.warmup):
+        layers[k % 2].forward_host(lg_h, x_h, wgu, wdn, outs[k % 2], streams[k % 2])
     if pg is not None:
         torch.distributed.barrier()
-        elapsed_ms, e2e_ms = max_over_ranks([elapsed_ms, e2e_ms], dev)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for s_ in streams:
+        s_.wait_event(e0)
+    for k in range(args.steps):
+        layers[k % 2].forward_host(lg_h, x_h, wgu, wdn, outs[k % 2], streams[k % 2])
+    for s_ in streams:
+        done = torch.cuda.Event()
+        done.record(s_)
+        stream.wait_event(done)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    for L_ in layers:
+        if L_.status() & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
+            raise RuntimeError("device status after the end-to-end steps")
+    if pg is not None:
+        torch.distributed.barrier()
+        elapsed_ms, e2e_ms, e2e_serial_ms = max_over_ranks([elapsed_ms, e2e_ms, e2e_serial_ms], dev)
 
     bwd = None
     if not args.no_backward and cfg.dtype == C.BF16 and cfg.F % 256 == 0:
-        del layer_h
+        del layer_h, layers
         torch.cuda.empty_cache()
         bwd = time_backward(cfg, inp, args, world, dev, stream, pg)
 
-    plans = plan_comparison(cfg, lg, dev) if rank == 0 else None
+    plans = plan_comparison(cfg, inp, dev) if rank == 0 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(cfg, inp, args.cpu_tokens)
@@ -488,6 +530,8 @@ def run_mine(args, world, rank, local):
                            "peaks": {"bf16_tflops": tensor_peak, "hbm_gbs": pk["hbm_gbs"], "kind": pk_kind}},
         "stages_ms": {"plan(topk+hist+plan+rowmaps)": med[0], "dispatch": med[1], "fc1": med[2], "fc2": med[3],
                       "combine": med[4]},
+        "step_ms": {"median": float(np.median(step_ms)), "min": float(step_ms.min()),
+                    "max": float(step_ms.max())},
         "stage_rates": {"fc1_tflops": fc1_flop / fc1_s / 1e12, "fc2_tflops": fc2_flop / fc2_s / 1e12,
                         "dispatch_gbs": gather_bytes / (mean[1] * 1e-3) / 1e9,
                         "combine_gbs": combine_bytes / (mean[4] * 1e-3) / 1e9},
@@ -496,7 +540,11 @@ def run_mine(args, world, rank, local):
         "planners": plans,
         "e2e": {"value": world * T / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * T * E + T * d * eb, "d2h_bytes_per_step": T * d * eb,
-                "ms_per_step": e2e_ms / args.steps},
+                "ms_per_step": e2e_ms / args.steps,
+                "path": "moe_layer_fwd_host per step (H2D of logits and x from pinned memory, the layer, D2H of "
+                        "out), two workspaces on two streams with steps alternating",
+                "one_stream_value": world * T / (e2e_serial_ms / args.steps * 1e-3),
+                "one_stream_ms_per_step": e2e_serial_ms / args.steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "layer_path": "moe_plan; moe_dispatch; moe_expert_fc1; moe_expert_fc2; moe_combine (the kernels of moe_layer_fwd)",
         "backward": bwd,
