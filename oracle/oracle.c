@@ -1010,3 +1010,184 @@ int orc_bwd_wgrad_elems(int64_t T, int32_t d, int32_t K, int32_t F, int32_t dtyp
 
 /* bf16 rounding exposed for pins of the rounding helper itself */
 uint16_t orc_double_to_bf16(double v) { return double_to_bf16(v); }
+
+/* ================================================= MX (block-scaled) forward
+ * [MegaFlux] §2.1 'Persistent MoE execution': the Blackwell MMA is block
+ * scaled (MXFP8 / MXFP4); §4.1 'Setup': the forward runs with MX operands,
+ * fp32 accumulation and bf16 outputs. [MoonEP] "A bandwidth-only model": an
+ * MX format stores one scale per 32 elements.
+ * READING: the pages name the formats but do not define them; they are read
+ * as the OCP Microscaling formats. A block is 32 consecutive elements along
+ * the contraction dimension; its scale is a power of two X = 2^(s - 127)
+ * stored as the 8-bit exponent s (E8M0); s = floor(log2(max |v|)) - 8 + 127
+ * for MXFP8 with E4M3 elements (8 = the exponent of E4M3's largest normal,
+ * 448 = 1.75 * 2^8), clamped to [0, 254], and s = 0 for an all-zero block;
+ * every element is v / X rounded to E4M3, nearest with ties to even,
+ * saturating at +-448. E4M3: 1 sign bit, 4 exponent bits (bias 7), 3
+ * mantissa bits, subnormals at exponent field 0, code 0x7F / 0xFF is NaN
+ * (never produced from finite input).
+ */
+
+/* The value of an E4M3 code (NaN codes give NaN). */
+static double e4m3_value(uint8_t c)
+{
+    const int sign = c >> 7, ef = (c >> 3) & 15, mf = c & 7;
+    double v;
+    if (ef == 15 && mf == 7) return NAN;
+    if (ef == 0) v = ldexp((double)mf, -9);                 /* subnormal: mf/8 * 2^-6 */
+    else v = ldexp(8.0 + mf, ef - 7 - 3);                  /* (1 + mf/8) * 2^(ef-7) */
+    return sign ? -v : v;
+}
+
+/* v rounded to E4M3: nearest, ties to even, saturating at 448; the sign of
+ * v is kept (a negative value that rounds to zero gives -0, code 0x80). */
+static uint8_t e4m3_encode(double v)
+{
+    const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    const double a = fabs(v);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal range: multiples of 2^-9; a rounding up to 2^-6 gives code 8, the smallest normal */
+        const double q = nearbyint(ldexp(a, 9));
+        return sign | (uint8_t)q;
+    }
+    int ex;
+    frexp(a, &ex);                 /* a = m * 2^ex, m in [0.5, 1) */
+    int e = ex - 1;                /* floor(log2 a), in [-6, 8] */
+    double r = nearbyint(ldexp(a, 3 - e));   /* 1.mmm scaled to [8, 16] */
+    if (r == 16.0) { r = 8.0; ++e; }
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)r - 8));
+}
+
+/* The E8M0 scale exponent of a block whose largest magnitude is amax. */
+static uint8_t mx_scale_code(double amax)
+{
+    if (amax == 0.0) return 0;
+    int ex;
+    frexp(amax, &ex);
+    int s = (ex - 1) - 8 + 127;
+    if (s < 0) s = 0;
+    if (s > 254) s = 254;
+    return (uint8_t)s;
+}
+
+/* Quantize the rows of an fp64 matrix [rows, K] (K a multiple of 32) to
+ * MXFP8: codes [rows, K] and scales [rows, K/32], both row-major. */
+static void mx_quantize_rows(int64_t rows, int32_t K, const double* v, uint8_t* codes, uint8_t* scales)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t b = 0; b < K / 32; ++b) {
+            const double* blk = v + r * K + (int64_t)b * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i)
+                if (fabs(blk[i]) > amax) amax = fabs(blk[i]);
+            const uint8_t s = mx_scale_code(amax);
+            scales[r * (K / 32) + b] = s;
+            const double X = ldexp(1.0, (int)s - 127);
+            for (int i = 0; i < 32; ++i) codes[r * K + (int64_t)b * 32 + i] = e4m3_encode(blk[i] / X);
+        }
+    }
+}
+
+static double mx_value(const uint8_t* codes, const uint8_t* scales, int32_t K, int64_t r, int32_t k)
+{
+    return e4m3_value(codes[r * K + k]) * ldexp(1.0, (int)scales[r * (K / 32) + k / 32] - 127);
+}
+
+/* MXFP8 quantization of a bf16 or fp32 matrix [rows, K]. */
+int orc_mx_quantize(int64_t rows, int32_t K, int32_t dtype, const void* x, uint8_t* codes, uint8_t* scales)
+{
+    if (K % 32 != 0) return ORC_ERR_ARG;
+    double* row = (double*)malloc(sizeof(double) * (size_t)K);
+    if (!row) return ORC_ERR_INTERNAL;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t k = 0; k < K; ++k) row[k] = load_elem(x, r * K + k, dtype);
+        mx_quantize_rows(1, K, row, codes + r * K, scales + r * (K / 32));
+    }
+    free(row);
+    return ORC_OK;
+}
+
+/* The values an MXFP8 matrix stands for, in fp64. */
+int orc_mx_dequantize(int64_t rows, int32_t K, const uint8_t* codes, const uint8_t* scales, double* out)
+{
+    if (K % 32 != 0) return ORC_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t k = 0; k < K; ++k) out[r * K + k] = mx_value(codes, scales, K, r, k);
+    return ORC_OK;
+}
+
+/* E4M3 codes <-> values, for the pins. */
+uint8_t orc_e4m3_encode(double v) { return e4m3_encode(v); }
+double orc_e4m3_value(uint8_t c) { return e4m3_value(c); }
+uint8_t orc_mx_scale_code(double amax) { return mx_scale_code(amax); }
+
+/* One routed entry of the MX expert FFN: token row xq (MXFP8 along d) through
+ * expert e. FC1 in fp64 over the dequantized operands (W1 = w_gate_up[e],
+ * MXFP8 along d), SwiGLU, h rounded to bf16 (FC1's bf16 output), then h
+ * quantized to MXFP8 along F (FC2's activation operand); FC2 in fp64 over
+ * dequantized h and W2 = w_down[e] (MXFP8 along F), y rounded to bf16.
+ * READING: FC1 writes bf16 (§4.1: bf16 outputs) and FC2's MXFP8 operand is
+ * quantized from those bf16 values. */
+static void mx_ffn_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* xs, int64_t xrow,
+                       const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s, int32_t e,
+                       double* hb /*[F]*/, uint8_t* hq /*[F]*/, uint8_t* hs /*[F/32]*/, double* y /*[d]*/)
+{
+    const int64_t g0 = (int64_t)e * 2 * F, u0 = g0 + F, dn0 = (int64_t)e * d;
+    for (int32_t j = 0; j < F; ++j) {
+        double a = 0.0, g = 0.0;
+        for (int32_t i = 0; i < d; ++i) {
+            const double xv = mx_value(xq, xs, d, xrow, i);
+            a += xv * mx_value(w1q, w1s, d, g0 + j, i);
+            g += xv * mx_value(w1q, w1s, d, u0 + j, i);
+        }
+        hb[j] = round_as(a / (1.0 + exp(-a)) * g, ORC_ROUND_BF16);
+    }
+    mx_quantize_rows(1, F, hb, hq, hs);
+    for (int32_t i = 0; i < d; ++i) {
+        double s = 0.0;
+        for (int32_t j = 0; j < F; ++j) s += mx_value(hq, hs, F, 0, j) * mx_value(w2q, w2s, F, dn0 + i, j);
+        y[i] = round_as(s, ORC_ROUND_BF16);
+    }
+}
+
+/* Sampled routed entries (token t, expert e) of the MX FFN: h (bf16 values),
+ * its MXFP8 codes and scales, and y (bf16 values). */
+int orc_mx_entry_ffn(int32_t d, int32_t F, int64_t n, const int64_t* tokens, const int32_t* experts,
+                     const uint8_t* xq, const uint8_t* xs, const uint8_t* w1q, const uint8_t* w1s,
+                     const uint8_t* w2q, const uint8_t* w2s, double* h_out /*[n,F]*/, uint8_t* hq_out /*[n,F]*/,
+                     uint8_t* hs_out /*[n,F/32]*/, double* y_out /*[n,d]*/)
+{
+    if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i)
+        mx_ffn_row(d, F, xq, xs, tokens[i], w1q, w1s, w2q, w2s, experts[i], h_out + (size_t)i * F,
+                   hq_out + (size_t)i * F, hs_out + (size_t)i * (F / 32), y_out + (size_t)i * d);
+    return ORC_OK;
+}
+
+/* Sampled tokens of the MX layer: the K entries of token t as above, then
+ * the weighted combine in fp64, rounded to bf16. */
+int orc_mx_token_out(int32_t d, int32_t F, int32_t K, int64_t n_tok, const int64_t* tokens,
+                     const uint8_t* xq, const uint8_t* xs, const int32_t* idx, const float* w,
+                     const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s,
+                     double* out /*[n_tok, d]*/)
+{
+    if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
+    double* hb = (double*)malloc(sizeof(double) * (size_t)F);
+    uint8_t* hq = (uint8_t*)malloc((size_t)F);
+    uint8_t* hs = (uint8_t*)malloc((size_t)F / 32);
+    double* y = (double*)malloc(sizeof(double) * (size_t)d * K);
+    if (!hb || !hq || !hs || !y) { free(hb); free(hq); free(hs); free(y); return ORC_ERR_INTERNAL; }
+    for (int64_t n = 0; n < n_tok; ++n) {
+        const int64_t t = tokens[n];
+        for (int32_t k = 0; k < K; ++k)
+            mx_ffn_row(d, F, xq, xs, t, w1q, w1s, w2q, w2s, idx[t * K + k], hb, hq, hs, y + (size_t)k * d);
+        for (int32_t i = 0; i < d; ++i) {
+            double s = 0.0;
+            for (int32_t k = 0; k < K; ++k) s += (double)w[t * K + k] * y[(size_t)k * d + i];
+            out[n * d + i] = round_as(s, ORC_ROUND_BF16);
+        }
+    }
+    free(hb); free(hq); free(hs); free(y);
+    return ORC_OK;
+}

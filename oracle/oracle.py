@@ -64,6 +64,18 @@ def lib():
         L.orc_bwd_tokens.argtypes = [i32, i32, i32, i32, i32, i32, i32, i64, P, P, P, P, P, P, P, P, P, P, P]
         L.orc_bwd_wgrad_elems.argtypes = [i64, i32, i32, i32, i32, i32, P, P, P, P, P, P, i32, i64, P, P, P, P]
         L.orc_double_to_bf16.restype = ctypes.c_uint16
+        L.orc_mx_quantize.argtypes = [i64, i32, i32, P, P, P]
+        L.orc_mx_dequantize.argtypes = [i64, i32, P, P, P]
+        L.orc_e4m3_encode.argtypes = [ctypes.c_double]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_value.restype = ctypes.c_double
+        L.orc_mx_scale_code.argtypes = [ctypes.c_double]
+        L.orc_mx_scale_code.restype = ctypes.c_uint8
+        L.orc_mx_entry_ffn.argtypes = [i32, i32, i64, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.orc_mx_token_out.argtypes = [i32, i32, i32, i64, P, P, P, P, P, P, P, P, P, P]
+        for f in ("orc_mx_quantize", "orc_mx_dequantize", "orc_mx_entry_ffn", "orc_mx_token_out"):
+            getattr(L, f).restype = ctypes.c_int
         for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_plan_blocks", "orc_row_maps", "orc_dispatch",
                   "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer", "orc_entry_ffn"):
             getattr(L, f).restype = ctypes.c_int
@@ -369,3 +381,79 @@ def timed_sample(logits, x, w_gu, w_down, *, K, R, tile, budget, gating, dtype,
     est = (t1 - t0) + per_tok * T
     return {"routing_s": t1 - t0, "ffn_s_per_token": per_tok, "layer_s_est": est,
             "sample_tokens": int(len(toks)), "measured_s": t2 - t0}
+
+
+# ---------------------------------------------------------------- MX (block-scaled) forward
+
+def e4m3_encode(v: float) -> int:
+    """A value rounded to an E4M3 code (nearest, ties to even, saturating at 448)."""
+    return int(lib().orc_e4m3_encode(float(v)))
+
+
+def e4m3_value(code: int) -> float:
+    return float(lib().orc_e4m3_value(int(code)))
+
+
+def mx_scale_code(amax: float) -> int:
+    """The E8M0 scale exponent of an MXFP8 block whose largest magnitude is amax."""
+    return int(lib().orc_mx_scale_code(float(amax)))
+
+
+def mx_quantize(x: np.ndarray, dtype: int):
+    """MXFP8 quantization of the rows of a [rows, K] matrix (bf16 bits or fp32), 32-element
+    blocks along K: (codes uint8 [rows, K], scale exponents uint8 [rows, K/32])."""
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    _check(lib().orc_mx_quantize(rows, K, dtype, _p(x), _p(codes), _p(scales)), "mx_quantize")
+    return codes, scales
+
+
+def mx_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = codes.shape
+    out = np.empty((rows, K), np.float64)
+    _check(lib().orc_mx_dequantize(rows, K, _p(codes), _p(scales), _p(out)), "mx_dequantize")
+    return out
+
+
+def mx_weights(w_gu: np.ndarray, w_down: np.ndarray, dtype: int):
+    """MXFP8 expert weights: W1 = w_gate_up [E, 2F, d] along d, W2 = w_down [E, d, F] along F."""
+    E, F2, d = w_gu.shape
+    F = F2 // 2
+    w1q, w1s = mx_quantize(np.ascontiguousarray(w_gu).reshape(E * F2, d), dtype)
+    w2q, w2s = mx_quantize(np.ascontiguousarray(w_down).reshape(E * d, F), dtype)
+    return w1q, w1s, w2q, w2s
+
+
+def mx_entry_ffn(tokens, experts, xq, xs, w1q, w1s, w2q, w2s, F: int):
+    """Routed entries of the MX expert FFN: h (bf16 values, fp64 array), h's MXFP8 codes and
+    scales, and y (bf16 values, fp64 array)."""
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    xq, xs, w1q, w1s, w2q, w2s = (np.ascontiguousarray(a, dtype=np.uint8) for a in (xq, xs, w1q, w1s, w2q, w2s))
+    d = xq.shape[1]
+    n = tokens.shape[0]
+    h = np.empty((n, F), np.float64)
+    hq = np.empty((n, F), np.uint8)
+    hs = np.empty((n, F // 32), np.uint8)
+    y = np.empty((n, d), np.float64)
+    _check(lib().orc_mx_entry_ffn(d, F, n, _p(tokens), _p(experts), _p(xq), _p(xs), _p(w1q), _p(w1s), _p(w2q),
+                                  _p(w2s), _p(h), _p(hq), _p(hs), _p(y)), "mx_entry_ffn")
+    return h, hq, hs, y
+
+
+def mx_token_out(tokens, xq, xs, idx, w, w1q, w1s, w2q, w2s, F: int) -> np.ndarray:
+    """Layer output rows (bf16 values, fp64 array) of selected tokens of the MX layer."""
+    tokens = np.ascontiguousarray(tokens, dtype=np.int64)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    xq, xs, w1q, w1s, w2q, w2s = (np.ascontiguousarray(a, dtype=np.uint8) for a in (xq, xs, w1q, w1s, w2q, w2s))
+    d = xq.shape[1]
+    K = idx.shape[1]
+    out = np.empty((tokens.shape[0], d), np.float64)
+    _check(lib().orc_mx_token_out(d, F, K, tokens.shape[0], _p(tokens), _p(xq), _p(xs), _p(idx), _p(w), _p(w1q),
+                                  _p(w1s), _p(w2q), _p(w2s), _p(out)), "mx_token_out")
+    return out
