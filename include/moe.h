@@ -308,6 +308,91 @@ moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void*
                          size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * ---- MXFP8 forward ([MegaFlux] §2.1 'Persistent MoE execution': block-scaled
+ * MX tensor-core MMA; §4.1 'Setup': the forward on MX operands with fp32
+ * accumulation and bf16 outputs; [MoonEP] "A bandwidth-only model": one
+ * scale per 32 elements).
+ *
+ * MXFP8 matrix [rows, K] (K a multiple of 128): codes uint8 [rows, K], one
+ * E4M3 byte per element, row-major; scales uint8, one E8M0 byte per 32
+ * consecutive elements of a row (value 2^(s - 127)), in 512-byte chunks:
+ * chunk (row / 128) * (K / 128) + col / 128 holds the scales of its 128 rows
+ * and four 32-blocks, the scale of row r, block b at byte
+ * 16 * (r % 32) + 4 * ((r % 128) / 32) + b % 4 of the chunk; that is
+ * ceil(rows / 128) * (K / 128) * 512 bytes. Quantization (OCP Microscaling):
+ * s = floor(log2 max|v|) - 8 + 127 clamped to [0, 254] (0 for an all-zero
+ * block), each element v / 2^(s-127) rounded to E4M3, nearest with ties to
+ * even, saturating at +-448.
+ * The MX calls take bf16 layers (cfg->dtype == MOE_BF16, tile 128, d % 256 ==
+ * 0, F % 128 == 0) and return MOE_ERR_UNSUPPORTED for others.
+ */
+enum {
+    MOE_MX_XQ = 0,   /* dispatched token rows: codes [rows_cap, d] */
+    MOE_MX_XS = 1,   /*   and their scales */
+    MOE_MX_HQ = 2,   /* FC1 output h: codes [rows_cap, F] */
+    MOE_MX_HS = 3,   /*   and their scales */
+    MOE_MX_W1Q = 4,  /* W1 codes [E * 2F, d], rows in FC1 tile order (see moe_mx_quantize_weights) */
+    MOE_MX_W1S = 5,  /*   and their scales */
+    MOE_MX_W2Q = 6,  /* W2 codes [E * d, F] */
+    MOE_MX_W2S = 7   /*   and their scales */
+};
+
+/* Bytes of one of the MX buffers above for cfg. */
+moe_status moe_mx_buffer_bytes(const moe_config* cfg, int32_t which, size_t* bytes);
+
+/*
+ * moe_mx_quantize_weights - MXFP8 expert weights, once, ahead of the layers.
+ *   w_gate_up bf16 [E, 2F, d], w_down bf16 [E, d, F] (device): as for moe_layer_fwd.
+ *   w1q, w1s (device, out): W1 along d. Rows are reordered for the MX GEMM's
+ *            FC1 column tiles: row e*2F + 128*t + i holds gate row e*2F +
+ *            64*t + i for i < 64 and up row e*2F + F + 64*t + (i - 64) for
+ *            i >= 64 (t < F/64).
+ *   w2q, w2s (device, out): W2 along F, rows unchanged.
+ * Sizes from moe_mx_buffer_bytes. No workspace; asynchronous on `stream`.
+ */
+moe_status moe_mx_quantize_weights(const moe_config* cfg, const void* w_gate_up, const void* w_down, void* w1q,
+                                   void* w1s, void* w2q, void* w2s, moe_stream_t stream);
+
+/*
+ * moe_dispatch_mx - step A6 with MXFP8 quantization: each token row of x
+ * (bf16 [T, d], device) is quantized along d once and its codes and scales
+ * are stored to the K rows of the plan's row map. Padding rows of xq/xs are
+ * not written. Needs the plan of moe_plan in ws (MOE_WS_PLAN or larger).
+ *   xq, xs (device, out): MOE_MX_XQ / MOE_MX_XS buffers.
+ */
+moe_status moe_dispatch_mx(const moe_config* cfg, const void* x, void* xq, void* xs, const void* ws,
+                           size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_fc1_mx - step A7 on MXFP8 operands: per planned block,
+ * h = silu(xq W1g^T) * (xq W1u^T) with the MMA's fp32 accumulation, rounded to
+ * bf16, then quantized to MXFP8 along F into hq / hs (MOE_MX_HQ / MOE_MX_HS,
+ * device, out). Padding rows of a block get zero codes and scale 0.
+ *   xq, xs: from moe_dispatch_mx; w1q, w1s: from moe_mx_quantize_weights.
+ */
+moe_status moe_expert_fc1_mx(const moe_config* cfg, const void* xq, const void* xs, const void* w1q,
+                             const void* w1s, void* hq, void* hs, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_expert_fc2_mx - step A8 on MXFP8 operands: yp = hq W2^T, fp32
+ * accumulation, stored as bf16 [rows_cap, d] (device, out); padding rows are
+ * zero. hq, hs: from moe_expert_fc1_mx; w2q, w2s: from moe_mx_quantize_weights.
+ */
+moe_status moe_expert_fc2_mx(const moe_config* cfg, const void* hq, const void* hs, const void* w2q,
+                             const void* w2s, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * moe_layer_fwd_mx - the whole layer on MXFP8 expert operands: moe_plan,
+ * moe_dispatch_mx, moe_expert_fc1_mx, moe_expert_fc2_mx and moe_combine, on
+ * a MOE_WS_LAYER workspace (xq/xs live where xp does, hq/hs where h does).
+ *   logits fp32 [T, E], x bf16 [T, d] (device); w1q/w1s/w2q/w2s from
+ *   moe_mx_quantize_weights (device); out bf16 [T, d] (device, out).
+ */
+moe_status moe_layer_fwd_mx(const moe_config* cfg, const float* logits, const void* x, const void* w1q,
+                            const void* w1s, const void* w2q, const void* w2s, void* out, void* ws,
+                            size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_plan_noalloc - moe_plan for callers that cannot allocate device
  * memory. The papers have no counterpart: this is an interface for callers
  * that are handed only their inputs and outputs (a plugin inside another

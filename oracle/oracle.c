@@ -1122,18 +1122,17 @@ uint8_t orc_e4m3_encode(double v) { return e4m3_encode(v); }
 double orc_e4m3_value(uint8_t c) { return e4m3_value(c); }
 uint8_t orc_mx_scale_code(double amax) { return mx_scale_code(amax); }
 
-/* One routed entry of the MX expert FFN: token row xq (MXFP8 along d) through
- * expert e. FC1 in fp64 over the dequantized operands (W1 = w_gate_up[e],
- * MXFP8 along d), SwiGLU, h rounded to bf16 (FC1's bf16 output), then h
- * quantized to MXFP8 along F (FC2's activation operand); FC2 in fp64 over
- * dequantized h and W2 = w_down[e] (MXFP8 along F), y rounded to bf16.
+/* FC1 of one routed entry of the MX expert FFN: token row xq (MXFP8 along
+ * d) through expert e's W1 = w_gate_up[e] (MXFP8 along d), in fp64 over the
+ * dequantized operands, SwiGLU, h rounded to bf16 (FC1's bf16 output), then
+ * h quantized to MXFP8 along F (FC2's activation operand).
  * READING: FC1 writes bf16 (§4.1: bf16 outputs) and FC2's MXFP8 operand is
  * quantized from those bf16 values. */
-static void mx_ffn_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* xs, int64_t xrow,
-                       const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s, int32_t e,
-                       double* hb /*[F]*/, uint8_t* hq /*[F]*/, uint8_t* hs /*[F/32]*/, double* y /*[d]*/)
+static void mx_fc1_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* xs, int64_t xrow,
+                       const uint8_t* w1q, const uint8_t* w1s, int32_t e,
+                       double* hb /*[F]*/, uint8_t* hq /*[F]*/, uint8_t* hs /*[F/32]*/)
 {
-    const int64_t g0 = (int64_t)e * 2 * F, u0 = g0 + F, dn0 = (int64_t)e * d;
+    const int64_t g0 = (int64_t)e * 2 * F, u0 = g0 + F;
     for (int32_t j = 0; j < F; ++j) {
         double a = 0.0, g = 0.0;
         for (int32_t i = 0; i < d; ++i) {
@@ -1144,11 +1143,52 @@ static void mx_ffn_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* x
         hb[j] = round_as(a / (1.0 + exp(-a)) * g, ORC_ROUND_BF16);
     }
     mx_quantize_rows(1, F, hb, hq, hs);
+}
+
+/* FC2 of one routed entry: an MXFP8 row of h (codes hq, scales hs) through
+ * expert e's W2 = w_down[e] (MXFP8 along F), fp64, y rounded to bf16. */
+static void mx_fc2_row(int32_t d, int32_t F, const uint8_t* hq, const uint8_t* hs, const uint8_t* w2q,
+                       const uint8_t* w2s, int32_t e, double* y /*[d]*/)
+{
+    const int64_t dn0 = (int64_t)e * d;
     for (int32_t i = 0; i < d; ++i) {
         double s = 0.0;
         for (int32_t j = 0; j < F; ++j) s += mx_value(hq, hs, F, 0, j) * mx_value(w2q, w2s, F, dn0 + i, j);
         y[i] = round_as(s, ORC_ROUND_BF16);
     }
+}
+
+static void mx_ffn_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* xs, int64_t xrow,
+                       const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s, int32_t e,
+                       double* hb /*[F]*/, uint8_t* hq /*[F]*/, uint8_t* hs /*[F/32]*/, double* y /*[d]*/)
+{
+    mx_fc1_row(d, F, xq, xs, xrow, w1q, w1s, e, hb, hq, hs);
+    mx_fc2_row(d, F, hq, hs, w2q, w2s, e, y);
+}
+
+/* FC1 alone for n rows of an MXFP8 activation matrix (row rows[i], expert
+ * experts[i]): h (bf16 values), its MXFP8 codes and scales. */
+int orc_mx_fc1_rows(int32_t d, int32_t F, int64_t n, const int64_t* rows, const int32_t* experts,
+                    const uint8_t* xq, const uint8_t* xs, const uint8_t* w1q, const uint8_t* w1s,
+                    double* h_out /*[n,F]*/, uint8_t* hq_out /*[n,F]*/, uint8_t* hs_out /*[n,F/32]*/)
+{
+    if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i)
+        mx_fc1_row(d, F, xq, xs, rows[i], w1q, w1s, experts[i], h_out + (size_t)i * F, hq_out + (size_t)i * F,
+                   hs_out + (size_t)i * (F / 32));
+    return ORC_OK;
+}
+
+/* FC2 alone for n MXFP8 rows of h (row i through expert experts[i]): y as
+ * bf16 values. */
+int orc_mx_fc2_rows(int32_t d, int32_t F, int64_t n, const int32_t* experts, const uint8_t* hq,
+                    const uint8_t* hs, const uint8_t* w2q, const uint8_t* w2s, double* y_out /*[n,d]*/)
+{
+    if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i)
+        mx_fc2_row(d, F, hq + (size_t)i * F, hs + (size_t)i * (F / 32), w2q, w2s, experts[i],
+                   y_out + (size_t)i * d);
+    return ORC_OK;
 }
 
 /* Sampled routed entries (token t, expert e) of the MX FFN: h (bf16 values),

@@ -74,7 +74,10 @@ def lib():
         L.orc_mx_scale_code.restype = ctypes.c_uint8
         L.orc_mx_entry_ffn.argtypes = [i32, i32, i64, P, P, P, P, P, P, P, P, P, P, P, P]
         L.orc_mx_token_out.argtypes = [i32, i32, i32, i64, P, P, P, P, P, P, P, P, P, P]
-        for f in ("orc_mx_quantize", "orc_mx_dequantize", "orc_mx_entry_ffn", "orc_mx_token_out"):
+        L.orc_mx_fc1_rows.argtypes = [i32, i32, i64, P, P, P, P, P, P, P, P, P]
+        L.orc_mx_fc2_rows.argtypes = [i32, i32, i64, P, P, P, P, P, P]
+        for f in ("orc_mx_quantize", "orc_mx_dequantize", "orc_mx_entry_ffn", "orc_mx_token_out",
+                  "orc_mx_fc1_rows", "orc_mx_fc2_rows"):
             getattr(L, f).restype = ctypes.c_int
         for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_plan_blocks", "orc_row_maps", "orc_dispatch",
                   "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer", "orc_entry_ffn"):
@@ -457,3 +460,29 @@ def mx_token_out(tokens, xq, xs, idx, w, w1q, w1s, w2q, w2s, F: int) -> np.ndarr
     _check(lib().orc_mx_token_out(d, F, K, tokens.shape[0], _p(tokens), _p(xq), _p(xs), _p(idx), _p(w), _p(w1q),
                                   _p(w1s), _p(w2q), _p(w2s), _p(out)), "mx_token_out")
     return out
+
+
+def mx_fc1_rows(rows, experts, xq, xs, w1q, w1s, F: int):
+    """FC1 of the MX FFN alone for rows of an MXFP8 activation matrix: h (bf16 values, fp64
+    array) and its MXFP8 codes and scales."""
+    rows = np.ascontiguousarray(rows, dtype=np.int64)
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    xq, xs, w1q, w1s = (np.ascontiguousarray(a, dtype=np.uint8) for a in (xq, xs, w1q, w1s))
+    d = xq.shape[1]
+    n = rows.shape[0]
+    h = np.empty((n, F), np.float64)
+    hq = np.empty((n, F), np.uint8)
+    hs = np.empty((n, F // 32), np.uint8)
+    _check(lib().orc_mx_fc1_rows(d, F, n, _p(rows), _p(experts), _p(xq), _p(xs), _p(w1q), _p(w1s), _p(h), _p(hq),
+                                 _p(hs)), "mx_fc1_rows")
+    return h, hq, hs
+
+
+def mx_fc2_rows(experts, hq, hs, w2q, w2s, d: int) -> np.ndarray:
+    """FC2 of the MX FFN alone: MXFP8 rows of h through their experts' W2 (bf16 values, fp64 array)."""
+    experts = np.ascontiguousarray(experts, dtype=np.int32)
+    hq, hs, w2q, w2s = (np.ascontiguousarray(a, dtype=np.uint8) for a in (hq, hs, w2q, w2s))
+    n, F = hq.shape
+    y = np.empty((n, d), np.float64)
+    _check(lib().orc_mx_fc2_rows(d, F, n, _p(experts), _p(hq), _p(hs), _p(w2q), _p(w2s), _p(y)), "mx_fc2_rows")
+    return y

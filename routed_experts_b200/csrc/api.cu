@@ -124,6 +124,27 @@ moe_status ffn_impl(const Shape& s, const WsLayout& L, const void* xp, const voi
     return fc_impl(s, L, 2, h, wdn, yp, ws, st);
 }
 
+moe_status mx_shape(const moe_config* cfg, Shape* s) {
+    moe_status r = make_shape(cfg, s);
+    if (r != MOE_OK) return r;
+    if (s->dtype != MOE_BF16 || s->tile != 128 || s->d % 256 != 0 || s->F % 128 != 0) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int64_t mx_bytes(const Shape& s, int which) {
+    switch (which) {
+        case MOE_MX_XQ: return s.rows_cap * s.d;
+        case MOE_MX_XS: return mx_scale_bytes(s.rows_cap, s.d);
+        case MOE_MX_HQ: return s.rows_cap * s.F;
+        case MOE_MX_HS: return mx_scale_bytes(s.rows_cap, s.F);
+        case MOE_MX_W1Q: return (int64_t)s.E * 2 * s.F * s.d;
+        case MOE_MX_W1S: return mx_scale_bytes((int64_t)s.E * 2 * s.F, s.d);
+        case MOE_MX_W2Q: return (int64_t)s.E * s.d * s.F;
+        case MOE_MX_W2S: return mx_scale_bytes((int64_t)s.E * s.d, s.F);
+    }
+    return -1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -382,6 +403,118 @@ moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void*
     if (e == cudaSuccess) e = launch_bwd_tc(s, 3, dag, xp, dw_gate_up, nullptr, P, st, kSpinBudget);
     if (e == cudaSuccess) e = launch_combine(s, dy, nullptr, dx, P, st);
     if (e == cudaSuccess && dlogits) e = launch_dlogits(s, logits, idx, w, dw, dlogits, st);
+    return from_cuda(e);
+}
+
+moe_status moe_mx_buffer_bytes(const moe_config* cfg, int32_t which, size_t* bytes) {
+    Shape s;
+    moe_status r = mx_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!bytes || which < MOE_MX_XQ || which > MOE_MX_W2S) return MOE_ERR_INVALID_ARG;
+    *bytes = (size_t)mx_bytes(s, which);
+    return MOE_OK;
+}
+
+moe_status moe_mx_quantize_weights(const moe_config* cfg, const void* w_gate_up, const void* w_down, void* w1q,
+                                   void* w1s, void* w2q, void* w2s, moe_stream_t stream) {
+    Shape s;
+    moe_status r = mx_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!w_gate_up || !w_down || !w1q || !w1s || !w2q || !w2s) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(w1q) || !aligned16(w1s) || !aligned16(w2q) ||
+        !aligned16(w2s))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_mx_quantize(w_gate_up, (int64_t)s.E * 2 * s.F, s.d, s.F, static_cast<uint8_t*>(w1q),
+                                       static_cast<uint8_t*>(w1s), st);
+    if (e == cudaSuccess)
+        e = launch_mx_quantize(w_down, (int64_t)s.E * s.d, s.F, 0, static_cast<uint8_t*>(w2q),
+                               static_cast<uint8_t*>(w2s), st);
+    return from_cuda(e);
+}
+
+moe_status moe_dispatch_mx(const moe_config* cfg, const void* x, void* xq, void* xs, const void* ws,
+                           size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = mx_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!x || !xq || !xs || !aligned16(x) || !aligned16(xq) || !aligned16(xs)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(const_cast<void*>(ws), L);
+    return from_cuda(launch_dispatch_mx(s, x, static_cast<uint8_t*>(xq), static_cast<uint8_t*>(xs), P,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status moe_expert_fc1_mx(const moe_config* cfg, const void* xq, const void* xs, const void* w1q,
+                             const void* w1s, void* hq, void* hs, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = mx_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!xq || !xs || !w1q || !w1s || !hq || !hs) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xq) || !aligned16(xs) || !aligned16(w1q) || !aligned16(w1s) || !aligned16(hq) || !aligned16(hs))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(ws, L);
+    return from_cuda(launch_ffn_mx(s, 1, static_cast<const uint8_t*>(xq), static_cast<const uint8_t*>(xs),
+                                   static_cast<const uint8_t*>(w1q), static_cast<const uint8_t*>(w1s), hq,
+                                   static_cast<uint8_t*>(hs), P, reinterpret_cast<cudaStream_t>(stream),
+                                   kSpinBudget));
+}
+
+moe_status moe_expert_fc2_mx(const moe_config* cfg, const void* hq, const void* hs, const void* w2q,
+                             const void* w2s, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = mx_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!hq || !hs || !w2q || !w2s || !yp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(hq) || !aligned16(hs) || !aligned16(w2q) || !aligned16(w2s) || !aligned16(yp))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(ws, L);
+    return from_cuda(launch_ffn_mx(s, 2, static_cast<const uint8_t*>(hq), static_cast<const uint8_t*>(hs),
+                                   static_cast<const uint8_t*>(w2q), static_cast<const uint8_t*>(w2s), yp, nullptr,
+                                   P, reinterpret_cast<cudaStream_t>(stream), kSpinBudget));
+}
+
+moe_status moe_layer_fwd_mx(const moe_config* cfg, const float* logits, const void* x, const void* w1q,
+                            const void* w1s, const void* w2q, const void* w2s, void* out, void* ws,
+                            size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = mx_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!logits || !x || !w1q || !w1s || !w2q || !w2s || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(logits) || !aligned16(x) || !aligned16(w1q) || !aligned16(w1s) || !aligned16(w2q) ||
+        !aligned16(w2s) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.layer_end)) != MOE_OK) return r;
+    // xq | xs in xp's place, hq | hs in h's place
+    const int64_t xs_at = align_up(mx_bytes(s, MOE_MX_XQ), 256), hs_at = align_up(mx_bytes(s, MOE_MX_HQ), 256);
+    if (xs_at + mx_bytes(s, MOE_MX_XS) > L.h - L.xp || hs_at + mx_bytes(s, MOE_MX_HS) > L.yp - L.h)
+        return MOE_ERR_UNSUPPORTED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    char* b = static_cast<char*>(ws);
+    int32_t* idx = reinterpret_cast<int32_t*>(b + L.idx);
+    float* w = reinterpret_cast<float*>(b + L.w);
+    int32_t* counts = reinterpret_cast<int32_t*>(b + L.counts);
+    uint8_t* xq = reinterpret_cast<uint8_t*>(b + L.xp);
+    uint8_t* xs = xq + xs_at;
+    uint8_t* hq = reinterpret_cast<uint8_t*>(b + L.h);
+    uint8_t* hs = hq + hs_at;
+    void* yp = b + L.yp;
+    if ((r = plan_impl(s, L, logits, idx, w, counts, ws, st)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(ws, L);
+    cudaError_t e = launch_dispatch_mx(s, x, xq, xs, P, st);
+    if (e == cudaSuccess)
+        e = launch_ffn_mx(s, 1, xq, xs, static_cast<const uint8_t*>(w1q), static_cast<const uint8_t*>(w1s), hq, hs, P,
+                          st, kSpinBudget);
+    if (e == cudaSuccess)
+        e = launch_ffn_mx(s, 2, hq, hs, static_cast<const uint8_t*>(w2q), static_cast<const uint8_t*>(w2s), yp,
+                          nullptr, P, st, kSpinBudget);
+    if (e == cudaSuccess) e = launch_combine(s, yp, w, out, P, st);
     return from_cuda(e);
 }
 

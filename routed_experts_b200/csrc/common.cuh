@@ -104,6 +104,17 @@ inline WsPtrs ws_ptrs(void* ws, const WsLayout& L) {
     return p;
 }
 
+// MXFP8 scales of a [rows, K] matrix (K a multiple of 128): one E8M0 byte per
+// 32 elements of a row, kept in 512-byte chunks, one per (128-row group,
+// 128-column group), chunk index (row / 128) * (K / 128) + column / 128.
+// Inside a chunk the scale of row r and 32-block b (both taken mod 128 and
+// mod 4) sits at byte 16 * (r % 32) + 4 * (r / 32) + b: 32 lines of 16 bytes,
+// the form in which the tensor cores' scale operand is copied into TMEM.
+__host__ __device__ inline int64_t mx_scale_offset(int64_t row, int64_t kblock, int64_t K) {
+    return ((row >> 7) * (K >> 7) + (kblock >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kblock & 3);
+}
+inline int64_t mx_scale_bytes(int64_t rows, int64_t K) { return (rows + 127) / 128 * (K / 128) * 512; }
+
 __device__ inline void set_status(uint32_t* header, uint32_t bits) {
     atomicOr(header + H_STATUS, bits);
 }
@@ -148,5 +159,20 @@ cudaError_t launch_zero_padding(const Shape& s, void* a, void* b, int64_t row_by
                                 cudaStream_t st);
 cudaError_t launch_dlogits(const Shape& s, const float* logits, const int32_t* idx, const float* w, const float* dw,
                            float* dl, cudaStream_t st);
+// MXFP8: a bf16 [rows, K] matrix to codes [rows, K] and chunked scales; with
+// interleave_F > 0 the rows are those of w_gate_up [E, 2F, K] reordered so
+// that every 128 rows of an expert hold 64 gate rows then the 64 matching up
+// rows (the FC1 column tiles of the MX GEMM).
+cudaError_t launch_mx_quantize(const void* x, int64_t rows, int K, int interleave_F, uint8_t* q, uint8_t* sc,
+                               cudaStream_t st);
+// The dispatch with MXFP8 quantization of each token row on the way.
+cudaError_t launch_dispatch_mx(const Shape& s, const void* x, uint8_t* xq, uint8_t* xs, const WsPtrs& ws,
+                               cudaStream_t st);
+// MX grouped GEMM: which 1 = FC1 + SwiGLU (a = xq/xs, w = W1 in the
+// interleaved MX layout, out = hq, out_sc = hs), 2 = FC2 (a = hq/hs, w = W2,
+// out = yp in bf16, out_sc unused).
+cudaError_t launch_ffn_mx(const Shape& s, int which, const uint8_t* a_q, const uint8_t* a_sc, const uint8_t* w_q,
+                          const uint8_t* w_sc, void* out, uint8_t* out_sc, const WsPtrs& ws, cudaStream_t st,
+                          long long spin_budget);
 
 }  // namespace moe

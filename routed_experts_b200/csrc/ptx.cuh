@@ -356,5 +356,53 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a
     return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
 }
 
+
+// ---- block-scaled (MX) MMA
+
+// Shared-memory descriptor of the scale factors of one k-step: 32 lines of
+// 16 bytes, contiguous (no swizzle, K-major core matrices of 8 lines x 16 B,
+// 128 bytes apart), the source of tmem_cp_sf_pair.
+__device__ __forceinline__ uint64_t sdesc_sf(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr & 0x3FFFF) >> 4);   // start address, 16-byte units
+    d |= (uint64_t)(16 >> 4) << 16;            // leading byte offset (one core matrix wide: unused)
+    d |= (uint64_t)(128 >> 4) << 32;           // stride byte offset: 8 lines x 16 B
+    d |= (uint64_t)1 << 46;                    // descriptor version for sm_100
+    return d;                                  // layout type 0: no swizzle
+}
+
+// Copies 32 lines x 128 bits of scale factors from shared memory into TMEM
+// columns taddr .. taddr+3 of lanes 0-31, repeated in each 32-lane quarter,
+// in both CTAs of the pair (each from its own shared memory).
+__device__ __forceinline__ void tmem_cp_sf_pair(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Instruction descriptor of a block-scaled MMA: E4M3 A and B (K-major),
+// fp32 accumulator, E8M0 scales one per 32 K-elements; a_sf / b_sf pick the
+// byte of the scale word (the 32-element K slice of a 128-deep k-step).
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int M, int N, uint32_t a_sf, uint32_t b_sf) {
+    return (b_sf << 4)                         // B scale byte
+           | (0u << 7)                         // A format: E4M3
+           | (0u << 10)                        // B format: E4M3
+           | ((uint32_t)(N >> 3) << 17)        // N / 8
+           | (1u << 23)                        // scale format: E8M0
+           | ((uint32_t)(M >> 4) << 24)        // M / 16
+           | (a_sf << 29);                     // A scale byte
+}
+
+// One block-scaled MMA over a CTA pair (M = 256, K = 32): D (+)= (A x SFA)
+// (B x SFB)^T, the scales read from TMEM at sfa / sfb (scale byte in bits
+// 30-31, as in the instruction descriptor).
+__device__ __forceinline__ void mma_mx_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+        : "memory");
+}
+
 }  // namespace ptx
 }  // namespace moe

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA = range(5)
 DEV_PLAN_INEXACT, DEV_TIMEOUT, DEV_BAD_INDEX = 1, 2, 4
 WS_PLAN, WS_LAYER, WS_LAYER_HOST, WS_LAYER_TRAIN = 0, 1, 2, 3
+MX_XQ, MX_XS, MX_HQ, MX_HS, MX_W1Q, MX_W1S, MX_W2Q, MX_W2S = range(8)
 
 
 class MoeError(RuntimeError):
@@ -70,11 +71,19 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         L.moe_probe_bounded_wait.argtypes = [P, ctypes.c_int64, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
+        L.moe_mx_buffer_bytes.argtypes = [C, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_mx_quantize_weights.argtypes = [C, P, P, P, P, P, P, P]
+        L.moe_dispatch_mx.argtypes = [C, P, P, P, P, S, P]
+        L.moe_expert_fc1_mx.argtypes = [C, P, P, P, P, P, P, P, S, P]
+        L.moe_expert_fc2_mx.argtypes = [C, P, P, P, P, P, P, S, P]
+        L.moe_layer_fwd_mx.argtypes = [C, P, P, P, P, P, P, P, P, S, P]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_ffn_fused", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
                   "moe_layer_fwd", "moe_layer_bwd", "moe_layer_fwd_train",
-                  "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait"):
+                  "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait",
+                  "moe_mx_buffer_bytes", "moe_mx_quantize_weights", "moe_dispatch_mx", "moe_expert_fc1_mx",
+                  "moe_expert_fc2_mx", "moe_layer_fwd_mx"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -228,6 +237,56 @@ def moe_read_status(ws, stream=None) -> int:
     return v.value
 
 
+# ---------------------------------------------------------------- MXFP8 forward
+
+def moe_mx_buffer_bytes(c, which: int) -> int:
+    v = ctypes.c_size_t(0)
+    _check(lib().moe_mx_buffer_bytes(ctypes.byref(config(c)), int(which), ctypes.byref(v)), "moe_mx_buffer_bytes")
+    return v.value
+
+
+def moe_mx_quantize_weights(c, w_gate_up, w_down, w1q, w1s, w2q, w2s, stream=None):
+    _check(lib().moe_mx_quantize_weights(ctypes.byref(config(c)), _ptr(w_gate_up), _ptr(w_down), _ptr(w1q),
+                                         _ptr(w1s), _ptr(w2q), _ptr(w2s), _stream(stream)), "moe_mx_quantize_weights")
+
+
+def moe_dispatch_mx(c, x, xq, xs, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_dispatch_mx(ctypes.byref(config(c)), _ptr(x), _ptr(xq), _ptr(xs), p, n, _stream(stream)),
+           "moe_dispatch_mx")
+
+
+def moe_expert_fc1_mx(c, xq, xs, w1q, w1s, hq, hs, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_expert_fc1_mx(ctypes.byref(config(c)), _ptr(xq), _ptr(xs), _ptr(w1q), _ptr(w1s), _ptr(hq),
+                                   _ptr(hs), p, n, _stream(stream)), "moe_expert_fc1_mx")
+
+
+def moe_expert_fc2_mx(c, hq, hs, w2q, w2s, yp, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_expert_fc2_mx(ctypes.byref(config(c)), _ptr(hq), _ptr(hs), _ptr(w2q), _ptr(w2s), _ptr(yp),
+                                   p, n, _stream(stream)), "moe_expert_fc2_mx")
+
+
+def moe_layer_fwd_mx(c, logits, x, w1q, w1s, w2q, w2s, out, ws, stream=None):
+    p, n = _ws(ws)
+    _check(lib().moe_layer_fwd_mx(ctypes.byref(config(c)), _ptr(logits), _ptr(x), _ptr(w1q), _ptr(w1s), _ptr(w2q),
+                                  _ptr(w2s), _ptr(out), p, n, _stream(stream)), "moe_layer_fwd_mx")
+
+
+def mx_buffer(c, which: int, device="cuda") -> torch.Tensor:
+    return torch.empty(moe_mx_buffer_bytes(c, which), dtype=torch.uint8, device=device)
+
+
+class MxWeights:
+    """A layer's expert weights in MXFP8, quantized on the device from bf16."""
+
+    def __init__(self, c, w_gate_up, w_down, stream=None):
+        dev = w_gate_up.device
+        self.w1q, self.w1s, self.w2q, self.w2s = (mx_buffer(c, k, dev) for k in (MX_W1Q, MX_W1S, MX_W2Q, MX_W2S))
+        moe_mx_quantize_weights(c, w_gate_up, w_down, self.w1q, self.w1s, self.w2q, self.w2s, stream)
+
+
 # ---------------------------------------------------------------- conveniences
 
 def act_dtype(c) -> torch.dtype:
@@ -292,6 +351,12 @@ class Layer:
         dl = torch.empty(c.T, c.E, dtype=torch.float32, device=dev) if dlogits else None
         moe_layer_bwd(c, logits, w_gate_up, w_down, d_out, dx, dwgu, dwdn, dl, self.ws, stream)
         return dx, dwgu, dwdn, dl
+
+    def forward_mx(self, logits, x, mxw: "MxWeights", out=None, stream=None):
+        """The layer on MXFP8 expert operands (weights from MxWeights)."""
+        out = self.out if out is None else out
+        moe_layer_fwd_mx(self.cfg, logits, x, mxw.w1q, mxw.w1s, mxw.w2q, mxw.w2s, out, self.ws, stream)
+        return out
 
     def status(self, stream=None) -> int:
         return moe_read_status(self.ws, stream)

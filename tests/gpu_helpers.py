@@ -231,3 +231,173 @@ def check_bwd_small(cfg, seed, device="cuda"):
     chosen = np.zeros((cfg.T, cfg.E), bool)
     np.put_along_axis(chosen, idx, True, axis=1)
     assert not dl.cpu().numpy()[~chosen].any()
+
+
+# ---------------------------------------------------------------- MXFP8 forward
+
+def mx_scale_index(rows: int, K: int) -> np.ndarray:
+    """For each (row, 32-block) of a [rows, K] MXFP8 matrix, the byte of its
+    scale in the chunked layout include/moe.h documents (512-byte chunks per
+    128 rows and 128 columns; row r, block b at 16 (r % 32) + 4 ((r % 128) / 32) + b % 4)."""
+    r = np.arange(rows, dtype=np.int64)[:, None]
+    b = np.arange(K // 32, dtype=np.int64)[None, :]
+    return ((r // 128) * (K // 128) + b // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + b % 4
+
+
+def mx_unchunk(sc: torch.Tensor | np.ndarray, rows: int, K: int) -> np.ndarray:
+    sc = sc.cpu().numpy() if isinstance(sc, torch.Tensor) else sc
+    return sc[mx_scale_index(rows, K)]
+
+
+def mx_chunk(logical: np.ndarray, K: int, nbytes: int) -> np.ndarray:
+    rows = logical.shape[0]
+    out = np.zeros(nbytes, np.uint8)
+    out[mx_scale_index(rows, K)] = logical
+    return out
+
+
+def w1_tile_rows(E: int, F: int) -> np.ndarray:
+    """Row order of the MX W1: row e*2F + 128 t + i is gate row 64 t + i (i < 64)
+    or up row F + 64 t + (i - 64) of expert e."""
+    i = np.arange(2 * F)
+    t, r = i // 128, i % 128
+    local = np.where(r < 64, 64 * t + r, F + 64 * t + (r - 64))
+    return (np.arange(E)[:, None] * 2 * F + local[None, :]).ravel()
+
+
+def mx_weights_on_device(cfg, inp: dict):
+    return M.MxWeights(cfg, inp["w_gate_up"], inp["w_down"])
+
+
+def mx_oracle_weights(cfg, inp: dict, experts=None):
+    """Oracle MXFP8 codes and scales of W1 / W2 (logical order) for the given experts (all by default)."""
+    es = range(cfg.E) if experts is None else experts
+    wgu = np.stack([I.to_numpy_bits(inp["w_gate_up"][e]) for e in es])
+    wdn = np.stack([I.to_numpy_bits(inp["w_down"][e]) for e in es])
+    return O.mx_weights(wgu, wdn, O.BF16)
+
+
+def run_mx_stages(cfg, inp: dict) -> dict:
+    """moe_plan, moe_dispatch_mx, moe_expert_fc1_mx, moe_expert_fc2_mx, moe_combine."""
+    dev = inp["x"].device
+    T, K, E, d, F = cfg.T, cfg.K, cfg.E, cfg.d, cfg.F
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
+    cap = M.moe_rows_capacity(cfg)
+    # padding rows of xq / xs are not written: fill them with NaN codes (0x7F) and scale 255
+    xq = torch.full((M.moe_mx_buffer_bytes(cfg, M.MX_XQ),), 0x7F, dtype=torch.uint8, device=dev)
+    xs = torch.full((M.moe_mx_buffer_bytes(cfg, M.MX_XS),), 0xFF, dtype=torch.uint8, device=dev)
+    hq = M.mx_buffer(cfg, M.MX_HQ, dev)
+    hs = M.mx_buffer(cfg, M.MX_HS, dev)
+    yp = torch.empty(cap, d, dtype=torch.bfloat16, device=dev)
+    out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    mxw = mx_weights_on_device(cfg, inp)
+    M.moe_plan(cfg, inp["logits"], idx, w, counts, ws)
+    M.moe_dispatch_mx(cfg, inp["x"], xq, xs, ws)
+    M.moe_expert_fc1_mx(cfg, xq, xs, mxw.w1q, mxw.w1s, hq, hs, ws)
+    M.moe_expert_fc2_mx(cfg, hq, hs, mxw.w2q, mxw.w2s, yp, ws)
+    M.moe_combine(cfg, yp, w, out, ws)
+    status = M.moe_read_status(ws)
+    return {"idx": idx, "w": w, "counts": counts, "xq": xq.view(cap, d), "xs": xs, "hq": hq.view(cap, F),
+            "hs": hs, "yp": yp, "out": out, "status": status, "plan": M.read_plan(cfg, ws), "ws": ws,
+            "rows_cap": cap, "mxw": mxw}
+
+
+def assert_mx_h_close(g_hq: np.ndarray, g_hs: np.ndarray, r_h: np.ndarray, r_hq: np.ndarray, r_hs: np.ndarray,
+                      what: str, max_code_frac: float = 2e-3):
+    """h after FC1 and MXFP8 quantization. The GPU forms h in fp32 and the
+    oracle in fp64, so where the bf16-rounded h lands on either side of a
+    rounding boundary the codes (or a block's scale) may differ; such
+    elements differ by at most one E4M3 step of the block and must stay
+    rare. Elementwise: |g - o| <= one step of E4M3 at o's magnitude (2^-3
+    relative) + 2^-9 of the block's scale; normwise <= 1e-2."""
+    gd = O.mx_dequantize(g_hq, g_hs)
+    rd = O.mx_dequantize(r_hq, r_hs)
+    code_diff = (g_hq != r_hq)
+    frac = code_diff.mean() if code_diff.size else 0.0
+    assert frac <= max_code_frac, f"{what}: {frac:.2e} of the codes differ"
+    scale = 2.0 ** (np.repeat(r_hs.astype(np.int64), 32, axis=1) - 127)
+    err = np.abs(gd - rd)
+    bad = err > 2.0 ** -3 * np.abs(rd) + 2.0 ** -9 * scale * 2
+    assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond one E4M3 step, max err {err.max():.3e}"
+    den = np.linalg.norm(rd)
+    if den > 0:
+        assert np.linalg.norm(gd - rd) / den <= 1e-2, f"{what}: normwise error"
+
+
+def check_mx_small(cfg, seed: int, device="cuda"):
+    """The MX layer stage by stage against the oracle on every element."""
+    inp = I.make_inputs(cfg, seed, device)
+    g = run_mx_stages(cfg, inp)
+    hin = host_inputs(inp)
+    ref = oracle_routing(cfg, hin)
+    assert g["rows_cap"] == ref["rows_cap"]
+    check_routing_and_plan(cfg, g, ref)
+    assert (g["status"] & ~O.PLAN_INEXACT) == 0, f"device status {g['status']}"
+    d, F, E, K = cfg.d, cfg.F, cfg.E, cfg.K
+    total = ref["plan"]["total_rows"]
+    src = ref["src_of"][:total]
+    valid = src >= 0
+    vrows = np.nonzero(valid)[0]
+    # weights: bit-exact codes and scales
+    w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp)
+    perm = w1_tile_rows(E, F)
+    gw1q = g["mxw"].w1q.view(E * 2 * F, d).cpu().numpy()
+    assert np.array_equal(gw1q, w1q[perm]), "W1 codes differ"
+    assert np.array_equal(mx_unchunk(g["mxw"].w1s, E * 2 * F, d), w1s[perm]), "W1 scales differ"
+    assert np.array_equal(g["mxw"].w2q.view(E * d, F).cpu().numpy(), w2q), "W2 codes differ"
+    assert np.array_equal(mx_unchunk(g["mxw"].w2s, E * d, F), w2s), "W2 scales differ"
+    # dispatch: every valid row holds its token's codes and scales, bit for bit
+    xq_ref, xs_ref = O.mx_quantize(hin["x"], O.BF16)
+    gxq = g["xq"][:total].cpu().numpy()
+    gxs = mx_unchunk(g["xs"], total, d)
+    assert np.array_equal(gxq[valid], xq_ref[src[valid]]), "dispatched codes differ"
+    assert np.array_equal(gxs[valid], xs_ref[src[valid]]), "dispatched scales differ"
+    # FC1 on the oracle's own operands
+    blocks = ref["plan"]["blocks"]
+    row_exp = np.zeros(total, np.int32)
+    for b in blocks:
+        row_exp[b[1]:b[1] + 128] = b[0]
+    xq_rows = xq_ref[src[valid]]
+    xs_rows = xs_ref[src[valid]]
+    rh, rhq, rhs = O.mx_fc1_rows(np.arange(len(vrows)), row_exp[valid], xq_rows, xs_rows, w1q, w1s, F)
+    ghq = g["hq"][:total].cpu().numpy()
+    ghs = mx_unchunk(g["hs"], total, F)
+    assert_mx_h_close(ghq[valid], ghs[valid], rh, rhq, rhs, "h (MXFP8)")
+    assert not ghq[~valid].any() and not ghs[~valid].any(), "padding rows of h must be zero codes and scales"
+    # FC2 on the oracle's h
+    ry = O.mx_fc2_rows(row_exp[valid], rhq, rhs, w2q, w2s, d)
+    gy = to_f64(g["yp"][:total])
+    assert_close(gy[valid], ry, C.BF16, "yp")
+    assert not gy[~valid].any(), "padding rows of yp must be zero"
+    # the whole layer
+    rout = O.mx_token_out(np.arange(cfg.T), xq_ref, xs_ref, ref["idx"], ref["w"], w1q, w1s, w2q, w2s, F)
+    assert_close(to_f64(g["out"]), rout, C.BF16, "out")
+    return g, ref, inp
+
+
+def check_mx_full_size(cfg, seed: int, n_tokens: int = 4, device="cuda"):
+    """Full-size MX layer through moe_layer_fwd_mx: bit-exact routing and plan
+    (moe_plan), and sampled tokens of out against the oracle."""
+    inp = I.make_inputs(cfg, seed, device)
+    hin = host_inputs(inp, with_weights=False)
+    ref = oracle_routing(cfg, hin)
+    layer = M.Layer(cfg, device)
+    mxw = mx_weights_on_device(cfg, inp)
+    out = layer.forward_mx(inp["logits"], inp["x"], mxw)
+    assert (layer.status() & ~O.PLAN_INEXACT) == 0
+    plan = M.read_plan(cfg, layer.ws)
+    assert np.array_equal(plan["row_of"].numpy(), ref["row_of"]), "row_of differs"
+    rng = np.random.default_rng(seed + 29)
+    toks = rng.choice(cfg.T, size=n_tokens, replace=False)
+    gout = to_f64(out[torch.as_tensor(toks, device=device)])
+    for i, t in enumerate(toks):
+        es = ref["idx"][t]
+        w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp, es)
+        xq, xs = O.mx_quantize(hin["x"][t:t + 1], O.BF16)
+        o = O.mx_token_out(np.array([0]), xq, xs, np.arange(cfg.K, dtype=np.int32)[None, :], ref["w"][t:t + 1],
+                           w1q, w1s, w2q, w2s, cfg.F)
+        assert_close(gout[i:i + 1], o, C.BF16, f"out[{t}]")
+    return out

@@ -161,3 +161,19 @@ def test_mx_token_out_is_the_weighted_sum_of_its_entries():
     _, _, _, y = O.mx_entry_ffn(np.repeat(np.arange(T), K), idx.ravel(), xq, xs, w1q, w1s, w2q, w2s, F)
     ref = (w.astype(np.float64)[:, :, None] * y.reshape(T, K, d)).sum(1)
     assert np.array_equal(out, O.bf16_bits_to_f64(_bf16(ref)))
+
+
+def test_mx_fc1_and_fc2_rows_compose_to_the_entry_ffn():
+    rng = np.random.default_rng(4)
+    E, d, F, T = 3, 64, 64, 4
+    x = _bf16(rng.standard_normal((T, d)))
+    w_gu = _bf16(rng.standard_normal((E, 2 * F, d)) * 0.2)
+    w_dn = _bf16(rng.standard_normal((E, d, F)) * 0.2)
+    xq, xs = O.mx_quantize(x, O.BF16)
+    w1q, w1s, w2q, w2s = O.mx_weights(w_gu, w_dn, O.BF16)
+    tokens = np.repeat(np.arange(T), E)
+    experts = np.tile(np.arange(E), T)
+    h, hq, hs, y = O.mx_entry_ffn(tokens, experts, xq, xs, w1q, w1s, w2q, w2s, F)
+    h1, hq1, hs1 = O.mx_fc1_rows(tokens, experts, xq, xs, w1q, w1s, F)
+    assert np.array_equal(h1, h) and np.array_equal(hq1, hq) and np.array_equal(hs1, hs)
+    assert np.array_equal(O.mx_fc2_rows(experts, hq, hs, w2q, w2s, d), y)
