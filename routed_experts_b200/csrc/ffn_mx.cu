@@ -57,7 +57,19 @@ constexpr int kMxSfBytes = 512;                             // 128 rows x 4 scal
 constexpr int kMxStageBytes = kMxABytes + kMxBBytes + 2 * kMxSfBytes;   // 25 KB
 constexpr uint32_t kMxTmemCols = 512;                       // allocation: a power of two >= 2*128 + 16
 constexpr uint32_t kMxSfCol = 2 * kMxN;                     // two sets of (4 SFA + 4 SFB) columns
-constexpr size_t kMxSmemBytes = 1024 /*align slack*/ + kMxStages * kMxStageBytes + kEpiBytes + sizeof(Smem) +
+
+// The control block: the bf16 kernel's, with one full / empty barrier pair
+// per stage of this kernel's ring.
+struct MxSmem {
+    uint64_t full[kMxStages], empty[kMxStages], acc_full[2], acc_empty[2], drain;
+    uint64_t item_full[kItemSlots], item_empty[kItemSlots], fwd_empty[kItemSlots];
+    int4 items[kItemSlots];       // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
+    uint32_t valid[kItemSlots];   // valid rows of the even CTA's block (low 16 bits) and the odd CTA's (high)
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+constexpr size_t kMxSmemBytes = 1024 /*align slack*/ + kMxStages * kMxStageBytes + kEpiBytes + sizeof(MxSmem) +
                                 2 * sizeof(int32_t) * (kMaxE + 1);
 static_assert(kMxSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kMxStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
@@ -168,7 +180,7 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_base = base + kMxStages * kMxStageBytes;
-    Smem* S = reinterpret_cast<Smem*>(epi_base + kEpiBytes);
+    MxSmem* S = reinterpret_cast<MxSmem*>(epi_base + kEpiBytes);
     int32_t* s_off = reinterpret_cast<int32_t*>(S + 1);
     int32_t* p_off = s_off + (a.E + 1);
     volatile int* abort_flag = &S->abort_flag;

@@ -80,16 +80,19 @@ __global__ void __launch_bounds__(kQWarps * 32)
 mx_quantize_kernel(const uint4* __restrict__ x, int64_t rows, int K, int interleave_F, uint8_t* __restrict__ q,
                    uint8_t* __restrict__ sc) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int segs = K / 256;
+    const int segs = (K + 255) / 256;   // K % 128 == 0: the last step of a row may be half full
     const int64_t units = rows * segs;
     for (int64_t u = (int64_t)blockIdx.x * kQWarps + warp; u < units; u += (int64_t)gridDim.x * kQWarps) {
         const int64_t r = u / segs;
         const int seg = (int)(u % segs);
         const int64_t col = (int64_t)seg * 256 + lane * 8;
-        const uint4 v = __ldg(x + (src_row(r, interleave_F) * K + col) / 8);
+        const bool in = col < K;   // whole groups of four lanes (32-blocks) are in or out together
+        const uint4 v = in ? __ldg(x + (src_row(r, interleave_F) * K + col) / 8) : make_uint4(0, 0, 0, 0);
         const uint32_t s = group_scale(amax8(v));
-        *reinterpret_cast<uint2*>(q + r * K + col) = e4m3x8(v, mx_inv_scale(s));
-        if ((lane & 3) == 0) sc[mx_scale_offset(r, col / 32, K)] = (uint8_t)s;
+        if (in) {
+            *reinterpret_cast<uint2*>(q + r * K + col) = e4m3x8(v, mx_inv_scale(s));
+            if ((lane & 3) == 0) sc[mx_scale_offset(r, col / 32, K)] = (uint8_t)s;
+        }
     }
 }
 
@@ -135,8 +138,8 @@ int grid_for(int64_t warps) {
 
 cudaError_t launch_mx_quantize(const void* x, int64_t rows, int K, int interleave_F, uint8_t* q, uint8_t* sc,
                                cudaStream_t st) {
-    if (K % 256 != 0 || rows <= 0) return cudaErrorInvalidValue;
-    mx_quantize_kernel<<<grid_for(rows * (K / 256)), kQWarps * 32, 0, st>>>(static_cast<const uint4*>(x), rows, K,
+    if (K % 128 != 0 || rows <= 0) return cudaErrorInvalidValue;
+    mx_quantize_kernel<<<grid_for(rows * ((K + 255) / 256)), kQWarps * 32, 0, st>>>(static_cast<const uint4*>(x), rows, K,
                                                                           interleave_F, q, sc);
     return cudaGetLastError();
 }
