@@ -51,6 +51,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-tokens", type=int, default=320, help="tokens of the oracle's FFN sample")
     p.add_argument("--no-backward", action="store_true", help="skip timing the layer's backward")
+    p.add_argument("--no-mx", action="store_true", help="skip timing the layer on MXFP8 operands")
     return p.parse_args()
 
 
@@ -326,6 +327,103 @@ def time_backward(cfg, inp, args, world, dev, stream, pg):
                     "gradient (8 launches); frac of the measured bf16 peak counts algorithmic FLOP"}
 
 
+def time_mx(cfg, inp, args, world, dev, stream, pg):
+    """The layer on MXFP8 expert operands (moe_layer_fwd_mx), W untimed and K
+    timed passes, plus its stages (plan, quantizing dispatch, FC1, FC2,
+    combine) timed by events between the calls; max over ranks. Weights are
+    quantized once, outside the timed region (an offline step)."""
+    from routed_experts_b200 import moe as M
+    lg, x, wgu, wdn = inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"]
+    T, d, E, F, K = cfg.T, cfg.d, cfg.E, cfg.F, cfg.K
+    q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    q0.record(stream)
+    mxw = M.MxWeights(cfg, wgu, wdn, stream)
+    q1.record(stream)
+    layer = M.Layer(cfg, dev)
+    ref = layer.forward(lg, x, wgu, wdn, stream=stream).float().clone()
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        if pg is not None:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1)
+        if pg is not None:
+            ms = max_over_ranks([ms], dev)[0]
+        return ms / args.steps
+
+    ms = timed(lambda: layer.forward_mx(lg, x, mxw, stream=stream))
+    out = layer.forward_mx(lg, x, mxw, stream=stream).float()
+    torch.cuda.synchronize(dev)
+    rel_to_bf16 = (torch.linalg.norm(out - ref) / torch.linalg.norm(ref)).item()
+    st = M.moe_read_status(layer.ws, stream)
+    if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
+        raise RuntimeError(f"device status {st} after the MX layer passes")
+    del layer
+    # the stages, events between the calls
+    idx = torch.empty(T, K, dtype=torch.int32, device=dev)
+    w = torch.empty(T, K, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
+    xq, xs, hq, hs = (M.mx_buffer(cfg, k, dev) for k in (M.MX_XQ, M.MX_XS, M.MX_HQ, M.MX_HS))
+    cap = M.moe_rows_capacity(cfg)
+    yp = torch.empty(cap, d, dtype=torch.bfloat16, device=dev)
+    o = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+    calls = (lambda: M.moe_plan(cfg, lg, idx, w, counts, ws, stream),
+             lambda: M.moe_dispatch_mx(cfg, x, xq, xs, ws, stream),
+             lambda: M.moe_expert_fc1_mx(cfg, xq, xs, mxw.w1q, mxw.w1s, hq, hs, ws, stream),
+             lambda: M.moe_expert_fc2_mx(cfg, hq, hs, mxw.w2q, mxw.w2s, yp, ws, stream),
+             lambda: M.moe_combine(cfg, yp, w, o, ws, stream))
+    for _ in range(args.warmup):
+        for f in calls:
+            f()
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(args.steps)]
+    for k in range(args.steps):
+        evs[k][0].record(stream)
+        for i, f in enumerate(calls):
+            f()
+            evs[k][i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    stage = np.array([[evs[k][i].elapsed_time(evs[k][i + 1]) for i in range(len(calls))] for k in range(args.steps)])
+    mean = stage.mean(axis=0)
+    if pg is not None:
+        mean = np.array(max_over_ranks(list(mean), dev))
+    pk, pk_kind = peaks()
+    fp8_peak = 2.0 * pk["bf16_tflops"]   # E4M3 dense rate = 2 x bf16 (4.5 vs 2.25 PFLOP/s nominal)
+    N = cfg.N
+    fc1_flop, fc2_flop = 2.0 * N * d * (2 * F), 2.0 * N * F * d
+    plan = M.read_plan(cfg, ws)
+    active = int((np.bincount(plan["blocks"][:, 0].numpy(), minlength=E) > 0).sum()) if plan["n_blocks"] else 0
+    w_bytes = active * 3 * F * d * (1 + 1 / 32)
+    alg_bytes = 4 * T * E + T * d * 2 + w_bytes + T * d * 2
+    t_roof = max((fc1_flop + fc2_flop) / (fp8_peak * 1e12), alg_bytes / (pk["hbm_gbs"] * 1e9))
+    disp_bytes = T * d * 2 + N * d * (1 + 1 / 32) + 4 * N
+    del mxw, xq, xs, hq, hs, yp
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "tokens_per_s": world * T / (ms * 1e-3),
+            "stages_ms": {"plan": mean[0], "dispatch_mx": mean[1], "fc1_mx": mean[2], "fc2_mx": mean[3],
+                          "combine": mean[4]},
+            "fc1_tflops": fc1_flop / (mean[2] * 1e-3) / 1e12, "fc2_tflops": fc2_flop / (mean[3] * 1e-3) / 1e12,
+            "fc1_frac": fc1_flop / (mean[2] * 1e-3) / 1e12 / fp8_peak,
+            "fc2_frac": fc2_flop / (mean[3] * 1e-3) / 1e12 / fp8_peak,
+            "fp8_peak_tflops": fp8_peak, "peak_kind": f"{pk_kind} bf16 burst x 2 (E4M3 / bf16 nominal ratio)",
+            "dispatch_mx_gbs": disp_bytes / (mean[1] * 1e-3) / 1e9,
+            "layer_roofline_frac": (t_roof * 1e3) / ms, "layer_roofline_ms": t_roof * 1e3,
+            "weight_quantize_ms": q0.elapsed_time(q1),
+            "rel_diff_to_bf16_layer": rel_to_bf16,
+            "note": "moe_layer_fwd_mx: plan, dispatch with MXFP8 quantization of x, FC1 + SwiGLU with h "
+                    "quantized to MXFP8 in the epilogue, FC2, combine; E4M3 elements, E8M0 scale per 32; "
+                    "weights quantized once outside the timed region"}
+
+
 def run_mine(args, world, rank, local):
     from routed_experts_b200 import moe as M
     cfg = C.NAMED[args.config]
@@ -470,6 +568,11 @@ def run_mine(args, world, rank, local):
         torch.cuda.empty_cache()
         bwd = time_backward(cfg, inp, args, world, dev, stream, pg)
 
+    mx = None
+    if not args.no_mx and cfg.dtype == C.BF16:
+        torch.cuda.empty_cache()
+        mx = time_mx(cfg, inp, args, world, dev, stream, pg)
+
     plans = plan_comparison(cfg, inp, dev) if rank == 0 else None
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -548,6 +651,7 @@ def run_mine(args, world, rank, local):
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "layer_path": "moe_plan; moe_dispatch; moe_expert_fc1; moe_expert_fc2; moe_combine (the kernels of moe_layer_fwd)",
         "backward": bwd,
+        "mx": mx,
         "fused_ffn": None if fused_ms is None else {
             "ms": fused_ms, "staged_fc1_fc2_ms": float(med[2] + med[3]),
             "note": "moe_expert_ffn_fused: FC1 and FC2 in one launch, FC2 tiles released per block pair "

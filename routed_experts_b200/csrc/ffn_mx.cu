@@ -16,17 +16,24 @@
 //     elements, so a k-step is 128 deep and takes four MMAs of
 //     tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale (M = 256, N = 128,
 //     K = 32);
-//   - each k-step also brings the scale factors of its 128 A rows and 128 B
-//     rows (512 bytes each, already in the chunked layout of
-//     mx_scale_offset) into shared memory with the same TMA barrier; the MMA
-//     thread copies them to TMEM (tcgen05.cp 32x128b.warpx4, four columns
-//     each) ahead of the k-step's MMAs, alternating between two column sets;
-//   - an item is 256 rows x 128 columns: two 128-column accumulators plus
-//     the scale columns fit in TMEM, where two 256-column accumulators would
-//     leave no room for the scales. FC1 items are 64 h columns: the weight
+//   - each k-step also brings the scale factors of its 128 A rows and 256 B
+//     rows (512 bytes per 128 rows, already in the chunked layout of
+//     mx_scale_offset) into a small ring beside the operand stages, on the
+//     same TMA barrier; the MMA thread copies them to TMEM (tcgen05.cp
+//     32x128b.warpx4, four columns per 128 rows) ahead of the k-step's MMAs,
+//     alternating between two column sets;
+//   - an item is 256 rows x 256 columns, issued as two N = 128 MMAs per K
+//     slice into two 128-column TMEM half-buffers. Three half-buffers rotate
+//     (item k takes buffers 2k mod 3 and 2k+1 mod 3) and the epilogue frees
+//     each half as soon as it has read it, so the next item's MMAs wait only
+//     for the first half of the previous item's epilogue; two full
+//     256-column accumulators would leave no TMEM for the scales. Each CTA
+//     holds 128 weight rows of the item as two 64-row halves. FC1's weight
 //     rows are stored with every 128 rows of an expert holding 64 gate rows
-//     then the matching 64 up rows (even CTA: gate, odd CTA: up), so both
-//     halves of SwiGLU sit side by side in each CTA's accumulator;
+//     then the matching 64 up rows, so each half-MMA's accumulator holds
+//     [64 gate | 64 up] columns (even CTA: gate, odd CTA: up) and a half is
+//     SwiGLU-complete: 64 h columns per half, 128 per item; an FC2 item is
+//     256 columns of d;
 //   - the FC1 epilogue applies SwiGLU, rounds h to bf16 (FC1's bf16 output)
 //     and quantizes it to MXFP8 along F right away: each thread holds 32
 //     consecutive h values of its row, exactly one scale block, so the
@@ -48,20 +55,23 @@ namespace {
 using namespace tc;
 
 constexpr int kMxBK = 128;                                  // K elements (bytes) per k-step
-constexpr int kMxN = 128;                                   // accumulator columns per item
-constexpr int kMxHalfN = 64;                                // weight rows each CTA holds
-constexpr int kMxStages = 7;
+constexpr int kMxHalf = 128;                                // accumulator columns of one half-item MMA (N)
+constexpr int kMxItemN = 2 * kMxHalf;                       // accumulator columns per item
+constexpr int kMxHalfRows = 64;                             // weight rows each CTA holds per half
+constexpr int kMxStages = 6;
 constexpr int kMxABytes = kBM * kMxBK;                      // 16 KB
-constexpr int kMxBBytes = kMxHalfN * kMxBK;                 // 8 KB
+constexpr int kMxBBytes = 2 * kMxHalfRows * kMxBK;          // 16 KB: the two halves' weight rows
+constexpr int kMxStageBytes = kMxABytes + kMxBBytes;        // 32 KB
 constexpr int kMxSfBytes = 512;                             // 128 rows x 4 scales
-constexpr int kMxStageBytes = kMxABytes + kMxBBytes + 2 * kMxSfBytes;   // 25 KB
-constexpr uint32_t kMxTmemCols = 512;                       // allocation: a power of two >= 2*128 + 16
-constexpr uint32_t kMxSfCol = 2 * kMxN;                     // two sets of (4 SFA + 4 SFB) columns
+constexpr int kMxSfStage = 3 * kMxSfBytes;                  // A, B of half 0, B of half 1
+constexpr int kMxBufs = 3;                                  // 128-column TMEM half-buffers
+constexpr uint32_t kMxTmemCols = 512;                       // allocation: a power of two >= 3*128 + 24
+constexpr uint32_t kMxSfCol = kMxBufs * kMxHalf;            // two sets of 12 scale columns from here
 
 // The control block: the bf16 kernel's, with one full / empty barrier pair
-// per stage of this kernel's ring.
+// per stage of this kernel's ring and per TMEM half-buffer.
 struct MxSmem {
-    uint64_t full[kMxStages], empty[kMxStages], acc_full[2], acc_empty[2], drain;
+    uint64_t full[kMxStages], empty[kMxStages], hfull[kMxBufs], hempty[kMxBufs], drain;
     uint64_t item_full[kItemSlots], item_empty[kItemSlots], fwd_empty[kItemSlots];
     int4 items[kItemSlots];       // expert (-1: no more work), column tile, first row of each CTA's block (-1: none)
     uint32_t valid[kItemSlots];   // valid rows of the even CTA's block (low 16 bits) and the odd CTA's (high)
@@ -69,14 +79,14 @@ struct MxSmem {
     int abort_flag;
 };
 
-constexpr size_t kMxSmemBytes = 1024 /*align slack*/ + kMxStages * kMxStageBytes + kEpiBytes + sizeof(MxSmem) +
-                                2 * sizeof(int32_t) * (kMaxE + 1);
+constexpr size_t kMxSmemBytes = 1024 /*align slack*/ + kMxStages * (kMxStageBytes + kMxSfStage) + kEpiBytes +
+                                sizeof(MxSmem) + 2 * sizeof(int32_t) * (kMaxE + 1);
 static_assert(kMxSmemBytes <= 232448, "shared memory per CTA");
 static_assert(kMxStageBytes % 1024 == 0, "stages keep the 1024-byte alignment of swizzled tiles");
 
 struct MxArgs {
     int Kdim;               // d (FC1) or F (FC2)
-    int n_tiles;            // F/64 (FC1) or d/128 (FC2)
+    int n_tiles;            // F/128 (FC1) or d/256 (FC2)
     int b_rows;             // rows of one expert in the weight matrix: 2F or d
     int E;
     int out_K;              // FC1: F, the row length of h (for its scale layout)
@@ -94,18 +104,20 @@ __device__ __forceinline__ uint32_t mx_scale_of(float amax) {
     return field > 8u ? field - 8u : 0u;
 }
 
-// The epilogue of one item for one warp (rows 32*quad .. 32*quad+31 of the
-// CTA's block). MODE 0: columns [0, 64) gate and [64, 128) up -> h codes of
-// columns j*64 .. j*64+63 and their two scales; MODE 1: 128 columns -> bf16 yp.
+// The epilogue of one half-item for one warp (rows 32*quad .. 32*quad+31 of
+// the CTA's block), reading the half-buffer at t_half. MODE 0: columns
+// [0, 64) gate and [64, 128) up -> h codes of columns col0 .. col0+63 and
+// their two scales; MODE 1: 128 columns -> bf16 yp columns col0 .. col0+127.
 template <int MODE>
-__device__ __forceinline__ void mx_epilogue_item(uint32_t t_row, int lane, int quad, uint8_t* stg, int& buf,
-                                                 const CUtensorMap* tmO, const MxArgs& a, int j, int row0, bool pad) {
+__device__ __forceinline__ void mx_epilogue_half(uint32_t t_half, int lane, int quad, uint8_t* stg, int& buf,
+                                                 const CUtensorMap* tmO, const MxArgs& a, int col0, int row0,
+                                                 bool pad) {
     if (MODE == 0) {
 #pragma unroll 1
-        for (int c = 0; c < kMxHalfN; c += 32) {
+        for (int c = 0; c < kMxHalfRows; c += 32) {
             uint32_t gt[32], up[32];
-            ptx::tmem_ld32(t_row + c, gt);
-            ptx::tmem_ld32(t_row + kMxHalfN + c, up);
+            ptx::tmem_ld32(t_half + c, gt);
+            ptx::tmem_ld32(t_half + kMxHalfRows + c, up);
             ptx::tmem_ld_wait();
             float h[32];
             float amax = 0.f;
@@ -135,18 +147,18 @@ __device__ __forceinline__ void mx_epilogue_item(uint32_t t_row, int lane, int q
             ptx::fence_proxy_async_shared();
             __syncwarp();
             if (lane == 0) {
-                ptx::tma_store_2d(tmO, tile, j * kMxHalfN + c, row0 + quad * 32);
+                ptx::tma_store_2d(tmO, tile, col0 + c, row0 + quad * 32);
                 ptx::bulk_commit_group();
             }
             buf ^= 1;
             const int64_t row = (int64_t)row0 + quad * 32 + lane;
-            a.out_sc[mx_scale_offset(row, (j * kMxHalfN + c) / 32, a.out_K)] = (uint8_t)s;
+            a.out_sc[mx_scale_offset(row, (col0 + c) / 32, a.out_K)] = (uint8_t)s;
         }
     } else {
 #pragma unroll 1
-        for (int c = 0; c < kMxN; c += 32) {
+        for (int c = 0; c < kMxHalf; c += 32) {
             uint32_t y[32];
-            ptx::tmem_ld32(t_row + c, y);
+            ptx::tmem_ld32(t_half + c, y);
             ptx::tmem_ld_wait();
             uint32_t pk[16];
 #pragma unroll
@@ -161,7 +173,7 @@ __device__ __forceinline__ void mx_epilogue_item(uint32_t t_row, int lane, int q
             ptx::fence_proxy_async_shared();
             __syncwarp();
             if (lane == 0) {
-                ptx::tma_store_2d(tmO, tile, j * kMxN + c, row0 + quad * 32);
+                ptx::tma_store_2d(tmO, tile, col0 + c, row0 + quad * 32);
                 ptx::bulk_commit_group();
             }
             buf ^= 1;
@@ -179,7 +191,8 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmO, MxArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* epi_base = base + kMxStages * kMxStageBytes;
+    uint8_t* sf_base = base + kMxStages * kMxStageBytes;          // the scale ring
+    uint8_t* epi_base = sf_base + kMxStages * kMxSfStage;
     MxSmem* S = reinterpret_cast<MxSmem*>(epi_base + kEpiBytes);
     int32_t* s_off = reinterpret_cast<int32_t*>(S + 1);
     int32_t* p_off = s_off + (a.E + 1);
@@ -190,7 +203,7 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     const bool even = rank == 0;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kMxStages; ++s) { ptx::mbar_init(&S->full[s], 1); ptx::mbar_init(&S->empty[s], 1); }
-        for (int q = 0; q < 2; ++q) { ptx::mbar_init(&S->acc_full[q], 1); ptx::mbar_init(&S->acc_empty[q], 8); }
+        for (int q = 0; q < kMxBufs; ++q) { ptx::mbar_init(&S->hfull[q], 1); ptx::mbar_init(&S->hempty[q], 8); }
         for (int q = 0; q < kItemSlots; ++q) {
             ptx::mbar_init(&S->item_full[q], 1);
             ptx::mbar_init(&S->item_empty[q], kItemConsumers);
@@ -321,18 +334,23 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (item.x < 0) break;
                 const int e = item.x, j = item.y;
                 const int row0 = even ? item.z : (item.w >= 0 ? item.w : item.z);
-                const int brow = e * a.b_rows + j * kMxN + (even ? 0 : kMxHalfN);
+                const int wrow = e * a.b_rows + j * kMxItemN;        // the item's first weight row
+                const int b_lo = wrow + (even ? 0 : kMxHalfRows);    // this CTA's rows of half 0
+                const int b_hi = b_lo + kMxHalf;                     // and of half 1
                 const int a_chunk0 = (row0 / 128) * kc;
-                const int b_chunk0 = ((e * a.b_rows + j * kMxN) / 128) * kc;
+                const int b_chunk0 = (wrow / 128) * kc, b_chunk1 = (wrow / 128 + 1) * kc;
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!role_wait(&S->empty[stage], phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
                     const uint32_t bar = ptx::map_to_rank(ptx::smem_addr(&S->full[stage]), 0);
                     uint8_t* st = base + stage * kMxStageBytes;
-                    if (even) ptx::mbar_arrive_expect_tx(&S->full[stage], 2 * kMxStageBytes);
+                    uint8_t* sf = sf_base + stage * kMxSfStage;
+                    if (even) ptx::mbar_arrive_expect_tx(&S->full[stage], 2 * (kMxStageBytes + kMxSfStage));
                     ptx::tma_load_2d_pair(st, &tmA, kb * kMxBK, row0, bar);
-                    ptx::tma_load_2d_pair(st + kMxABytes, &tmB, kb * kMxBK, brow, bar);
-                    ptx::tma_load_2d_pair(st + kMxABytes + kMxBBytes, &tmSA, 0, (a_chunk0 + kb) * 4, bar);
-                    ptx::tma_load_2d_pair(st + kMxABytes + kMxBBytes + kMxSfBytes, &tmSB, 0, (b_chunk0 + kb) * 4, bar);
+                    ptx::tma_load_2d_pair(st + kMxABytes, &tmB, kb * kMxBK, b_lo, bar);
+                    ptx::tma_load_2d_pair(st + kMxABytes + kMxBBytes / 2, &tmB, kb * kMxBK, b_hi, bar);
+                    ptx::tma_load_2d_pair(sf, &tmSA, 0, (a_chunk0 + kb) * 4, bar);
+                    ptx::tma_load_2d_pair(sf + kMxSfBytes, &tmSB, 0, (b_chunk0 + kb) * 4, bar);
+                    ptx::tma_load_2d_pair(sf + 2 * kMxSfBytes, &tmSB, 0, (b_chunk1 + kb) * 4, bar);
                     ++fills;
                     if (++stage == kMxStages) { stage = 0; phase ^= 1; }
                 }
@@ -355,25 +373,33 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 if (!take_item(k, item)) { ok = false; break; }
                 release_item(k);
                 if (item.x < 0) break;
-                const int acc = k & 1;
-                const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
-                if (!role_wait_cluster(&S->acc_empty[acc], acc_phase ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
+                // this item's half-buffers and how often each was used before
+                const int s0 = 2 * k, s1 = 2 * k + 1;
+                const int b0 = s0 % kMxBufs, b1 = s1 % kMxBufs;
+                const uint32_t p0 = (uint32_t)((s0 / kMxBufs) & 1), p1 = (uint32_t)((s1 / kMxBufs) & 1);
+                if (!role_wait_cluster(&S->hempty[b0], p0 ^ 1, a.spin, abort_flag, a.header) ||
+                    !role_wait_cluster(&S->hempty[b1], p1 ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
                 ptx::tc_fence_after();
-                const uint32_t d_tmem = tmem + (uint32_t)(acc * kMxN);
+                const uint32_t d0 = tmem + (uint32_t)(b0 * kMxHalf), d1 = tmem + (uint32_t)(b1 * kMxHalf);
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!role_wait(&S->full[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
                     ptx::tc_fence_after();
                     const uint32_t a_addr = ptx::smem_addr(base + stage * kMxStageBytes);
                     const uint32_t b_addr = a_addr + kMxABytes;
-                    const uint32_t sfa_addr = b_addr + kMxBBytes;
-                    const uint32_t sfa_t = tmem + kMxSfCol + 8u * sf_set, sfb_t = sfa_t + 4u;
-                    ptx::tmem_cp_sf_pair(sfa_t, ptx::sdesc_sf(sfa_addr));
-                    ptx::tmem_cp_sf_pair(sfb_t, ptx::sdesc_sf(sfa_addr + kMxSfBytes));
+                    const uint32_t sf_addr = ptx::smem_addr(sf_base + stage * kMxSfStage);
+                    const uint32_t sfa_t = tmem + kMxSfCol + 12u * sf_set;
+                    ptx::tmem_cp_sf_pair(sfa_t, ptx::sdesc_sf(sf_addr));
+                    ptx::tmem_cp_sf_pair(sfa_t + 4u, ptx::sdesc_sf(sf_addr + kMxSfBytes));
+                    ptx::tmem_cp_sf_pair(sfa_t + 8u, ptx::sdesc_sf(sf_addr + 2 * kMxSfBytes));
 #pragma unroll
                     for (uint32_t ks = 0; ks < kMxBK / 32; ++ks) {
-                        ptx::mma_mx_pair(d_tmem, ptx::sdesc_k_sw128(a_addr + ks * 32), ptx::sdesc_k_sw128(b_addr + ks * 32),
-                                         ptx::idesc_mx_e4m3(2 * kBM, kMxN, ks, ks), sfa_t | (ks << 30),
-                                         sfb_t | (ks << 30), (kb | (int)ks) != 0 ? 1u : 0u);
+                        const uint32_t idesc = ptx::idesc_mx_e4m3(2 * kBM, kMxHalf, ks, ks);
+                        const uint32_t acc = (kb | (int)ks) != 0 ? 1u : 0u;
+                        const uint64_t adesc = ptx::sdesc_k_sw128(a_addr + ks * 32);
+                        ptx::mma_mx_pair(d0, adesc, ptx::sdesc_k_sw128(b_addr + ks * 32), idesc, sfa_t | (ks << 30),
+                                         (sfa_t + 4u) | (ks << 30), acc);
+                        ptx::mma_mx_pair(d1, adesc, ptx::sdesc_k_sw128(b_addr + kMxBBytes / 2 + ks * 32), idesc,
+                                         sfa_t | (ks << 30), (sfa_t + 8u) | (ks << 30), acc);
                     }
                     issued = true;
                     sf_set ^= 1u;
@@ -383,9 +409,11 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     if (++stage == kMxStages) { stage = 0; phase ^= 1; }
                 }
                 if (ok) {
-                    const uint32_t full_addr = ptx::smem_addr(&S->acc_full[acc]);
-                    ptx::mma_commit_pair(full_addr);
-                    ptx::mma_commit_pair(ptx::map_to_rank(full_addr, 1));
+                    const uint32_t f0 = ptx::smem_addr(&S->hfull[b0]), f1 = ptx::smem_addr(&S->hfull[b1]);
+                    ptx::mma_commit_pair(f0);
+                    ptx::mma_commit_pair(ptx::map_to_rank(f0, 1));
+                    ptx::mma_commit_pair(f1);
+                    ptx::mma_commit_pair(ptx::map_to_rank(f1, 1));
                 }
             }
             if (!ok && issued) {
@@ -410,18 +438,24 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             const int j = item.y;
             const bool pad = m >= (int)(even ? (vv & 0xffffu) : (vv >> 16));
             const int row0 = even ? item.z : item.w;   // -1: this CTA's half of the pair is empty
-            const int acc = k & 1;
-            const uint32_t acc_phase = (uint32_t)((k >> 1) & 1);
-            if (!role_wait(&S->acc_full[acc], acc_phase, a.spin, abort_flag, a.header)) break;
-            ptx::tc_fence_after();
-            const uint32_t t_acc = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(acc * kMxN);
-            if (row0 >= 0) mx_epilogue_item<MODE>(t_acc, lane, quad, stg, buf, &tmO, a, j, row0, pad);
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-                if (even) ptx::mbar_arrive(&S->acc_empty[acc]);
-                else ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->acc_empty[acc]), 0));
+            bool ok = true;
+            for (int half = 0; half < 2 && ok; ++half) {
+                const int sl = 2 * k + half;
+                const int b = sl % kMxBufs;
+                const uint32_t par = (uint32_t)((sl / kMxBufs) & 1);
+                if (!role_wait(&S->hfull[b], par, a.spin, abort_flag, a.header)) { ok = false; break; }
+                ptx::tc_fence_after();
+                const uint32_t t_half = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(b * kMxHalf);
+                const int col0 = MODE == 0 ? j * 2 * kMxHalfRows + half * kMxHalfRows : j * kMxItemN + half * kMxHalf;
+                if (row0 >= 0) mx_epilogue_half<MODE>(t_half, lane, quad, stg, buf, &tmO, a, col0, row0, pad);
+                ptx::tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if (even) ptx::mbar_arrive(&S->hempty[b]);
+                    else ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->hempty[b]), 0));
+                }
             }
+            if (!ok) break;
         }
         if (lane == 0) ptx::bulk_wait_group<0>();   // the stores are done before the CTA exits
     }
@@ -463,7 +497,7 @@ cudaError_t launch_ffn_mx(const Shape& s, int which, const uint8_t* a_q, const u
     const bool fc1 = which == 1;
     MxArgs a;
     a.Kdim = fc1 ? s.d : s.F;
-    a.n_tiles = fc1 ? s.F / kMxHalfN : s.d / kMxN;
+    a.n_tiles = fc1 ? s.F / (2 * kMxHalfRows) : s.d / kMxItemN;
     a.b_rows = fc1 ? 2 * s.F : s.d;
     a.E = s.E;
     a.out_K = s.F;
@@ -480,7 +514,7 @@ cudaError_t launch_ffn_mx(const Shape& s, int which, const uint8_t* a_q, const u
     const uint64_t chunks_b = rows_b / 128 * (a.Kdim / 128);
     CUtensorMap tA, tB, tSA, tSB, tO;
     if (!make_tmap_u8(&tA, a_q, (uint64_t)a.Kdim, rows_a, kMxBK, kBM, true) ||
-        !make_tmap_u8(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxBK, kMxHalfN, true) ||
+        !make_tmap_u8(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxBK, kMxHalfRows, true) ||
         !make_tmap_u8(&tSA, a_sc, 128, chunks_a * 4, 128, 4, false) ||
         !make_tmap_u8(&tSB, w_sc, 128, chunks_b * 4, 128, 4, false))
         return cudaErrorInvalidValue;

@@ -327,8 +327,10 @@ def assert_mx_h_close(g_hq: np.ndarray, g_hs: np.ndarray, r_h: np.ndarray, r_hq:
         assert np.linalg.norm(gd - rd) / den <= 1e-2, f"{what}: normwise error"
 
 
-def check_mx_small(cfg, seed: int, device="cuda"):
-    """The MX layer stage by stage against the oracle on every element."""
+def check_mx_small(cfg, seed: int, device="cuda", max_rows: int = 768, max_tokens: int = 192):
+    """The MX layer stage by stage against the oracle: weights and dispatched
+    rows on every element; h and yp on every valid row up to max_rows (a
+    seeded sample beyond), out on every token up to max_tokens (likewise)."""
     inp = I.make_inputs(cfg, seed, device)
     g = run_mx_stages(cfg, inp)
     hin = host_inputs(inp)
@@ -340,7 +342,6 @@ def check_mx_small(cfg, seed: int, device="cuda"):
     total = ref["plan"]["total_rows"]
     src = ref["src_of"][:total]
     valid = src >= 0
-    vrows = np.nonzero(valid)[0]
     # weights: bit-exact codes and scales
     w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp)
     perm = w1_tile_rows(E, F)
@@ -355,30 +356,35 @@ def check_mx_small(cfg, seed: int, device="cuda"):
     gxs = mx_unchunk(g["xs"], total, d)
     assert np.array_equal(gxq[valid], xq_ref[src[valid]]), "dispatched codes differ"
     assert np.array_equal(gxs[valid], xs_ref[src[valid]]), "dispatched scales differ"
-    # FC1 on the oracle's own operands
+    # FC1 on the oracle's own operands: every valid row of small layers, a
+    # seeded sample of at most max_rows rows (all blocks' row positions) otherwise
     blocks = ref["plan"]["blocks"]
     row_exp = np.zeros(total, np.int32)
     for b in blocks:
         row_exp[b[1]:b[1] + 128] = b[0]
-    xq_rows = xq_ref[src[valid]]
-    xs_rows = xs_ref[src[valid]]
-    rh, rhq, rhs = O.mx_fc1_rows(np.arange(len(vrows)), row_exp[valid], xq_rows, xs_rows, w1q, w1s, F)
+    rng = np.random.default_rng(seed + 5)
+    vrows = np.nonzero(valid)[0]
+    if len(vrows) > max_rows:
+        vrows = np.sort(rng.choice(vrows, size=max_rows, replace=False))
+    rh, rhq, rhs = O.mx_fc1_rows(np.arange(len(vrows)), row_exp[vrows], xq_ref[src[vrows]], xs_ref[src[vrows]],
+                                 w1q, w1s, F)
     ghq = g["hq"][:total].cpu().numpy()
     ghs = mx_unchunk(g["hs"], total, F)
-    assert_mx_h_close(ghq[valid], ghs[valid], rh, rhq, rhs, "h (MXFP8)")
+    assert_mx_h_close(ghq[vrows], ghs[vrows], rh, rhq, rhs, "h (MXFP8)")
     assert not ghq[~valid].any() and not ghs[~valid].any(), "padding rows of h must be zero codes and scales"
     # FC2 on the oracle's h
-    ry = O.mx_fc2_rows(row_exp[valid], rhq, rhs, w2q, w2s, d)
+    ry = O.mx_fc2_rows(row_exp[vrows], rhq, rhs, w2q, w2s, d)
     gy = to_f64(g["yp"][:total])
-    assert_close(gy[valid], ry, C.BF16, "yp")
+    assert_close(gy[vrows], ry, C.BF16, "yp")
     assert not gy[~valid].any(), "padding rows of yp must be zero"
-    # the whole layer
-    rout = O.mx_token_out(np.arange(cfg.T), xq_ref, xs_ref, ref["idx"], ref["w"], w1q, w1s, w2q, w2s, F)
-    assert_close(to_f64(g["out"]), rout, C.BF16, "out")
+    # the whole layer, on all tokens or a seeded sample
+    toks = np.arange(cfg.T) if cfg.T <= max_tokens else np.sort(rng.choice(cfg.T, size=max_tokens, replace=False))
+    rout = O.mx_token_out(toks, xq_ref, xs_ref, ref["idx"], ref["w"], w1q, w1s, w2q, w2s, F)
+    assert_close(to_f64(g["out"])[toks], rout, C.BF16, "out")
     return g, ref, inp
 
 
-def check_mx_full_size(cfg, seed: int, n_tokens: int = 4, device="cuda"):
+def check_mx_full_size(cfg, seed: int, n_tokens: int = 3, device="cuda"):
     """Full-size MX layer through moe_layer_fwd_mx: bit-exact routing and plan
     (moe_plan), and sampled tokens of out against the oracle."""
     inp = I.make_inputs(cfg, seed, device)

@@ -63,6 +63,6 @@ def test_mx_layer_is_close_to_the_bf16_layer():
     assert rel > 1e-4, "the MX layer should not be the bf16 layer"
 
 
-@pytest.mark.parametrize("name", ["olmoe", "dsv3"])
-def test_mx_layer_full_size_sampled(name):
-    check_mx_full_size(C.NAMED[name], 0)
+@pytest.mark.parametrize("name,n_tokens", [("olmoe", 3), ("dsv3", 1)])
+def test_mx_layer_full_size_sampled(name, n_tokens):
+    check_mx_full_size(C.NAMED[name], 0, n_tokens=n_tokens)
