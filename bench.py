@@ -359,7 +359,8 @@ def time_mx(cfg, inp, args, world, dev, stream, pg):
             ms = max_over_ranks([ms], dev)[0]
         return ms / args.steps
 
-    ms = timed(lambda: layer.forward_mx(lg, x, mxw, stream=stream))
+    with ClockSampler(dev) as clk:
+        ms = timed(lambda: layer.forward_mx(lg, x, mxw, stream=stream))
     out = layer.forward_mx(lg, x, mxw, stream=stream).float()
     torch.cuda.synchronize(dev)
     rel_to_bf16 = (torch.linalg.norm(out - ref) / torch.linalg.norm(ref)).item()
@@ -419,6 +420,7 @@ def time_mx(cfg, inp, args, world, dev, stream, pg):
             "layer_roofline_frac": (t_roof * 1e3) / ms, "layer_roofline_ms": t_roof * 1e3,
             "weight_quantize_ms": q0.elapsed_time(q1),
             "rel_diff_to_bf16_layer": rel_to_bf16,
+            "clocks": clk.summary(),
             "note": "moe_layer_fwd_mx: plan, dispatch with MXFP8 quantization of x, FC1 + SwiGLU with h "
                     "quantized to MXFP8 in the epilogue, FC2, combine; E4M3 elements, E8M0 scale per 32; "
                     "weights quantized once outside the timed region"}
@@ -562,16 +564,16 @@ def run_mine(args, world, rank, local):
         torch.distributed.barrier()
         elapsed_ms, e2e_ms, e2e_serial_ms = max_over_ranks([elapsed_ms, e2e_ms, e2e_serial_ms], dev)
 
-    bwd = None
-    if not args.no_backward and cfg.dtype == C.BF16 and cfg.F % 256 == 0:
-        del layer_h, layers
-        torch.cuda.empty_cache()
-        bwd = time_backward(cfg, inp, args, world, dev, stream, pg)
-
+    del layer_h, layers
+    torch.cuda.empty_cache()
     mx = None
     if not args.no_mx and cfg.dtype == C.BF16:
-        torch.cuda.empty_cache()
         mx = time_mx(cfg, inp, args, world, dev, stream, pg)
+
+    bwd = None
+    if not args.no_backward and cfg.dtype == C.BF16 and cfg.F % 256 == 0:
+        torch.cuda.empty_cache()
+        bwd = time_backward(cfg, inp, args, world, dev, stream, pg)
 
     plans = plan_comparison(cfg, inp, dev) if rank == 0 else None
     cpu = None

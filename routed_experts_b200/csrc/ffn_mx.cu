@@ -13,27 +13,27 @@
 // TMA warp, an MMA warp and four epilogue warps per CTA, every wait bounded)
 // with these differences:
 //   - operands are E4M3 bytes: one 128-byte swizzled row holds 128 K
-//     elements, so a k-step is 128 deep and takes four MMAs of
-//     tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale (M = 256, N = 128,
-//     K = 32);
+//     elements, so a k-step is 128 deep: four K = 32 slices of
+//     tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale (M = 256);
 //   - each k-step also brings the scale factors of its 128 A rows and 256 B
 //     rows (512 bytes per 128 rows, already in the chunked layout of
 //     mx_scale_offset) into a small ring beside the operand stages, on the
 //     same TMA barrier; the MMA thread copies them to TMEM (tcgen05.cp
 //     32x128b.warpx4, four columns per 128 rows) ahead of the k-step's MMAs,
 //     alternating between two column sets;
-//   - an item is 256 rows x 256 columns, issued as two N = 128 MMAs per K
-//     slice into two 128-column TMEM half-buffers. Three half-buffers rotate
-//     (item k takes buffers 2k mod 3 and 2k+1 mod 3) and the epilogue frees
-//     each half as soon as it has read it, so the next item's MMAs wait only
-//     for the first half of the previous item's epilogue; two full
-//     256-column accumulators would leave no TMEM for the scales. Each CTA
-//     holds 128 weight rows of the item as two 64-row halves. FC1's weight
-//     rows are stored with every 128 rows of an expert holding 64 gate rows
-//     then the matching 64 up rows, so each half-MMA's accumulator holds
-//     [64 gate | 64 up] columns (even CTA: gate, odd CTA: up) and a half is
-//     SwiGLU-complete: 64 h columns per half, 128 per item; an FC2 item is
-//     256 columns of d;
+//   - an item is 256 rows x 256 columns held in two 128-column TMEM
+//     half-buffers. Three half-buffers rotate (item k takes buffers 2k mod 3
+//     and 2k+1 mod 3) and the epilogue frees each half as soon as it has read
+//     it, so the next item's MMAs wait only for the first half of the
+//     previous item's epilogue; two full 256-column accumulators would leave
+//     no TMEM for the scales. When the item's half-buffers are adjacent (two
+//     items in three) one N = 256 MMA per K slice covers both and each CTA
+//     holds 128 consecutive weight rows of the item; otherwise two N = 128
+//     MMAs per K slice fill them and each CTA holds 64 rows of each half;
+//   - FC1's weight rows are stored with every 128 rows of an expert holding
+//     64 gate rows then the matching 64 up rows, so either way a half-buffer
+//     holds [64 gate | 64 up] columns and is SwiGLU-complete: 64 h columns
+//     per half, 128 per item. An FC2 item is 256 columns of d;
 //   - the FC1 epilogue applies SwiGLU, rounds h to bf16 (FC1's bf16 output)
 //     and quantizes it to MXFP8 along F right away: each thread holds 32
 //     consecutive h values of its row, exactly one scale block, so the
@@ -335,8 +335,12 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const int e = item.x, j = item.y;
                 const int row0 = even ? item.z : (item.w >= 0 ? item.w : item.z);
                 const int wrow = e * a.b_rows + j * kMxItemN;        // the item's first weight row
-                const int b_lo = wrow + (even ? 0 : kMxHalfRows);    // this CTA's rows of half 0
-                const int b_hi = b_lo + kMxHalf;                     // and of half 1
+                // half-buffers 2k mod 3 and 2k+1 mod 3 are adjacent unless the first is the last:
+                // then one N = 256 MMA reads 128 contiguous rows per CTA (CTA c: rows 128c ..),
+                // else two N = 128 MMAs read 64 rows of each half per CTA (CTA c: rows 64c ..)
+                const bool wide = (2 * k) % kMxBufs != kMxBufs - 1;
+                const int b_lo = wrow + (wide ? (even ? 0 : kMxHalf) : (even ? 0 : kMxHalfRows));
+                const int b_hi = b_lo + (wide ? kMxHalfRows : kMxHalf);
                 const int a_chunk0 = (row0 / 128) * kc;
                 const int b_chunk0 = (wrow / 128) * kc, b_chunk1 = (wrow / 128 + 1) * kc;
                 for (int kb = 0; kb < kb_count; ++kb) {
@@ -381,6 +385,7 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     !role_wait_cluster(&S->hempty[b1], p1 ^ 1, a.spin, abort_flag, a.header)) { ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t d0 = tmem + (uint32_t)(b0 * kMxHalf), d1 = tmem + (uint32_t)(b1 * kMxHalf);
+                const bool wide = b1 == b0 + 1;   // adjacent half-buffers: one N = 256 MMA per K slice
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!role_wait(&S->full[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
                     ptx::tc_fence_after();
@@ -391,15 +396,26 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     ptx::tmem_cp_sf_pair(sfa_t, ptx::sdesc_sf(sf_addr));
                     ptx::tmem_cp_sf_pair(sfa_t + 4u, ptx::sdesc_sf(sf_addr + kMxSfBytes));
                     ptx::tmem_cp_sf_pair(sfa_t + 8u, ptx::sdesc_sf(sf_addr + 2 * kMxSfBytes));
+                    if (wide) {
+                        // one N = 256 MMA per K slice over both half-buffers (d1 = d0 + 128); its
+                        // B scales are the 8 columns from sfa_t + 4 (rows 0-127, then 128-255)
 #pragma unroll
-                    for (uint32_t ks = 0; ks < kMxBK / 32; ++ks) {
-                        const uint32_t idesc = ptx::idesc_mx_e4m3(2 * kBM, kMxHalf, ks, ks);
-                        const uint32_t acc = (kb | (int)ks) != 0 ? 1u : 0u;
-                        const uint64_t adesc = ptx::sdesc_k_sw128(a_addr + ks * 32);
-                        ptx::mma_mx_pair(d0, adesc, ptx::sdesc_k_sw128(b_addr + ks * 32), idesc, sfa_t | (ks << 30),
-                                         (sfa_t + 4u) | (ks << 30), acc);
-                        ptx::mma_mx_pair(d1, adesc, ptx::sdesc_k_sw128(b_addr + kMxBBytes / 2 + ks * 32), idesc,
-                                         sfa_t | (ks << 30), (sfa_t + 8u) | (ks << 30), acc);
+                        for (uint32_t ks = 0; ks < kMxBK / 32; ++ks)
+                            ptx::mma_mx_pair(d0, ptx::sdesc_k_sw128(a_addr + ks * 32),
+                                             ptx::sdesc_k_sw128(b_addr + ks * 32),
+                                             ptx::idesc_mx_e4m3(2 * kBM, kMxItemN, ks, ks), sfa_t | (ks << 30),
+                                             (sfa_t + 4u) | (ks << 30), (kb | (int)ks) != 0 ? 1u : 0u);
+                    } else {
+#pragma unroll
+                        for (uint32_t ks = 0; ks < kMxBK / 32; ++ks) {
+                            const uint32_t idesc = ptx::idesc_mx_e4m3(2 * kBM, kMxHalf, ks, ks);
+                            const uint32_t acc = (kb | (int)ks) != 0 ? 1u : 0u;
+                            const uint64_t adesc = ptx::sdesc_k_sw128(a_addr + ks * 32);
+                            ptx::mma_mx_pair(d0, adesc, ptx::sdesc_k_sw128(b_addr + ks * 32), idesc,
+                                             sfa_t | (ks << 30), (sfa_t + 4u) | (ks << 30), acc);
+                            ptx::mma_mx_pair(d1, adesc, ptx::sdesc_k_sw128(b_addr + kMxBBytes / 2 + ks * 32), idesc,
+                                             sfa_t | (ks << 30), (sfa_t + 8u) | (ks << 30), acc);
+                        }
                     }
                     issued = true;
                     sf_set ^= 1u;
