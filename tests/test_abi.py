@@ -144,6 +144,62 @@ def test_fused_ffn_checks_its_arguments(M):
                                   None) == M.MOE_ERR_UNSUPPORTED
 
 
+def test_mx_buffer_sizes(M):
+    cfg = C.OLMOE
+    cap = M.moe_rows_capacity(cfg)
+    E, d, F = cfg.E, cfg.d, cfg.F
+
+    def scale_bytes(rows, K):
+        return -(-rows // 128) * (K // 128) * 512
+
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_XQ) == cap * d
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_XS) == scale_bytes(cap, d)
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_HQ) == cap * F
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_HS) == scale_bytes(cap, F)
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_W1Q) == E * 2 * F * d
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_W1S) == E * 2 * F * d // 32
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_W2Q) == E * d * F
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_W2S) == E * d * F // 32
+    L = M.lib()
+    n = ctypes.c_size_t(0)
+    assert L.moe_mx_buffer_bytes(ctypes.byref(M.config(cfg)), 8, ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
+    # fp32 layers and widths the MX GEMM does not tile are unsupported
+    for bad in (C.TINY, cfg.replace(F=1000), cfg.replace(d=2176)):
+        assert L.moe_mx_buffer_bytes(ctypes.byref(M.config(bad)), 0, ctypes.byref(n)) in \
+            (M.MOE_ERR_UNSUPPORTED, M.MOE_ERR_INVALID_ARG), bad
+
+
+def test_mx_calls_check_their_arguments(M):
+    L = M.lib()
+    fake = ctypes.c_void_p(1 << 20)      # never dereferenced: every check below fails first
+    odd = ctypes.c_void_p((1 << 20) + 8)
+    s = ctypes.c_size_t
+    bf = C.TINY.replace(dtype=C.BF16, tile=128, d=256, F=256)
+    cfg = ctypes.byref(M.config(bf))
+    plan_need = M.moe_workspace_size(bf, M.WS_PLAN)
+    layer_need = M.moe_workspace_size(bf, M.WS_LAYER)
+    # weights: a null or misaligned pointer, or an unsupported shape (the call has no workspace to check)
+    assert L.moe_mx_quantize_weights(cfg, fake, fake, fake, None, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_mx_quantize_weights(cfg, fake, odd, fake, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    tiny = ctypes.byref(M.config(C.TINY))
+    assert L.moe_mx_quantize_weights(tiny, fake, fake, fake, fake, fake, fake, None) == M.MOE_ERR_UNSUPPORTED
+    assert L.moe_dispatch_mx(cfg, fake, fake, fake, fake, s(plan_need - 1), None) == M.MOE_ERR_WORKSPACE
+    assert L.moe_dispatch_mx(cfg, fake, None, fake, fake, s(plan_need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_fc1_mx(cfg, fake, fake, fake, fake, fake, fake, fake, s(plan_need - 1), None) == \
+        M.MOE_ERR_WORKSPACE
+    assert L.moe_expert_fc1_mx(cfg, fake, odd, fake, fake, fake, fake, fake, s(plan_need), None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_fc2_mx(cfg, fake, fake, fake, fake, fake, fake, s(plan_need - 1), None) == \
+        M.MOE_ERR_WORKSPACE
+    assert L.moe_expert_fc2_mx(cfg, fake, fake, fake, None, fake, fake, s(plan_need), None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_fwd_mx(cfg, fake, fake, fake, fake, fake, fake, fake, fake, s(layer_need - 1), None) == \
+        M.MOE_ERR_WORKSPACE
+    assert L.moe_layer_fwd_mx(cfg, fake, fake, fake, fake, fake, fake, None, fake, s(layer_need), None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_fwd_mx(tiny, fake, fake, fake, fake, fake, fake, fake, fake, s(layer_need), None) == \
+        M.MOE_ERR_UNSUPPORTED
+
+
 def test_binding_refuses_to_run_without_library(tmp_path, monkeypatch):
     from routed_experts_b200 import moe
     monkeypatch.setattr(moe, "_lib", None)
