@@ -1071,9 +1071,54 @@ static uint8_t mx_scale_code(double amax)
     return (uint8_t)s;
 }
 
-/* Quantize the rows of an fp64 matrix [rows, K] (K a multiple of 32) to
- * MXFP8: codes [rows, K] and scales [rows, K/32], both row-major. */
-static void mx_quantize_rows(int64_t rows, int32_t K, const double* v, uint8_t* codes, uint8_t* scales)
+/* MXFP4 ([MegaFlux] §4.1: MXFP4 weights in the forward; [MoonEP] "A
+ * bandwidth-only model": packed 4-bit elements plus one scale per 32).
+ * READING: OCP E2M1 elements: 1 sign bit, 2 exponent bits (bias 1), 1
+ * mantissa bit, subnormal at exponent field 0; magnitudes 0, 0.5, 1, 1.5, 2,
+ * 3, 4, 6; no NaN or infinity. The block scale uses the exponent of E2M1's
+ * largest normal (6 = 1.5 * 2^2): s = floor(log2 max|v|) - 2 + 127. Here a
+ * code is kept one per byte (0..15); packing two per byte is storage. */
+static double e2m1_value(uint8_t c)
+{
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    return (c & 8) ? -mag[c & 7] : mag[c & 7];
+}
+
+/* v rounded to E2M1: the nearest of the eight magnitudes, ties to the even
+ * code, saturating at 6; the sign of v is kept. */
+static uint8_t e2m1_encode(double v)
+{
+    const uint8_t sign = signbit(v) ? 8 : 0;
+    const double a = fabs(v);
+    uint8_t best = 0;
+    double bd = INFINITY;
+    for (uint8_t c = 0; c < 8; ++c) {
+        const double dd = fabs(e2m1_value(c) - a);
+        if (dd < bd || (dd == bd && (c & 1) == 0)) { bd = dd; best = c; }
+    }
+    return sign | best;
+}
+
+enum { ORC_MX_E4M3 = 0, ORC_MX_E2M1 = 1 };
+
+static int elem_emax(int fmt) { return fmt == ORC_MX_E2M1 ? 2 : 8; }
+
+/* The scale exponent of a block with largest magnitude amax for element format fmt. */
+static uint8_t mx_scale_code_fmt(double amax, int fmt)
+{
+    if (amax == 0.0) return 0;
+    int ex;
+    frexp(amax, &ex);
+    int s = (ex - 1) - elem_emax(fmt) + 127;
+    if (s < 0) s = 0;
+    if (s > 254) s = 254;
+    return (uint8_t)s;
+}
+
+/* Quantize the rows of an fp64 matrix [rows, K] (K a multiple of 32) to an MX
+ * format: codes [rows, K] and scales [rows, K/32], both row-major. */
+static void mx_quantize_rows_fmt(int64_t rows, int32_t K, int fmt, const double* v, uint8_t* codes,
+                                 uint8_t* scales)
 {
     for (int64_t r = 0; r < rows; ++r) {
         for (int32_t b = 0; b < K / 32; ++b) {
@@ -1081,17 +1126,31 @@ static void mx_quantize_rows(int64_t rows, int32_t K, const double* v, uint8_t* 
             double amax = 0.0;
             for (int i = 0; i < 32; ++i)
                 if (fabs(blk[i]) > amax) amax = fabs(blk[i]);
-            const uint8_t s = mx_scale_code(amax);
+            const uint8_t s = mx_scale_code_fmt(amax, fmt);
             scales[r * (K / 32) + b] = s;
             const double X = ldexp(1.0, (int)s - 127);
-            for (int i = 0; i < 32; ++i) codes[r * K + (int64_t)b * 32 + i] = e4m3_encode(blk[i] / X);
+            for (int i = 0; i < 32; ++i)
+                codes[r * K + (int64_t)b * 32 + i] = fmt == ORC_MX_E2M1 ? e2m1_encode(blk[i] / X)
+                                                                         : e4m3_encode(blk[i] / X);
         }
     }
 }
 
+static void mx_quantize_rows(int64_t rows, int32_t K, const double* v, uint8_t* codes, uint8_t* scales)
+{
+    mx_quantize_rows_fmt(rows, K, ORC_MX_E4M3, v, codes, scales);
+}
+
+static double mx_value_fmt(const uint8_t* codes, const uint8_t* scales, int32_t K, int64_t r, int32_t k, int fmt)
+{
+    const uint8_t c = codes[r * K + k];
+    return (fmt == ORC_MX_E2M1 ? e2m1_value(c) : e4m3_value(c)) *
+           ldexp(1.0, (int)scales[r * (K / 32) + k / 32] - 127);
+}
+
 static double mx_value(const uint8_t* codes, const uint8_t* scales, int32_t K, int64_t r, int32_t k)
 {
-    return e4m3_value(codes[r * K + k]) * ldexp(1.0, (int)scales[r * (K / 32) + k / 32] - 127);
+    return mx_value_fmt(codes, scales, K, r, k, ORC_MX_E4M3);
 }
 
 /* MXFP8 quantization of a bf16 or fp32 matrix [rows, K]. */
@@ -1117,6 +1176,35 @@ int orc_mx_dequantize(int64_t rows, int32_t K, const uint8_t* codes, const uint8
     return ORC_OK;
 }
 
+/* Quantization of a bf16 or fp32 matrix [rows, K] to an MX format (fmt 0:
+ * MXFP8 E4M3, 1: MXFP4 E2M1, one code per byte). */
+int orc_mx_quantize_fmt(int64_t rows, int32_t K, int32_t dtype, int32_t fmt, const void* x, uint8_t* codes,
+                        uint8_t* scales)
+{
+    if (K % 32 != 0 || (fmt != ORC_MX_E4M3 && fmt != ORC_MX_E2M1)) return ORC_ERR_ARG;
+    double* row = (double*)malloc(sizeof(double) * (size_t)K);
+    if (!row) return ORC_ERR_INTERNAL;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int32_t k = 0; k < K; ++k) row[k] = load_elem(x, r * K + k, dtype);
+        mx_quantize_rows_fmt(1, K, fmt, row, codes + r * K, scales + r * (K / 32));
+    }
+    free(row);
+    return ORC_OK;
+}
+
+int orc_mx_dequantize_fmt(int64_t rows, int32_t K, int32_t fmt, const uint8_t* codes, const uint8_t* scales,
+                          double* out)
+{
+    if (K % 32 != 0 || (fmt != ORC_MX_E4M3 && fmt != ORC_MX_E2M1)) return ORC_ERR_ARG;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int32_t k = 0; k < K; ++k) out[r * K + k] = mx_value_fmt(codes, scales, K, r, k, fmt);
+    return ORC_OK;
+}
+
+uint8_t orc_e2m1_encode(double v) { return e2m1_encode(v); }
+double orc_e2m1_value(uint8_t c) { return e2m1_value(c); }
+uint8_t orc_mx_scale_code_fmt(double amax, int32_t fmt) { return mx_scale_code_fmt(amax, fmt); }
+
 /* E4M3 codes <-> values, for the pins. */
 uint8_t orc_e4m3_encode(double v) { return e4m3_encode(v); }
 double orc_e4m3_value(uint8_t c) { return e4m3_value(c); }
@@ -1129,7 +1217,7 @@ uint8_t orc_mx_scale_code(double amax) { return mx_scale_code(amax); }
  * READING: FC1 writes bf16 (§4.1: bf16 outputs) and FC2's MXFP8 operand is
  * quantized from those bf16 values. */
 static void mx_fc1_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* xs, int64_t xrow,
-                       const uint8_t* w1q, const uint8_t* w1s, int32_t e,
+                       const uint8_t* w1q, const uint8_t* w1s, int32_t wfmt, int32_t e,
                        double* hb /*[F]*/, uint8_t* hq /*[F]*/, uint8_t* hs /*[F/32]*/)
 {
     const int64_t g0 = (int64_t)e * 2 * F, u0 = g0 + F;
@@ -1137,8 +1225,8 @@ static void mx_fc1_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* x
         double a = 0.0, g = 0.0;
         for (int32_t i = 0; i < d; ++i) {
             const double xv = mx_value(xq, xs, d, xrow, i);
-            a += xv * mx_value(w1q, w1s, d, g0 + j, i);
-            g += xv * mx_value(w1q, w1s, d, u0 + j, i);
+            a += xv * mx_value_fmt(w1q, w1s, d, g0 + j, i, wfmt);
+            g += xv * mx_value_fmt(w1q, w1s, d, u0 + j, i, wfmt);
         }
         hb[j] = round_as(a / (1.0 + exp(-a)) * g, ORC_ROUND_BF16);
     }
@@ -1148,45 +1236,46 @@ static void mx_fc1_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* x
 /* FC2 of one routed entry: an MXFP8 row of h (codes hq, scales hs) through
  * expert e's W2 = w_down[e] (MXFP8 along F), fp64, y rounded to bf16. */
 static void mx_fc2_row(int32_t d, int32_t F, const uint8_t* hq, const uint8_t* hs, const uint8_t* w2q,
-                       const uint8_t* w2s, int32_t e, double* y /*[d]*/)
+                       const uint8_t* w2s, int32_t wfmt, int32_t e, double* y /*[d]*/)
 {
     const int64_t dn0 = (int64_t)e * d;
     for (int32_t i = 0; i < d; ++i) {
         double s = 0.0;
-        for (int32_t j = 0; j < F; ++j) s += mx_value(hq, hs, F, 0, j) * mx_value(w2q, w2s, F, dn0 + i, j);
+        for (int32_t j = 0; j < F; ++j)
+            s += mx_value(hq, hs, F, 0, j) * mx_value_fmt(w2q, w2s, F, dn0 + i, j, wfmt);
         y[i] = round_as(s, ORC_ROUND_BF16);
     }
 }
 
 static void mx_ffn_row(int32_t d, int32_t F, const uint8_t* xq, const uint8_t* xs, int64_t xrow,
-                       const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s, int32_t e,
-                       double* hb /*[F]*/, uint8_t* hq /*[F]*/, uint8_t* hs /*[F/32]*/, double* y /*[d]*/)
+                       const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s, int32_t wfmt,
+                       int32_t e, double* hb /*[F]*/, uint8_t* hq /*[F]*/, uint8_t* hs /*[F/32]*/, double* y /*[d]*/)
 {
-    mx_fc1_row(d, F, xq, xs, xrow, w1q, w1s, e, hb, hq, hs);
-    mx_fc2_row(d, F, hq, hs, w2q, w2s, e, y);
+    mx_fc1_row(d, F, xq, xs, xrow, w1q, w1s, wfmt, e, hb, hq, hs);
+    mx_fc2_row(d, F, hq, hs, w2q, w2s, wfmt, e, y);
 }
 
 /* FC1 alone for n rows of an MXFP8 activation matrix (row rows[i], expert
  * experts[i]): h (bf16 values), its MXFP8 codes and scales. */
 int orc_mx_fc1_rows(int32_t d, int32_t F, int64_t n, const int64_t* rows, const int32_t* experts,
-                    const uint8_t* xq, const uint8_t* xs, const uint8_t* w1q, const uint8_t* w1s,
+                    const uint8_t* xq, const uint8_t* xs, const uint8_t* w1q, const uint8_t* w1s, int32_t wfmt,
                     double* h_out /*[n,F]*/, uint8_t* hq_out /*[n,F]*/, uint8_t* hs_out /*[n,F/32]*/)
 {
     if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
     for (int64_t i = 0; i < n; ++i)
-        mx_fc1_row(d, F, xq, xs, rows[i], w1q, w1s, experts[i], h_out + (size_t)i * F, hq_out + (size_t)i * F,
-                   hs_out + (size_t)i * (F / 32));
+        mx_fc1_row(d, F, xq, xs, rows[i], w1q, w1s, wfmt, experts[i], h_out + (size_t)i * F,
+                   hq_out + (size_t)i * F, hs_out + (size_t)i * (F / 32));
     return ORC_OK;
 }
 
 /* FC2 alone for n MXFP8 rows of h (row i through expert experts[i]): y as
  * bf16 values. */
 int orc_mx_fc2_rows(int32_t d, int32_t F, int64_t n, const int32_t* experts, const uint8_t* hq,
-                    const uint8_t* hs, const uint8_t* w2q, const uint8_t* w2s, double* y_out /*[n,d]*/)
+                    const uint8_t* hs, const uint8_t* w2q, const uint8_t* w2s, int32_t wfmt, double* y_out /*[n,d]*/)
 {
     if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
     for (int64_t i = 0; i < n; ++i)
-        mx_fc2_row(d, F, hq + (size_t)i * F, hs + (size_t)i * (F / 32), w2q, w2s, experts[i],
+        mx_fc2_row(d, F, hq + (size_t)i * F, hs + (size_t)i * (F / 32), w2q, w2s, wfmt, experts[i],
                    y_out + (size_t)i * d);
     return ORC_OK;
 }
@@ -1195,12 +1284,12 @@ int orc_mx_fc2_rows(int32_t d, int32_t F, int64_t n, const int32_t* experts, con
  * its MXFP8 codes and scales, and y (bf16 values). */
 int orc_mx_entry_ffn(int32_t d, int32_t F, int64_t n, const int64_t* tokens, const int32_t* experts,
                      const uint8_t* xq, const uint8_t* xs, const uint8_t* w1q, const uint8_t* w1s,
-                     const uint8_t* w2q, const uint8_t* w2s, double* h_out /*[n,F]*/, uint8_t* hq_out /*[n,F]*/,
-                     uint8_t* hs_out /*[n,F/32]*/, double* y_out /*[n,d]*/)
+                     const uint8_t* w2q, const uint8_t* w2s, int32_t wfmt, double* h_out /*[n,F]*/,
+                     uint8_t* hq_out /*[n,F]*/, uint8_t* hs_out /*[n,F/32]*/, double* y_out /*[n,d]*/)
 {
     if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
     for (int64_t i = 0; i < n; ++i)
-        mx_ffn_row(d, F, xq, xs, tokens[i], w1q, w1s, w2q, w2s, experts[i], h_out + (size_t)i * F,
+        mx_ffn_row(d, F, xq, xs, tokens[i], w1q, w1s, w2q, w2s, wfmt, experts[i], h_out + (size_t)i * F,
                    hq_out + (size_t)i * F, hs_out + (size_t)i * (F / 32), y_out + (size_t)i * d);
     return ORC_OK;
 }
@@ -1209,7 +1298,7 @@ int orc_mx_entry_ffn(int32_t d, int32_t F, int64_t n, const int64_t* tokens, con
  * the weighted combine in fp64, rounded to bf16. */
 int orc_mx_token_out(int32_t d, int32_t F, int32_t K, int64_t n_tok, const int64_t* tokens,
                      const uint8_t* xq, const uint8_t* xs, const int32_t* idx, const float* w,
-                     const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s,
+                     const uint8_t* w1q, const uint8_t* w1s, const uint8_t* w2q, const uint8_t* w2s, int32_t wfmt,
                      double* out /*[n_tok, d]*/)
 {
     if (d % 32 != 0 || F % 32 != 0) return ORC_ERR_ARG;
@@ -1221,7 +1310,7 @@ int orc_mx_token_out(int32_t d, int32_t F, int32_t K, int64_t n_tok, const int64
     for (int64_t n = 0; n < n_tok; ++n) {
         const int64_t t = tokens[n];
         for (int32_t k = 0; k < K; ++k)
-            mx_ffn_row(d, F, xq, xs, t, w1q, w1s, w2q, w2s, idx[t * K + k], hb, hq, hs, y + (size_t)k * d);
+            mx_ffn_row(d, F, xq, xs, t, w1q, w1s, w2q, w2s, wfmt, idx[t * K + k], hb, hq, hs, y + (size_t)k * d);
         for (int32_t i = 0; i < d; ++i) {
             double s = 0.0;
             for (int32_t k = 0; k < K; ++k) s += (double)w[t * K + k] * y[(size_t)k * d + i];

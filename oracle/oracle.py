@@ -72,12 +72,20 @@ def lib():
         L.orc_e4m3_value.restype = ctypes.c_double
         L.orc_mx_scale_code.argtypes = [ctypes.c_double]
         L.orc_mx_scale_code.restype = ctypes.c_uint8
-        L.orc_mx_entry_ffn.argtypes = [i32, i32, i64, P, P, P, P, P, P, P, P, P, P, P, P]
-        L.orc_mx_token_out.argtypes = [i32, i32, i32, i64, P, P, P, P, P, P, P, P, P, P]
-        L.orc_mx_fc1_rows.argtypes = [i32, i32, i64, P, P, P, P, P, P, P, P, P]
-        L.orc_mx_fc2_rows.argtypes = [i32, i32, i64, P, P, P, P, P, P]
+        L.orc_mx_entry_ffn.argtypes = [i32, i32, i64, P, P, P, P, P, P, P, P, i32, P, P, P, P]
+        L.orc_mx_token_out.argtypes = [i32, i32, i32, i64, P, P, P, P, P, P, P, P, P, i32, P]
+        L.orc_mx_quantize_fmt.argtypes = [i64, i32, i32, i32, P, P, P]
+        L.orc_mx_dequantize_fmt.argtypes = [i64, i32, i32, P, P, P]
+        L.orc_e2m1_encode.argtypes = [ctypes.c_double]
+        L.orc_e2m1_encode.restype = ctypes.c_uint8
+        L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+        L.orc_e2m1_value.restype = ctypes.c_double
+        L.orc_mx_scale_code_fmt.argtypes = [ctypes.c_double, i32]
+        L.orc_mx_scale_code_fmt.restype = ctypes.c_uint8
+        L.orc_mx_fc1_rows.argtypes = [i32, i32, i64, P, P, P, P, P, P, i32, P, P, P]
+        L.orc_mx_fc2_rows.argtypes = [i32, i32, i64, P, P, P, P, P, i32, P]
         for f in ("orc_mx_quantize", "orc_mx_dequantize", "orc_mx_entry_ffn", "orc_mx_token_out",
-                  "orc_mx_fc1_rows", "orc_mx_fc2_rows"):
+                  "orc_mx_fc1_rows", "orc_mx_fc2_rows", "orc_mx_quantize_fmt", "orc_mx_dequantize_fmt"):
             getattr(L, f).restype = ctypes.c_int
         for f in ("orc_topk_gate", "orc_histogram", "orc_plan", "orc_plan_blocks", "orc_row_maps", "orc_dispatch",
                   "orc_expert_ffn", "orc_combine", "orc_token_out", "orc_dense_layer", "orc_entry_ffn"):
@@ -388,6 +396,41 @@ def timed_sample(logits, x, w_gu, w_down, *, K, R, tile, budget, gating, dtype,
 
 # ---------------------------------------------------------------- MX (block-scaled) forward
 
+MX_E4M3, MX_E2M1 = 0, 1   # element formats: MXFP8 (E4M3), MXFP4 (E2M1, one code per byte here)
+
+
+def e2m1_encode(v: float) -> int:
+    """A value rounded to an E2M1 code (nearest, ties to even, saturating at 6)."""
+    return int(lib().orc_e2m1_encode(float(v)))
+
+
+def e2m1_value(code: int) -> float:
+    return float(lib().orc_e2m1_value(int(code)))
+
+
+def mx_scale_code_fmt(amax: float, fmt: int) -> int:
+    return int(lib().orc_mx_scale_code_fmt(float(amax), int(fmt)))
+
+
+def mx_quantize_fmt(x: np.ndarray, dtype: int, fmt: int):
+    """MX quantization of the rows of a [rows, K] matrix in element format fmt: (codes uint8 [rows, K],
+    one code per byte, scale exponents uint8 [rows, K/32])."""
+    x = np.ascontiguousarray(x)
+    rows, K = x.shape
+    codes = np.empty((rows, K), np.uint8)
+    scales = np.empty((rows, K // 32), np.uint8)
+    _check(lib().orc_mx_quantize_fmt(rows, K, dtype, fmt, _p(x), _p(codes), _p(scales)), "mx_quantize_fmt")
+    return codes, scales
+
+
+def mx_dequantize_fmt(codes: np.ndarray, scales: np.ndarray, fmt: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    scales = np.ascontiguousarray(scales, dtype=np.uint8)
+    rows, K = codes.shape
+    out = np.empty((rows, K), np.float64)
+    _check(lib().orc_mx_dequantize_fmt(rows, K, fmt, _p(codes), _p(scales), _p(out)), "mx_dequantize_fmt")
+    return out
+
 def e4m3_encode(v: float) -> int:
     """A value rounded to an E4M3 code (nearest, ties to even, saturating at 448)."""
     return int(lib().orc_e4m3_encode(float(v)))
@@ -422,16 +465,17 @@ def mx_dequantize(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     return out
 
 
-def mx_weights(w_gu: np.ndarray, w_down: np.ndarray, dtype: int):
-    """MXFP8 expert weights: W1 = w_gate_up [E, 2F, d] along d, W2 = w_down [E, d, F] along F."""
+def mx_weights(w_gu: np.ndarray, w_down: np.ndarray, dtype: int, fmt: int = MX_E4M3):
+    """MX expert weights (fmt: MXFP8 or MXFP4): W1 = w_gate_up [E, 2F, d] along d, W2 = w_down
+    [E, d, F] along F."""
     E, F2, d = w_gu.shape
     F = F2 // 2
-    w1q, w1s = mx_quantize(np.ascontiguousarray(w_gu).reshape(E * F2, d), dtype)
-    w2q, w2s = mx_quantize(np.ascontiguousarray(w_down).reshape(E * d, F), dtype)
+    w1q, w1s = mx_quantize_fmt(np.ascontiguousarray(w_gu).reshape(E * F2, d), dtype, fmt)
+    w2q, w2s = mx_quantize_fmt(np.ascontiguousarray(w_down).reshape(E * d, F), dtype, fmt)
     return w1q, w1s, w2q, w2s
 
 
-def mx_entry_ffn(tokens, experts, xq, xs, w1q, w1s, w2q, w2s, F: int):
+def mx_entry_ffn(tokens, experts, xq, xs, w1q, w1s, w2q, w2s, F: int, wfmt: int = MX_E4M3):
     """Routed entries of the MX expert FFN: h (bf16 values, fp64 array), h's MXFP8 codes and
     scales, and y (bf16 values, fp64 array)."""
     tokens = np.ascontiguousarray(tokens, dtype=np.int64)
@@ -444,11 +488,11 @@ def mx_entry_ffn(tokens, experts, xq, xs, w1q, w1s, w2q, w2s, F: int):
     hs = np.empty((n, F // 32), np.uint8)
     y = np.empty((n, d), np.float64)
     _check(lib().orc_mx_entry_ffn(d, F, n, _p(tokens), _p(experts), _p(xq), _p(xs), _p(w1q), _p(w1s), _p(w2q),
-                                  _p(w2s), _p(h), _p(hq), _p(hs), _p(y)), "mx_entry_ffn")
+                                  _p(w2s), wfmt, _p(h), _p(hq), _p(hs), _p(y)), "mx_entry_ffn")
     return h, hq, hs, y
 
 
-def mx_token_out(tokens, xq, xs, idx, w, w1q, w1s, w2q, w2s, F: int) -> np.ndarray:
+def mx_token_out(tokens, xq, xs, idx, w, w1q, w1s, w2q, w2s, F: int, wfmt: int = MX_E4M3) -> np.ndarray:
     """Layer output rows (bf16 values, fp64 array) of selected tokens of the MX layer."""
     tokens = np.ascontiguousarray(tokens, dtype=np.int64)
     idx = np.ascontiguousarray(idx, dtype=np.int32)
@@ -458,11 +502,11 @@ def mx_token_out(tokens, xq, xs, idx, w, w1q, w1s, w2q, w2s, F: int) -> np.ndarr
     K = idx.shape[1]
     out = np.empty((tokens.shape[0], d), np.float64)
     _check(lib().orc_mx_token_out(d, F, K, tokens.shape[0], _p(tokens), _p(xq), _p(xs), _p(idx), _p(w), _p(w1q),
-                                  _p(w1s), _p(w2q), _p(w2s), _p(out)), "mx_token_out")
+                                  _p(w1s), _p(w2q), _p(w2s), wfmt, _p(out)), "mx_token_out")
     return out
 
 
-def mx_fc1_rows(rows, experts, xq, xs, w1q, w1s, F: int):
+def mx_fc1_rows(rows, experts, xq, xs, w1q, w1s, F: int, wfmt: int = MX_E4M3):
     """FC1 of the MX FFN alone for rows of an MXFP8 activation matrix: h (bf16 values, fp64
     array) and its MXFP8 codes and scales."""
     rows = np.ascontiguousarray(rows, dtype=np.int64)
@@ -473,16 +517,17 @@ def mx_fc1_rows(rows, experts, xq, xs, w1q, w1s, F: int):
     h = np.empty((n, F), np.float64)
     hq = np.empty((n, F), np.uint8)
     hs = np.empty((n, F // 32), np.uint8)
-    _check(lib().orc_mx_fc1_rows(d, F, n, _p(rows), _p(experts), _p(xq), _p(xs), _p(w1q), _p(w1s), _p(h), _p(hq),
-                                 _p(hs)), "mx_fc1_rows")
+    _check(lib().orc_mx_fc1_rows(d, F, n, _p(rows), _p(experts), _p(xq), _p(xs), _p(w1q), _p(w1s), wfmt, _p(h),
+                                 _p(hq), _p(hs)), "mx_fc1_rows")
     return h, hq, hs
 
 
-def mx_fc2_rows(experts, hq, hs, w2q, w2s, d: int) -> np.ndarray:
+def mx_fc2_rows(experts, hq, hs, w2q, w2s, d: int, wfmt: int = MX_E4M3) -> np.ndarray:
     """FC2 of the MX FFN alone: MXFP8 rows of h through their experts' W2 (bf16 values, fp64 array)."""
     experts = np.ascontiguousarray(experts, dtype=np.int32)
     hq, hs, w2q, w2s = (np.ascontiguousarray(a, dtype=np.uint8) for a in (hq, hs, w2q, w2s))
     n, F = hq.shape
     y = np.empty((n, d), np.float64)
-    _check(lib().orc_mx_fc2_rows(d, F, n, _p(experts), _p(hq), _p(hs), _p(w2q), _p(w2s), _p(y)), "mx_fc2_rows")
+    _check(lib().orc_mx_fc2_rows(d, F, n, _p(experts), _p(hq), _p(hs), _p(w2q), _p(w2s), wfmt, _p(y)),
+           "mx_fc2_rows")
     return y

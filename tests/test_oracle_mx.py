@@ -177,3 +177,68 @@ def test_mx_fc1_and_fc2_rows_compose_to_the_entry_ffn():
     h1, hq1, hs1 = O.mx_fc1_rows(tokens, experts, xq, xs, w1q, w1s, F)
     assert np.array_equal(h1, h) and np.array_equal(hq1, hq) and np.array_equal(hs1, hs)
     assert np.array_equal(O.mx_fc2_rows(experts, hq, hs, w2q, w2s, d), y)
+
+
+# ---------------------------------------------------------------- MXFP4 (E2M1) weights
+
+def test_e2m1_table():
+    # the format's own facts: 1 sign, 2 exponent bits (bias 1), 1 mantissa bit, subnormal 0.5
+    assert [O.e2m1_value(c) for c in range(8)] == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert [O.e2m1_value(c) for c in range(8, 16)] == [-0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def test_e2m1_encode_ties_and_saturation():
+    # midpoints go to the even code (mantissa bit 0)
+    for v, c in ((0.25, 0), (0.75, 2), (1.25, 2), (1.75, 4), (2.5, 4), (3.5, 6), (5.0, 6), (6.0, 7), (7.0, 7),
+                 (100.0, 7), (0.2, 0), (0.3, 1), (-1.3, 8 | 3), (-0.1, 8)):
+        assert O.e2m1_encode(v) == c, v
+    rng = np.random.default_rng(9)
+    vals = np.array([O.e2m1_value(c) for c in range(8)])
+    for v in rng.uniform(-7, 7, 2000):
+        c = O.e2m1_encode(v)
+        d = np.abs(vals - abs(v))
+        assert abs(O.e2m1_value(c & 7) - abs(v)) == d.min() or abs(v) > 6
+        assert (c >= 8) == (v < 0)
+
+
+def test_mxfp4_scale_and_error_bound():
+    rng = np.random.default_rng(12)
+    for amax in 2.0 ** rng.uniform(-60, 60, 2000):
+        X = 2.0 ** (O.mx_scale_code_fmt(amax, O.MX_E2M1) - 127)
+        assert 4.0 <= amax / X < 8.0          # the block maximum lands in E2M1's top binade (or saturates)
+    x = rng.standard_normal((8, 128)).astype(np.float32)
+    q, s = O.mx_quantize_fmt(x, O.FP32, O.MX_E2M1)
+    assert q.max() < 16
+    dq = O.mx_dequantize_fmt(q, s, O.MX_E2M1)
+    X = np.repeat(2.0 ** (s.astype(np.int64) - 127), 32, axis=1)
+    v = x.astype(np.float64) / X
+    err = np.abs(dq / X - v)
+    # half a step of the value's binade (steps 0.5 below 2, 1 in [2, 4), 2 in [4, 6]); saturation above 6
+    step = np.where(np.abs(v) < 2, 0.5, np.where(np.abs(v) < 4, 1.0, 2.0))
+    assert np.all((err <= step / 2 + 1e-12) | (np.abs(v) > 6))
+
+
+def test_mx_ffn_with_mxfp4_weights_on_exact_inputs():
+    """MXFP4 weights that E2M1 represents exactly: the MX FFN's h equals the plain oracle's h."""
+    rng = np.random.default_rng(6)
+    E, d, F, T = 2, 64, 64, 3
+    vals = np.array([O.e2m1_value(c) for c in range(16)])
+
+    def grid(rows, K):
+        v = rng.choice(vals, size=(rows, K // 32, 32))
+        v[:, :, 0] = rng.choice([4.0, 6.0, -4.0, -6.0], size=(rows, K // 32))
+        return (v * 2.0 ** rng.integers(-9, -5, size=(rows, K // 32, 1))).reshape(rows, K).astype(np.float32)
+
+    x = _grid_matrix(rng, T, d)
+    w_gu = grid(E * 2 * F, d).reshape(E, 2 * F, d)
+    w_dn = grid(E * d, F).reshape(E, d, F)
+    xq, xs = O.mx_quantize(x, O.FP32)
+    w1q, w1s, w2q, w2s = O.mx_weights(w_gu, w_dn, O.FP32, O.MX_E2M1)
+    assert np.array_equal(O.mx_dequantize_fmt(w1q, w1s, O.MX_E2M1), w_gu.reshape(E * 2 * F, d).astype(np.float64))
+    tokens = np.repeat(np.arange(T), E)
+    experts = np.tile(np.arange(E), T)
+    h, hq, hs, y = O.mx_entry_ffn(tokens, experts, xq, xs, w1q, w1s, w2q, w2s, F, O.MX_E2M1)
+    h_ref, _ = O.entry_ffn(tokens, experts, x, w_gu, w_dn, O.FP32, O.ROUND_BF16)
+    assert np.array_equal(h, h_ref)
+    y2 = O.mx_fc2_rows(experts, hq, hs, w2q, w2s, d, O.MX_E2M1)
+    assert np.array_equal(y2, y)
