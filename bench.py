@@ -327,17 +327,18 @@ def time_backward(cfg, inp, args, world, dev, stream, pg):
                     "gradient (8 launches); frac of the measured bf16 peak counts algorithmic FLOP"}
 
 
-def time_mx(cfg, inp, args, world, dev, stream, pg):
-    """The layer on MXFP8 expert operands (moe_layer_fwd_mx), W untimed and K
-    timed passes, plus its stages (plan, quantizing dispatch, FC1, FC2,
-    combine) timed by events between the calls; max over ranks. Weights are
-    quantized once, outside the timed region (an offline step)."""
+def time_mx(cfg, inp, args, world, dev, stream, pg, wfmt=0):
+    """The layer on MX expert operands (moe_layer_fwd_mx; wfmt 0: MXFP8 weights,
+    1: MXFP4 weights; activations MXFP8), W untimed and K timed passes, plus its
+    stages (plan, quantizing dispatch, FC1, FC2, combine) timed by events
+    between the calls; max over ranks. Weights are quantized once, outside the
+    timed region (an offline step)."""
     from routed_experts_b200 import moe as M
     lg, x, wgu, wdn = inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"]
     T, d, E, F, K = cfg.T, cfg.d, cfg.E, cfg.F, cfg.K
     q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     q0.record(stream)
-    mxw = M.MxWeights(cfg, wgu, wdn, stream)
+    mxw = M.MxWeights(cfg, wgu, wdn, stream, wfmt=wfmt)
     q1.record(stream)
     layer = M.Layer(cfg, dev)
     ref = layer.forward(lg, x, wgu, wdn, stream=stream).float().clone()
@@ -379,8 +380,8 @@ def time_mx(cfg, inp, args, world, dev, stream, pg):
     o = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
     calls = (lambda: M.moe_plan(cfg, lg, idx, w, counts, ws, stream),
              lambda: M.moe_dispatch_mx(cfg, x, xq, xs, ws, stream),
-             lambda: M.moe_expert_fc1_mx(cfg, xq, xs, mxw.w1q, mxw.w1s, hq, hs, ws, stream),
-             lambda: M.moe_expert_fc2_mx(cfg, hq, hs, mxw.w2q, mxw.w2s, yp, ws, stream),
+             lambda: M.moe_expert_fc1_mx(cfg, xq, xs, mxw.w1q, mxw.w1s, hq, hs, ws, stream, wfmt),
+             lambda: M.moe_expert_fc2_mx(cfg, hq, hs, mxw.w2q, mxw.w2s, yp, ws, stream, wfmt),
              lambda: M.moe_combine(cfg, yp, w, o, ws, stream))
     for _ in range(args.warmup):
         for f in calls:
@@ -403,7 +404,7 @@ def time_mx(cfg, inp, args, world, dev, stream, pg):
     fc1_flop, fc2_flop = 2.0 * N * d * (2 * F), 2.0 * N * F * d
     plan = M.read_plan(cfg, ws)
     active = int((np.bincount(plan["blocks"][:, 0].numpy(), minlength=E) > 0).sum()) if plan["n_blocks"] else 0
-    w_bytes = active * 3 * F * d * (1 + 1 / 32)
+    w_bytes = active * 3 * F * d * ((0.5 if wfmt else 1.0) + 1 / 32)
     alg_bytes = 4 * T * E + T * d * 2 + w_bytes + T * d * 2
     t_roof = max((fc1_flop + fc2_flop) / (fp8_peak * 1e12), alg_bytes / (pk["hbm_gbs"] * 1e9))
     disp_bytes = T * d * 2 + N * d * (1 + 1 / 32) + 4 * N
@@ -421,8 +422,9 @@ def time_mx(cfg, inp, args, world, dev, stream, pg):
             "weight_quantize_ms": q0.elapsed_time(q1),
             "rel_diff_to_bf16_layer": rel_to_bf16,
             "clocks": clk.summary(),
+            "weights": "MXFP4 (E2M1)" if wfmt else "MXFP8 (E4M3)",
             "note": "moe_layer_fwd_mx: plan, dispatch with MXFP8 quantization of x, FC1 + SwiGLU with h "
-                    "quantized to MXFP8 in the epilogue, FC2, combine; E4M3 elements, E8M0 scale per 32; "
+                    "quantized to MXFP8 in the epilogue, FC2, combine; E8M0 scale per 32 elements; "
                     "weights quantized once outside the timed region"}
 
 
@@ -566,9 +568,11 @@ def run_mine(args, world, rank, local):
 
     del layer_h, layers
     torch.cuda.empty_cache()
-    mx = None
+    mx = mx4 = None
     if not args.no_mx and cfg.dtype == C.BF16:
-        mx = time_mx(cfg, inp, args, world, dev, stream, pg)
+        mx = time_mx(cfg, inp, args, world, dev, stream, pg, 0)
+        torch.cuda.empty_cache()
+        mx4 = time_mx(cfg, inp, args, world, dev, stream, pg, 1)
 
     bwd = None
     if not args.no_backward and cfg.dtype == C.BF16 and cfg.F % 256 == 0:
@@ -654,6 +658,7 @@ def run_mine(args, world, rank, local):
         "layer_path": "moe_plan; moe_dispatch; moe_expert_fc1; moe_expert_fc2; moe_combine (the kernels of moe_layer_fwd)",
         "backward": bwd,
         "mx": mx,
+        "mx_fp4_weights": mx4,
         "fused_ffn": None if fused_ms is None else {
             "ms": fused_ms, "staged_fc1_fc2_ms": float(med[2] + med[3]),
             "note": "moe_expert_ffn_fused: FC1 and FC2 in one launch, FC2 tiles released per block pair "

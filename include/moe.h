@@ -326,22 +326,32 @@ moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void*
  * The MX calls take bf16 layers (cfg->dtype == MOE_BF16, tile 128, d % 256 ==
  * 0, F % 128 == 0) and return MOE_ERR_UNSUPPORTED for others.
  */
+/* Element format of MX expert weights: MXFP8 (E4M3, one byte per element) or
+ * MXFP4 ([MegaFlux] §4.1's forward weights: E2M1, values 0, 0.5, 1, 1.5, 2, 3,
+ * 4, 6 and their negatives, two codes per byte, element 2i in the low nibble
+ * of byte i; scale s = floor(log2 max|v|) - 2 + 127 clamped to [0, 254];
+ * nearest with ties to even, saturating at +-6). Activations and h are
+ * always MXFP8. */
+enum { MOE_MX_W_E4M3 = 0, MOE_MX_W_E2M1 = 1 };
+
 enum {
     MOE_MX_XQ = 0,   /* dispatched token rows: codes [rows_cap, d] */
     MOE_MX_XS = 1,   /*   and their scales */
     MOE_MX_HQ = 2,   /* FC1 output h: codes [rows_cap, F] */
     MOE_MX_HS = 3,   /*   and their scales */
-    MOE_MX_W1Q = 4,  /* W1 codes [E * 2F, d], rows in FC1 tile order (see moe_mx_quantize_weights) */
+    MOE_MX_W1Q = 4,  /* W1 codes [E * 2F, d] (E4M3) or [E * 2F, d / 2] (E2M1), rows in FC1 tile order */
     MOE_MX_W1S = 5,  /*   and their scales */
-    MOE_MX_W2Q = 6,  /* W2 codes [E * d, F] */
+    MOE_MX_W2Q = 6,  /* W2 codes [E * d, F] (E4M3) or [E * d, F / 2] (E2M1) */
     MOE_MX_W2S = 7   /*   and their scales */
 };
 
-/* Bytes of one of the MX buffers above for cfg. */
-moe_status moe_mx_buffer_bytes(const moe_config* cfg, int32_t which, size_t* bytes);
+/* Bytes of one of the MX buffers above for cfg and weight format wfmt (which
+ * only the weight codes depend on). */
+moe_status moe_mx_buffer_bytes(const moe_config* cfg, int32_t which, int32_t wfmt, size_t* bytes);
 
 /*
- * moe_mx_quantize_weights - MXFP8 expert weights, once, ahead of the layers.
+ * moe_mx_quantize_weights - MX expert weights (wfmt: MOE_MX_W_E4M3 or
+ * MOE_MX_W_E2M1), once, ahead of the layers.
  *   w_gate_up bf16 [E, 2F, d], w_down bf16 [E, d, F] (device): as for moe_layer_fwd.
  *   w1q, w1s (device, out): W1 along d. Rows are reordered for the MX GEMM's
  *            FC1 column tiles: row e*2F + 128*t + i holds gate row e*2F +
@@ -350,8 +360,8 @@ moe_status moe_mx_buffer_bytes(const moe_config* cfg, int32_t which, size_t* byt
  *   w2q, w2s (device, out): W2 along F, rows unchanged.
  * Sizes from moe_mx_buffer_bytes. No workspace; asynchronous on `stream`.
  */
-moe_status moe_mx_quantize_weights(const moe_config* cfg, const void* w_gate_up, const void* w_down, void* w1q,
-                                   void* w1s, void* w2q, void* w2s, moe_stream_t stream);
+moe_status moe_mx_quantize_weights(const moe_config* cfg, const void* w_gate_up, const void* w_down, int32_t wfmt,
+                                   void* w1q, void* w1s, void* w2q, void* w2s, moe_stream_t stream);
 
 /*
  * moe_dispatch_mx - step A6 with MXFP8 quantization: each token row of x
@@ -368,28 +378,33 @@ moe_status moe_dispatch_mx(const moe_config* cfg, const void* x, void* xq, void*
  * h = silu(xq W1g^T) * (xq W1u^T) with the MMA's fp32 accumulation, rounded to
  * bf16, then quantized to MXFP8 along F into hq / hs (MOE_MX_HQ / MOE_MX_HS,
  * device, out). Padding rows of a block get zero codes and scale 0.
- *   xq, xs: from moe_dispatch_mx; w1q, w1s: from moe_mx_quantize_weights.
+ *   xq, xs: from moe_dispatch_mx; w1q, w1s: from moe_mx_quantize_weights with
+ *   weight format wfmt.
  */
 moe_status moe_expert_fc1_mx(const moe_config* cfg, const void* xq, const void* xs, const void* w1q,
-                             const void* w1s, void* hq, void* hs, void* ws, size_t ws_bytes, moe_stream_t stream);
+                             const void* w1s, int32_t wfmt, void* hq, void* hs, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
 
 /*
  * moe_expert_fc2_mx - step A8 on MXFP8 operands: yp = hq W2^T, fp32
  * accumulation, stored as bf16 [rows_cap, d] (device, out); padding rows are
- * zero. hq, hs: from moe_expert_fc1_mx; w2q, w2s: from moe_mx_quantize_weights.
+ * zero. hq, hs: from moe_expert_fc1_mx; w2q, w2s: from moe_mx_quantize_weights
+ * with weight format wfmt.
  */
 moe_status moe_expert_fc2_mx(const moe_config* cfg, const void* hq, const void* hs, const void* w2q,
-                             const void* w2s, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream);
+                             const void* w2s, int32_t wfmt, void* yp, void* ws, size_t ws_bytes,
+                             moe_stream_t stream);
 
 /*
  * moe_layer_fwd_mx - the whole layer on MXFP8 expert operands: moe_plan,
  * moe_dispatch_mx, moe_expert_fc1_mx, moe_expert_fc2_mx and moe_combine, on
  * a MOE_WS_LAYER workspace (xq/xs live where xp does, hq/hs where h does).
  *   logits fp32 [T, E], x bf16 [T, d] (device); w1q/w1s/w2q/w2s from
- *   moe_mx_quantize_weights (device); out bf16 [T, d] (device, out).
+ *   moe_mx_quantize_weights with weight format wfmt (device); out bf16 [T, d]
+ *   (device, out).
  */
 moe_status moe_layer_fwd_mx(const moe_config* cfg, const float* logits, const void* x, const void* w1q,
-                            const void* w1s, const void* w2q, const void* w2s, void* out, void* ws,
+                            const void* w1s, const void* w2q, const void* w2s, int32_t wfmt, void* out, void* ws,
                             size_t ws_bytes, moe_stream_t stream);
 
 /*

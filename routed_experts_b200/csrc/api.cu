@@ -131,15 +131,18 @@ moe_status mx_shape(const moe_config* cfg, Shape* s) {
     return MOE_OK;
 }
 
-int64_t mx_bytes(const Shape& s, int which) {
+bool wfmt_ok(int32_t wfmt) { return wfmt == MOE_MX_W_E4M3 || wfmt == MOE_MX_W_E2M1; }
+
+int64_t mx_bytes(const Shape& s, int which, int wfmt = MOE_MX_W_E4M3) {
+    const int64_t per = wfmt == MOE_MX_W_E2M1 ? 2 : 1;   // weight elements per code byte
     switch (which) {
         case MOE_MX_XQ: return s.rows_cap * s.d;
         case MOE_MX_XS: return mx_scale_bytes(s.rows_cap, s.d);
         case MOE_MX_HQ: return s.rows_cap * s.F;
         case MOE_MX_HS: return mx_scale_bytes(s.rows_cap, s.F);
-        case MOE_MX_W1Q: return (int64_t)s.E * 2 * s.F * s.d;
+        case MOE_MX_W1Q: return (int64_t)s.E * 2 * s.F * s.d / per;
         case MOE_MX_W1S: return mx_scale_bytes((int64_t)s.E * 2 * s.F, s.d);
-        case MOE_MX_W2Q: return (int64_t)s.E * s.d * s.F;
+        case MOE_MX_W2Q: return (int64_t)s.E * s.d * s.F / per;
         case MOE_MX_W2S: return mx_scale_bytes((int64_t)s.E * s.d, s.F);
     }
     return -1;
@@ -406,29 +409,29 @@ moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void*
     return from_cuda(e);
 }
 
-moe_status moe_mx_buffer_bytes(const moe_config* cfg, int32_t which, size_t* bytes) {
+moe_status moe_mx_buffer_bytes(const moe_config* cfg, int32_t which, int32_t wfmt, size_t* bytes) {
     Shape s;
     moe_status r = mx_shape(cfg, &s);
     if (r != MOE_OK) return r;
-    if (!bytes || which < MOE_MX_XQ || which > MOE_MX_W2S) return MOE_ERR_INVALID_ARG;
-    *bytes = (size_t)mx_bytes(s, which);
+    if (!bytes || which < MOE_MX_XQ || which > MOE_MX_W2S || !wfmt_ok(wfmt)) return MOE_ERR_INVALID_ARG;
+    *bytes = (size_t)mx_bytes(s, which, wfmt);
     return MOE_OK;
 }
 
-moe_status moe_mx_quantize_weights(const moe_config* cfg, const void* w_gate_up, const void* w_down, void* w1q,
-                                   void* w1s, void* w2q, void* w2s, moe_stream_t stream) {
+moe_status moe_mx_quantize_weights(const moe_config* cfg, const void* w_gate_up, const void* w_down, int32_t wfmt,
+                                   void* w1q, void* w1s, void* w2q, void* w2s, moe_stream_t stream) {
     Shape s;
     moe_status r = mx_shape(cfg, &s);
     if (r != MOE_OK) return r;
-    if (!w_gate_up || !w_down || !w1q || !w1s || !w2q || !w2s) return MOE_ERR_INVALID_ARG;
+    if (!w_gate_up || !w_down || !w1q || !w1s || !w2q || !w2s || !wfmt_ok(wfmt)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(w1q) || !aligned16(w1s) || !aligned16(w2q) ||
         !aligned16(w2s))
         return MOE_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_mx_quantize(w_gate_up, (int64_t)s.E * 2 * s.F, s.d, s.F, static_cast<uint8_t*>(w1q),
-                                       static_cast<uint8_t*>(w1s), st);
+    cudaError_t e = launch_mx_quantize(w_gate_up, (int64_t)s.E * 2 * s.F, s.d, s.F, wfmt,
+                                       static_cast<uint8_t*>(w1q), static_cast<uint8_t*>(w1s), st);
     if (e == cudaSuccess)
-        e = launch_mx_quantize(w_down, (int64_t)s.E * s.d, s.F, 0, static_cast<uint8_t*>(w2q),
+        e = launch_mx_quantize(w_down, (int64_t)s.E * s.d, s.F, 0, wfmt, static_cast<uint8_t*>(w2q),
                                static_cast<uint8_t*>(w2s), st);
     return from_cuda(e);
 }
@@ -447,45 +450,47 @@ moe_status moe_dispatch_mx(const moe_config* cfg, const void* x, void* xq, void*
 }
 
 moe_status moe_expert_fc1_mx(const moe_config* cfg, const void* xq, const void* xs, const void* w1q,
-                             const void* w1s, void* hq, void* hs, void* ws, size_t ws_bytes, moe_stream_t stream) {
+                             const void* w1s, int32_t wfmt, void* hq, void* hs, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
     Shape s;
     moe_status r = mx_shape(cfg, &s);
     if (r != MOE_OK) return r;
-    if (!xq || !xs || !w1q || !w1s || !hq || !hs) return MOE_ERR_INVALID_ARG;
+    if (!xq || !xs || !w1q || !w1s || !hq || !hs || !wfmt_ok(wfmt)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(xq) || !aligned16(xs) || !aligned16(w1q) || !aligned16(w1s) || !aligned16(hq) || !aligned16(hs))
         return MOE_ERR_INVALID_ARG;
     const WsLayout L = make_layout(s);
     if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
     const WsPtrs P = ws_ptrs(ws, L);
     return from_cuda(launch_ffn_mx(s, 1, static_cast<const uint8_t*>(xq), static_cast<const uint8_t*>(xs),
-                                   static_cast<const uint8_t*>(w1q), static_cast<const uint8_t*>(w1s), hq,
+                                   static_cast<const uint8_t*>(w1q), static_cast<const uint8_t*>(w1s), wfmt, hq,
                                    static_cast<uint8_t*>(hs), P, reinterpret_cast<cudaStream_t>(stream),
                                    kSpinBudget));
 }
 
 moe_status moe_expert_fc2_mx(const moe_config* cfg, const void* hq, const void* hs, const void* w2q,
-                             const void* w2s, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream) {
+                             const void* w2s, int32_t wfmt, void* yp, void* ws, size_t ws_bytes,
+                             moe_stream_t stream) {
     Shape s;
     moe_status r = mx_shape(cfg, &s);
     if (r != MOE_OK) return r;
-    if (!hq || !hs || !w2q || !w2s || !yp) return MOE_ERR_INVALID_ARG;
+    if (!hq || !hs || !w2q || !w2s || !yp || !wfmt_ok(wfmt)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(hq) || !aligned16(hs) || !aligned16(w2q) || !aligned16(w2s) || !aligned16(yp))
         return MOE_ERR_INVALID_ARG;
     const WsLayout L = make_layout(s);
     if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
     const WsPtrs P = ws_ptrs(ws, L);
     return from_cuda(launch_ffn_mx(s, 2, static_cast<const uint8_t*>(hq), static_cast<const uint8_t*>(hs),
-                                   static_cast<const uint8_t*>(w2q), static_cast<const uint8_t*>(w2s), yp, nullptr,
-                                   P, reinterpret_cast<cudaStream_t>(stream), kSpinBudget));
+                                   static_cast<const uint8_t*>(w2q), static_cast<const uint8_t*>(w2s), wfmt, yp,
+                                   nullptr, P, reinterpret_cast<cudaStream_t>(stream), kSpinBudget));
 }
 
 moe_status moe_layer_fwd_mx(const moe_config* cfg, const float* logits, const void* x, const void* w1q,
-                            const void* w1s, const void* w2q, const void* w2s, void* out, void* ws,
+                            const void* w1s, const void* w2q, const void* w2s, int32_t wfmt, void* out, void* ws,
                             size_t ws_bytes, moe_stream_t stream) {
     Shape s;
     moe_status r = mx_shape(cfg, &s);
     if (r != MOE_OK) return r;
-    if (!logits || !x || !w1q || !w1s || !w2q || !w2s || !out) return MOE_ERR_INVALID_ARG;
+    if (!logits || !x || !w1q || !w1s || !w2q || !w2s || !out || !wfmt_ok(wfmt)) return MOE_ERR_INVALID_ARG;
     if (!aligned16(logits) || !aligned16(x) || !aligned16(w1q) || !aligned16(w1s) || !aligned16(w2q) ||
         !aligned16(w2s) || !aligned16(out))
         return MOE_ERR_INVALID_ARG;
@@ -509,10 +514,10 @@ moe_status moe_layer_fwd_mx(const moe_config* cfg, const float* logits, const vo
     const WsPtrs P = ws_ptrs(ws, L);
     cudaError_t e = launch_dispatch_mx(s, x, xq, xs, P, st);
     if (e == cudaSuccess)
-        e = launch_ffn_mx(s, 1, xq, xs, static_cast<const uint8_t*>(w1q), static_cast<const uint8_t*>(w1s), hq, hs, P,
-                          st, kSpinBudget);
+        e = launch_ffn_mx(s, 1, xq, xs, static_cast<const uint8_t*>(w1q), static_cast<const uint8_t*>(w1s), wfmt, hq,
+                          hs, P, st, kSpinBudget);
     if (e == cudaSuccess)
-        e = launch_ffn_mx(s, 2, hq, hs, static_cast<const uint8_t*>(w2q), static_cast<const uint8_t*>(w2s), yp,
+        e = launch_ffn_mx(s, 2, hq, hs, static_cast<const uint8_t*>(w2q), static_cast<const uint8_t*>(w2s), wfmt, yp,
                           nullptr, P, st, kSpinBudget);
     if (e == cudaSuccess) e = launch_combine(s, yp, w, out, P, st);
     return from_cuda(e);

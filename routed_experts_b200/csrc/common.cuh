@@ -159,20 +159,21 @@ cudaError_t launch_zero_padding(const Shape& s, void* a, void* b, int64_t row_by
                                 cudaStream_t st);
 cudaError_t launch_dlogits(const Shape& s, const float* logits, const int32_t* idx, const float* w, const float* dw,
                            float* dl, cudaStream_t st);
-// MXFP8: a bf16 [rows, K] matrix to codes [rows, K] and chunked scales; with
-// interleave_F > 0 the rows are those of w_gate_up [E, 2F, K] reordered so
-// that every 128 rows of an expert hold 64 gate rows then the 64 matching up
-// rows (the FC1 column tiles of the MX GEMM).
-cudaError_t launch_mx_quantize(const void* x, int64_t rows, int K, int interleave_F, uint8_t* q, uint8_t* sc,
-                               cudaStream_t st);
+// MX quantization of a bf16 [rows, K] matrix (fmt MOE_MX_W_E4M3: codes
+// [rows, K]; MOE_MX_W_E2M1: codes [rows, K/2], two per byte) with chunked
+// scales; with interleave_F > 0 the rows are those of w_gate_up [E, 2F, K]
+// reordered so that every 128 rows of an expert hold 64 gate rows then the
+// 64 matching up rows (the FC1 column tiles of the MX GEMM).
+cudaError_t launch_mx_quantize(const void* x, int64_t rows, int K, int interleave_F, int fmt, uint8_t* q,
+                               uint8_t* sc, cudaStream_t st);
 // The dispatch with MXFP8 quantization of each token row on the way.
 cudaError_t launch_dispatch_mx(const Shape& s, const void* x, uint8_t* xq, uint8_t* xs, const WsPtrs& ws,
                                cudaStream_t st);
 // MX grouped GEMM: which 1 = FC1 + SwiGLU (a = xq/xs, w = W1 in the
 // interleaved MX layout, out = hq, out_sc = hs), 2 = FC2 (a = hq/hs, w = W2,
-// out = yp in bf16, out_sc unused).
+// out = yp in bf16, out_sc unused); wfmt: the weights' element format.
 cudaError_t launch_ffn_mx(const Shape& s, int which, const uint8_t* a_q, const uint8_t* a_sc, const uint8_t* w_q,
-                          const uint8_t* w_sc, void* out, uint8_t* out_sc, const WsPtrs& ws, cudaStream_t st,
-                          long long spin_budget);
+                          const uint8_t* w_sc, int wfmt, void* out, uint8_t* out_sc, const WsPtrs& ws,
+                          cudaStream_t st, long long spin_budget);
 
 }  // namespace moe

@@ -40,6 +40,11 @@
 //     block maximum needs no communication. Codes are stored by TMA (32 x 32
 //     byte tiles), scales by plain byte stores into the chunked layout. FC2
 //     stores bf16 yp as the bf16 kernel does.
+// Weights may be MXFP4 instead ([MegaFlux] §4.1: MXFP4 weights, MXFP8
+// activations): E2M1 codes packed two per byte in memory, which TMA unpacks
+// (CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B) into the same 128-byte shared-memory
+// rows, one element per byte; the MMA reads them as E2M1 (B format field)
+// and the barrier counts the packed bytes.
 // Experts with a single block run in a pair beside an empty half.
 #include <cuda_fp8.h>
 #include <cudaTypedefs.h>
@@ -181,10 +186,11 @@ __device__ __forceinline__ void mx_epilogue_half(uint32_t t_half, int lane, int 
     }
 }
 
-// MODE 0: FC1 + SwiGLU -> MXFP8 h; MODE 1: FC2 -> bf16 yp. tmA / tmB: E4M3
-// operands (128-byte swizzle); tmSA / tmSB: their chunked scales viewed as
+// MODE 0: FC1 + SwiGLU -> MXFP8 h; MODE 1: FC2 -> bf16 yp. WF: the weights'
+// element format (MOE_MX_W_E4M3 or MOE_MX_W_E2M1). tmA / tmB: the operands
+// (128-byte swizzle); tmSA / tmSB: their chunked scales viewed as
 // [chunks * 4, 128] bytes; tmO: the output.
-template <int MODE>
+template <int MODE, int WF>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
               const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -348,7 +354,11 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     const uint32_t bar = ptx::map_to_rank(ptx::smem_addr(&S->full[stage]), 0);
                     uint8_t* st = base + stage * kMxStageBytes;
                     uint8_t* sf = sf_base + stage * kMxSfStage;
-                    if (even) ptx::mbar_arrive_expect_tx(&S->full[stage], 2 * (kMxStageBytes + kMxSfStage));
+                    // E2M1 weights count their packed bytes (half a byte per element)
+                    if (even)
+                        ptx::mbar_arrive_expect_tx(&S->full[stage],
+                                                   2 * (kMxABytes + (WF == MOE_MX_W_E2M1 ? kMxBBytes / 2 : kMxBBytes) +
+                                                        kMxSfStage));
                     ptx::tma_load_2d_pair(st, &tmA, kb * kMxBK, row0, bar);
                     ptx::tma_load_2d_pair(st + kMxABytes, &tmB, kb * kMxBK, b_lo, bar);
                     ptx::tma_load_2d_pair(st + kMxABytes + kMxBBytes / 2, &tmB, kb * kMxBK, b_hi, bar);
@@ -369,6 +379,8 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (even CTA)
         if (lane == 0 && even) {
+            // B format field of the instruction descriptor (bits 10-12): E4M3 0, E2M1 5
+            constexpr uint32_t kBFormat = WF == MOE_MX_W_E2M1 ? (5u << 10) : 0u;
             int stage = 0;
             uint32_t phase = 0, sf_set = 0;
             bool ok = true, issued = false;
@@ -403,12 +415,12 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                         for (uint32_t ks = 0; ks < kMxBK / 32; ++ks)
                             ptx::mma_mx_pair(d0, ptx::sdesc_k_sw128(a_addr + ks * 32),
                                              ptx::sdesc_k_sw128(b_addr + ks * 32),
-                                             ptx::idesc_mx_e4m3(2 * kBM, kMxItemN, ks, ks), sfa_t | (ks << 30),
+                                             ptx::idesc_mx_e4m3(2 * kBM, kMxItemN, ks, ks) | kBFormat, sfa_t | (ks << 30),
                                              (sfa_t + 4u) | (ks << 30), (kb | (int)ks) != 0 ? 1u : 0u);
                     } else {
 #pragma unroll
                         for (uint32_t ks = 0; ks < kMxBK / 32; ++ks) {
-                            const uint32_t idesc = ptx::idesc_mx_e4m3(2 * kBM, kMxHalf, ks, ks);
+                            const uint32_t idesc = ptx::idesc_mx_e4m3(2 * kBM, kMxHalf, ks, ks) | kBFormat;
                             const uint32_t acc = (kb | (int)ks) != 0 ? 1u : 0u;
                             const uint64_t adesc = ptx::sdesc_k_sw128(a_addr + ks * 32);
                             ptx::mma_mx_pair(d0, adesc, ptx::sdesc_k_sw128(b_addr + ks * 32), idesc,
@@ -500,12 +512,38 @@ bool make_tmap_u8(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t row
     return r == CUDA_SUCCESS;
 }
 
+// Packed E2M1 codes [rows, inner elements] (inner / 2 bytes per row), loaded
+// as [box_rows, 128] elements unpacked to one byte each, 128-byte swizzle.
+bool make_tmap_e2m1(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner / 2};
+    cuuint32_t box[2] = {128, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int WF>
+cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA, const CUtensorMap& tSB,
+                       const CUtensorMap& tO, const MxArgs& a, int grid, cudaStream_t st) {
+    cudaError_t err = cudaFuncSetAttribute(ffn_mx_kernel<MODE, WF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           (int)kMxSmemBytes);
+    if (err != cudaSuccess) return err;
+    ffn_mx_kernel<MODE, WF><<<grid, kThreads, kMxSmemBytes, st>>>(tA, tB, tSA, tSB, tO, a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_ffn_mx(const Shape& s, int which, const uint8_t* a_q, const uint8_t* a_sc, const uint8_t* w_q,
-                          const uint8_t* w_sc, void* out, uint8_t* out_sc, const WsPtrs& ws, cudaStream_t st,
-                          long long spin_budget) {
+                          const uint8_t* w_sc, int wfmt, void* out, uint8_t* out_sc, const WsPtrs& ws,
+                          cudaStream_t st, long long spin_budget) {
     if (s.d % 256 != 0 || s.F % 128 != 0) return cudaErrorInvalidValue;
+    if (wfmt != MOE_MX_W_E4M3 && wfmt != MOE_MX_W_E2M1) return cudaErrorInvalidValue;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -529,26 +567,20 @@ cudaError_t launch_ffn_mx(const Shape& s, int which, const uint8_t* a_q, const u
     const uint64_t chunks_a = (uint64_t)((s.rows_cap + 127) / 128) * (a.Kdim / 128);
     const uint64_t chunks_b = rows_b / 128 * (a.Kdim / 128);
     CUtensorMap tA, tB, tSA, tSB, tO;
-    if (!make_tmap_u8(&tA, a_q, (uint64_t)a.Kdim, rows_a, kMxBK, kBM, true) ||
-        !make_tmap_u8(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxBK, kMxHalfRows, true) ||
+    const bool b_ok = wfmt == MOE_MX_W_E2M1 ? make_tmap_e2m1(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxHalfRows)
+                                            : make_tmap_u8(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxBK, kMxHalfRows, true);
+    if (!make_tmap_u8(&tA, a_q, (uint64_t)a.Kdim, rows_a, kMxBK, kBM, true) || !b_ok ||
         !make_tmap_u8(&tSA, a_sc, 128, chunks_a * 4, 128, 4, false) ||
         !make_tmap_u8(&tSB, w_sc, 128, chunks_b * 4, 128, 4, false))
         return cudaErrorInvalidValue;
     const bool out_ok = fc1 ? make_tmap_u8(&tO, out, (uint64_t)s.F, rows_a, 32, 32, false)
                             : make_tmap_out(&tO, out, (uint64_t)s.d, rows_a);
     if (!out_ok) return cudaErrorInvalidValue;
-    if (fc1) {
-        cudaError_t err = cudaFuncSetAttribute(ffn_mx_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kMxSmemBytes);
-        if (err != cudaSuccess) return err;
-        ffn_mx_kernel<0><<<sms, kThreads, kMxSmemBytes, st>>>(tA, tB, tSA, tSB, tO, a);
-    } else {
-        cudaError_t err = cudaFuncSetAttribute(ffn_mx_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)kMxSmemBytes);
-        if (err != cudaSuccess) return err;
-        ffn_mx_kernel<1><<<sms, kThreads, kMxSmemBytes, st>>>(tA, tB, tSA, tSB, tO, a);
-    }
-    return cudaGetLastError();
+    if (wfmt == MOE_MX_W_E2M1)
+        return fc1 ? launch_one<0, MOE_MX_W_E2M1>(tA, tB, tSA, tSB, tO, a, sms, st)
+                   : launch_one<1, MOE_MX_W_E2M1>(tA, tB, tSA, tSB, tO, a, sms, st);
+    return fc1 ? launch_one<0, MOE_MX_W_E4M3>(tA, tB, tSA, tSB, tO, a, sms, st)
+               : launch_one<1, MOE_MX_W_E4M3>(tA, tB, tSA, tSB, tO, a, sms, st);
 }
 
 }  // namespace moe

@@ -19,6 +19,13 @@
 // two xor-shuffles away. Each lane converts its 8 values and stores 8 bytes;
 // the block's first lane stores the scale byte at its place in the chunked
 // scale layout (mx_scale_offset).
+//
+// Weights may also be quantized to MXFP4 ([MegaFlux] §4.1: MXFP4 weights):
+// E2M1 elements (0, 0.5, 1, 1.5, 2, 3, 4, 6; nearest, ties to even,
+// saturating at 6) with s = floor(log2 max|v|) - 2 + 127 (2 = the exponent
+// of E2M1's largest normal, 6 = 1.5 * 2^2), two codes per byte, element 2i
+// in the low nibble of byte i.
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -28,9 +35,12 @@ namespace {
 
 constexpr int kQWarps = 8;
 
+// The scale exponent of a block with fp32 maximum amax; EMAX is the exponent
+// of the element format's largest normal (8 for E4M3, 2 for E2M1).
+template <uint32_t EMAX = 8>
 __device__ __forceinline__ uint32_t mx_scale_of(float amax) {
     const uint32_t field = (__float_as_uint(amax) >> 23) & 0xFFu;
-    return field > 8u ? field - 8u : 0u;
+    return field > EMAX ? field - EMAX : 0u;
 }
 
 __device__ __forceinline__ float mx_inv_scale(uint32_t s) { return __uint_as_float((254u - s) << 23); }
@@ -47,10 +57,11 @@ __device__ __forceinline__ float amax8(const uint4& v) {
 }
 
 // The block scale of the 32 elements held by this lane's group of four.
+template <uint32_t EMAX = 8>
 __device__ __forceinline__ uint32_t group_scale(float m) {
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
     m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-    return mx_scale_of(m);
+    return mx_scale_of<EMAX>(m);
 }
 
 // 8 bf16 values times inv, rounded to E4M3, element 0 in the lowest byte.
@@ -68,6 +79,21 @@ __device__ __forceinline__ uint2 e4m3x8(const uint4& v, float inv) {
     return make_uint2(w[0], w[1]);
 }
 
+// 8 bf16 values times inv, rounded to E2M1, two per byte, element 0 in the
+// lowest nibble.
+__device__ __forceinline__ uint32_t e2m1x8(const uint4& v, float inv) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+    uint32_t w = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 f = __bfloat1622float2(p[i]);
+        f.x *= inv;
+        f.y *= inv;
+        w |= (uint32_t)__nv_cvt_float2_to_fp4x2(f, __NV_E2M1, cudaRoundNearest) << (8 * i);
+    }
+    return w;
+}
+
 // Row r of the quantized matrix reads input row src_row(r).
 __device__ __forceinline__ int64_t src_row(int64_t r, int interleave_F) {
     if (interleave_F <= 0) return r;
@@ -76,6 +102,7 @@ __device__ __forceinline__ int64_t src_row(int64_t r, int interleave_F) {
     return e * per + (t < 64 ? jt * 64 + t : interleave_F + jt * 64 + (t - 64));
 }
 
+template <int FMT>   // MOE_MX_W_E4M3 or MOE_MX_W_E2M1
 __global__ void __launch_bounds__(kQWarps * 32)
 mx_quantize_kernel(const uint4* __restrict__ x, int64_t rows, int K, int interleave_F, uint8_t* __restrict__ q,
                    uint8_t* __restrict__ sc) {
@@ -88,9 +115,12 @@ mx_quantize_kernel(const uint4* __restrict__ x, int64_t rows, int K, int interle
         const int64_t col = (int64_t)seg * 256 + lane * 8;
         const bool in = col < K;   // whole groups of four lanes (32-blocks) are in or out together
         const uint4 v = in ? __ldg(x + (src_row(r, interleave_F) * K + col) / 8) : make_uint4(0, 0, 0, 0);
-        const uint32_t s = group_scale(amax8(v));
+        const uint32_t s = group_scale<FMT == MOE_MX_W_E2M1 ? 2u : 8u>(amax8(v));
         if (in) {
-            *reinterpret_cast<uint2*>(q + r * K + col) = e4m3x8(v, mx_inv_scale(s));
+            if (FMT == MOE_MX_W_E2M1)
+                *reinterpret_cast<uint32_t*>(q + (r * K + col) / 2) = e2m1x8(v, mx_inv_scale(s));
+            else
+                *reinterpret_cast<uint2*>(q + r * K + col) = e4m3x8(v, mx_inv_scale(s));
             if ((lane & 3) == 0) sc[mx_scale_offset(r, col / 32, K)] = (uint8_t)s;
         }
     }
@@ -113,7 +143,7 @@ dispatch_mx_kernel(const uint4* __restrict__ x, uint8_t* __restrict__ xq, uint8_
         for (int seg = 0; seg < d / 256; ++seg) {
             const int64_t col = (int64_t)seg * 256 + lane * 8;
             const uint4 v = __ldg(x + ((int64_t)t * d + col) / 8);
-            const uint32_t s = group_scale(amax8(v));
+            const uint32_t s = group_scale<8u>(amax8(v));
             const uint2 c = e4m3x8(v, mx_inv_scale(s));
             for (int k = 0; k < K; ++k) {
                 const int row = __shfl_sync(0xffffffffu, my_row, k);
@@ -136,11 +166,17 @@ int grid_for(int64_t warps) {
 
 }  // namespace
 
-cudaError_t launch_mx_quantize(const void* x, int64_t rows, int K, int interleave_F, uint8_t* q, uint8_t* sc,
-                               cudaStream_t st) {
+cudaError_t launch_mx_quantize(const void* x, int64_t rows, int K, int interleave_F, int fmt, uint8_t* q,
+                               uint8_t* sc, cudaStream_t st) {
     if (K % 128 != 0 || rows <= 0) return cudaErrorInvalidValue;
-    mx_quantize_kernel<<<grid_for(rows * ((K + 255) / 256)), kQWarps * 32, 0, st>>>(static_cast<const uint4*>(x), rows, K,
-                                                                          interleave_F, q, sc);
+    const int grid = grid_for(rows * ((K + 255) / 256));
+    const uint4* x4 = static_cast<const uint4*>(x);
+    if (fmt == MOE_MX_W_E2M1)
+        mx_quantize_kernel<MOE_MX_W_E2M1><<<grid, kQWarps * 32, 0, st>>>(x4, rows, K, interleave_F, q, sc);
+    else if (fmt == MOE_MX_W_E4M3)
+        mx_quantize_kernel<MOE_MX_W_E4M3><<<grid, kQWarps * 32, 0, st>>>(x4, rows, K, interleave_F, q, sc);
+    else
+        return cudaErrorInvalidValue;
     return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
 DEV_PLAN_INEXACT, DEV_TIMEOUT, DEV_BAD_INDEX = 1, 2, 4
 WS_PLAN, WS_LAYER, WS_LAYER_HOST, WS_LAYER_TRAIN = 0, 1, 2, 3
 MX_XQ, MX_XS, MX_HQ, MX_HS, MX_W1Q, MX_W1S, MX_W2Q, MX_W2S = range(8)
+MX_W_E4M3, MX_W_E2M1 = 0, 1   # weight element formats: MXFP8, MXFP4
 
 
 class MoeError(RuntimeError):
@@ -71,12 +72,13 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         L.moe_probe_bounded_wait.argtypes = [P, ctypes.c_int64, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
-        L.moe_mx_buffer_bytes.argtypes = [C, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
-        L.moe_mx_quantize_weights.argtypes = [C, P, P, P, P, P, P, P]
+        I32 = ctypes.c_int32
+        L.moe_mx_buffer_bytes.argtypes = [C, I32, I32, ctypes.POINTER(ctypes.c_size_t)]
+        L.moe_mx_quantize_weights.argtypes = [C, P, P, I32, P, P, P, P, P]
         L.moe_dispatch_mx.argtypes = [C, P, P, P, P, S, P]
-        L.moe_expert_fc1_mx.argtypes = [C, P, P, P, P, P, P, P, S, P]
-        L.moe_expert_fc2_mx.argtypes = [C, P, P, P, P, P, P, S, P]
-        L.moe_layer_fwd_mx.argtypes = [C, P, P, P, P, P, P, P, P, S, P]
+        L.moe_expert_fc1_mx.argtypes = [C, P, P, P, P, I32, P, P, P, S, P]
+        L.moe_expert_fc2_mx.argtypes = [C, P, P, P, P, I32, P, P, S, P]
+        L.moe_layer_fwd_mx.argtypes = [C, P, P, P, P, P, P, I32, P, P, S, P]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_ffn_fused", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
@@ -239,15 +241,17 @@ def moe_read_status(ws, stream=None) -> int:
 
 # ---------------------------------------------------------------- MXFP8 forward
 
-def moe_mx_buffer_bytes(c, which: int) -> int:
+def moe_mx_buffer_bytes(c, which: int, wfmt: int = MX_W_E4M3) -> int:
     v = ctypes.c_size_t(0)
-    _check(lib().moe_mx_buffer_bytes(ctypes.byref(config(c)), int(which), ctypes.byref(v)), "moe_mx_buffer_bytes")
+    _check(lib().moe_mx_buffer_bytes(ctypes.byref(config(c)), int(which), int(wfmt), ctypes.byref(v)),
+           "moe_mx_buffer_bytes")
     return v.value
 
 
-def moe_mx_quantize_weights(c, w_gate_up, w_down, w1q, w1s, w2q, w2s, stream=None):
-    _check(lib().moe_mx_quantize_weights(ctypes.byref(config(c)), _ptr(w_gate_up), _ptr(w_down), _ptr(w1q),
-                                         _ptr(w1s), _ptr(w2q), _ptr(w2s), _stream(stream)), "moe_mx_quantize_weights")
+def moe_mx_quantize_weights(c, w_gate_up, w_down, w1q, w1s, w2q, w2s, stream=None, wfmt: int = MX_W_E4M3):
+    _check(lib().moe_mx_quantize_weights(ctypes.byref(config(c)), _ptr(w_gate_up), _ptr(w_down), int(wfmt),
+                                         _ptr(w1q), _ptr(w1s), _ptr(w2q), _ptr(w2s), _stream(stream)),
+           "moe_mx_quantize_weights")
 
 
 def moe_dispatch_mx(c, x, xq, xs, ws, stream=None):
@@ -256,35 +260,38 @@ def moe_dispatch_mx(c, x, xq, xs, ws, stream=None):
            "moe_dispatch_mx")
 
 
-def moe_expert_fc1_mx(c, xq, xs, w1q, w1s, hq, hs, ws, stream=None):
+def moe_expert_fc1_mx(c, xq, xs, w1q, w1s, hq, hs, ws, stream=None, wfmt: int = MX_W_E4M3):
     p, n = _ws(ws)
-    _check(lib().moe_expert_fc1_mx(ctypes.byref(config(c)), _ptr(xq), _ptr(xs), _ptr(w1q), _ptr(w1s), _ptr(hq),
-                                   _ptr(hs), p, n, _stream(stream)), "moe_expert_fc1_mx")
+    _check(lib().moe_expert_fc1_mx(ctypes.byref(config(c)), _ptr(xq), _ptr(xs), _ptr(w1q), _ptr(w1s), int(wfmt),
+                                   _ptr(hq), _ptr(hs), p, n, _stream(stream)), "moe_expert_fc1_mx")
 
 
-def moe_expert_fc2_mx(c, hq, hs, w2q, w2s, yp, ws, stream=None):
+def moe_expert_fc2_mx(c, hq, hs, w2q, w2s, yp, ws, stream=None, wfmt: int = MX_W_E4M3):
     p, n = _ws(ws)
-    _check(lib().moe_expert_fc2_mx(ctypes.byref(config(c)), _ptr(hq), _ptr(hs), _ptr(w2q), _ptr(w2s), _ptr(yp),
-                                   p, n, _stream(stream)), "moe_expert_fc2_mx")
+    _check(lib().moe_expert_fc2_mx(ctypes.byref(config(c)), _ptr(hq), _ptr(hs), _ptr(w2q), _ptr(w2s), int(wfmt),
+                                   _ptr(yp), p, n, _stream(stream)), "moe_expert_fc2_mx")
 
 
-def moe_layer_fwd_mx(c, logits, x, w1q, w1s, w2q, w2s, out, ws, stream=None):
+def moe_layer_fwd_mx(c, logits, x, w1q, w1s, w2q, w2s, out, ws, stream=None, wfmt: int = MX_W_E4M3):
     p, n = _ws(ws)
     _check(lib().moe_layer_fwd_mx(ctypes.byref(config(c)), _ptr(logits), _ptr(x), _ptr(w1q), _ptr(w1s), _ptr(w2q),
-                                  _ptr(w2s), _ptr(out), p, n, _stream(stream)), "moe_layer_fwd_mx")
+                                  _ptr(w2s), int(wfmt), _ptr(out), p, n, _stream(stream)), "moe_layer_fwd_mx")
 
 
-def mx_buffer(c, which: int, device="cuda") -> torch.Tensor:
-    return torch.empty(moe_mx_buffer_bytes(c, which), dtype=torch.uint8, device=device)
+def mx_buffer(c, which: int, device="cuda", wfmt: int = MX_W_E4M3) -> torch.Tensor:
+    return torch.empty(moe_mx_buffer_bytes(c, which, wfmt), dtype=torch.uint8, device=device)
 
 
 class MxWeights:
-    """A layer's expert weights in MXFP8, quantized on the device from bf16."""
+    """A layer's expert weights in MXFP8 (wfmt MX_W_E4M3) or MXFP4 (MX_W_E2M1), quantized on the
+    device from bf16."""
 
-    def __init__(self, c, w_gate_up, w_down, stream=None):
+    def __init__(self, c, w_gate_up, w_down, stream=None, wfmt: int = MX_W_E4M3):
         dev = w_gate_up.device
-        self.w1q, self.w1s, self.w2q, self.w2s = (mx_buffer(c, k, dev) for k in (MX_W1Q, MX_W1S, MX_W2Q, MX_W2S))
-        moe_mx_quantize_weights(c, w_gate_up, w_down, self.w1q, self.w1s, self.w2q, self.w2s, stream)
+        self.wfmt = wfmt
+        self.w1q, self.w1s, self.w2q, self.w2s = (mx_buffer(c, k, dev, wfmt)
+                                                  for k in (MX_W1Q, MX_W1S, MX_W2Q, MX_W2S))
+        moe_mx_quantize_weights(c, w_gate_up, w_down, self.w1q, self.w1s, self.w2q, self.w2s, stream, wfmt)
 
 
 # ---------------------------------------------------------------- conveniences
@@ -355,7 +362,7 @@ class Layer:
     def forward_mx(self, logits, x, mxw: "MxWeights", out=None, stream=None):
         """The layer on MXFP8 expert operands (weights from MxWeights)."""
         out = self.out if out is None else out
-        moe_layer_fwd_mx(self.cfg, logits, x, mxw.w1q, mxw.w1s, mxw.w2q, mxw.w2s, out, self.ws, stream)
+        moe_layer_fwd_mx(self.cfg, logits, x, mxw.w1q, mxw.w1s, mxw.w2q, mxw.w2s, out, self.ws, stream, mxw.wfmt)
         return out
 
     def status(self, stream=None) -> int:

@@ -265,19 +265,33 @@ def w1_tile_rows(E: int, F: int) -> np.ndarray:
     return (np.arange(E)[:, None] * 2 * F + local[None, :]).ravel()
 
 
-def mx_weights_on_device(cfg, inp: dict):
-    return M.MxWeights(cfg, inp["w_gate_up"], inp["w_down"])
+def mx_weights_on_device(cfg, inp: dict, wfmt: int = M.MX_W_E4M3):
+    return M.MxWeights(cfg, inp["w_gate_up"], inp["w_down"], wfmt=wfmt)
 
 
-def mx_oracle_weights(cfg, inp: dict, experts=None):
-    """Oracle MXFP8 codes and scales of W1 / W2 (logical order) for the given experts (all by default)."""
+def mx_oracle_weights(cfg, inp: dict, experts=None, wfmt: int = M.MX_W_E4M3):
+    """Oracle MX codes (one per byte) and scales of W1 / W2 (logical order) for the given experts (all by
+    default), in weight format wfmt."""
     es = range(cfg.E) if experts is None else experts
     wgu = np.stack([I.to_numpy_bits(inp["w_gate_up"][e]) for e in es])
     wdn = np.stack([I.to_numpy_bits(inp["w_down"][e]) for e in es])
-    return O.mx_weights(wgu, wdn, O.BF16)
+    return O.mx_weights(wgu, wdn, O.BF16, wfmt)
 
 
-def run_mx_stages(cfg, inp: dict) -> dict:
+def mx_weight_codes(q: torch.Tensor, rows: int, K: int, wfmt: int) -> np.ndarray:
+    """Weight codes from the device, one per byte: E2M1 codes are packed two per
+    byte, element 2i in the low nibble of byte i."""
+    a = q.cpu().numpy()
+    if wfmt == M.MX_W_E4M3:
+        return a.reshape(rows, K)
+    a = a.reshape(rows, K // 2)
+    out = np.empty((rows, K), np.uint8)
+    out[:, 0::2] = a & 0xF
+    out[:, 1::2] = a >> 4
+    return out
+
+
+def run_mx_stages(cfg, inp: dict, wfmt: int = M.MX_W_E4M3) -> dict:
     """moe_plan, moe_dispatch_mx, moe_expert_fc1_mx, moe_expert_fc2_mx, moe_combine."""
     dev = inp["x"].device
     T, K, E, d, F = cfg.T, cfg.K, cfg.E, cfg.d, cfg.F
@@ -293,11 +307,11 @@ def run_mx_stages(cfg, inp: dict) -> dict:
     hs = M.mx_buffer(cfg, M.MX_HS, dev)
     yp = torch.empty(cap, d, dtype=torch.bfloat16, device=dev)
     out = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
-    mxw = mx_weights_on_device(cfg, inp)
+    mxw = mx_weights_on_device(cfg, inp, wfmt)
     M.moe_plan(cfg, inp["logits"], idx, w, counts, ws)
     M.moe_dispatch_mx(cfg, inp["x"], xq, xs, ws)
-    M.moe_expert_fc1_mx(cfg, xq, xs, mxw.w1q, mxw.w1s, hq, hs, ws)
-    M.moe_expert_fc2_mx(cfg, hq, hs, mxw.w2q, mxw.w2s, yp, ws)
+    M.moe_expert_fc1_mx(cfg, xq, xs, mxw.w1q, mxw.w1s, hq, hs, ws, wfmt=wfmt)
+    M.moe_expert_fc2_mx(cfg, hq, hs, mxw.w2q, mxw.w2s, yp, ws, wfmt=wfmt)
     M.moe_combine(cfg, yp, w, out, ws)
     status = M.moe_read_status(ws)
     return {"idx": idx, "w": w, "counts": counts, "xq": xq.view(cap, d), "xs": xs, "hq": hq.view(cap, F),
@@ -327,12 +341,13 @@ def assert_mx_h_close(g_hq: np.ndarray, g_hs: np.ndarray, r_h: np.ndarray, r_hq:
         assert np.linalg.norm(gd - rd) / den <= 1e-2, f"{what}: normwise error"
 
 
-def check_mx_small(cfg, seed: int, device="cuda", max_rows: int = 768, max_tokens: int = 192):
+def check_mx_small(cfg, seed: int, device="cuda", max_rows: int = 768, max_tokens: int = 192,
+                   wfmt: int = M.MX_W_E4M3):
     """The MX layer stage by stage against the oracle: weights and dispatched
     rows on every element; h and yp on every valid row up to max_rows (a
     seeded sample beyond), out on every token up to max_tokens (likewise)."""
     inp = I.make_inputs(cfg, seed, device)
-    g = run_mx_stages(cfg, inp)
+    g = run_mx_stages(cfg, inp, wfmt)
     hin = host_inputs(inp)
     ref = oracle_routing(cfg, hin)
     assert g["rows_cap"] == ref["rows_cap"]
@@ -343,12 +358,12 @@ def check_mx_small(cfg, seed: int, device="cuda", max_rows: int = 768, max_token
     src = ref["src_of"][:total]
     valid = src >= 0
     # weights: bit-exact codes and scales
-    w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp)
+    w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp, wfmt=wfmt)
     perm = w1_tile_rows(E, F)
-    gw1q = g["mxw"].w1q.view(E * 2 * F, d).cpu().numpy()
+    gw1q = mx_weight_codes(g["mxw"].w1q, E * 2 * F, d, wfmt)
     assert np.array_equal(gw1q, w1q[perm]), "W1 codes differ"
     assert np.array_equal(mx_unchunk(g["mxw"].w1s, E * 2 * F, d), w1s[perm]), "W1 scales differ"
-    assert np.array_equal(g["mxw"].w2q.view(E * d, F).cpu().numpy(), w2q), "W2 codes differ"
+    assert np.array_equal(mx_weight_codes(g["mxw"].w2q, E * d, F, wfmt), w2q), "W2 codes differ"
     assert np.array_equal(mx_unchunk(g["mxw"].w2s, E * d, F), w2s), "W2 scales differ"
     # dispatch: every valid row holds its token's codes and scales, bit for bit
     xq_ref, xs_ref = O.mx_quantize(hin["x"], O.BF16)
@@ -367,31 +382,31 @@ def check_mx_small(cfg, seed: int, device="cuda", max_rows: int = 768, max_token
     if len(vrows) > max_rows:
         vrows = np.sort(rng.choice(vrows, size=max_rows, replace=False))
     rh, rhq, rhs = O.mx_fc1_rows(np.arange(len(vrows)), row_exp[vrows], xq_ref[src[vrows]], xs_ref[src[vrows]],
-                                 w1q, w1s, F)
+                                 w1q, w1s, F, wfmt)
     ghq = g["hq"][:total].cpu().numpy()
     ghs = mx_unchunk(g["hs"], total, F)
     assert_mx_h_close(ghq[vrows], ghs[vrows], rh, rhq, rhs, "h (MXFP8)")
     assert not ghq[~valid].any() and not ghs[~valid].any(), "padding rows of h must be zero codes and scales"
     # FC2 on the oracle's h
-    ry = O.mx_fc2_rows(row_exp[vrows], rhq, rhs, w2q, w2s, d)
+    ry = O.mx_fc2_rows(row_exp[vrows], rhq, rhs, w2q, w2s, d, wfmt)
     gy = to_f64(g["yp"][:total])
     assert_close(gy[vrows], ry, C.BF16, "yp")
     assert not gy[~valid].any(), "padding rows of yp must be zero"
     # the whole layer, on all tokens or a seeded sample
     toks = np.arange(cfg.T) if cfg.T <= max_tokens else np.sort(rng.choice(cfg.T, size=max_tokens, replace=False))
-    rout = O.mx_token_out(toks, xq_ref, xs_ref, ref["idx"], ref["w"], w1q, w1s, w2q, w2s, F)
+    rout = O.mx_token_out(toks, xq_ref, xs_ref, ref["idx"], ref["w"], w1q, w1s, w2q, w2s, F, wfmt)
     assert_close(to_f64(g["out"])[toks], rout, C.BF16, "out")
     return g, ref, inp
 
 
-def check_mx_full_size(cfg, seed: int, n_tokens: int = 3, device="cuda"):
+def check_mx_full_size(cfg, seed: int, n_tokens: int = 3, device="cuda", wfmt: int = M.MX_W_E4M3):
     """Full-size MX layer through moe_layer_fwd_mx: bit-exact routing and plan
     (moe_plan), and sampled tokens of out against the oracle."""
     inp = I.make_inputs(cfg, seed, device)
     hin = host_inputs(inp, with_weights=False)
     ref = oracle_routing(cfg, hin)
     layer = M.Layer(cfg, device)
-    mxw = mx_weights_on_device(cfg, inp)
+    mxw = mx_weights_on_device(cfg, inp, wfmt)
     out = layer.forward_mx(inp["logits"], inp["x"], mxw)
     assert (layer.status() & ~O.PLAN_INEXACT) == 0
     plan = M.read_plan(cfg, layer.ws)
@@ -401,9 +416,9 @@ def check_mx_full_size(cfg, seed: int, n_tokens: int = 3, device="cuda"):
     gout = to_f64(out[torch.as_tensor(toks, device=device)])
     for i, t in enumerate(toks):
         es = ref["idx"][t]
-        w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp, es)
+        w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp, es, wfmt)
         xq, xs = O.mx_quantize(hin["x"][t:t + 1], O.BF16)
         o = O.mx_token_out(np.array([0]), xq, xs, np.arange(cfg.K, dtype=np.int32)[None, :], ref["w"][t:t + 1],
-                           w1q, w1s, w2q, w2s, cfg.F)
+                           w1q, w1s, w2q, w2s, cfg.F, wfmt)
         assert_close(gout[i:i + 1], o, C.BF16, f"out[{t}]")
     return out

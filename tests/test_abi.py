@@ -160,12 +160,18 @@ def test_mx_buffer_sizes(M):
     assert M.moe_mx_buffer_bytes(cfg, M.MX_W1S) == E * 2 * F * d // 32
     assert M.moe_mx_buffer_bytes(cfg, M.MX_W2Q) == E * d * F
     assert M.moe_mx_buffer_bytes(cfg, M.MX_W2S) == E * d * F // 32
+    # MXFP4 weights: two codes per byte, the same scales, activations unchanged
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_W1Q, M.MX_W_E2M1) == E * 2 * F * d // 2
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_W2Q, M.MX_W_E2M1) == E * d * F // 2
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_W1S, M.MX_W_E2M1) == E * 2 * F * d // 32
+    assert M.moe_mx_buffer_bytes(cfg, M.MX_XQ, M.MX_W_E2M1) == cap * d
     L = M.lib()
     n = ctypes.c_size_t(0)
-    assert L.moe_mx_buffer_bytes(ctypes.byref(M.config(cfg)), 8, ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_mx_buffer_bytes(ctypes.byref(M.config(cfg)), 8, 0, ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_mx_buffer_bytes(ctypes.byref(M.config(cfg)), 0, 2, ctypes.byref(n)) == M.MOE_ERR_INVALID_ARG
     # fp32 layers and widths the MX GEMM does not tile are unsupported
     for bad in (C.TINY, cfg.replace(F=1000), cfg.replace(d=2176)):
-        assert L.moe_mx_buffer_bytes(ctypes.byref(M.config(bad)), 0, ctypes.byref(n)) in \
+        assert L.moe_mx_buffer_bytes(ctypes.byref(M.config(bad)), 0, 0, ctypes.byref(n)) in \
             (M.MOE_ERR_UNSUPPORTED, M.MOE_ERR_INVALID_ARG), bad
 
 
@@ -179,24 +185,30 @@ def test_mx_calls_check_their_arguments(M):
     plan_need = M.moe_workspace_size(bf, M.WS_PLAN)
     layer_need = M.moe_workspace_size(bf, M.WS_LAYER)
     # weights: a null or misaligned pointer, or an unsupported shape (the call has no workspace to check)
-    assert L.moe_mx_quantize_weights(cfg, fake, fake, fake, None, fake, fake, None) == M.MOE_ERR_INVALID_ARG
-    assert L.moe_mx_quantize_weights(cfg, fake, odd, fake, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_mx_quantize_weights(cfg, fake, fake, 0, fake, None, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_mx_quantize_weights(cfg, fake, odd, 0, fake, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
+    assert L.moe_mx_quantize_weights(cfg, fake, fake, 7, fake, fake, fake, fake, None) == M.MOE_ERR_INVALID_ARG
     tiny = ctypes.byref(M.config(C.TINY))
-    assert L.moe_mx_quantize_weights(tiny, fake, fake, fake, fake, fake, fake, None) == M.MOE_ERR_UNSUPPORTED
+    assert L.moe_mx_quantize_weights(tiny, fake, fake, 0, fake, fake, fake, fake, None) == M.MOE_ERR_UNSUPPORTED
     assert L.moe_dispatch_mx(cfg, fake, fake, fake, fake, s(plan_need - 1), None) == M.MOE_ERR_WORKSPACE
     assert L.moe_dispatch_mx(cfg, fake, None, fake, fake, s(plan_need), None) == M.MOE_ERR_INVALID_ARG
-    assert L.moe_expert_fc1_mx(cfg, fake, fake, fake, fake, fake, fake, fake, s(plan_need - 1), None) == \
+    assert L.moe_expert_fc1_mx(cfg, fake, fake, fake, fake, 0, fake, fake, fake, s(plan_need - 1), None) == \
         M.MOE_ERR_WORKSPACE
-    assert L.moe_expert_fc1_mx(cfg, fake, odd, fake, fake, fake, fake, fake, s(plan_need), None) == \
+    assert L.moe_expert_fc1_mx(cfg, fake, odd, fake, fake, 0, fake, fake, fake, s(plan_need), None) == \
         M.MOE_ERR_INVALID_ARG
-    assert L.moe_expert_fc2_mx(cfg, fake, fake, fake, fake, fake, fake, s(plan_need - 1), None) == \
-        M.MOE_ERR_WORKSPACE
-    assert L.moe_expert_fc2_mx(cfg, fake, fake, fake, None, fake, fake, s(plan_need), None) == M.MOE_ERR_INVALID_ARG
-    assert L.moe_layer_fwd_mx(cfg, fake, fake, fake, fake, fake, fake, fake, fake, s(layer_need - 1), None) == \
-        M.MOE_ERR_WORKSPACE
-    assert L.moe_layer_fwd_mx(cfg, fake, fake, fake, fake, fake, fake, None, fake, s(layer_need), None) == \
+    assert L.moe_expert_fc1_mx(cfg, fake, fake, fake, fake, 3, fake, fake, fake, s(plan_need), None) == \
         M.MOE_ERR_INVALID_ARG
-    assert L.moe_layer_fwd_mx(tiny, fake, fake, fake, fake, fake, fake, fake, fake, s(layer_need), None) == \
+    assert L.moe_expert_fc2_mx(cfg, fake, fake, fake, fake, 1, fake, fake, s(plan_need - 1), None) == \
+        M.MOE_ERR_WORKSPACE
+    assert L.moe_expert_fc2_mx(cfg, fake, fake, fake, None, 1, fake, fake, s(plan_need), None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_fwd_mx(cfg, fake, fake, fake, fake, fake, fake, 0, fake, fake, s(layer_need - 1), None) == \
+        M.MOE_ERR_WORKSPACE
+    assert L.moe_layer_fwd_mx(cfg, fake, fake, fake, fake, fake, fake, 0, None, fake, s(layer_need), None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_fwd_mx(cfg, fake, fake, fake, fake, fake, fake, -1, fake, fake, s(layer_need), None) == \
+        M.MOE_ERR_INVALID_ARG
+    assert L.moe_layer_fwd_mx(tiny, fake, fake, fake, fake, fake, fake, 0, fake, fake, s(layer_need), None) == \
         M.MOE_ERR_UNSUPPORTED
 
 

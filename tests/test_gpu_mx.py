@@ -25,13 +25,19 @@ MX_SIGMOID = C.LayerConfig("mx_sigmoid", T=768, d=768, E=12, K=3, F=128, R=4, ti
                            gating=C.GATE_SIGMOID_TOPK, zipf_s=0.8)
 
 
+FMTS = [M.MX_W_E4M3, M.MX_W_E2M1]
+FMT_IDS = ["mxfp8_w", "mxfp4_w"]
+
+
+@pytest.mark.parametrize("wfmt", FMTS, ids=FMT_IDS)
 @pytest.mark.parametrize("cfg", [MX_SMALL, MX_SKEW, MX_SIGMOID], ids=lambda c: c.name)
-def test_mx_layer_small(cfg):
-    check_mx_small(cfg, 0)
+def test_mx_layer_small(cfg, wfmt):
+    check_mx_small(cfg, 0, wfmt=wfmt)
 
 
-def test_mx_layer_second_seed_and_block_planner():
-    check_mx_small(MX_SKEW.replace(name="mx_skew_blocks", plan_mode=C.PLAN_BLOCKS), 3)
+@pytest.mark.parametrize("wfmt", FMTS, ids=FMT_IDS)
+def test_mx_layer_second_seed_and_block_planner(wfmt):
+    check_mx_small(MX_SKEW.replace(name="mx_skew_blocks", plan_mode=C.PLAN_BLOCKS), 3, wfmt=wfmt)
 
 
 def test_mx_layer_entry_matches_the_stages():
@@ -40,7 +46,7 @@ def test_mx_layer_entry_matches_the_stages():
     cfg = MX_SKEW
     from .gpu_helpers import run_mx_stages
     inp = I.make_inputs(cfg, 1, "cuda")
-    g = run_mx_stages(cfg, inp)
+    g = run_mx_stages(cfg, inp, M.MX_W_E2M1)
     layer = M.Layer(cfg, "cuda")
     out = layer.forward_mx(inp["logits"], inp["x"], g["mxw"])
     torch.cuda.synchronize()
@@ -49,20 +55,24 @@ def test_mx_layer_entry_matches_the_stages():
     assert torch.equal(out2, out), "the MX layer is deterministic"
 
 
-def test_mx_layer_is_close_to_the_bf16_layer():
-    """MXFP8 operands move the output by about the E4M3 rounding (2^-4
-    relative per operand), not more: a check of scale handling at size."""
+@pytest.mark.parametrize("wfmt,bound", [(M.MX_W_E4M3, 0.08), (M.MX_W_E2M1, 0.3)], ids=FMT_IDS)
+def test_mx_layer_is_close_to_the_bf16_layer(wfmt, bound):
+    """MX operands move the output by about their rounding (E4M3: 2^-4
+    relative per element; E2M1 weights: up to 1/6 relative), not more: a
+    check of scale handling at size."""
     from routed_experts_b200 import inputs as I
     cfg = MX_SKEW
     inp = I.make_inputs(cfg, 2, "cuda")
     layer = M.Layer(cfg, "cuda")
     ref = layer.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"]).float().clone()
-    out = layer.forward_mx(inp["logits"], inp["x"], M.MxWeights(cfg, inp["w_gate_up"], inp["w_down"])).float()
+    mxw = M.MxWeights(cfg, inp["w_gate_up"], inp["w_down"], wfmt=wfmt)
+    out = layer.forward_mx(inp["logits"], inp["x"], mxw).float()
     rel = (torch.linalg.norm(out - ref) / torch.linalg.norm(ref)).item()
-    assert rel < 0.08, rel
+    assert rel < bound, rel
     assert rel > 1e-4, "the MX layer should not be the bf16 layer"
 
 
+@pytest.mark.parametrize("wfmt", FMTS, ids=FMT_IDS)
 @pytest.mark.parametrize("name,n_tokens", [("olmoe", 3), ("dsv3", 1)])
-def test_mx_layer_full_size_sampled(name, n_tokens):
-    check_mx_full_size(C.NAMED[name], 0, n_tokens=n_tokens)
+def test_mx_layer_full_size_sampled(name, n_tokens, wfmt):
+    check_mx_full_size(C.NAMED[name], 0, n_tokens=n_tokens, wfmt=wfmt)
