@@ -242,3 +242,17 @@ def test_mx_ffn_with_mxfp4_weights_on_exact_inputs():
     assert np.array_equal(h, h_ref)
     y2 = O.mx_fc2_rows(experts, hq, hs, w2q, w2s, d, O.MX_E2M1)
     assert np.array_equal(y2, y)
+
+
+def test_e4m3_encode_matches_torch_float8_e4m3fn():
+    """The oracle's encoder against a library conversion (PyTorch's
+    float8_e4m3fn, round to nearest even) on values within the finite range,
+    including every midpoint between neighbouring codes and subnormals."""
+    import torch
+    codes, vals = _table()
+    rng = np.random.default_rng(21)
+    mags = np.concatenate([2.0 ** rng.uniform(-12, np.log2(448.0), 6000), (vals[:-1] + vals[1:]) / 2, vals])
+    v = np.concatenate([mags, -mags]).astype(np.float32)   # fp32-representable inputs for both sides
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([O.e4m3_encode(float(t)) for t in v], np.uint8)
+    assert np.array_equal(got, ref)
