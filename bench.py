@@ -497,25 +497,30 @@ def run_mine(args, world, rank, local):
     if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
         raise RuntimeError(f"device status {st} after the timed steps")
 
-    # the fused FFN (FC1 and FC2 in one launch) on the same plan and xp, K passes
-    fused_ms = None
+    # the fused FFN (FC1 and FC2 in one launch) on the same plan and xp, K passes; then the
+    # same with FC1 gathering x through the row map (dispatch, FC1 and FC2 in one launch)
+    fused_ms = gather_ms = None
     if cfg.dtype == C.BF16:
-        for _ in range(args.warmup):
-            M.moe_expert_ffn_fused(cfg, xp, wgu, wdn, h, yp, ws, stream)
-        if pg is not None:
-            torch.distributed.barrier()
-        torch.cuda.synchronize(dev)
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(args.steps):
-            M.moe_expert_ffn_fused(cfg, xp, wgu, wdn, h, yp, ws, stream)
-        f1.record(stream)
-        torch.cuda.synchronize(dev)
-        fused_ms = f0.elapsed_time(f1)
-        if pg is not None:
-            fused_ms = max_over_ranks([fused_ms], dev)[0]
-        fused_ms /= args.steps
+        def timed_passes(fn):
+            for _ in range(args.warmup):
+                fn()
+            if pg is not None:
+                torch.distributed.barrier()
+            torch.cuda.synchronize(dev)
+            f0 = torch.cuda.Event(enable_timing=True)
+            f1 = torch.cuda.Event(enable_timing=True)
+            f0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            f1.record(stream)
+            torch.cuda.synchronize(dev)
+            t = f0.elapsed_time(f1)
+            if pg is not None:
+                t = max_over_ranks([t], dev)[0]
+            return t / args.steps
+
+        fused_ms = timed_passes(lambda: M.moe_expert_ffn_fused(cfg, xp, wgu, wdn, h, yp, ws, stream))
+        gather_ms = timed_passes(lambda: M.moe_expert_ffn_fused_gather(cfg, x, wgu, wdn, h, yp, ws, stream))
 
     # end to end through the public API with host buffers: H2D of logits and x
     # from pinned memory, the layer, D2H of the output, every step
@@ -660,9 +665,11 @@ def run_mine(args, world, rank, local):
         "mx": mx,
         "mx_fp4_weights": mx4,
         "fused_ffn": None if fused_ms is None else {
-            "ms": fused_ms, "staged_fc1_fc2_ms": float(med[2] + med[3]),
-            "note": "moe_expert_ffn_fused: FC1 and FC2 in one launch, FC2 tiles released per block pair "
-                    "(the staged FC1 and FC2 launches are what the layer runs)"},
+            "ms": fused_ms, "gather_ms": gather_ms, "staged_fc1_fc2_ms": float(med[2] + med[3]),
+            "staged_dispatch_fc1_fc2_ms": float(med[1] + med[2] + med[3]),
+            "note": "moe_expert_ffn_fused: FC1 and FC2 in one launch, FC2 tiles released per block pair; "
+                    "moe_expert_ffn_fused_gather: the same with FC1 gathering x through the row map "
+                    "(the staged launches are what the layer runs)"},
         "clocks": clk.summary(),
     }
     if cpu is not None:

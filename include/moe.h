@@ -225,6 +225,18 @@ moe_status moe_expert_ffn_fused(const moe_config* cfg, const void* xp, const voi
                                 void* h, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_expert_ffn_fused_gather - steps A6 to A8 in one launch (bf16 layers):
+ * moe_expert_ffn_fused with FC1's activation rows read straight from x
+ * [T, d] (device) through the plan's row map (TMA four-row gathers; padding
+ * rows repeat their block's first token and are stored as zero h and yp
+ * rows), so xp is never written. Same h and yp bits as moe_dispatch followed
+ * by moe_expert_ffn. Other dtypes return MOE_ERR_UNSUPPORTED.
+ */
+moe_status moe_expert_ffn_fused_gather(const moe_config* cfg, const void* x, const void* w_gate_up,
+                                       const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream);
+
+/*
  * moe_expert_fc1_gather - steps A6 and A7 in one pass (bf16 layers only):
  * FC1 + SwiGLU whose activation rows are gathered straight from x [T, d]
  * (device) through the plan's row map, so no xp buffer is written or read

@@ -250,6 +250,23 @@ moe_status moe_expert_ffn_fused(const moe_config* cfg, const void* xp, const voi
                                       kSpinBudget));
 }
 
+moe_status moe_expert_ffn_fused_gather(const moe_config* cfg, const void* x, const void* w_gate_up,
+                                       const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
+                                       moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!x || !w_gate_up || !w_down || !h || !yp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(h) || !aligned16(yp))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(ws, L);
+    return from_cuda(launch_ffn_fused(s, x, w_gate_up, w_down, h, yp, P, reinterpret_cast<cudaStream_t>(stream),
+                                      kSpinBudget, true));
+}
+
 moe_status moe_expert_fc1(const moe_config* cfg, const void* xp, const void* w_gate_up, void* h, void* ws,
                           size_t ws_bytes, moe_stream_t stream) {
     Shape s;

@@ -145,9 +145,11 @@ cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const 
 cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact = nullptr);
-// FC1 then FC2 in one launch (bf16): h and yp as launch_ffn_tc's which = 1 and 2
-cudaError_t launch_ffn_fused(const Shape& s, const void* xp, const void* w_gate_up, const void* w_down, void* h,
-                             void* yp, const WsPtrs& ws, cudaStream_t st, long long spin_budget);
+// FC1 then FC2 in one launch (bf16): h and yp as launch_ffn_tc's which = 1 and 2;
+// a_src is xp, or x [T, d] read through the row map when gather is set
+cudaError_t launch_ffn_fused(const Shape& s, const void* a_src, const void* w_gate_up, const void* w_down, void* h,
+                             void* yp, const WsPtrs& ws, cudaStream_t st, long long spin_budget,
+                             bool gather = false);
 // backward (bf16): mode 0 DGrad W2 + SwiGLU derivative (a_mat = dY, b_mat = w_down, ag, out = dAG),
 // 1 DGrad W1 (a_mat = dAG, b_mat = w_gate_up, out = dXp), 2 WGrad W2 (a_mat = dY, b_mat = h,
 // out = dW2 fp32), 3 WGrad W1 (a_mat = dAG, b_mat = xp, out = dW1 fp32)

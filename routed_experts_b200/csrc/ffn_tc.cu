@@ -176,7 +176,9 @@ __device__ __forceinline__ void epilogue_item(uint32_t t_row, int lane, int quad
 // out an FC2 item of a block pair only once all FC1 column tiles of that pair
 // are stored (a per-pair count each epilogue warp raises with a release add
 // after its TMA stores complete; bounded wait, acquire), so FC2 reads h while
-// it is still in L2. tmA2 / tmB2 / tmO2 are FC2's operands and output.
+// it is still in L2. tmA2 / tmB2 / tmO2 are FC2's operands and output;
+// MODE 5: MODE 4 with FC1's A gathered from x as in MODE 2 (dispatch, FC1
+// and FC2 in one launch).
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -232,7 +234,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
         ptx::prefetch_tmap(&tmB);
         ptx::prefetch_tmap(&tmO);
         if (MODE == 3) ptx::prefetch_tmap(&tmP);
-        if (MODE == 4) { ptx::prefetch_tmap(&tmA2); ptx::prefetch_tmap(&tmB2); ptx::prefetch_tmap(&tmO2); }
+        if (MODE >= 4) { ptx::prefetch_tmap(&tmA2); ptx::prefetch_tmap(&tmB2); ptx::prefetch_tmap(&tmO2); }
     }
     __syncthreads();
     ptx::cluster_sync();   // the peer's barriers exist before any remote arrive, store or copy
@@ -241,10 +243,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = S->tmem_base;
-    constexpr bool kFused = MODE == 4;
+    constexpr bool kFused = MODE == 4 || MODE == 5;
     const int n_items = p_off[a.E] * (a.n_tiles + (kFused ? a.n_tiles2 : 0));
     const int kb_count = a.Kdim / kBK;
-    constexpr bool kGather = MODE == 2;
+    constexpr bool kGather = MODE == 2 || MODE == 5;   // FC1 items only
     // an item's phase (fused FFN: FC2 items carry it in the column field's bit 16)
     auto is_fc2 = [&](const int4& item) { return kFused ? (item.y >> 16) != 0 : MODE == 1; };
 
@@ -323,7 +325,7 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 item.y = __shfl_sync(0xffffffffu, item.y, 0);
                 item.z = __shfl_sync(0xffffffffu, item.z, 0);
                 item.w = __shfl_sync(0xffffffffu, item.w, 0);
-                if (kGather && item.x >= 0) {
+                if (kGather && item.x >= 0 && (item.y >> 16) == 0) {
                     // tokens of the rows of both blocks; a padding row takes its block's first token
                     const int r_even = item.z, r_odd = item.w >= 0 ? item.w : item.z;
                     const int first_even = __ldg(a.src_of + r_even), first_odd = __ldg(a.src_of + r_odd);
@@ -392,7 +394,8 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
             int4 item;
             if (!take_item(k, item)) { ok = false; break; }
             int4 tok = make_int4(0, 0, 0, 0);   // gathered FC1: tokens of this lane's four rows
-            if (kGather && item.x >= 0) tok = *reinterpret_cast<const int4*>(&S->rows[slot_of(k)][4 * lane]);
+            const bool gath = kGather && item.x >= 0 && (item.y >> 16) == 0;   // warp-uniform
+            if (gath) tok = *reinterpret_cast<const int4*>(&S->rows[slot_of(k)][4 * lane]);
             __syncwarp();
             if (lane == 0) release_item(k);
             if (item.x < 0) break;
@@ -411,10 +414,10 @@ ffn_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 uint8_t* st = base + stage * kStageBytes;
                 if (lane == 0) {
                     if (even) ptx::mbar_arrive_expect_tx(&S->full[stage], 2 * kStageBytes);
-                    if (!kGather) ptx::tma_load_2d_pair(st, mA, kb * kBK, row0, bar);
+                    if (!gath) ptx::tma_load_2d_pair(st, mA, kb * kBK, row0, bar);
                     ptx::tma_load_2d_pair(st + kABytes, mB, kb * kBK, brow, bar);
                 }
-                if (kGather) ptx::tma_gather4_pair(st + 4 * 128 * lane, &tmA, kb * kBK, tok.x, tok.y, tok.z, tok.w, bar);
+                if (gath) ptx::tma_gather4_pair(st + 4 * 128 * lane, &tmA, kb * kBK, tok.x, tok.y, tok.z, tok.w, bar);
                 ++fills;
                 if (++stage == kStages) { stage = 0; phase ^= 1; }
             }
@@ -784,7 +787,7 @@ template <int MODE>
 cudaError_t launch_mode(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tO, const CUtensorMap& tP,
                         TcArgs a, int grid, cudaStream_t st, int32_t* single_queue,
                         const CUtensorMap* t2 = nullptr) {
-    constexpr bool kSingles = MODE != 2 && MODE != 4;
+    constexpr bool kSingles = MODE != 2 && MODE != 4 && MODE != 5;
     a.lone_apart = kSingles ? 1 : 0;
     cudaError_t err = cudaFuncSetAttribute(ffn_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)kSmemBytes);
@@ -889,8 +892,8 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     return launch_mode<1>(tA, tB, tO, tO, a, sms, st, ws.gemm_q + 8);
 }
 
-cudaError_t launch_ffn_fused(const Shape& s, const void* xp, const void* w_gate_up, const void* w_down, void* h,
-                             void* yp, const WsPtrs& ws, cudaStream_t st, long long spin_budget) {
+cudaError_t launch_ffn_fused(const Shape& s, const void* a_src, const void* w_gate_up, const void* w_down, void* h,
+                             void* yp, const WsPtrs& ws, cudaStream_t st, long long spin_budget, bool gather) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -905,10 +908,12 @@ cudaError_t launch_ffn_fused(const Shape& s, const void* xp, const void* w_gate_
     a.queue = ws.gemm_q;
     a.src_of = ws.src_of;
     a.ready = ws.pair_ready;
-    // FC1: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h; FC2: h [rows_cap, F] x w_down [E*d, F] -> yp
+    // FC1: xp [rows_cap, d] (or x [T, d] gathered through the row map) x w_gate_up [E*2F, d] -> h;
+    // FC2: h [rows_cap, F] x w_down [E*d, F] -> yp
     CUtensorMap tA, tB, tO, t2[3];
-    if (!make_tmap(&tA, xp, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
-        !make_tmap(&tB, w_gate_up, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
+    const bool a_ok = gather ? make_tmap(&tA, a_src, (uint64_t)s.d, (uint64_t)s.T, 1)
+                             : make_tmap(&tA, a_src, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM);
+    if (!a_ok || !make_tmap(&tB, w_gate_up, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
         !make_tmap_out(&tO, h, (uint64_t)s.F, (uint64_t)s.rows_cap) ||
         !make_tmap(&t2[0], h, (uint64_t)s.F, (uint64_t)s.rows_cap, kBM) ||
         !make_tmap(&t2[1], w_down, (uint64_t)s.F, (uint64_t)s.E * s.d, kHalfN) ||
@@ -921,7 +926,8 @@ cudaError_t launch_ffn_fused(const Shape& s, const void* xp, const void* w_gate_
     a.Kdim2 = s.F;
     a.n_tiles2 = s.d / kN;
     a.b_rows2 = s.d;
-    return launch_mode<4>(tA, tB, tO, tO, a, sms, st, nullptr, t2);
+    return gather ? launch_mode<5>(tA, tB, tO, tO, a, sms, st, nullptr, t2)
+                  : launch_mode<4>(tA, tB, tO, tO, a, sms, st, nullptr, t2);
 }
 
 }  // namespace moe

@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_ffn.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_expert_fc1.argtypes = [C, P, P, P, P, S, P]
         L.moe_expert_ffn_fused.argtypes = [C, P, P, P, P, P, P, S, P]
+        L.moe_expert_ffn_fused_gather.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_expert_fc2.argtypes = [C, P, P, P, P, S, P]
         L.moe_expert_fc1_gather.argtypes = [C, P, P, P, P, S, P]
         L.moe_combine.argtypes = [C, P, P, P, P, S, P]
@@ -81,7 +82,7 @@ def lib() -> ctypes.CDLL:
         L.moe_layer_fwd_mx.argtypes = [C, P, P, P, P, P, P, I32, P, P, S, P]
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
-                  "moe_expert_ffn", "moe_expert_ffn_fused", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
+                  "moe_expert_ffn", "moe_expert_ffn_fused", "moe_expert_ffn_fused_gather", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
                   "moe_layer_fwd", "moe_layer_bwd", "moe_layer_fwd_train",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait",
                   "moe_mx_buffer_bytes", "moe_mx_quantize_weights", "moe_dispatch_mx", "moe_expert_fc1_mx",
@@ -168,6 +169,13 @@ def moe_expert_ffn_fused(c, xp, w_gate_up, w_down, h, yp, ws, stream=None):
     p, n = _ws(ws)
     _check(lib().moe_expert_ffn_fused(ctypes.byref(config(c)), _ptr(xp), _ptr(w_gate_up), _ptr(w_down), _ptr(h),
                                       _ptr(yp), p, n, _stream(stream)), "moe_expert_ffn_fused")
+
+
+def moe_expert_ffn_fused_gather(c, x, w_gate_up, w_down, h, yp, ws, stream=None):
+    """Dispatch, FC1 and FC2 in one launch: FC1 reads x through the plan's row map."""
+    p, n = _ws(ws)
+    _check(lib().moe_expert_ffn_fused_gather(ctypes.byref(config(c)), _ptr(x), _ptr(w_gate_up), _ptr(w_down),
+                                             _ptr(h), _ptr(yp), p, n, _stream(stream)), "moe_expert_ffn_fused_gather")
 
 
 def moe_expert_fc1(c, xp, w_gate_up, h, ws, stream=None):

@@ -142,6 +142,13 @@ def test_fused_ffn_checks_its_arguments(M):
     n = M.moe_workspace_size(C.TINY, M.WS_PLAN)
     assert L.moe_expert_ffn_fused(ctypes.byref(M.config(C.TINY)), fake, fake, fake, fake, fake, fake, s(n),
                                   None) == M.MOE_ERR_UNSUPPORTED
+    g = L.moe_expert_ffn_fused_gather
+    assert g(cfg, fake, fake, fake, fake, fake, fake, s(need - 1), None) == M.MOE_ERR_WORKSPACE
+    assert g(cfg, None, fake, fake, fake, fake, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    odd = ctypes.c_void_p((1 << 20) + 4)
+    assert g(cfg, fake, fake, fake, odd, fake, fake, s(need), None) == M.MOE_ERR_INVALID_ARG
+    assert g(ctypes.byref(M.config(C.TINY)), fake, fake, fake, fake, fake, fake, s(n), None) == \
+        M.MOE_ERR_UNSUPPORTED
 
 
 def test_mx_buffer_sizes(M):

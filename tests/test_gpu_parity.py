@@ -195,8 +195,9 @@ def test_qwen3_skew_sweep_plans(cfg):
 @pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, WIDE_BF16, C.OLMOE, C.DSV3], ids=lambda c: c.name)
 def test_fused_ffn_matches_the_staged_launches(cfg):
     """FC1 and FC2 in one launch, FC2 tiles released per block pair by the
-    readiness counts, give the same bits as the separate launches; a second
-    call without a new plan does too (the counts start from zero again)."""
+    readiness counts, give the same bits as the separate launches, with FC1
+    reading xp or gathering x through the row map; a second call without a
+    new plan does too (the counts start from zero again)."""
     inp = I.make_inputs(cfg, 3, "cuda")
     g = run_stages(cfg, inp)
     for _ in range(2):
@@ -207,5 +208,12 @@ def test_fused_ffn_matches_the_staged_launches(cfg):
         total = g["plan"]["total_rows"]
         assert torch.equal(h2[:total], g["h"][:total])
         assert torch.equal(y2[:total], g["yp"][:total])
+        # dispatch, FC1 and FC2 in one launch: FC1 reads x through the row map
+        h3 = torch.full_like(g["h"], float("nan"))
+        y3 = torch.full_like(g["yp"], float("nan"))
+        M.moe_expert_ffn_fused_gather(cfg, inp["x"], inp["w_gate_up"], inp["w_down"], h3, y3, g["ws"])
+        assert M.moe_read_status(g["ws"]) & ~M.DEV_PLAN_INEXACT == 0
+        assert torch.equal(h3[:total], g["h"][:total])
+        assert torch.equal(y3[:total], g["yp"][:total])
     del g, inp
     torch.cuda.empty_cache()
