@@ -199,7 +199,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(est),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic (seeded; see DESIGN.md input recipe)",
+            "data": "synthetic (seeded SplitMix64 + Box-Muller inputs, the recipe in routed_experts_b200/inputs.py)",
             "config": {"workload": cfg.name, **C.describe(cfg)},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": sample},
@@ -628,7 +628,7 @@ def run_mine(args, world, rank, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "bf16" if cfg.dtype == C.BF16 else "fp32",
-        "data": "synthetic (seeded SplitMix64 + Box-Muller inputs; see DESIGN.md input recipe)",
+        "data": "synthetic (seeded SplitMix64 + Box-Muller inputs, the recipe in routed_experts_b200/inputs.py)",
         "config": {"workload": cfg.name, **C.describe(cfg), "seed": args.seed,
                    "l2": "no flush: one step touches ~%.1f GB (weights %.2f GB) >> 126 MB L2"
                          % ((alg_bytes + 3 * cap * d * eb + 2 * cap * F * eb) / 1e9, weight_bytes / 1e9),
