@@ -320,10 +320,10 @@ moe_status moe_layer_bwd(const moe_config* cfg, const float* logits, const void*
                          size_t ws_bytes, moe_stream_t stream);
 
 /*
- * ---- MXFP8 forward ([MegaFlux] §2.1 'Persistent MoE execution': block-scaled
- * MX tensor-core MMA; §4.1 'Setup': the forward on MX operands with fp32
- * accumulation and bf16 outputs; [MoonEP] "A bandwidth-only model": one
- * scale per 32 elements).
+ * ---- MX forward: MXFP8 activations with MXFP4 or MXFP8 weights ([MegaFlux]
+ * §2.1 'Persistent MoE execution': block-scaled MX tensor-core MMA; §4.1
+ * 'Setup': the forward on MX operands with fp32 accumulation and bf16
+ * outputs; [MoonEP] "A bandwidth-only model": one scale per 32 elements).
  *
  * MXFP8 matrix [rows, K] (K a multiple of 128): codes uint8 [rows, K], one
  * E4M3 byte per element, row-major; scales uint8, one E8M0 byte per 32
@@ -386,7 +386,7 @@ moe_status moe_dispatch_mx(const moe_config* cfg, const void* x, void* xq, void*
                            size_t ws_bytes, moe_stream_t stream);
 
 /*
- * moe_expert_fc1_mx - step A7 on MXFP8 operands: per planned block,
+ * moe_expert_fc1_mx - step A7 on MX operands: per planned block,
  * h = silu(xq W1g^T) * (xq W1u^T) with the MMA's fp32 accumulation, rounded to
  * bf16, then quantized to MXFP8 along F into hq / hs (MOE_MX_HQ / MOE_MX_HS,
  * device, out). Padding rows of a block get zero codes and scale 0.
@@ -398,7 +398,7 @@ moe_status moe_expert_fc1_mx(const moe_config* cfg, const void* xq, const void* 
                              moe_stream_t stream);
 
 /*
- * moe_expert_fc2_mx - step A8 on MXFP8 operands: yp = hq W2^T, fp32
+ * moe_expert_fc2_mx - step A8 on MX operands: yp = hq W2^T, fp32
  * accumulation, stored as bf16 [rows_cap, d] (device, out); padding rows are
  * zero. hq, hs: from moe_expert_fc1_mx; w2q, w2s: from moe_mx_quantize_weights
  * with weight format wfmt.
@@ -408,7 +408,7 @@ moe_status moe_expert_fc2_mx(const moe_config* cfg, const void* hq, const void* 
                              moe_stream_t stream);
 
 /*
- * moe_layer_fwd_mx - the whole layer on MXFP8 expert operands: moe_plan,
+ * moe_layer_fwd_mx - the whole layer on MX expert operands: moe_plan,
  * moe_dispatch_mx, moe_expert_fc1_mx, moe_expert_fc2_mx and moe_combine, on
  * a MOE_WS_LAYER workspace (xq/xs live where xp does, hq/hs where h does).
  *   logits fp32 [T, E], x bf16 [T, d] (device); w1q/w1s/w2q/w2s from
