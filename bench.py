@@ -45,11 +45,12 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=20)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--config", default="olmoe", choices=sorted(C.NAMED))
+    p.add_argument("--config", default="dsv3", choices=sorted(C.NAMED))
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--impl", default="mine", choices=["mine", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-tokens", type=int, default=320, help="tokens of the oracle's FFN sample")
+    p.add_argument("--cpu-tokens", type=int, default=None,
+                   help="tokens of the oracle's FFN sample (default: sized to a few seconds per leg)")
     p.add_argument("--no-backward", action="store_true", help="skip timing the layer's backward")
     p.add_argument("--no-mx", action="store_true", help="skip timing the layer on MXFP8 operands")
     return p.parse_args()
@@ -175,34 +176,131 @@ def dist_setup(args):
     return world, rank, local
 
 
+# ------------------------------------------------------------------ the CPU oracle, timed
+
+# Rough fp64 rate of the oracle's plain loops on one core (FLOP/s), used only
+# to size the token samples so that each leg takes seconds, not hours.
+ORACLE_FLOPS_GUESS = 1.8e9
+
+
+def host_facts() -> dict:
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "logical_cpus": os.cpu_count(), "usable_cpus": len(os.sched_getaffinity(0))}
+
+
+def oracle_tokens_for(cfg, seconds: float, lo: int, hi: int) -> int:
+    """Tokens of the oracle's FFN sample that take about `seconds` on one core."""
+    per_token = 6.0 * cfg.d * cfg.F * cfg.K / ORACLE_FLOPS_GUESS
+    return int(max(lo, min(hi, cfg.T, round(seconds / per_token))))
+
+
+def oracle_leg(cfg, logits, x, expert_weights, n_tokens: int, workers: int) -> dict:
+    """One timed pass of the CPU oracle on a bounded sample of the layer.
+
+    Routing, gating, histogram, planning and row maps run over every token
+    on one thread (the planner is sequential). The expert FFN and combine
+    run for `n_tokens` evenly spaced tokens, split into `workers` shards that
+    run on that many threads at once (each shard is one single-threaded
+    oracle call; ctypes releases the interpreter lock around it). The
+    whole-layer time is the routing time plus the sample's wall time per
+    token times T. `expert_weights(experts)` returns host bit arrays of those
+    experts' weights (fetched outside the timed parts)."""
+    import concurrent.futures
+    from oracle import oracle as O
+    T, E, K = cfg.T, cfg.E, cfg.K
+    t0 = time.perf_counter()
+    idx, w = O.topk_gate(logits, K, cfg.gating)
+    counts = O.histogram(idx, E)
+    pl = O.plan(T, E, K, cfg.R, cfg.tile, cfg.budget, counts, getattr(cfg, "plan_mode", 0))
+    O.row_maps(idx, E, pl["pieces"], O.rows_capacity(T * K, E, cfg.R, cfg.budget, cfg.tile))
+    routing_s = time.perf_counter() - t0
+    toks = np.unique(np.linspace(0, T - 1, num=min(n_tokens, T)).astype(np.int64))
+    experts, sub = np.unique(idx[toks], return_inverse=True)
+    wgu, wdn = expert_weights(experts)
+    sub_idx = np.ascontiguousarray(sub.reshape(len(toks), K).astype(np.int32))
+    xs = np.ascontiguousarray(x[toks])
+    ws_ = np.ascontiguousarray(w[toks])
+    shards = [s_ for s_ in np.array_split(np.arange(len(toks), dtype=np.int64), workers) if len(s_)]
+    rm = O.default_round_mode(cfg.dtype)
+    t1 = time.perf_counter()
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(shards)) as ex:
+        list(ex.map(lambda sh: O.token_out(sh, xs, sub_idx, ws_, wgu, wdn, cfg.dtype, rm), shards))
+    ffn_s = time.perf_counter() - t1
+    per_tok = ffn_s / len(toks)
+    return {"routing_s": routing_s, "ffn_wall_s": ffn_s, "sample_tokens": int(len(toks)),
+            "threads": len(shards), "layer_s_est": routing_s + per_tok * T,
+            "step_s": routing_s + ffn_s}
+
+
+def oracle_sample_text(cfg, leg: dict) -> str:
+    return (f"top-k, gating, histogram, plan and row maps over all {cfg.T} tokens on one thread "
+            f"({leg['routing_s']:.2f} s); expert FFN and combine over {leg['sample_tokens']} evenly spaced tokens on "
+            f"{leg['threads']} thread(s) ({leg['ffn_wall_s']:.2f} s wall), scaled to {cfg.T} tokens; fp64 C oracle, "
+            f"each call single-threaded")
+
+
+def bench_config(cfg, seed: int, world: int) -> dict:
+    """The `config` object of the JSON line (identical in both arms)."""
+    eb = cfg.elem_bytes
+    w_bytes = 3 * cfg.E * cfg.F * cfg.d * eb
+    buf_bytes = (cfg.N + (cfg.E + cfg.R * cfg.budget) * cfg.tile) * (2 * cfg.d + cfg.F) * eb
+    big = w_bytes + buf_bytes > 126e6
+    l2 = (f"no flush: inputs larger than L2 (expert weights {w_bytes / 1e9:.2f} GB, padded xp/h/yp "
+          f"{buf_bytes / 1e9:.2f} GB, against a 126 MB L2)" if big else
+          f"no flush; the working set ({(w_bytes + buf_bytes) / 1e6:.1f} MB) fits in L2 (a parity-sized shape)")
+    return {"workload": cfg.name, **C.describe(cfg), "seed": seed, "l2": l2,
+            "parallelism": f"replicas x{world} (independent layers, no collective)"}
+
+
 # ------------------------------------------------------------------ reference arm
 
 def run_reference(args, world, rank):
+    """The CPU oracle as the reference arm, rank 0 only: each step is one
+    oracle_leg on all usable host cores over a bounded token sample."""
     if rank != 0:
         return
-    from oracle import oracle as O
     cfg = C.NAMED[args.config]
-    inp = I.make_inputs(cfg, args.seed, "cpu")
-    h = {k: I.to_numpy_bits(v) for k, v in inp.items()}
-    kw = dict(K=cfg.K, R=cfg.R, tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype)
-    n_tok = max(2, args.cpu_tokens // 16)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"   # input generation only
+    inp = I.make_inputs(cfg, args.seed, dev, weights=False)
+    logits, x = I.to_numpy_bits(inp["logits"]), I.to_numpy_bits(inp["x"])
+    workers = max(1, len(os.sched_getaffinity(0)))
+    n_tok = workers * oracle_tokens_for(cfg, 2.0, 1, 64) if args.cpu_tokens is None else args.cpu_tokens
+
+    cache = {}
+
+    def weights(experts):
+        missing = [int(e) for e in experts if int(e) not in cache]
+        if missing:
+            wgu, wdn = I.expert_weights(cfg, args.seed, missing, dev)
+            for i, e in enumerate(missing):
+                cache[e] = (I.to_numpy_bits(wgu[i]), I.to_numpy_bits(wdn[i]))
+        return (np.stack([cache[int(e)][0] for e in experts]), np.stack([cache[int(e)][1] for e in experts]))
+
+    oracle_leg(cfg, logits, x, weights, n_tok, workers)   # fetches the sample's weights once
     for _ in range(args.warmup):
-        O.timed_sample(h["logits"], h["x"], h["w_gate_up"], h["w_down"], n_tokens=2, **kw)
-    est = []
-    for _ in range(args.steps):
-        r = O.timed_sample(h["logits"], h["x"], h["w_gate_up"], h["w_down"], n_tokens=n_tok, **kw)
-        est.append(r["layer_s_est"])
-    total = sum(est)
-    value = cfg.T * len(est) / total
-    sample = (f"per step: top-k, gating, histogram, plan and row maps over all {cfg.T} tokens; expert FFN and "
-              f"combine over {n_tok} evenly spaced tokens, scaled by T/{n_tok}; single-threaded fp64 C oracle")
+        oracle_leg(cfg, logits, x, weights, n_tok, workers)
+    legs = [oracle_leg(cfg, logits, x, weights, n_tok, workers) for _ in range(args.steps)]
+    est = sum(l_["layer_s_est"] for l_ in legs)
+    value = cfg.T * len(legs) / est
+    measured = sum(l_["step_s"] for l_ in legs)
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(est),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * measured / len(legs),
+            "layer_ms_est": 1e3 * est / len(legs),
+            "timing": "ms_per_step is the measured wall time of one sampled step; value is the whole layer's "
+                      "tokens/s extrapolated from it (layer_ms_est per layer)",
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded SplitMix64 + Box-Muller inputs, the recipe in routed_experts_b200/inputs.py)",
-            "config": {"workload": cfg.name, **C.describe(cfg)},
-            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": sample},
+            "config": bench_config(cfg, args.seed, world),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": legs[0]["threads"], "kind": "oracle",
+                             "sample": oracle_sample_text(cfg, legs[0]), "host": host_facts()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -259,16 +357,42 @@ def plan_comparison(cfg, inp, dev, reps=20):
 
 
 def cpu_baseline(cfg, inp, n_tokens):
-    from oracle import oracle as O
-    h = {k: I.to_numpy_bits(v) for k, v in inp.items()}
-    r = O.timed_sample(h["logits"], h["x"], h["w_gate_up"], h["w_down"], K=cfg.K, R=cfg.R, tile=cfg.tile,
-                       budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype, n_tokens=n_tokens)
-    return {"value": cfg.T / r["layer_s_est"], "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": (f"top-k, gating, histogram, plan and row maps over all {cfg.T} tokens "
-                       f"({r['routing_s']:.2f} s) plus expert FFN and combine over {r['sample_tokens']} evenly "
-                       f"spaced tokens ({r['ffn_s_per_token'] * 1e3:.1f} ms/token), scaled to {cfg.T} tokens; "
-                       f"{r['measured_s']:.1f} s of single-threaded fp64 C"),
-            "measured_s": r["measured_s"]}
+    """The oracle on the host cores beside the GPU run: one leg on a single
+    thread and one on every usable core, each on a bounded token sample."""
+    logits, x = I.to_numpy_bits(inp["logits"]), I.to_numpy_bits(inp["x"])
+
+    def weights(experts):
+        sel = torch.as_tensor(np.asarray(experts, dtype=np.int64), device=inp["w_gate_up"].device)
+        return I.to_numpy_bits(inp["w_gate_up"][sel]), I.to_numpy_bits(inp["w_down"][sel])
+
+    workers = max(1, len(os.sched_getaffinity(0)))
+    one = oracle_leg(cfg, logits, x, weights, n_tokens or oracle_tokens_for(cfg, 12.0, 8, 320), 1)
+    allc = oracle_leg(cfg, logits, x, weights, workers * oracle_tokens_for(cfg, 8.0, 1, 256), workers)
+    return {"value": cfg.T / allc["layer_s_est"], "unit": "tokens/s", "cores": allc["threads"], "kind": "oracle",
+            "sample": oracle_sample_text(cfg, allc), "host": host_facts(),
+            "single_core": {"value": cfg.T / one["layer_s_est"], "unit": "tokens/s", "cores": 1,
+                            "sample": oracle_sample_text(cfg, one)}}
+
+
+def skew_descriptors(cfg, counts: np.ndarray, plan: dict) -> dict:
+    """Routing skew of the step's input and the balance the plan reached:
+    kappa = max/mean entries per expert ([MegaFlux] §4.1, the workloads'
+    skew measure), MaxVio = how far the busiest expert sits above the mean,
+    as a ratio minus one ([MoonEP] "Per-expert breakdown"), and the virtual
+    ranks' loads (entries, and 128-row tiles after padding) over their mean
+    before planning (home experts only) and after."""
+    c = np.asarray(counts, dtype=np.float64)
+    mean_e = cfg.N / cfg.E
+    home = c.reshape(cfg.R, cfg.E // cfg.R).sum(axis=1)
+    C_ = cfg.N / cfg.R
+    loads = plan["rank_load"].numpy().astype(np.float64)
+    tiles = np.diff(plan["rank_row0"].numpy()) / cfg.tile
+    return {"kappa": float(c.max() / mean_e), "maxvio": float(c.max() / mean_e - 1.0),
+            "experts_chosen": int((c > 0).sum()),
+            "rank_load_max_over_mean_before": float(home.max() / C_),
+            "rank_load_min_over_mean_before": float(home.min() / C_),
+            "rank_load_max_over_mean_after": float(loads.max() / C_),
+            "rank_tiles_max_over_mean_after": float(tiles.max() / tiles.mean())}
 
 
 def time_backward(cfg, inp, args, world, dev, stream, pg):
@@ -629,10 +753,7 @@ def run_mine(args, world, rank, local):
         "vs_baseline": None,
         "dtype": "bf16" if cfg.dtype == C.BF16 else "fp32",
         "data": "synthetic (seeded SplitMix64 + Box-Muller inputs, the recipe in routed_experts_b200/inputs.py)",
-        "config": {"workload": cfg.name, **C.describe(cfg), "seed": args.seed,
-                   "l2": "no flush: one step touches ~%.1f GB (weights %.2f GB) >> 126 MB L2"
-                         % ((alg_bytes + 3 * cap * d * eb + 2 * cap * F * eb) / 1e9, weight_bytes / 1e9),
-                   "parallelism": f"replicas x{world} (independent layers, no collective)"},
+        "config": bench_config(cfg, args.seed, world),
         "roofline": {"bound": "tensor", "kernel": "ffn_tc_kernel<FC1+SwiGLU>",
                      "achieved": fc1_flop / fc1_s / 1e12, "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": fc1_flop / fc1_s / 1e12 / tensor_peak,
@@ -651,6 +772,7 @@ def run_mine(args, world, rank, local):
                         "combine_gbs": combine_bytes / (mean[4] * 1e-3) / 1e9},
         "plan": {"moves": plan["moves"], "replicas": plan["replicas"], "status": plan["status"],
                  "padded_rows": plan["total_rows"] - N, "blocks": plan["n_blocks"]},
+        "skew": skew_descriptors(cfg, counts.cpu().numpy(), plan),
         "planners": plans,
         "e2e": {"value": world * T / (e2e_ms / args.steps * 1e-3), "unit": "tokens/s",
                 "h2d_bytes_per_step": 4 * T * E + T * d * eb, "d2h_bytes_per_step": T * d * eb,
@@ -673,7 +795,7 @@ def run_mine(args, world, rank, local):
         "clocks": clk.summary(),
     }
     if cpu is not None:
-        line["cpu_baseline"] = {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")}
+        line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
 
 

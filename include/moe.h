@@ -430,16 +430,19 @@ moe_status moe_layer_fwd_mx(const moe_config* cfg, const float* logits, const vo
  *   logits, topk_idx, topk_w, counts: as in moe_plan.
  *   row_of  int32 [T*K] (device, out): padded row of entry (t, k), as in
  *           moe_plan_layout.
- *   header  uint32 [8] (device, out): device status bits, n_pieces,
- *           n_blocks, total_rows, moves, replicas in total, 0, 0 - as the
- *           header of moe_plan_layout.
+ *   header  uint32 [8] (device, out): the header of moe_plan_layout: device
+ *           status bits, n_pieces, n_blocks, total_rows, moves, replicas in
+ *           total, then for MOE_PLAN_BLOCKS tau and the winning candidate,
+ *           else 0, 0.
  * The planner's scratch lives in one static device array of
  * MOE_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
  * the library keeps reserved until the process exits. A shape whose scratch
  * exceeds it returns MOE_ERR_WORKSPACE (moe_workspace_size with MOE_WS_PLAN
  * gives the bytes a shape needs). The call allocates and frees nothing.
- * The first call on each device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
+ * Every call looks up the array's device address on the current device (a
+ * lookup, not an allocation; it stays right after a cudaDeviceReset). The
+ * first lookup on a device loads the library's device code there, so make
+ * the first call on each device before any stream capture.
  * Every call shares the one array and it keeps the last call's contents;
  * calls that overlap on the GPU (for example on two streams at once) race
  * on it, so order them on one stream or with events.

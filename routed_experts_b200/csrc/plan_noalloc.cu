@@ -13,11 +13,13 @@
 //
 // The array's name is only a host-side stand-in in host code; a kernel given
 // it would fault, or on systems where the GPU can reach host memory would
-// silently use the wrong memory. Its device address is looked up once per
-// device with cudaGetSymbolAddress, with that device current, on the first
-// call made on that device, and the kernels receive that address.
-#include <mutex>
-
+// silently use the wrong memory. Every call therefore looks up the array's
+// device address on the current device with cudaGetSymbolAddress (a lookup,
+// no allocation) and hands that address to the kernels. Looking it up on
+// every call rather than once keeps the address right after a
+// cudaDeviceReset, which reloads the library's module and may move the array.
+// The first lookup on a device loads the module there, so that first call
+// belongs before any stream capture.
 #include "common.cuh"
 
 namespace {
@@ -25,11 +27,6 @@ namespace {
 // Largest scratch one call can use; every GPU that loads the library keeps
 // this much device memory reserved until the process exits.
 constexpr size_t kScratchBytes = MOE_NOALLOC_SCRATCH_BYTES;
-
-// Device addresses of the scratch array, one per device, looked up on first use.
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mu;
-void* g_scratch_dev[kMaxDevices] = {};
 
 }  // namespace
 
@@ -39,19 +36,11 @@ namespace {
 
 // The device address of g_plan_scratch on the current device.
 cudaError_t scratch_address(void** out) {
-    int dev = -1;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_plan_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_setup_mu);
-    if (g_scratch_dev[dev] == nullptr) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_plan_scratch);
-        if (e != cudaSuccess) return e;
-        if (p == nullptr) return cudaErrorInvalidSymbol;
-        g_scratch_dev[dev] = p;
-    }
-    *out = g_scratch_dev[dev];
+    if (p == nullptr) return cudaErrorInvalidSymbol;
+    *out = p;
     return cudaSuccess;
 }
 

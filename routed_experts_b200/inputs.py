@@ -97,21 +97,23 @@ def uniform(key: int, start: int, n: int, device="cpu") -> torch.Tensor:
     return _lsr(z, 11).to(torch.float64) * (2.0 ** -53)
 
 
-def normal(key: int, n: int, device="cpu", out_dtype=torch.float64, std: float = 1.0) -> torch.Tensor:
-    """n standard normals (times std) of stream ``key``, drawn in chunks, stored as out_dtype."""
+def normal(key: int, n: int, device="cpu", out_dtype=torch.float64, std: float = 1.0,
+           start: int = 0) -> torch.Tensor:
+    """Normals start..start+n-1 (times std) of stream ``key``, drawn in chunks, stored as out_dtype."""
     out = torch.empty(n, dtype=out_dtype, device=device)
     pos = 0
     while pos < n:
         m = min(_CHUNK, n - pos)
-        # element j of the tensor is the cos (j even) or sin (j odd) output of
+        # element j of the stream is the cos (j even) or sin (j odd) output of
         # pair j//2, which uses uniforms 2*(j//2) and 2*(j//2)+1
-        p0 = pos // 2
-        npairs = (pos + m - 1) // 2 - p0 + 1
+        a = start + pos
+        p0 = a // 2
+        npairs = (a + m - 1) // 2 - p0 + 1
         u = uniform(key, 2 * p0, 2 * npairs, device).view(-1, 2)
         r = torch.sqrt(-2.0 * torch.log1p(-u[:, 0]))
         th = (2.0 * math.pi) * u[:, 1]
         v = torch.stack((r * torch.cos(th), r * torch.sin(th)), dim=1).reshape(-1)
-        v = v[pos - 2 * p0: pos - 2 * p0 + m]
+        v = v[a - 2 * p0: a - 2 * p0 + m]
         if std != 1.0:
             v = v * std
         if out_dtype == torch.bfloat16:
@@ -182,6 +184,24 @@ def make_inputs(cfg: LayerConfig, seed: int = 0, device="cpu", weights: bool = T
     out["logits"] = lg.to(torch.float32).contiguous()
     out["x"] = x.contiguous()
     return out
+
+
+def expert_weights(cfg: LayerConfig, seed: int, experts, device="cpu"):
+    """The expert weights of ``make_inputs`` for the listed experts only:
+    (w_gate_up [n, 2F, d], w_down [n, d, F]), bit-identical to those experts'
+    slices of the full tensors (the streams are counter-based, so each
+    expert's elements are drawn from their own positions)."""
+    dt = torch.bfloat16 if cfg.dtype == BF16 else torch.float32
+    d, F = cfg.d, cfg.F
+    es = [int(e) for e in experts]
+    wgu = torch.empty(len(es), 2 * F, d, dtype=dt, device=device)
+    wdn = torch.empty(len(es), d, F, dtype=dt, device=device)
+    for i, e in enumerate(es):
+        wgu[i] = normal(stream_key(seed, TID_WGU), 2 * F * d, device, dt, cfg.w_std,
+                        start=e * 2 * F * d).view(2 * F, d)
+        wdn[i] = normal(stream_key(seed, TID_WDOWN), d * F, device, dt, cfg.w_std,
+                        start=e * d * F).view(d, F)
+    return wgu, wdn
 
 
 def make_grad_out(cfg: LayerConfig, seed: int = 0, device="cpu") -> torch.Tensor:

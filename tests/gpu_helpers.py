@@ -2,6 +2,9 @@
 stage, and compare every stage with the CPU oracle on the same inputs."""
 from __future__ import annotations
 
+import concurrent.futures
+import os
+
 import numpy as np
 import torch
 
@@ -35,29 +38,192 @@ def to_f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def run_stages(cfg, inp: dict) -> dict:
-    """moe_plan, moe_dispatch, moe_expert_ffn, moe_combine on device inputs."""
+# Bit patterns written into h and yp before a call: rows no entry maps to
+# (padding) must come back either untouched or zero, never anything else.
+SENTINEL = {C.BF16: 0x7FAB, C.FP32: 0x7FC0ABCD}
+
+
+def sentinel_like(shape, cfg, device) -> torch.Tensor:
+    if cfg.dtype == C.BF16:
+        return torch.full(shape, SENTINEL[C.BF16], dtype=torch.int16, device=device).view(torch.bfloat16)
+    return torch.full(shape, SENTINEL[C.FP32], dtype=torch.int32, device=device).view(torch.float32)
+
+
+PATHS = ("staged", "fused", "fused_gather", "fc1_gather", "layer")
+
+
+def run_path(cfg, inp: dict, path: str = "staged") -> dict:
+    """moe_plan, then the FFN through one of the library's paths, then
+    moe_combine, on device inputs:
+      staged        moe_dispatch, moe_expert_ffn (FC1 launch, FC2 launch)
+      fused         moe_dispatch, moe_expert_ffn_fused (FC1 and FC2 in one launch)
+      fused_gather  moe_expert_ffn_fused_gather (dispatch, FC1 and FC2 in one launch)
+      fc1_gather    moe_expert_fc1_gather (dispatch and FC1 in one launch), moe_expert_fc2
+      layer         moe_layer_fwd alone (h and yp stay inside its workspace)."""
     dev = inp["x"].device
     T, K, E, d, F = cfg.T, cfg.K, cfg.E, cfg.d, cfg.F
     dt = M.act_dtype(cfg)
+    cap = M.moe_rows_capacity(cfg)
+    if path == "layer":
+        layer = M.Layer(cfg, dev)
+        out = layer.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"])
+        status = layer.status()
+        return {"out": out, "status": status, "plan": M.read_plan(cfg, layer.ws), "ws": layer.ws, "rows_cap": cap,
+                "idx": None}
     idx = torch.empty(T, K, dtype=torch.int32, device=dev)
     w = torch.empty(T, K, dtype=torch.float32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
     ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
-    cap = M.moe_rows_capacity(cfg)
-    # dispatch leaves padding rows of xp alone: NaN there must not reach h, yp or out
-    xp = torch.full((cap, d), float("nan"), dtype=dt, device=dev)
-    h = torch.empty(cap, F, dtype=dt, device=dev)
-    yp = torch.empty(cap, d, dtype=dt, device=dev)
+    h = sentinel_like((cap, F), cfg, dev)
+    yp = sentinel_like((cap, d), cfg, dev)
     out = torch.empty(T, d, dtype=dt, device=dev)
     M.moe_plan(cfg, inp["logits"], idx, w, counts, ws)
-    M.moe_dispatch(cfg, inp["x"], xp, ws)
-    M.moe_expert_ffn(cfg, xp, inp["w_gate_up"], inp["w_down"], h, yp, ws)
+    xp = None
+    if path in ("staged", "fused"):
+        # dispatch leaves padding rows of xp alone: NaN there must not reach h, yp or out
+        xp = torch.full((cap, d), float("nan"), dtype=dt, device=dev)
+        M.moe_dispatch(cfg, inp["x"], xp, ws)
+    if path == "staged":
+        M.moe_expert_ffn(cfg, xp, inp["w_gate_up"], inp["w_down"], h, yp, ws)
+    elif path == "fused":
+        M.moe_expert_ffn_fused(cfg, xp, inp["w_gate_up"], inp["w_down"], h, yp, ws)
+    elif path == "fused_gather":
+        M.moe_expert_ffn_fused_gather(cfg, inp["x"], inp["w_gate_up"], inp["w_down"], h, yp, ws)
+    elif path == "fc1_gather":
+        M.moe_expert_fc1_gather(cfg, inp["x"], inp["w_gate_up"], h, ws)
+        M.moe_expert_fc2(cfg, h, inp["w_down"], yp, ws)
+    else:
+        raise ValueError(path)
     M.moe_combine(cfg, yp, w, out, ws)
     status = M.moe_read_status(ws)
     plan = M.read_plan(cfg, ws)
     return {"idx": idx, "w": w, "counts": counts, "xp": xp, "h": h, "yp": yp, "out": out,
             "status": status, "plan": plan, "ws": ws, "rows_cap": cap}
+
+
+def run_stages(cfg, inp: dict) -> dict:
+    """moe_plan, moe_dispatch, moe_expert_ffn, moe_combine on device inputs."""
+    return run_path(cfg, inp, "staged")
+
+
+def check_padding_rows(t: torch.Tensor, valid: np.ndarray, cfg, what: str):
+    """Rows no entry maps to hold either the sentinel written before the call
+    or zero in every element."""
+    pad = torch.as_tensor(np.nonzero(~valid)[0], device=t.device)
+    if not len(pad):
+        return
+    bits = t[pad].view(torch.int16 if cfg.dtype == C.BF16 else torch.int32)
+    sent = SENTINEL[cfg.dtype]
+    if cfg.dtype == C.BF16:
+        sent = sent - (1 << 16) if sent >= (1 << 15) else sent
+    ok = (bits == sent).all(dim=1) | (bits == 0).all(dim=1)
+    assert bool(ok.all()), f"{what}: {int((~ok).sum())} padding rows written with values"
+
+
+# ---------------------------------------------------------------- the oracle on many cores
+
+ORACLE_THREADS = max(1, min(64, len(os.sched_getaffinity(0))))
+
+
+def _threaded(fn, n: int, *arrays):
+    """fn over ORACLE_THREADS contiguous shards of range(n), run on that many
+    threads (each call is one single-threaded oracle call; ctypes releases
+    the interpreter lock around it). Returns the shards' results in order."""
+    shards = [s_ for s_ in np.array_split(np.arange(n), ORACLE_THREADS) if len(s_)]
+    with concurrent.futures.ThreadPoolExecutor(max_workers=len(shards)) as ex:
+        return list(ex.map(fn, shards))
+
+
+def par_entry_ffn(tokens, experts, x, wgu, wdn, dtype, rm):
+    """O.entry_ffn over shards of the entries, on several threads."""
+    tokens = np.asarray(tokens, np.int64)
+    experts = np.asarray(experts, np.int32)
+    parts = _threaded(lambda sh: O.entry_ffn(tokens[sh], experts[sh], x, wgu, wdn, dtype, rm), len(tokens))
+    return np.concatenate([p[0] for p in parts]), np.concatenate([p[1] for p in parts])
+
+
+def par_token_out(tokens, x, idx, w, wgu, wdn, dtype, rm):
+    """O.token_out over shards of the tokens, on several threads."""
+    tokens = np.asarray(tokens, np.int64)
+    return np.concatenate(_threaded(lambda sh: O.token_out(tokens[sh], x, idx, w, wgu, wdn, dtype, rm),
+                                    len(tokens)))
+
+
+# ---------------------------------------------------------------- a test-side reference at full size
+
+class CloseOnGpu:
+    """The bf16 output bound of assert_close, accumulated over many slices on
+    the GPU: elementwise |g - o| <= atol + rtol |o| and the normwise error."""
+
+    def __init__(self, dtype: int, what: str):
+        self.atol, self.rtol, self.nrm = TOL[dtype]
+        self.what = what
+        self.bad = 0
+        self.n = 0
+        self.err2 = 0.0
+        self.ref2 = 0.0
+        self.max_err = 0.0
+
+    def add(self, got: torch.Tensor, ref: torch.Tensor):
+        g, o = got.double(), ref.double()
+        err = (g - o).abs()
+        self.bad += int((err > self.atol + self.rtol * o.abs()).sum())
+        self.n += err.numel()
+        self.err2 += float((err * err).sum())
+        self.ref2 += float((o * o).sum())
+        if err.numel():
+            self.max_err = max(self.max_err, float(err.max()))
+
+    def check(self):
+        assert self.bad == 0, f"{self.what}: {self.bad} of {self.n} elements out of tolerance, max err {self.max_err:.3e}"
+        if self.ref2 > 0:
+            rel = (self.err2 / self.ref2) ** 0.5
+            assert rel <= self.nrm, f"{self.what}: normwise error {rel:.3e} > {self.nrm}"
+
+
+def check_every_row_fp64(cfg, inp: dict, ref: dict, g: dict):
+    """Every valid row of h and yp, and every token of out, against a
+    test-side fp64 evaluation of the same formula on the GPU (torch matmuls
+    per expert, bf16 rounding where the layer stores: h = bf16(silu(a) g),
+    y = bf16(h W2^T), out = bf16(sum_k w_k y_k) in fp64). It reaches every
+    work item of a full-size layer, which the oracle's one-by-one rows
+    cannot; the oracle pins it through the sampled rows beside it."""
+    dev = inp["x"].device
+    F = cfg.F
+    blocks = ref["plan"]["blocks"]
+    total = ref["plan"]["total_rows"]
+    src = torch.as_tensor(ref["src_of"][:total], device=dev, dtype=torch.int64)
+    y_ref = torch.zeros(total, cfg.d, dtype=torch.float32, device=dev)
+    ch, cy = CloseOnGpu(cfg.dtype, "h (every valid row)"), CloseOnGpu(cfg.dtype, "yp (every valid row)")
+    rdt = torch.bfloat16 if cfg.dtype == C.BF16 else torch.float32
+    for e in np.unique(blocks[:, 0]):
+        eb = blocks[blocks[:, 0] == e]
+        rows = torch.as_tensor(np.concatenate([np.arange(b[1], b[1] + b[2]) for b in eb]), device=dev)
+        xe = inp["x"][src[rows]].double()
+        w1 = inp["w_gate_up"][int(e)].double()
+        a = xe @ w1[:F].T
+        gg = xe @ w1[F:].T
+        h = (a / (1.0 + torch.exp(-a)) * gg).to(rdt)
+        y = (h.double() @ inp["w_down"][int(e)].double().T).to(rdt)
+        if g.get("h") is not None:
+            ch.add(g["h"][rows], h)
+            cy.add(g["yp"][rows], y)
+        y_ref[rows] = y.float()
+        del xe, w1, a, gg, h, y
+    if g.get("h") is not None:
+        ch.check()
+        cy.check()
+    row_of = torch.as_tensor(ref["row_of"], device=dev, dtype=torch.int64).view(cfg.T, cfg.K)
+    wk = torch.as_tensor(ref["w"], device=dev).double()
+    co = CloseOnGpu(cfg.dtype, "out (every token)")
+    step = max(1, (1 << 28) // (cfg.K * cfg.d * 8))
+    for t0 in range(0, cfg.T, step):
+        t1 = min(cfg.T, t0 + step)
+        acc = torch.zeros(t1 - t0, cfg.d, dtype=torch.float64, device=dev)
+        for k in range(cfg.K):
+            acc += wk[t0:t1, k:k + 1] * y_ref[row_of[t0:t1, k]].double()
+        co.add(g["out"][t0:t1], acc.to(rdt))
+    co.check()
 
 
 def host_inputs(inp: dict, with_weights: bool = True) -> dict:
@@ -67,9 +233,10 @@ def host_inputs(inp: dict, with_weights: bool = True) -> dict:
 
 def check_routing_and_plan(cfg, g: dict, ref: dict):
     """Bit-exact checks of top-k, counts, plan and row maps; weights within 1e-6."""
-    assert np.array_equal(g["idx"].cpu().numpy(), ref["idx"]), "top-k indices differ"
-    np.testing.assert_allclose(g["w"].cpu().numpy(), ref["w"], rtol=0, atol=W_ATOL)
-    assert np.array_equal(g["counts"].cpu().numpy(), ref["counts"]), "counts differ"
+    if g.get("idx") is not None:
+        assert np.array_equal(g["idx"].cpu().numpy(), ref["idx"]), "top-k indices differ"
+        np.testing.assert_allclose(g["w"].cpu().numpy(), ref["w"], rtol=0, atol=W_ATOL)
+        assert np.array_equal(g["counts"].cpu().numpy(), ref["counts"]), "counts differ"
     gp, rp = g["plan"], ref["plan"]
     assert gp["moves"] == rp["moves"]
     assert (gp["status"] & O.PLAN_INEXACT) == rp["status"]
@@ -97,91 +264,123 @@ def oracle_routing(cfg, hin: dict) -> dict:
             "rows_cap": cap}
 
 
-def check_full_small(cfg, seed: int, device="cuda"):
-    """Every stage against the oracle, every element (sizes the oracle runs in seconds)."""
+def f64_to_bits(v: np.ndarray, dtype: int) -> np.ndarray:
+    """Values that are exactly representable in the layer's type, as its bits."""
+    f = np.asarray(v, np.float64).astype(np.float32)
+    return (f.view(np.uint32) >> 16).astype(np.uint16) if dtype == C.BF16 else f
+
+
+def row_experts(blocks: np.ndarray, total: int) -> np.ndarray:
+    """The expert of every padded row (-1 outside blocks)."""
+    e = np.full(total, -1, np.int32)
+    for b in blocks:
+        e[b[1]:b[1] + b[2]] = b[0]
+    return e
+
+
+def check_full_small(cfg, seed: int, device="cuda", path: str = "staged", threads: bool = False):
+    """Every stage against the oracle, every element (sizes the oracle runs in
+    seconds). With threads=True the oracle's FFN runs as one entry_ffn per
+    valid row, sharded over host threads, and its combine on those rows
+    (the same arithmetic as the oracle's layer, for layers too large for one
+    thread)."""
     inp = I.make_inputs(cfg, seed, device)
-    g = run_stages(cfg, inp)
+    g = run_path(cfg, inp, path)
     hin = host_inputs(inp)
-    ref = O.layer(hin["logits"], hin["x"], hin["w_gate_up"], hin["w_down"], K=cfg.K, R=cfg.R,
-                  tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype,
-                  plan_mode=getattr(cfg, "plan_mode", 0))
+    rm = O.default_round_mode(cfg.dtype)
+    if not threads:
+        ref = O.layer(hin["logits"], hin["x"], hin["w_gate_up"], hin["w_down"], K=cfg.K, R=cfg.R,
+                      tile=cfg.tile, budget=cfg.budget, gating=cfg.gating, dtype=cfg.dtype,
+                      plan_mode=getattr(cfg, "plan_mode", 0))
+    else:
+        ref = oracle_routing(cfg, hin)
     assert g["rows_cap"] == ref["rows_cap"]
     check_routing_and_plan(cfg, g, ref)
     assert (g["status"] & ~O.PLAN_INEXACT) == 0, f"device status {g['status']}"
     total = ref["plan"]["total_rows"]
-    valid = ref["src_of"][:total] >= 0
-    assert np.array_equal(I.to_numpy_bits(g["xp"][:total])[valid], ref["xp"][:total][valid]), "xp differs"
-    gh, gy = to_f64(g["h"][:total]), to_f64(g["yp"][:total])
-    rh, ry = O.to_f64(ref["h"][:total], cfg.dtype), O.to_f64(ref["yp"][:total], cfg.dtype)
-    assert_close(gh[valid], rh[valid], cfg.dtype, "h")
-    assert_close(gy[valid], ry[valid], cfg.dtype, "yp")
-    assert not gh[~valid].any() and not gy[~valid].any(), "padding rows must be zero"
+    src = ref["src_of"][:total]
+    valid = src >= 0
+    if threads:
+        vrows = np.nonzero(valid)[0]
+        rh, ry = par_entry_ffn(src[vrows], row_experts(ref["plan"]["blocks"], total)[vrows], hin["x"],
+                               hin["w_gate_up"], hin["w_down"], cfg.dtype, rm)
+        yp_bits = np.zeros((ref["rows_cap"], cfg.d), np.uint16 if cfg.dtype == C.BF16 else np.float32)
+        yp_bits[vrows] = f64_to_bits(ry, cfg.dtype)
+        ref["out"] = O.combine(yp_bits, ref["row_of"], ref["w"], cfg.dtype, rm)
+        ref_h = np.zeros((total, cfg.F)); ref_h[vrows] = rh
+        ref_y = np.zeros((total, cfg.d)); ref_y[vrows] = ry
+    else:
+        ref_h = O.to_f64(ref["h"][:total], cfg.dtype)
+        ref_y = O.to_f64(ref["yp"][:total], cfg.dtype)
+    if g.get("xp") is not None:
+        assert np.array_equal(I.to_numpy_bits(g["xp"][:total])[valid], hin["x"][src[valid]]), "xp differs"
+    if g.get("h") is not None:
+        assert_close(to_f64(g["h"][:total])[valid], ref_h[valid], cfg.dtype, "h")
+        assert_close(to_f64(g["yp"][:total])[valid], ref_y[valid], cfg.dtype, "yp")
+        check_padding_rows(g["h"][:total], valid, cfg, "h")
+        check_padding_rows(g["yp"][:total], valid, cfg, "yp")
     assert_close(to_f64(g["out"]), O.to_f64(ref["out"], cfg.dtype), cfg.dtype, "out")
     return g, ref, inp
 
 
-class ExpertWeights:
-    """Host copies of single experts' weights, fetched on demand."""
+def check_routing_full_size(cfg, seed: int, device="cuda"):
+    """Routing, gating, counts, plan and row maps of a full-size layer, bit-exact (weights within 1e-6)."""
+    inp = I.make_inputs(cfg, seed, device, weights=False)
+    dev = inp["x"].device
+    idx = torch.empty(cfg.T, cfg.K, dtype=torch.int32, device=dev)
+    w = torch.empty(cfg.T, cfg.K, dtype=torch.float32, device=dev)
+    counts = torch.empty(cfg.E, dtype=torch.int32, device=dev)
+    ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
+    M.moe_plan(cfg, inp["logits"], idx, w, counts, ws)
+    status = M.moe_read_status(ws)
+    assert (status & ~O.PLAN_INEXACT) == 0, f"device status {status}"
+    g = {"idx": idx, "w": w, "counts": counts, "plan": M.read_plan(cfg, ws)}
+    ref = oracle_routing(cfg, host_inputs(inp, with_weights=False))
+    check_routing_and_plan(cfg, g, ref)
+    return ref
 
-    def __init__(self, inp: dict):
-        self.wgu, self.wdn = inp["w_gate_up"], inp["w_down"]
-        self.cache = {}
 
-    def stack(self, experts):
-        es = list(experts)
-        for e in es:
-            if e not in self.cache:
-                self.cache[e] = (I.to_numpy_bits(self.wgu[e]), I.to_numpy_bits(self.wdn[e]))
-        return (np.stack([self.cache[e][0] for e in es]), np.stack([self.cache[e][1] for e in es]))
-
-
-def check_full_size(cfg, seed: int, n_tokens: int = 8, n_rows: int = 32, device="cuda"):
-    """Full-size layer: bit-exact routing, plan, row maps and dispatch; sampled
-    rows of h and yp and sampled tokens of out against the oracle."""
+def check_full_size(cfg, seed: int, path: str = "staged", n_tokens: int = 64, device="cuda"):
+    """A full-size layer through one of the library's paths:
+      * routing, plan and row maps bit-exact, and the dispatched rows;
+      * every valid row of h and yp, and every token of out, against the
+        test-side fp64 evaluation (check_every_row_fp64);
+      * one row of h and yp in every planned block, with the row inside the
+        block drawn at random, and n_tokens tokens of out spread over the
+        token range, against the oracle (one by one, sharded over threads);
+      * rows no entry maps to untouched or zero."""
     inp = I.make_inputs(cfg, seed, device)
-    g = run_stages(cfg, inp)
+    g = run_path(cfg, inp, path)
     hin = host_inputs(inp, with_weights=False)
     ref = oracle_routing(cfg, hin)
     check_routing_and_plan(cfg, g, ref)
     assert (g["status"] & ~O.PLAN_INEXACT) == 0, f"device status {g['status']}"
     total = ref["plan"]["total_rows"]
     src = ref["src_of"][:total]
-    # dispatch: every row is the token row it names (or zero), bit for bit
-    xp = I.to_numpy_bits(g["xp"][:total])
     x = hin["x"]
     valid = src >= 0
-    assert np.array_equal(xp[valid], x[src[valid]]), "xp rows differ from their token rows"
-    del xp
-    # padding rows of h and yp are zero (xp holds NaN there)
-    pad = torch.as_tensor(np.nonzero(~valid)[0], device=device)
-    if len(pad):
-        assert not g["h"][pad].any() and not g["yp"][pad].any(), "padding rows of h and yp must be zero"
+    if g.get("xp") is not None:
+        xp = I.to_numpy_bits(g["xp"][:total])
+        assert np.array_equal(xp[valid], x[src[valid]]), "xp rows differ from their token rows"
+        del xp
+    if g.get("h") is not None:
+        check_padding_rows(g["h"][:total], valid, cfg, "h")
+        check_padding_rows(g["yp"][:total], valid, cfg, "yp")
+    check_every_row_fp64(cfg, inp, ref, g)
+    wgu, wdn = I.to_numpy_bits(inp["w_gate_up"]), I.to_numpy_bits(inp["w_down"])
+    rm = O.default_round_mode(cfg.dtype)
     rng = np.random.default_rng(seed + 17)
-    ew = ExpertWeights(inp)
-    # sampled rows of h and yp, from a few experts
     blocks = ref["plan"]["blocks"]
-    experts = rng.choice(np.unique(blocks[:, 0]), size=min(4, len(np.unique(blocks[:, 0]))), replace=False)
-    rows, exps = [], []
-    for k, e in enumerate(experts):
-        eb = blocks[blocks[:, 0] == e]
-        cand = np.concatenate([np.arange(b[1], b[1] + b[2]) for b in eb])
-        pick = rng.choice(cand, size=min(n_rows // len(experts), len(cand)), replace=False)
-        rows += pick.tolist()
-        exps += [k] * len(pick)
-    rows = np.array(rows)
-    wgu, wdn = ew.stack(experts)
-    rh, ry = O.entry_ffn(src[rows], np.array(exps), x, wgu, wdn, cfg.dtype, O.default_round_mode(cfg.dtype))
-    assert_close(to_f64(g["h"][torch.as_tensor(rows, device=device)]), rh, cfg.dtype, "sampled h rows")
-    assert_close(to_f64(g["yp"][torch.as_tensor(rows, device=device)]), ry, cfg.dtype, "sampled yp rows")
-    # sampled tokens of the output
-    toks = rng.choice(cfg.T, size=n_tokens, replace=False)
-    gout = to_f64(g["out"][torch.as_tensor(toks, device=device)])
-    for i, t in enumerate(toks):
-        es = ref["idx"][t]
-        wgu, wdn = ew.stack(es)
-        o = O.token_out(np.array([0]), x[t:t + 1], np.arange(cfg.K, dtype=np.int32)[None, :],
-                        ref["w"][t:t + 1], wgu, wdn, cfg.dtype, O.default_round_mode(cfg.dtype))
-        assert_close(gout[i:i + 1], o, cfg.dtype, f"out[{t}]")
+    if g.get("h") is not None:
+        rows = np.array([b[1] + rng.integers(b[2]) for b in blocks], np.int64)
+        rh, ry = par_entry_ffn(src[rows], blocks[:, 0], x, wgu, wdn, cfg.dtype, rm)
+        sel = torch.as_tensor(rows, device=device)
+        assert_close(to_f64(g["h"][sel]), rh, cfg.dtype, "h, one row per block")
+        assert_close(to_f64(g["yp"][sel]), ry, cfg.dtype, "yp, one row per block")
+    toks = np.unique(np.clip(np.linspace(0, cfg.T - 1, n_tokens).astype(np.int64) +
+                             rng.integers(0, max(1, cfg.T // n_tokens), n_tokens), 0, cfg.T - 1))
+    o = par_token_out(toks, x, ref["idx"], ref["w"], wgu, wdn, cfg.dtype, rm)
+    assert_close(to_f64(g["out"][torch.as_tensor(toks, device=device)]), o, cfg.dtype, "out, spread tokens")
     return g, ref, inp
 
 
@@ -399,26 +598,63 @@ def check_mx_small(cfg, seed: int, device="cuda", max_rows: int = 768, max_token
     return g, ref, inp
 
 
-def check_mx_full_size(cfg, seed: int, n_tokens: int = 3, device="cuda", wfmt: int = M.MX_W_E4M3):
-    """Full-size MX layer through moe_layer_fwd_mx: bit-exact routing and plan
-    (moe_plan), and sampled tokens of out against the oracle."""
+def par_mx_oracle_weights(cfg, inp: dict, wfmt: int):
+    """Oracle MX codes and scales of every expert's W1 and W2 (logical order),
+    one oracle call per expert, sharded over host threads."""
+    E = cfg.E
+
+    def one(sh):
+        res = []
+        for e in sh:
+            res.append(O.mx_weights(I.to_numpy_bits(inp["w_gate_up"][int(e)])[None],
+                                    I.to_numpy_bits(inp["w_down"][int(e)])[None], O.BF16, wfmt))
+        return res
+
+    parts = [r for chunk in _threaded(one, E) for r in chunk]
+    return tuple(np.concatenate([p[i] for p in parts]) for i in range(4))
+
+
+def check_mx_full_size(cfg, seed: int, n_tokens: int = 32, device="cuda", wfmt: int = M.MX_W_E4M3):
+    """Full-size MX layer through the staged MX calls: bit-exact routing, plan
+    and dispatched codes and scales; one row of h (codes and scales) and of
+    yp in every planned block, and n_tokens tokens of out spread over the
+    token range, against the oracle; the layer entry gives the same bits."""
     inp = I.make_inputs(cfg, seed, device)
+    g = run_mx_stages(cfg, inp, wfmt)
     hin = host_inputs(inp, with_weights=False)
     ref = oracle_routing(cfg, hin)
-    layer = M.Layer(cfg, device)
-    mxw = mx_weights_on_device(cfg, inp, wfmt)
-    out = layer.forward_mx(inp["logits"], inp["x"], mxw)
-    assert (layer.status() & ~O.PLAN_INEXACT) == 0
-    plan = M.read_plan(cfg, layer.ws)
-    assert np.array_equal(plan["row_of"].numpy(), ref["row_of"]), "row_of differs"
+    check_routing_and_plan(cfg, g, ref)
+    assert (g["status"] & ~O.PLAN_INEXACT) == 0, f"device status {g['status']}"
+    d, F = cfg.d, cfg.F
+    total = ref["plan"]["total_rows"]
+    src = ref["src_of"][:total]
+    valid = src >= 0
+    xq_ref, xs_ref = O.mx_quantize(hin["x"], O.BF16)
+    gxq = g["xq"][:total].cpu().numpy()
+    gxs = mx_unchunk(g["xs"], total, d)
+    assert np.array_equal(gxq[valid], xq_ref[src[valid]]), "dispatched codes differ"
+    assert np.array_equal(gxs[valid], xs_ref[src[valid]]), "dispatched scales differ"
+    del gxq, gxs
+    w1q, w1s, w2q, w2s = par_mx_oracle_weights(cfg, inp, wfmt)
     rng = np.random.default_rng(seed + 29)
-    toks = rng.choice(cfg.T, size=n_tokens, replace=False)
-    gout = to_f64(out[torch.as_tensor(toks, device=device)])
-    for i, t in enumerate(toks):
-        es = ref["idx"][t]
-        w1q, w1s, w2q, w2s = mx_oracle_weights(cfg, inp, es, wfmt)
-        xq, xs = O.mx_quantize(hin["x"][t:t + 1], O.BF16)
-        o = O.mx_token_out(np.array([0]), xq, xs, np.arange(cfg.K, dtype=np.int32)[None, :], ref["w"][t:t + 1],
-                           w1q, w1s, w2q, w2s, cfg.F, wfmt)
-        assert_close(gout[i:i + 1], o, C.BF16, f"out[{t}]")
-    return out
+    blocks = ref["plan"]["blocks"]
+    rows = np.array([b[1] + rng.integers(b[2]) for b in blocks], np.int64)
+    exps = blocks[:, 0].astype(np.int32)
+    parts = _threaded(lambda sh: O.mx_fc1_rows(np.arange(len(sh)), exps[sh], xq_ref[src[rows[sh]]],
+                                               xs_ref[src[rows[sh]]], w1q, w1s, F, wfmt), len(rows))
+    rh, rhq, rhs = (np.concatenate([p[i] for p in parts]) for i in range(3))
+    ghq = g["hq"][torch.as_tensor(rows, device=device)].cpu().numpy()
+    ghs_all = mx_unchunk(g["hs"], total, F)
+    assert_mx_h_close(ghq, ghs_all[rows], rh, rhq, rhs, "h (MXFP8), one row per block")
+    ry = np.concatenate(_threaded(lambda sh: O.mx_fc2_rows(exps[sh], rhq[sh], rhs[sh], w2q, w2s, d, wfmt),
+                                  len(rows)))
+    assert_close(to_f64(g["yp"][torch.as_tensor(rows, device=device)]), ry, C.BF16, "yp, one row per block")
+    toks = np.unique(np.linspace(0, cfg.T - 1, n_tokens).astype(np.int64))
+    rout = np.concatenate(_threaded(lambda sh: O.mx_token_out(toks[sh], xq_ref, xs_ref, ref["idx"], ref["w"], w1q,
+                                                               w1s, w2q, w2s, F, wfmt), len(toks)))
+    assert_close(to_f64(g["out"][torch.as_tensor(toks, device=device)]), rout, C.BF16, "out, spread tokens")
+    layer = M.Layer(cfg, device)
+    out = layer.forward_mx(inp["logits"], inp["x"], g["mxw"])
+    assert (layer.status() & ~O.PLAN_INEXACT) == 0
+    assert torch.equal(out, g["out"]), "moe_layer_fwd_mx differs from the staged MX calls"
+    return g

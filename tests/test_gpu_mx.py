@@ -73,6 +73,8 @@ def test_mx_layer_is_close_to_the_bf16_layer(wfmt, bound):
 
 
 @pytest.mark.parametrize("wfmt", FMTS, ids=FMT_IDS)
-@pytest.mark.parametrize("name,n_tokens", [("olmoe", 3), ("dsv3", 1)])
-def test_mx_layer_full_size_sampled(name, n_tokens, wfmt):
-    check_mx_full_size(C.NAMED[name], 0, n_tokens=n_tokens, wfmt=wfmt)
+@pytest.mark.parametrize("name", ["olmoe", "dsv3"])
+def test_mx_layer_full_size(name, wfmt):
+    # one row of h and yp in every planned block, 32 tokens of out
+    check_mx_full_size(C.NAMED[name], 0, n_tokens=32, wfmt=wfmt)
+    torch.cuda.empty_cache()

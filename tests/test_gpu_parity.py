@@ -14,7 +14,7 @@ from routed_experts_b200 import configs as C
 from routed_experts_b200 import inputs as I
 from routed_experts_b200 import moe as M
 
-from .gpu_helpers import check_full_size, check_full_small, run_stages, to_f64
+from .gpu_helpers import check_full_size, check_full_small, check_routing_full_size, run_path, run_stages, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -27,6 +27,12 @@ MED_BF16 = C.LayerConfig("med_bf16", T=1024, d=512, E=16, K=4, F=384, R=4, tile=
 WIDE_BF16 = C.LayerConfig("wide_bf16", T=256, d=768, E=32, K=8, F=128, R=8, tile=128, budget=4,
                           zipf_s=1.5)
 TINY_TILES = [C.TINY.replace(name=f"tiny_t{t}", tile=t) for t in (16, 32, 64, 128)]
+# Large enough that every cluster of CTA pairs takes several work items of
+# FC1 and of FC2 (about 300 each over 74 pairs), the operand ring wraps
+# inside every item (16 or 8 k-steps against 6 stages) and both TMEM
+# accumulators alternate; small enough for the oracle on a few cores.
+RING_BF16 = C.LayerConfig("ring_bf16", T=4096, d=1024, E=16, K=4, F=512, R=8, tile=128, budget=2,
+                          zipf_s=1.0)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -121,25 +127,6 @@ def test_layer_call_matches_staged_calls(cfg):
     assert torch.equal(out_h, staged.cpu())
 
 
-@pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, WIDE_BF16, C.OLMOE, C.DSV3], ids=lambda c: c.name)
-def test_gathered_fc1_matches_dispatch_then_fc1(cfg):
-    """FC1 reading x through the row map gives bit-identical h (padding rows
-    zero in both) to dispatch + FC1, and the whole-layer call gives
-    bit-identical output to the staged calls."""
-    inp = I.make_inputs(cfg, 2, "cuda")
-    g = run_stages(cfg, inp)
-    h2 = torch.empty_like(g["h"])
-    M.moe_expert_fc1_gather(cfg, inp["x"], inp["w_gate_up"], h2, g["ws"])
-    total = g["plan"]["total_rows"]
-    assert torch.equal(h2[:total], g["h"][:total])
-    layer = M.Layer(cfg)
-    out = layer.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"])
-    assert layer.status() & ~M.DEV_PLAN_INEXACT == 0
-    assert torch.equal(out, g["out"])
-    del layer, g, inp
-    torch.cuda.empty_cache()
-
-
 def test_gathered_fc1_is_bf16_only():
     cfg = C.TINY
     ws = M.alloc_workspace(cfg)
@@ -172,11 +159,14 @@ def test_block_planner_small_layers(cfg):
 
 @pytest.mark.parametrize("cfg", [C.OLMOE, C.QWEN3, C.EXTREME, C.DSV3], ids=lambda c: c.name)
 def test_block_planner_full_size(cfg):
-    check_full_size(cfg.replace(name=cfg.name + "_blocks", plan_mode=C.PLAN_BLOCKS), 0, n_tokens=4, n_rows=16)
+    check_full_size(cfg.replace(name=cfg.name + "_blocks", plan_mode=C.PLAN_BLOCKS), 0, n_tokens=32)
     torch.cuda.empty_cache()
 
 
-FULL = [C.OLMOE, C.QWEN3, C.EXTREME, C.DSV3]
+# The extreme-skew shape's second reading of its hot expert: the +30 bias
+# on half of the tokens only (the expert still takes the largest share).
+EXTREME_HOT50 = C.EXTREME.replace(name="extreme_hot50", hot_frac=0.5)
+FULL = [C.OLMOE, C.QWEN3, C.EXTREME, C.DSV3, EXTREME_HOT50]
 
 
 @pytest.mark.parametrize("cfg", FULL, ids=lambda c: c.name)
@@ -185,35 +175,67 @@ def test_full_size_layer(cfg):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("cfg", C.QWEN3_SWEEP, ids=lambda c: c.name)
-def test_qwen3_skew_sweep_plans(cfg):
-    # routing, plan, row maps and dispatch at full size for every skew level
-    check_full_size(cfg, 1, n_tokens=2, n_rows=8)
+@pytest.mark.parametrize("seed", [1, 2])
+@pytest.mark.parametrize("cfg", FULL + list(C.QWEN3_SWEEP), ids=lambda c: c.name)
+def test_full_size_routing_other_seeds(cfg, seed):
+    # routing, gating, counts, plan and row maps for the other realizations
+    check_routing_full_size(cfg, seed)
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, WIDE_BF16, C.OLMOE, C.DSV3], ids=lambda c: c.name)
-def test_fused_ffn_matches_the_staged_launches(cfg):
-    """FC1 and FC2 in one launch, FC2 tiles released per block pair by the
-    readiness counts, give the same bits as the separate launches, with FC1
-    reading xp or gathering x through the row map; a second call without a
-    new plan does too (the counts start from zero again)."""
+@pytest.mark.parametrize("seed", [1, 2])
+@pytest.mark.parametrize("cfg", [C.OLMOE, C.DSV3], ids=lambda c: c.name)
+def test_full_size_layer_other_seeds(cfg, seed):
+    check_full_size(cfg, seed, n_tokens=32)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cfg", C.QWEN3_SWEEP, ids=lambda c: c.name)
+def test_qwen3_skew_sweep(cfg):
+    # every skew level at full size: the plan bit-exact, every block sampled
+    check_full_size(cfg, 1, n_tokens=32)
+    torch.cuda.empty_cache()
+
+
+FUSED_PATHS = ["fused", "fused_gather", "fc1_gather", "layer"]
+
+
+@pytest.mark.parametrize("path", FUSED_PATHS)
+@pytest.mark.parametrize("cfg", [C.OLMOE, C.DSV3], ids=lambda c: c.name)
+def test_full_size_other_paths(cfg, path):
+    """The fused launches, FC1 with the dispatch folded in, and the whole-layer
+    entry against the oracle and the fp64 reference at full size."""
+    check_full_size(cfg, 3, path=path, n_tokens=32)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("path", ["staged", "fused", "fused_gather", "fc1_gather"])
+def test_every_element_of_a_layer_whose_clusters_take_several_items(path):
+    check_full_small(RING_BF16, 0, path=path, threads=True)
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, WIDE_BF16], ids=lambda c: c.name)
+@pytest.mark.parametrize("path", ["fused", "fused_gather", "fc1_gather"])
+def test_small_layers_other_paths(cfg, path):
+    check_full_small(cfg, 3, path=path)
+
+
+@pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, C.OLMOE], ids=lambda c: c.name)
+@pytest.mark.parametrize("path", ["fused", "fused_gather"])
+def test_fused_ffn_is_repeatable(cfg, path):
+    """A second fused call on the same workspace, without a new plan, gives
+    the same bits (its readiness counts and queues start from zero again)."""
     inp = I.make_inputs(cfg, 3, "cuda")
-    g = run_stages(cfg, inp)
-    for _ in range(2):
-        h2 = torch.full_like(g["h"], float("nan"))
-        y2 = torch.full_like(g["yp"], float("nan"))
-        M.moe_expert_ffn_fused(cfg, g["xp"], inp["w_gate_up"], inp["w_down"], h2, y2, g["ws"])
-        assert M.moe_read_status(g["ws"]) & ~M.DEV_PLAN_INEXACT == 0
-        total = g["plan"]["total_rows"]
-        assert torch.equal(h2[:total], g["h"][:total])
-        assert torch.equal(y2[:total], g["yp"][:total])
-        # dispatch, FC1 and FC2 in one launch: FC1 reads x through the row map
-        h3 = torch.full_like(g["h"], float("nan"))
-        y3 = torch.full_like(g["yp"], float("nan"))
-        M.moe_expert_ffn_fused_gather(cfg, inp["x"], inp["w_gate_up"], inp["w_down"], h3, y3, g["ws"])
-        assert M.moe_read_status(g["ws"]) & ~M.DEV_PLAN_INEXACT == 0
-        assert torch.equal(h3[:total], g["h"][:total])
-        assert torch.equal(y3[:total], g["yp"][:total])
-    del g, inp
+    a = run_path(cfg, inp, path)
+    h2, y2 = torch.empty_like(a["h"]), torch.empty_like(a["yp"])
+    if path == "fused":
+        M.moe_expert_ffn_fused(cfg, a["xp"], inp["w_gate_up"], inp["w_down"], h2, y2, a["ws"])
+    else:
+        M.moe_expert_ffn_fused_gather(cfg, inp["x"], inp["w_gate_up"], inp["w_down"], h2, y2, a["ws"])
+    assert M.moe_read_status(a["ws"]) & ~M.DEV_PLAN_INEXACT == 0
+    valid = torch.as_tensor(np.nonzero(a["plan"]["src_of"].numpy() >= 0)[0], device="cuda")
+    assert torch.equal(h2[valid], a["h"][valid])
+    assert torch.equal(y2[valid], a["yp"][valid])
+    del a, inp
     torch.cuda.empty_cache()

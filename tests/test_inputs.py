@@ -93,3 +93,20 @@ def test_named_configs_are_consistent(cfg):
     assert cfg.d % 64 == 0 and cfg.F % 64 == 0
     if cfg.dtype == C.BF16:
         assert cfg.tile == 128
+
+
+def test_expert_weights_match_slices_of_the_full_tensors(monkeypatch):
+    # odd offsets and a chunk boundary inside an expert's range
+    monkeypatch.setattr(I, "_CHUNK", 1000)
+    cfg = C.LayerConfig("ew", T=16, d=64, E=5, K=2, F=48, R=1, tile=16, budget=0)
+    full = I.make_inputs(cfg, 3)
+    wgu, wdn = I.expert_weights(cfg, 3, [4, 1, 2])
+    assert torch.equal(wgu, full["w_gate_up"][[4, 1, 2]])
+    assert torch.equal(wdn, full["w_down"][[4, 1, 2]])
+
+
+def test_normal_with_an_offset_is_a_slice():
+    key = I.stream_key(9, 1)
+    ref = I.normal(key, 101)
+    for start in (0, 1, 2, 37, 64):
+        assert torch.equal(I.normal(key, 101 - start, start=start), ref[start:])

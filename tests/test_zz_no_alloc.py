@@ -66,7 +66,7 @@ def _compare(got, ref):
     np.testing.assert_allclose(g_w.numpy(), r_w.numpy(), rtol=0, atol=W_ATOL)
     assert torch.equal(g_counts, r_counts)
     assert torch.equal(g_row, r_row)
-    assert torch.equal(g_hdr[:6], r_hdr[:6])
+    assert torch.equal(g_hdr, r_hdr)
 
 
 def test_no_alloc_plan_matches_plan_on_two_calls_in_a_row(M):
@@ -82,6 +82,17 @@ def test_no_alloc_plan_matches_plan_on_two_calls_in_a_row(M):
     _compare(_no_alloc(M, second, in2), ref2)
     # and the same layer twice
     _compare(_no_alloc(M, second, in2), ref2)
+
+
+def test_no_alloc_block_planner_header(M):
+    # MegaFlux's block-granular planner fills header words 6 and 7 (tau and
+    # the winning candidate); they must match moe_plan's too
+    cfg = C.OLMOE.replace(plan_mode=C.PLAN_BLOCKS)
+    inp = I.make_inputs(cfg, 2, "cuda", weights=False)
+    ref = _with_workspace(M, cfg, inp)
+    assert int(ref[4][6]) > 0
+    _compare(_no_alloc(M, cfg, inp), ref)
+    _compare(_no_alloc(M, cfg, inp), ref)
 
 
 def test_no_alloc_rejects_shapes_beyond_the_static_scratch(M):
