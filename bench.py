@@ -140,7 +140,7 @@ def source_sha(*rel):
     return h.hexdigest()[:16]
 
 
-GEMM_SOURCES = ("routed_experts_b200/csrc/ffn_tc.cu", "routed_experts_b200/csrc/ptx.cuh",
+GEMM_SOURCES = ("routed_experts_b200/csrc/ffn_tn.cu", "routed_experts_b200/csrc/ptx.cuh",
                 "routed_experts_b200/csrc/common.cuh", "routed_experts_b200/csrc/tc_common.cuh")
 
 
@@ -754,7 +754,7 @@ def run_mine(args, world, rank, local):
         "dtype": "bf16" if cfg.dtype == C.BF16 else "fp32",
         "data": "synthetic (seeded SplitMix64 + Box-Muller inputs, the recipe in routed_experts_b200/inputs.py)",
         "config": bench_config(cfg, args.seed, world),
-        "roofline": {"bound": "tensor", "kernel": "ffn_tc_kernel<FC1+SwiGLU>",
+        "roofline": {"bound": "tensor", "kernel": "ffn_tn_kernel<0> (FC1 + SwiGLU)",
                      "achieved": fc1_flop / fc1_s / 1e12, "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": fc1_flop / fc1_s / 1e12 / tensor_peak,
                      "traffic": ncu_traffic(f"fc1@{cfg.name}"),

@@ -172,9 +172,9 @@ moe_status moe_plan(const moe_config* cfg, const float* logits, int32_t* topk_id
 /*
  * moe_dispatch - step A6: xp[row] = x[src_of[row]] for every valid row
  * ([MegaFlux] §1: routed activations go to the ranks that compute their
- * experts). Padding rows of xp are not written: moe_expert_ffn and
- * moe_expert_fc1/fc2 store zero h and yp rows for them whatever xp holds
- * there, so their contents never reach the output.
+ * experts). Padding rows of xp are not written. Whatever they hold never
+ * reaches a valid row of h or yp, nor the output: every output element of
+ * the expert FFN depends on its own token row alone.
  *   x   [T, d] (device), xp [rows_cap, d] (device, out).
  */
 moe_status moe_dispatch(const moe_config* cfg, const void* x, void* xp, const void* ws,
@@ -189,10 +189,14 @@ moe_status moe_dispatch(const moe_config* cfg, const void* x, void* xp, const vo
  *              projection, rows F..2F-1 the up projection (K-major).
  *   w_down     [E, d, F] (device, K-major).
  *   h          [rows_cap, F] (device, out): silu(xp.gate) * (xp.up) on
- *              valid rows, zero on padding rows.
- *   yp         [rows_cap, d] (device, out): h . w_down on valid rows, zero
- *              on padding rows.
- * fp32 accumulation; in bf16 mode h and yp are rounded to bf16 once.
+ *              valid rows.
+ *   yp         [rows_cap, d] (device, out): h . w_down on valid rows.
+ * Rows of h and yp that no entry maps to (padding) hold unspecified values:
+ * bf16 layers leave them as they were, fp32 layers write zero. fp32
+ * accumulation; in bf16 mode h and yp are rounded to bf16 once.
+ * bf16 layers run on the tensor cores with the token rows as the MMA's N
+ * dimension, so each block costs its valid rows rounded up to 16 rather
+ * than a whole tile.
  */
 moe_status moe_expert_ffn(const moe_config* cfg, const void* xp, const void* w_gate_up,
                           const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
@@ -218,8 +222,9 @@ moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_do
  * readiness is a count in the workspace, raised with a release by each
  * epilogue warp after its stores and read with an acquire by the scheduler;
  * the wait is bounded and reports MOE_DEV_TIMEOUT. Same arguments, outputs
- * and rounding as moe_expert_ffn (one-block experts run on a CTA pair beside
- * an empty half here).
+ * on valid rows and rounding as moe_expert_ffn; padding rows of h and yp are
+ * written as zero. It computes whole 128-row tiles (one-block experts on a
+ * CTA pair beside an empty half).
  */
 moe_status moe_expert_ffn_fused(const moe_config* cfg, const void* xp, const void* w_gate_up, const void* w_down,
                                 void* h, void* yp, void* ws, size_t ws_bytes, moe_stream_t stream);
@@ -229,8 +234,9 @@ moe_status moe_expert_ffn_fused(const moe_config* cfg, const void* xp, const voi
  * moe_expert_ffn_fused with FC1's activation rows read straight from x
  * [T, d] (device) through the plan's row map (TMA four-row gathers; padding
  * rows repeat their block's first token and are stored as zero h and yp
- * rows), so xp is never written. Same h and yp bits as moe_dispatch followed
- * by moe_expert_ffn. Other dtypes return MOE_ERR_UNSUPPORTED.
+ * rows), so xp is never written. The same formula and rounding as
+ * moe_dispatch followed by moe_expert_ffn on valid rows. Other dtypes
+ * return MOE_ERR_UNSUPPORTED.
  */
 moe_status moe_expert_ffn_fused_gather(const moe_config* cfg, const void* x, const void* w_gate_up,
                                        const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
@@ -241,8 +247,9 @@ moe_status moe_expert_ffn_fused_gather(const moe_config* cfg, const void* x, con
  * FC1 + SwiGLU whose activation rows are gathered straight from x [T, d]
  * (device) through the plan's row map, so no xp buffer is written or read
  * ([MegaFlux] §2.1: token movement overlapped with the tiled FC1 work).
- * h [rows_cap, F] (device, out) holds the same values as moe_dispatch +
- * moe_expert_fc1 on every row (padding rows zero). It needs no xp buffer (rows_cap * d elements less memory)
+ * h [rows_cap, F] (device, out) holds what moe_dispatch + moe_expert_fc1
+ * give on valid rows (the same formula and rounding; padding rows are
+ * written as zero). It needs no xp buffer (rows_cap * d elements less memory)
  * but runs FC1 at about half the speed of moe_expert_fc1: each 16 KB
  * activation tile takes 32 four-row gathers instead of one tile copy.
  * fp32 layers return MOE_ERR_UNSUPPORTED.
@@ -464,6 +471,24 @@ moe_status moe_read_status(const void* ws, moe_stream_t stream, uint32_t* dev_bi
  * exercised without hanging or faulting a GPU.
  */
 moe_status moe_probe_bounded_wait(uint32_t* status_word, int64_t budget_cycles, moe_stream_t stream);
+
+/*
+ * moe_probe_expert_ffn_timeout - a check of the expert FFN's failure
+ * handling (bf16 layers; other dtypes return MOE_ERR_UNSUPPORTED):
+ * moe_expert_ffn with every device-side wait of its tensor-core kernels
+ * given budget_cycles clock cycles (1 .. 2^34) instead of about two seconds.
+ * With a budget shorter than a copy or an MMA takes, waits run out: the
+ * kernels OR MOE_DEV_TIMEOUT into the workspace's status word, stop both
+ * CTAs of each pair, let every copy and MMA in flight finish, free their
+ * tensor memory and return. h and yp are then undefined; the GEMM work
+ * queues in the workspace are left at zero, so the next call runs normally
+ * (moe_plan clears the status word). No papers' counterpart: it lets the
+ * timeout path of the real kernels run on a GPU without a kernel broken on
+ * purpose.
+ */
+moe_status moe_probe_expert_ffn_timeout(const moe_config* cfg, const void* xp, const void* w_gate_up,
+                                        const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
+                                        int64_t budget_cycles, moe_stream_t stream);
 
 /* A static string naming a moe_status. */
 const char* moe_status_string(moe_status s);

@@ -556,6 +556,26 @@ moe_status moe_probe_bounded_wait(uint32_t* status_word, int64_t budget_cycles, 
                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
+moe_status moe_probe_expert_ffn_timeout(const moe_config* cfg, const void* xp, const void* w_gate_up,
+                                        const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
+                                        int64_t budget_cycles, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (budget_cycles < 1 || budget_cycles > ((int64_t)1 << 34)) return MOE_ERR_INVALID_ARG;
+    if (!xp || !w_gate_up || !w_down || !h || !yp) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(xp) || !aligned16(w_gate_up) || !aligned16(w_down) || !aligned16(h) || !aligned16(yp))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    const WsPtrs P = ws_ptrs(ws, L);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_ffn_tn(s, 1, xp, w_gate_up, h, P, st, (long long)budget_cycles);
+    if (e == cudaSuccess) e = launch_ffn_tn(s, 2, h, w_down, yp, P, st, (long long)budget_cycles);
+    return from_cuda(e);
+}
+
 const char* moe_status_string(moe_status s) {
     switch (s) {
         case MOE_OK: return "MOE_OK";

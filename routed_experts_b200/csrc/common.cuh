@@ -143,6 +143,11 @@ cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void*
 cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                             const WsPtrs& ws, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st);
+// The grouped GEMM with the token rows as the MMA's N (which = 1: FC1 + SwiGLU,
+// 2: FC2; bf16): the MMA covers each block's valid rows rounded up to 16; rows
+// of h and yp past a block's valid ones are not written.
+cudaError_t launch_ffn_tn(const Shape& s, int which, const void* a_mat, const void* w, void* out,
+                          const WsPtrs& ws, cudaStream_t st, long long spin_budget);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact = nullptr);
 // FC1 then FC2 in one launch (bf16): h and yp as launch_ffn_tc's which = 1 and 2;

@@ -1,7 +1,12 @@
 // ffn_tc.cu - the grouped SwiGLU expert FFN on the 5th-generation tensor cores
-// (steps A7, A8 for bf16 layers): a persistent, warp-specialised tcgen05 GEMM
-// over the planned token blocks, run by CTA pairs, fed by TMA, accumulating
-// in TMEM.
+// (steps A7, A8 for bf16 layers) with the token rows as the MMA's M: a
+// persistent, warp-specialised tcgen05 GEMM over the planned token blocks, run
+// by CTA pairs, fed by TMA, accumulating in TMEM. It computes whole 128-row
+// blocks, and serves the launches that need that: FC1 gathering x through the
+// row map, the training forward (which keeps the pre-activations and zero
+// padding rows for the backward) and the fused FC1 -> FC2 launches. The
+// staged FC1 and FC2 of the layer run on ffn_tn.cu, which covers each
+// block's valid rows rounded up to 16 instead.
 //
 // [MegaFlux] "MegaFlux: Skew-Resilient MoE Megakernels via Pipelined Expert
 // Replication", §2.1 'Persistent MoE execution': persistent CTAs with
@@ -829,6 +834,8 @@ cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaSt
 
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact) {
+    // FC1 + SwiGLU (which = 1) and FC2 (which = 2) run on the token-N kernel (ffn_tn.cu)
+    if (which == 1 || which == 2) return launch_ffn_tn(s, which, a_mat, w, out, ws, st, spin_budget);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -868,28 +875,7 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
         a.b_rows = 2 * s.F;
         return launch_mode<3>(tA, tB, tO, tP, a, sms, st, ws.gemm_q + 8);
     }
-    if (which == 1) {
-        // FC1 + SwiGLU: xp [rows_cap, d] x w_gate_up [E*2F, d] -> h [rows_cap, F]
-        if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||
-            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
-            !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap))
-            return cudaErrorInvalidValue;
-        a.Kdim = s.d;
-        a.n_tiles = s.F / 128;
-        a.F = s.F;
-        a.b_rows = 2 * s.F;
-        return launch_mode<0>(tA, tB, tO, tO, a, sms, st, ws.gemm_q + 8);
-    }
-    // FC2: h [rows_cap, F] x w_down [E*d, F] -> yp [rows_cap, d]
-    if (!make_tmap(&tA, a_mat, (uint64_t)s.F, (uint64_t)s.rows_cap, kBM) ||
-        !make_tmap(&tB, w, (uint64_t)s.F, (uint64_t)s.E * s.d, kHalfN) ||
-        !make_tmap_out(&tO, out, (uint64_t)s.d, (uint64_t)s.rows_cap))
-        return cudaErrorInvalidValue;
-    a.Kdim = s.F;
-    a.n_tiles = s.d / 256;
-    a.F = 0;
-    a.b_rows = s.d;
-    return launch_mode<1>(tA, tB, tO, tO, a, sms, st, ws.gemm_q + 8);
+    return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_ffn_fused(const Shape& s, const void* a_src, const void* w_gate_up, const void* w_down, void* h,

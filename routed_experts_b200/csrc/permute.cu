@@ -20,9 +20,9 @@
 // experts. On one GPU that is a copy of token rows, done as a scatter: one
 // warp per token reads its row of x once (16-byte vectors) and stores it to
 // the K rows the row map names, so x is read from memory once even when it
-// does not fit in L2. Padding rows of xp are not written: the FFN writes
-// zero h and yp rows for them whatever xp holds there, and nothing reads
-// them after that.
+// does not fit in L2. Padding rows of xp are not written: each output
+// element of the expert FFN depends on its own token row alone, so nothing
+// they hold reaches a valid row of h or yp.
 #include "common.cuh"
 
 namespace moe {

@@ -590,21 +590,36 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
         ws.sched_off[tid] = eb_off;
         if (tid == E - 1) { ws.exp_piece_off[E] = ep_off + np_e; ws.sched_off[E] = eb_off + nb_e; }
         int pi = ep_off, bi = eb_off;
-        // the owner's prefix starts at 0; later slices were cut from the tail,
-        // so reverse creation order is ascending start order
+        // The expert's schedule lists its whole blocks first, then the partial
+        // last block of each piece, larger first (ties in start order), so the
+        // GEMM's consecutive block pairs hold blocks of about the same size.
+        // Pieces in start order: the owner's prefix starts at 0; later slices
+        // were cut from the tail, so reverse creation order is ascending start.
         if (own_pid[tid] >= 0) {
             const int pid = own_pid[tid];
             ws.exp_piece_idx[pi++] = pid;
-            const int nt = (rem[tid] + a.tile - 1) / a.tile;
-            for (int i = 0; i < nt; ++i) ws.sched[bi++] = pfb[pid] + i;
+            for (int i = 0; i < rem[tid] / a.tile; ++i) ws.sched[bi++] = pfb[pid] + i;
         }
         for (int i = nrep - 1; i >= 0; --i) {
             if (rep[5 * i + 1] != tid) continue;
             const int pid = rep[5 * i + 4];
             ws.exp_piece_idx[pi++] = pid;
-            const int nt = (rep[5 * i + 3] + a.tile - 1) / a.tile;
-            for (int j = 0; j < nt; ++j) ws.sched[bi++] = pfb[pid] + j;
+            for (int j = 0; j < rep[5 * i + 3] / a.tile; ++j) ws.sched[bi++] = pfb[pid] + j;
         }
+        const int part0 = bi;
+        auto add_partial = [&](int pid, int len) {
+            const int v = len % a.tile;
+            if (v == 0) return;
+            int k = bi++;
+            while (k > part0 && ws.blocks[(int64_t)kBlockInts * ws.sched[k - 1] + 2] < v) {
+                ws.sched[k] = ws.sched[k - 1];
+                --k;
+            }
+            ws.sched[k] = pfb[pid] + len / a.tile;
+        };
+        if (own_pid[tid] >= 0) add_partial(own_pid[tid], rem[tid]);
+        for (int i = nrep - 1; i >= 0; --i)
+            if (rep[5 * i + 1] == tid) add_partial(rep[5 * i + 4], rep[5 * i + 3]);
     }
     if (tid == 0) {
         ws.header[H_STATUS] = s_status;

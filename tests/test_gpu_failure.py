@@ -58,3 +58,46 @@ def test_probe_rejects_bad_budget():
         M.moe_probe_bounded_wait(status, -1)
     with pytest.raises(M.MoeError):
         M.moe_probe_bounded_wait(status, 1 << 40)
+
+
+# The real GEMM's abort path: moe_expert_ffn with every device-side wait of
+# its tensor-core kernels cut to a few clock cycles. Waits run out while
+# copies and MMAs are in flight; both CTAs of every pair must stop, drain what
+# they issued, free tensor memory and return, and the next calls on the same
+# workspace must give the right result (queues back at zero).
+MED = C.LayerConfig("abort_med", T=1024, d=512, E=16, K=4, F=384, R=4, tile=128, budget=2, zipf_s=1.2)
+
+
+@pytest.mark.parametrize("budget", [1, 300, 3000])
+def test_expert_ffn_timeout_path_returns_and_recovers(budget):
+    from routed_experts_b200 import inputs as I
+    from .gpu_helpers import run_path
+    inp = I.make_inputs(MED, 7, "cuda")
+    ref = run_path(MED, inp, "staged")
+    assert ref["status"] & M.DEV_TIMEOUT == 0
+    h = torch.zeros_like(ref["h"])
+    y = torch.zeros_like(ref["yp"])
+    t0 = time.perf_counter()
+    for _ in range(3):
+        M.moe_probe_expert_ffn_timeout(MED, ref["xp"], inp["w_gate_up"], inp["w_down"], h, y, ref["ws"], budget)
+    status = M.moe_read_status(ref["ws"])
+    assert time.perf_counter() - t0 < 60.0
+    if budget == 1:
+        assert status & M.DEV_TIMEOUT
+    # a new plan clears the status; the normal FFN on the same workspace is right again
+    M.moe_plan(MED, inp["logits"], ref["idx"], ref["w"], ref["counts"], ref["ws"])
+    M.moe_expert_ffn(MED, ref["xp"], inp["w_gate_up"], inp["w_down"], h, y, ref["ws"])
+    assert M.moe_read_status(ref["ws"]) & ~M.DEV_PLAN_INEXACT == 0
+    valid = torch.as_tensor((ref["plan"]["src_of"].numpy() >= 0).nonzero()[0], device="cuda")
+    assert torch.equal(h[valid], ref["h"][valid])
+    assert torch.equal(y[valid], ref["yp"][valid])
+
+
+def test_expert_ffn_timeout_probe_rejects_bad_arguments():
+    ws = M.alloc_workspace(SMALL)
+    x = torch.zeros(16, device="cuda", dtype=torch.bfloat16)
+    for budget in (0, 1 << 40):
+        with pytest.raises(M.MoeError):
+            M.moe_probe_expert_ffn_timeout(SMALL, x, x, x, x, x, ws, budget)
+    with pytest.raises(M.MoeError):
+        M.moe_probe_expert_ffn_timeout(C.TINY, x, x, x, x, x, ws, 100)
