@@ -59,16 +59,23 @@ namespace {
 
 using namespace tc;
 
-constexpr int kMxBK = 128;                                  // K elements (bytes) per k-step
+constexpr int kMxBK = 128;                                  // K elements (bytes) per slab
 constexpr int kMxHalf = 128;                                // accumulator columns of one half-item MMA (N)
 constexpr int kMxItemN = 2 * kMxHalf;                       // accumulator columns per item
 constexpr int kMxHalfRows = 64;                             // weight rows each CTA holds per half
-constexpr int kMxStages = 6;
-constexpr int kMxABytes = kBM * kMxBK;                      // 16 KB
-constexpr int kMxBBytes = 2 * kMxHalfRows * kMxBK;          // 16 KB: the two halves' weight rows
-constexpr int kMxStageBytes = kMxABytes + kMxBBytes;        // 32 KB
-constexpr int kMxSfBytes = 512;                             // 128 rows x 4 scales
-constexpr int kMxSfStage = 3 * kMxSfBytes;                  // A, B of half 0, B of half 1
+// A stage holds kMxSlabs 128-deep K slabs, each operand (and each scale
+// operand) brought by one TMA copy covering all of them: the operand feed
+// is paced by copies more than by bytes.
+constexpr int kMxSlabs = 2;
+constexpr int kMxStages = 6 / kMxSlabs;
+constexpr int kMxSlabA = kBM * kMxBK;                       // 16 KB: 128 activation rows of one slab
+constexpr int kMxSlabB = 2 * kMxHalfRows * kMxBK;           // 16 KB: the two halves' weight rows of one slab
+constexpr int kMxABytes = kMxSlabs * kMxSlabA;
+constexpr int kMxBBytes = kMxSlabs * kMxSlabB;
+constexpr int kMxStageBytes = kMxABytes + kMxBBytes;
+constexpr int kMxSfBytes = 512;                             // 128 rows x 4 scales of one slab
+constexpr int kMxSfOp = kMxSlabs * kMxSfBytes;              // one scale operand's chunks of a stage
+constexpr int kMxSfStage = 3 * kMxSfOp;                     // A, B of half 0, B of half 1
 constexpr int kMxBufs = 3;                                  // 128-column TMEM half-buffers
 constexpr uint32_t kMxTmemCols = 512;                       // allocation: a power of two >= 3*128 + 24
 constexpr uint32_t kMxSfCol = kMxBufs * kMxHalf;            // two sets of 12 scale columns from here
@@ -193,6 +200,7 @@ __device__ __forceinline__ void mx_epilogue_half(uint32_t t_half, int lane, int 
 template <int MODE, int WF>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+              const __grid_constant__ CUtensorMap tmB2,
               const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
               const __grid_constant__ CUtensorMap tmO, MxArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -241,6 +249,7 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     if (warp == 0 && lane == 0) {
         ptx::prefetch_tmap(&tmA);
         ptx::prefetch_tmap(&tmB);
+        ptx::prefetch_tmap(&tmB2);
         ptx::prefetch_tmap(&tmSA);
         ptx::prefetch_tmap(&tmSB);
         ptx::prefetch_tmap(&tmO);
@@ -253,7 +262,10 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
     ptx::tc_fence_after();
     const uint32_t tmem = S->tmem_base;
     const int n_items = p_off[a.E] * a.n_tiles;
-    const int kb_count = a.Kdim / kMxBK;
+    // stages per item: the last one holds a single slab when K / 128 is odd (its
+    // copies still bring two, the second beyond K or unused, and no MMA reads it)
+    const int n_slabs = a.Kdim / kMxBK;
+    const int kb_count = (n_slabs + kMxSlabs - 1) / kMxSlabs;
 
     auto slot_of = [](int k) { return k % kItemSlots; };
     auto parity_of = [](int k) { return (uint32_t)((k / kItemSlots) & 1); };
@@ -343,10 +355,11 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 const int wrow = e * a.b_rows + j * kMxItemN;        // the item's first weight row
                 // half-buffers 2k mod 3 and 2k+1 mod 3 are adjacent unless the first is the last:
                 // then one N = 256 MMA reads 128 contiguous rows per CTA (CTA c: rows 128c ..),
-                // else two N = 128 MMAs read 64 rows of each half per CTA (CTA c: rows 64c ..)
+                // brought by one 128-row copy; else two N = 128 MMAs read 64 rows of each half per
+                // CTA (CTA c: rows 64c ..), brought by two 64-row copies
                 const bool wide = (2 * k) % kMxBufs != kMxBufs - 1;
                 const int b_lo = wrow + (wide ? (even ? 0 : kMxHalf) : (even ? 0 : kMxHalfRows));
-                const int b_hi = b_lo + (wide ? kMxHalfRows : kMxHalf);
+                const int b_hi = b_lo + kMxHalf;
                 const int a_chunk0 = (row0 / 128) * kc;
                 const int b_chunk0 = (wrow / 128) * kc, b_chunk1 = (wrow / 128 + 1) * kc;
                 for (int kb = 0; kb < kb_count; ++kb) {
@@ -354,17 +367,22 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                     const uint32_t bar = ptx::map_to_rank(ptx::smem_addr(&S->full[stage]), 0);
                     uint8_t* st = base + stage * kMxStageBytes;
                     uint8_t* sf = sf_base + stage * kMxSfStage;
+                    const int ks0 = kb * kMxSlabs;   // the stage's first K slab
                     // E2M1 weights count their packed bytes (half a byte per element)
                     if (even)
                         ptx::mbar_arrive_expect_tx(&S->full[stage],
                                                    2 * (kMxABytes + (WF == MOE_MX_W_E2M1 ? kMxBBytes / 2 : kMxBBytes) +
                                                         kMxSfStage));
-                    ptx::tma_load_2d_pair(st, &tmA, kb * kMxBK, row0, bar);
-                    ptx::tma_load_2d_pair(st + kMxABytes, &tmB, kb * kMxBK, b_lo, bar);
-                    ptx::tma_load_2d_pair(st + kMxABytes + kMxBBytes / 2, &tmB, kb * kMxBK, b_hi, bar);
-                    ptx::tma_load_2d_pair(sf, &tmSA, 0, (a_chunk0 + kb) * 4, bar);
-                    ptx::tma_load_2d_pair(sf + kMxSfBytes, &tmSB, 0, (b_chunk0 + kb) * 4, bar);
-                    ptx::tma_load_2d_pair(sf + 2 * kMxSfBytes, &tmSB, 0, (b_chunk1 + kb) * 4, bar);
+                    ptx::tma_load_3d_pair(st, &tmA, 0, row0, ks0, bar);
+                    if (wide) {
+                        ptx::tma_load_3d_pair(st + kMxABytes, &tmB2, 0, b_lo, ks0, bar);
+                    } else {
+                        ptx::tma_load_3d_pair(st + kMxABytes, &tmB, 0, b_lo, ks0, bar);
+                        ptx::tma_load_3d_pair(st + kMxABytes + kMxBBytes / 2, &tmB, 0, b_hi, ks0, bar);
+                    }
+                    ptx::tma_load_2d_pair(sf, &tmSA, 0, (a_chunk0 + ks0) * 4, bar);
+                    ptx::tma_load_2d_pair(sf + kMxSfOp, &tmSB, 0, (b_chunk0 + ks0) * 4, bar);
+                    ptx::tma_load_2d_pair(sf + 2 * kMxSfOp, &tmSB, 0, (b_chunk1 + ks0) * 4, bar);
                     ++fills;
                     if (++stage == kMxStages) { stage = 0; phase ^= 1; }
                 }
@@ -401,36 +419,49 @@ ffn_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ C
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!role_wait(&S->full[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    const uint32_t a_addr = ptx::smem_addr(base + stage * kMxStageBytes);
-                    const uint32_t b_addr = a_addr + kMxABytes;
-                    const uint32_t sf_addr = ptx::smem_addr(sf_base + stage * kMxSfStage);
-                    const uint32_t sfa_t = tmem + kMxSfCol + 12u * sf_set;
-                    ptx::tmem_cp_sf_pair(sfa_t, ptx::sdesc_sf(sf_addr));
-                    ptx::tmem_cp_sf_pair(sfa_t + 4u, ptx::sdesc_sf(sf_addr + kMxSfBytes));
-                    ptx::tmem_cp_sf_pair(sfa_t + 8u, ptx::sdesc_sf(sf_addr + 2 * kMxSfBytes));
-                    if (wide) {
-                        // one N = 256 MMA per K slice over both half-buffers (d1 = d0 + 128); its
-                        // B scales are the 8 columns from sfa_t + 4 (rows 0-127, then 128-255)
+                    const uint32_t a_stage = ptx::smem_addr(base + stage * kMxStageBytes);
+                    const uint32_t b_stage = a_stage + kMxABytes;
+                    const uint32_t sf_stage = ptx::smem_addr(sf_base + stage * kMxSfStage);
 #pragma unroll
-                        for (uint32_t ks = 0; ks < kMxBK / 32; ++ks)
-                            ptx::mma_mx_pair(d0, ptx::sdesc_k_sw128(a_addr + ks * 32),
-                                             ptx::sdesc_k_sw128(b_addr + ks * 32),
-                                             ptx::idesc_mx_e4m3(2 * kBM, kMxItemN, ks, ks) | kBFormat, sfa_t | (ks << 30),
-                                             (sfa_t + 4u) | (ks << 30), (kb | (int)ks) != 0 ? 1u : 0u);
-                    } else {
+                    for (int sl = 0; sl < kMxSlabs; ++sl) {
+                        if (kb * kMxSlabs + sl >= n_slabs) break;
+                        // slab sl: activation rows at sl * 16 KB; weight rows: wide, 128 rows at
+                        // sl * 16 KB; else the low half's 64 rows at sl * 8 KB and the high half's at
+                        // kMxBBytes / 2 + sl * 8 KB; each scale operand's chunk at sl * 512 B
+                        const uint32_t a_addr = a_stage + sl * kMxSlabA;
+                        const uint32_t b_addr = wide ? b_stage + sl * kMxSlabB : b_stage + sl * (kMxSlabB / 2);
+                        const uint32_t b_hi_addr = b_stage + kMxBBytes / 2 + sl * (kMxSlabB / 2);
+                        const uint32_t sf_addr = sf_stage + sl * kMxSfBytes;
+                        const uint32_t sfa_t = tmem + kMxSfCol + 12u * sf_set;
+                        ptx::tmem_cp_sf_pair(sfa_t, ptx::sdesc_sf(sf_addr));
+                        ptx::tmem_cp_sf_pair(sfa_t + 4u, ptx::sdesc_sf(sf_addr + kMxSfOp));
+                        ptx::tmem_cp_sf_pair(sfa_t + 8u, ptx::sdesc_sf(sf_addr + 2 * kMxSfOp));
+                        const int kk = kb * kMxSlabs + sl;   // K slab index: the first one starts the accumulation
+                        if (wide) {
+                            // one N = 256 MMA per K slice over both half-buffers (d1 = d0 + 128); its
+                            // B scales are the 8 columns from sfa_t + 4 (rows 0-127, then 128-255)
 #pragma unroll
-                        for (uint32_t ks = 0; ks < kMxBK / 32; ++ks) {
-                            const uint32_t idesc = ptx::idesc_mx_e4m3(2 * kBM, kMxHalf, ks, ks) | kBFormat;
-                            const uint32_t acc = (kb | (int)ks) != 0 ? 1u : 0u;
-                            const uint64_t adesc = ptx::sdesc_k_sw128(a_addr + ks * 32);
-                            ptx::mma_mx_pair(d0, adesc, ptx::sdesc_k_sw128(b_addr + ks * 32), idesc,
-                                             sfa_t | (ks << 30), (sfa_t + 4u) | (ks << 30), acc);
-                            ptx::mma_mx_pair(d1, adesc, ptx::sdesc_k_sw128(b_addr + kMxBBytes / 2 + ks * 32), idesc,
-                                             sfa_t | (ks << 30), (sfa_t + 8u) | (ks << 30), acc);
+                            for (uint32_t ks = 0; ks < kMxBK / 32; ++ks)
+                                ptx::mma_mx_pair(d0, ptx::sdesc_k_sw128(a_addr + ks * 32),
+                                                 ptx::sdesc_k_sw128(b_addr + ks * 32),
+                                                 ptx::idesc_mx_e4m3(2 * kBM, kMxItemN, ks, ks) | kBFormat,
+                                                 sfa_t | (ks << 30), (sfa_t + 4u) | (ks << 30),
+                                                 (kk | (int)ks) != 0 ? 1u : 0u);
+                        } else {
+#pragma unroll
+                            for (uint32_t ks = 0; ks < kMxBK / 32; ++ks) {
+                                const uint32_t idesc = ptx::idesc_mx_e4m3(2 * kBM, kMxHalf, ks, ks) | kBFormat;
+                                const uint32_t acc = (kk | (int)ks) != 0 ? 1u : 0u;
+                                const uint64_t adesc = ptx::sdesc_k_sw128(a_addr + ks * 32);
+                                ptx::mma_mx_pair(d0, adesc, ptx::sdesc_k_sw128(b_addr + ks * 32), idesc,
+                                                 sfa_t | (ks << 30), (sfa_t + 4u) | (ks << 30), acc);
+                                ptx::mma_mx_pair(d1, adesc, ptx::sdesc_k_sw128(b_hi_addr + ks * 32), idesc,
+                                                 sfa_t | (ks << 30), (sfa_t + 8u) | (ks << 30), acc);
+                            }
                         }
+                        sf_set ^= 1u;
                     }
                     issued = true;
-                    sf_set ^= 1u;
                     const uint32_t empty_addr = ptx::smem_addr(&S->empty[stage]);
                     ptx::mma_commit_pair(empty_addr);
                     ptx::mma_commit_pair(ptx::map_to_rank(empty_addr, 1));
@@ -512,28 +543,45 @@ bool make_tmap_u8(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t row
     return r == CUDA_SUCCESS;
 }
 
-// Packed E2M1 codes [rows, inner elements] (inner / 2 bytes per row), loaded
-// as [box_rows, 128] elements unpacked to one byte each, 128-byte swizzle.
-bool make_tmap_e2m1(CUtensorMap* tm, const void* ptr, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+// An E4M3 code matrix [rows, K] as 3-D (128, row, K/128 slab), box (128,
+// box_rows, kMxSlabs): kMxSlabs 128-byte K slabs of box_rows rows, slab
+// after slab, 128-byte swizzle.
+bool make_tmap_slabs_u8(CUtensorMap* tm, const void* ptr, uint64_t K, uint64_t rows, uint32_t box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {inner, rows};
-    cuuint64_t strides[1] = {inner / 2};
-    cuuint32_t box[2] = {128, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+    cuuint64_t dims[3] = {(cuuint64_t)kMxBK, rows, K / kMxBK};
+    cuuint64_t strides[2] = {K, (cuuint64_t)kMxBK};
+    cuuint32_t box[3] = {(cuuint32_t)kMxBK, box_rows, (cuuint32_t)kMxSlabs};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// Packed E2M1 codes [rows, K elements] (K / 2 bytes per row) as 3-D (128,
+// row, K/128 slab), box (128, box_rows, kMxSlabs) elements, unpacked to one
+// byte each in shared memory, 128-byte swizzle.
+bool make_tmap_e2m1(CUtensorMap* tm, const void* ptr, uint64_t K, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kMxBK, rows, K / kMxBK};
+    cuuint64_t strides[2] = {K / 2, (cuuint64_t)kMxBK / 2};
+    cuuint32_t box[3] = {(cuuint32_t)kMxBK, box_rows, (cuuint32_t)kMxSlabs};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 template <int MODE, int WF>
-cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tSA, const CUtensorMap& tSB,
-                       const CUtensorMap& tO, const MxArgs& a, int grid, cudaStream_t st) {
+cudaError_t launch_one(const CUtensorMap& tA, const CUtensorMap& tB, const CUtensorMap& tB2, const CUtensorMap& tSA,
+                       const CUtensorMap& tSB, const CUtensorMap& tO, const MxArgs& a, int grid, cudaStream_t st) {
     cudaError_t err = cudaFuncSetAttribute(ffn_mx_kernel<MODE, WF>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)kMxSmemBytes);
     if (err != cudaSuccess) return err;
-    ffn_mx_kernel<MODE, WF><<<grid, kThreads, kMxSmemBytes, st>>>(tA, tB, tSA, tSB, tO, a);
+    ffn_mx_kernel<MODE, WF><<<grid, kThreads, kMxSmemBytes, st>>>(tA, tB, tB2, tSA, tSB, tO, a);
     return cudaGetLastError();
 }
 
@@ -566,21 +614,25 @@ cudaError_t launch_ffn_mx(const Shape& s, int which, const uint8_t* a_q, const u
     const uint64_t rows_b = (uint64_t)s.E * a.b_rows;
     const uint64_t chunks_a = (uint64_t)((s.rows_cap + 127) / 128) * (a.Kdim / 128);
     const uint64_t chunks_b = rows_b / 128 * (a.Kdim / 128);
-    CUtensorMap tA, tB, tSA, tSB, tO;
-    const bool b_ok = wfmt == MOE_MX_W_E2M1 ? make_tmap_e2m1(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxHalfRows)
-                                            : make_tmap_u8(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxBK, kMxHalfRows, true);
-    if (!make_tmap_u8(&tA, a_q, (uint64_t)a.Kdim, rows_a, kMxBK, kBM, true) || !b_ok ||
-        !make_tmap_u8(&tSA, a_sc, 128, chunks_a * 4, 128, 4, false) ||
-        !make_tmap_u8(&tSB, w_sc, 128, chunks_b * 4, 128, 4, false))
+    CUtensorMap tA, tB, tB2, tSA, tSB, tO;
+    const bool e2m1 = wfmt == MOE_MX_W_E2M1;
+    const bool b_ok = e2m1 ? make_tmap_e2m1(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxHalfRows) &&
+                                 make_tmap_e2m1(&tB2, w_q, (uint64_t)a.Kdim, rows_b, kMxHalf)
+                           : make_tmap_slabs_u8(&tB, w_q, (uint64_t)a.Kdim, rows_b, kMxHalfRows) &&
+                                 make_tmap_slabs_u8(&tB2, w_q, (uint64_t)a.Kdim, rows_b, kMxHalf);
+    // scales: a stage's kMxSlabs consecutive 512-byte chunks of each operand in one copy
+    if (!make_tmap_slabs_u8(&tA, a_q, (uint64_t)a.Kdim, rows_a, kBM) || !b_ok ||
+        !make_tmap_u8(&tSA, a_sc, 128, chunks_a * 4, 128, 4 * kMxSlabs, false) ||
+        !make_tmap_u8(&tSB, w_sc, 128, chunks_b * 4, 128, 4 * kMxSlabs, false))
         return cudaErrorInvalidValue;
     const bool out_ok = fc1 ? make_tmap_u8(&tO, out, (uint64_t)s.F, rows_a, 32, 32, false)
                             : make_tmap_out(&tO, out, (uint64_t)s.d, rows_a);
     if (!out_ok) return cudaErrorInvalidValue;
     if (wfmt == MOE_MX_W_E2M1)
-        return fc1 ? launch_one<0, MOE_MX_W_E2M1>(tA, tB, tSA, tSB, tO, a, sms, st)
-                   : launch_one<1, MOE_MX_W_E2M1>(tA, tB, tSA, tSB, tO, a, sms, st);
-    return fc1 ? launch_one<0, MOE_MX_W_E4M3>(tA, tB, tSA, tSB, tO, a, sms, st)
-               : launch_one<1, MOE_MX_W_E4M3>(tA, tB, tSA, tSB, tO, a, sms, st);
+        return fc1 ? launch_one<0, MOE_MX_W_E2M1>(tA, tB, tB2, tSA, tSB, tO, a, sms, st)
+                   : launch_one<1, MOE_MX_W_E2M1>(tA, tB, tB2, tSA, tSB, tO, a, sms, st);
+    return fc1 ? launch_one<0, MOE_MX_W_E4M3>(tA, tB, tB2, tSA, tSB, tO, a, sms, st)
+               : launch_one<1, MOE_MX_W_E4M3>(tA, tB, tB2, tSA, tSB, tO, a, sms, st);
 }
 
 }  // namespace moe
