@@ -70,6 +70,8 @@ struct PlanArgs {
     int max_rep;
     int plan_mode;
     int max_pairs;   // length of the fused FFN's readiness counters
+    int sort_off;    // byte offset in dynamic shared memory of the partial-block sort scratch
+    int packed;      // loads fit the greedy's packed (value, index) keys
 };
 
 // ---------------------------------------------------------------- warp helpers
@@ -227,12 +229,13 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
         for (int c = tid; c < a.n_chunks; c += kThreads) f |= ws.chunk_flags[c];
         if (f) atomicOr(&s_status, f);
     }
+    auto chunk_count = [&](int c, int e) -> int { return __ldg(ws.chunk_counts + (int64_t)c * E + e); };
     const int g = tid / E, e0 = tid % E;
     if (g < a.G) {
         const int c0 = (int)((int64_t)g * a.n_chunks / a.G), c1 = (int)((int64_t)(g + 1) * a.n_chunks / a.G);
         int s = 0;
 #pragma unroll 8
-        for (int c = c0; c < c1; ++c) s += __ldg(ws.chunk_counts + (int64_t)c * E + e0);
+        for (int c = c0; c < c1; ++c) s += chunk_count(c, e0);
         part[g * E + e0] = s;
     }
     __syncthreads();
@@ -255,7 +258,7 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
 #pragma unroll 8
         for (int c = c0; c < c1; ++c) {
             ws.chunk_base[(int64_t)c * E + e0] = run;
-            run += __ldg(ws.chunk_counts + (int64_t)c * E + e0);
+            run += chunk_count(c, e0);
         }
     }
     if (tid < R) {
@@ -273,9 +276,23 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
         int moves = 0, nrep = 0;
         uint32_t st = 0;
         for (;;) {
-            // hungriest rank: lowest load, lowest index on ties
+            // hungriest rank: lowest load, lowest index on ties; biggest donor: highest
+            // load, lowest index on ties. With loads below 2^23 both are one warp
+            // reduction of a packed key (load above the rank's 8 bits).
             int mv = INT_MAX, mr = INT_MAX;
             int xv = INT_MIN, xr = INT_MAX;
+            if (a.packed) {
+                uint32_t kmin = 0xffffffffu, kmax = 0u;
+                for (int r = lane; r < R; r += 32) {
+                    const uint32_t l = (uint32_t)L[r];
+                    kmin = min(kmin, (l << 8) | (uint32_t)r);
+                    kmax = max(kmax, (l << 8) | (uint32_t)(255 - r));
+                }
+                kmin = __reduce_min_sync(0xffffffffu, kmin);
+                kmax = __reduce_max_sync(0xffffffffu, kmax);
+                mv = (int)(kmin >> 8); mr = (int)(kmin & 255u);
+                xv = (int)(kmax >> 8); xr = 255 - (int)(kmax & 255u);
+            } else {
             for (int r = lane; r < R; r += 32) {
                 const int l = L[r];
                 if (l < mv) { mv = l; mr = r; }
@@ -290,6 +307,7 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
                 const int pr = __shfl_xor_sync(0xffffffffu, xr, off);
                 if (pv > xv || (pv == xv && pr < xr)) { xv = pv; xr = pr; }
             }
+            }
             const int recv = mr, donor = xr;
             if (mv >= C) break;
             if (moves == cap) { st |= MOE_DEV_PLAN_INEXACT; break; }
@@ -298,6 +316,17 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
             while (need > 0) {
                 // donor's biggest remaining expert, lowest id on ties
                 int bv = 0, be = INT_MAX;
+                if (a.packed) {
+                    // remaining entries above the expert's 10-bit position among the donor's
+                    uint32_t kb = 0u;
+                    for (int e = donor * a.per + lane; e < (donor + 1) * a.per; e += 32) {
+                        const int r_ = rem[e];
+                        if (r_ > 0) kb = max(kb, ((uint32_t)r_ << 10) | (uint32_t)(1023 - (e - donor * a.per)));
+                    }
+                    kb = __reduce_max_sync(0xffffffffu, kb);
+                    bv = (int)(kb >> 10);
+                    be = donor * a.per + 1023 - (int)(kb & 1023u);
+                } else {
                 for (int e = donor * a.per + lane; e < (donor + 1) * a.per; e += 32) {
                     const int r_ = rem[e];
                     if (r_ > bv) { bv = r_; be = e; }
@@ -307,6 +336,7 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
                     const int ov = __shfl_xor_sync(0xffffffffu, bv, off);
                     const int oe = __shfl_xor_sync(0xffffffffu, be, off);
                     if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+                }
                 }
                 if (bv <= 0) break;                       // donor holds nothing
                 if (used[recv] >= a.budget) break;        // no replica slot left
@@ -606,20 +636,24 @@ plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
             ws.exp_piece_idx[pi++] = pid;
             for (int j = 0; j < rep[5 * i + 3] / a.tile; ++j) ws.sched[bi++] = pfb[pid] + j;
         }
-        const int part0 = bi;
+        // partial last blocks: insertion-sorted by their valid rows (stable) in this
+        // expert's own stretch of shared scratch (one slot per piece of the expert)
+        int32_t* srt = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(sm) + a.sort_off) + ep_off;
+        int np_part = 0;
         auto add_partial = [&](int pid, int len) {
             const int v = len % a.tile;
             if (v == 0) return;
-            int k = bi++;
-            while (k > part0 && ws.blocks[(int64_t)kBlockInts * ws.sched[k - 1] + 2] < v) {
-                ws.sched[k] = ws.sched[k - 1];
+            int k = np_part++;
+            while (k > 0 && pq[4 * srt[k - 1] + 2] % a.tile < v) {
+                srt[k] = srt[k - 1];
                 --k;
             }
-            ws.sched[k] = pfb[pid] + len / a.tile;
+            srt[k] = pid;
         };
         if (own_pid[tid] >= 0) add_partial(own_pid[tid], rem[tid]);
         for (int i = nrep - 1; i >= 0; --i)
             if (rep[5 * i + 1] == tid) add_partial(rep[5 * i + 4], rep[5 * i + 3]);
+        for (int k = 0; k < np_part; ++k) ws.sched[bi++] = pfb[srt[k]] + pq[4 * srt[k] + 2] / a.tile;
     }
     if (tid == 0) {
         ws.header[H_STATUS] = s_status;
@@ -654,6 +688,12 @@ cudaError_t launch_plan(const Shape& s, int32_t* counts_out, const WsPtrs& ws, c
     if (s.plan_mode == MOE_PLAN_BLOCKS)
         smem += sizeof(int32_t) * ((size_t)s.E + 12 * s.R + 4 * s.per + 4 + 2 * a.max_rep) +
                 (((size_t)4 * s.E + 15) & ~(size_t)15) + sizeof(int16_t) * 4 * (size_t)s.E * s.R;
+    smem = (smem + 15) & ~(size_t)15;
+    a.sort_off = (int)smem;                                   // one int per piece
+    smem += sizeof(int32_t) * ((size_t)s.E + a.max_rep);
+    smem = (smem + 15) & ~(size_t)15;
+    // packed greedy keys: a rank's load and an expert's count stay below 2^22
+    a.packed = s.N < ((int64_t)1 << 22) && s.R <= 256 && s.per <= 1024 ? 1 : 0;
     cudaError_t err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
