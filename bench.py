@@ -4,7 +4,9 @@
 
 One step = one pass of the whole layer (top-k and gating, histogram, planner,
 row maps, dispatch, FC1 + SwiGLU, FC2, combine) over one batch of seeded
-synthetic inputs already resident in HBM, through the C ABI. Under torchrun
+synthetic inputs already resident in HBM: one moe_layer_fwd call through the
+C ABI. The stages are timed in a second pass, one ABI call per stage, and
+FC2 with the combine folded in (moe_expert_fc2_combine) in a third. Under torchrun
 every rank runs its own independent layer (its own tokens, replicated
 weights, no collective on the data path: weak scaling); the timed region is
 bracketed by a barrier and a device synchronisation, and the time is the
@@ -36,7 +38,7 @@ from routed_experts_b200 import configs as C  # noqa: E402
 from routed_experts_b200 import inputs as I  # noqa: E402
 
 METRIC = "routed MoE layer tokens/s at 1 B200; % of bf16 tensor / HBM roofline"
-LAUNCHES_PER_STEP = 7   # topk_hist, plan, row_maps, gather, fc1, fc2, combine
+LAUNCHES_PER_STEP = 7   # moe_layer_fwd: topk_hist, plan, row_maps, gather, fc1, fc2, combine
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -570,56 +572,74 @@ def run_mine(args, world, rank, local):
     idx = torch.empty(T, K, dtype=torch.int32, device=dev)
     w = torch.empty(T, K, dtype=torch.float32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
-    ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
+    ws = M.alloc_workspace(cfg, M.WS_LAYER, dev)
     cap = M.moe_rows_capacity(cfg)
     xp = torch.empty(cap, d, dtype=dt, device=dev)
     h = torch.empty(cap, F, dtype=dt, device=dev)
     yp = torch.empty(cap, d, dtype=dt, device=dev)
     out = torch.empty(T, d, dtype=dt, device=dev)
     lg, x, wgu, wdn = inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"]
+    fold = cfg.dtype == C.BF16
 
-    n_ev = 6
-    def step(evs=None):
-        # the kernels moe_layer_fwd runs, one ABI call per stage so each stage can be timed
-        if evs is not None: evs[0].record(stream)
-        M.moe_plan(cfg, lg, idx, w, counts, ws, stream)
-        if evs is not None: evs[1].record(stream)
-        M.moe_dispatch(cfg, x, xp, ws, stream)
-        if evs is not None: evs[2].record(stream)
-        M.moe_expert_fc1(cfg, xp, wgu, h, ws, stream)
-        if evs is not None: evs[3].record(stream)
-        M.moe_expert_fc2(cfg, h, wdn, yp, ws, stream)
-        if evs is not None: evs[4].record(stream)
-        M.moe_combine(cfg, yp, w, out, ws, stream)
-        if evs is not None: evs[5].record(stream)
-
+    # the timed step: the whole layer, one moe_layer_fwd call
+    layer = M.Layer(cfg, dev)
     for _ in range(args.warmup):
-        step()
-    st = M.moe_read_status(ws, stream)
+        layer.forward(lg, x, wgu, wdn, stream=stream)
+    st = layer.status(stream)
     if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
         raise RuntimeError(f"device status {st} after warm-up")
-    plan = M.read_plan(cfg, ws)
-
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    step_evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     if pg is not None:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
     with ClockSampler(dev) as clk:
-        t0.record(stream)
         for k in range(args.steps):
-            step(evs[k])
-        t1.record(stream)
+            step_evs[k].record(stream)
+            layer.forward(lg, x, wgu, wdn, stream=stream)
+        step_evs[args.steps].record(stream)
         torch.cuda.synchronize(dev)
     if pg is not None:
         torch.distributed.barrier()
-    elapsed_ms = t0.elapsed_time(t1)
-    stage_ms = np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n_ev - 1)] for e in evs])
-    step_ms = np.array([e[0].elapsed_time(e[n_ev - 1]) for e in evs])   # each step, launch to last stage
-    st = M.moe_read_status(ws, stream)
+    elapsed_ms = step_evs[0].elapsed_time(step_evs[args.steps])
+    step_ms = np.array([step_evs[k].elapsed_time(step_evs[k + 1]) for k in range(args.steps)])
+    st = layer.status(stream)
     if st & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
         raise RuntimeError(f"device status {st} after the timed steps")
+    del layer
+
+    # the same kernels, one ABI call per stage, so that each stage can be timed
+    def stages(evs, fold_fc2=False):
+        evs[0].record(stream)
+        M.moe_plan(cfg, lg, idx, w, counts, ws, stream)
+        evs[1].record(stream)
+        M.moe_dispatch(cfg, x, xp, ws, stream)
+        evs[2].record(stream)
+        M.moe_expert_fc1(cfg, xp, wgu, h, ws, stream)
+        evs[3].record(stream)
+        if fold_fc2:
+            M.moe_expert_fc2_combine(cfg, h, wdn, w, yp, out, ws, stream)
+            evs[4].record(stream)
+            return
+        M.moe_expert_fc2(cfg, h, wdn, yp, ws, stream)
+        evs[4].record(stream)
+        M.moe_combine(cfg, yp, w, out, ws, stream)
+        evs[5].record(stream)
+
+    def time_stages(fold_fc2):
+        n = 5 if fold_fc2 else 6
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps + args.warmup)]
+        torch.cuda.synchronize(dev)
+        for e in evs:
+            stages(e, fold_fc2)
+        torch.cuda.synchronize(dev)
+        st_ = M.moe_read_status(ws, stream)
+        if st_ & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
+            raise RuntimeError(f"device status {st_} after the stage pass")
+        return np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n - 1)] for e in evs[args.warmup:]])
+
+    fold_ms = time_stages(True) if fold else None
+    stage_ms = time_stages(False)
+    plan = M.read_plan(cfg, ws)
 
     # the fused FFN (FC1 and FC2 in one launch) on the same plan and xp, K passes; then the
     # same with FC1 gathering x through the row map (dispatch, FC1 and FC2 in one launch)
@@ -765,6 +785,10 @@ def run_mine(args, world, rank, local):
                            "peaks": {"bf16_tflops": tensor_peak, "hbm_gbs": pk["hbm_gbs"], "kind": pk_kind}},
         "stages_ms": {"plan(topk+hist+plan+rowmaps)": med[0], "dispatch": med[1], "fc1": med[2], "fc2": med[3],
                       "combine": med[4]},
+        "fc2_combine_fold_ms": None if fold_ms is None else {
+            "median": float(np.median(fold_ms[:, 3])), "separate_fc2_plus_combine": float(med[3] + med[4]),
+            "note": "moe_expert_fc2_combine (FC2 with the top-k sum in its epilogue, bit-identical; its call "
+                    "clears the arrival counters first) against moe_expert_fc2 + moe_combine"},
         "step_ms": {"median": float(np.median(step_ms)), "min": float(step_ms.min()),
                     "max": float(step_ms.max())},
         "stage_rates": {"fc1_tflops": fc1_flop / fc1_s / 1e12, "fc2_tflops": fc2_flop / fc2_s / 1e12,
@@ -782,7 +806,7 @@ def run_mine(args, world, rank, local):
                 "one_stream_value": world * T / (e2e_serial_ms / args.steps * 1e-3),
                 "one_stream_ms_per_step": e2e_serial_ms / args.steps},
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "layer_path": "moe_plan; moe_dispatch; moe_expert_fc1; moe_expert_fc2; moe_combine (the kernels of moe_layer_fwd)",
+        "layer_path": "moe_layer_fwd: top-k + histogram, plan, row maps, dispatch, FC1 + SwiGLU, FC2, combine",
         "backward": bwd,
         "mx": mx,
         "mx_fp4_weights": mx4,

@@ -268,8 +268,31 @@ moe_status moe_combine(const moe_config* cfg, const void* yp, const float* topk_
                        const void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * moe_expert_fc2_combine - steps A8 and A9 in one launch (bf16 layers):
+ * moe_expert_fc2 with the weighted top-k sum folded into its epilogue
+ * ([MegaFlux] §2.1 "Fixed-placement MegaMoE forward": a token's output is
+ * formed as soon as its expert rows are done; §1: the outputs are combined
+ * by the routing weights). yp [rows_cap, d] (device, out) is written as by
+ * moe_expert_fc2, and out [T, d] (device, out) is bit-identical to
+ * moe_combine(yp, topk_w): the same fixed k order, fp32 sum and one
+ * rounding. Each (token, 32 columns) has an arrival counter; the epilogue
+ * whose rows complete a token's K rows of those columns sums them.
+ *   h [rows_cap, F], w_down [E, d, F], topk_w fp32 [T, K] (device).
+ *   ws  a MOE_WS_LAYER workspace holding the plan of moe_plan (the counters
+ *       live in its layer part; the call clears them first).
+ * Returns MOE_ERR_UNSUPPORTED for fp32 layers, MOE_ERR_WORKSPACE when
+ * ws_bytes is below moe_workspace_size(MOE_WS_LAYER).
+ * It is slower than moe_expert_fc2 followed by moe_combine on one GPU: FC2
+ * walks the experts in order, so most tokens complete in its last items and
+ * their sums fall on the epilogue warps there. moe_layer_fwd does not use it.
+ */
+moe_status moe_expert_fc2_combine(const moe_config* cfg, const void* h, const void* w_down, const float* topk_w,
+                                  void* yp, void* out, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
  * moe_layer_fwd - the whole layer, A1 to A9, on device buffers, with
- * top-k, xp, h and yp carved from a MOE_WS_LAYER workspace.
+ * top-k, xp, h and yp carved from a MOE_WS_LAYER workspace: the kernels of
+ * moe_plan, moe_dispatch, moe_expert_fc1, moe_expert_fc2 and moe_combine.
  */
 moe_status moe_layer_fwd(const moe_config* cfg, const float* logits, const void* x,
                          const void* w_gate_up, const void* w_down, void* out, void* ws,

@@ -72,6 +72,7 @@ WsLayout make_layout(const Shape& s) {
     L.idx = take(sizeof(int32_t) * s.N);
     L.w = take(sizeof(float) * s.N);
     L.counts = take(sizeof(int32_t) * s.E);
+    L.arrivals = take(sizeof(int32_t) * (int64_t)s.T * (s.d / 32));
     L.xp = take((int64_t)s.eb * s.rows_cap * s.d);
     L.h = take((int64_t)s.eb * s.rows_cap * s.F);
     L.yp = take((int64_t)s.eb * s.rows_cap * s.d);
@@ -302,6 +303,25 @@ moe_status moe_expert_fc2(const moe_config* cfg, const void* h, const void* w_do
     const WsLayout L = make_layout(s);
     if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
     return fc_impl(s, L, 2, h, w_down, yp, ws, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_expert_fc2_combine(const moe_config* cfg, const void* h, const void* w_down, const float* topk_w,
+                                  void* yp, void* out, void* ws, size_t ws_bytes, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (!h || !w_down || !topk_w || !yp || !out) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(h) || !aligned16(w_down) || !aligned16(topk_w) || !aligned16(yp) || !aligned16(out))
+        return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.layer_end)) != MOE_OK) return r;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t* arrivals = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + L.arrivals);
+    if (cudaMemsetAsync(arrivals, 0, sizeof(int32_t) * (size_t)s.T * (s.d / 32), st) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    const FoldArgs fold{topk_w, out, arrivals};
+    return from_cuda(launch_ffn_tn(s, 2, h, w_down, yp, ws_ptrs(ws, L), st, kSpinBudget, &fold));
 }
 
 moe_status moe_combine(const moe_config* cfg, const void* yp, const float* topk_w, void* out, const void* ws,

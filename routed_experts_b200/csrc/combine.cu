@@ -20,6 +20,8 @@ template <bool BF16, int KMAX>
 __global__ void __launch_bounds__(kCWarps * 32)
 combine_kernel(const uint4* __restrict__ yp, const float* __restrict__ w, uint4* __restrict__ out,
                int T, int K, int nvec, int64_t rows_cap, WsPtrs ws) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t bad = 0;
     for (int t = blockIdx.x * kCWarps + warp; t < T; t += gridDim.x * kCWarps) {
@@ -92,14 +94,15 @@ cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void*
     const int grid = (int)(want < cap ? want : cap);
     const uint4* y4 = static_cast<const uint4*>(yp);
     uint4* o4 = static_cast<uint4*>(out);
-#define MOE_COMBINE(B, KM) combine_kernel<B, KM><<<grid, kCWarps * 32, 0, st>>>(y4, w, o4, s.T, s.K, nvec, s.rows_cap, ws)
+#define MOE_COMBINE(B, KM) \
+    return launch_pdl(combine_kernel<B, KM>, dim3(grid), dim3(kCWarps * 32), 0, st, y4, w, o4, s.T, s.K, nvec, \
+                      s.rows_cap, ws)
     const bool bf = s.dtype == MOE_BF16;
     if (s.K <= 2) { if (bf) MOE_COMBINE(true, 2); else MOE_COMBINE(false, 2); }
     else if (s.K <= 4) { if (bf) MOE_COMBINE(true, 4); else MOE_COMBINE(false, 4); }
     else if (s.K <= 8) { if (bf) MOE_COMBINE(true, 8); else MOE_COMBINE(false, 8); }
     else { if (bf) MOE_COMBINE(true, 16); else MOE_COMBINE(false, 16); }
 #undef MOE_COMBINE
-    return cudaGetLastError();
 }
 
 }  // namespace moe

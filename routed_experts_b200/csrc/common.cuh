@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "moe.h"
 
 namespace moe {
@@ -45,7 +47,7 @@ struct WsLayout {
         blocks, sched_off, sched, rank_load, rank_replicas, rank_row0, row_of, src_of, gemm_q, pair_ready;
     int64_t plan_end;
     // MOE_WS_LAYER extras
-    int64_t idx, w, counts, xp, h, yp;
+    int64_t idx, w, counts, arrivals, xp, h, yp;
     int64_t layer_end;
     // MOE_WS_LAYER_HOST extras
     int64_t logits_dev, x_dev, out_dev;
@@ -119,6 +121,32 @@ __device__ inline void set_status(uint32_t* header, uint32_t bits) {
     atomicOr(header + H_STATUS, bits);
 }
 
+// Programmatic dependent launch along the layer's chain of kernels. A kernel
+// launched by launch_pdl may have its CTAs placed while the kernel before it
+// in the stream is still running; it calls pdl_wait() first, which returns
+// once that kernel has completed with its memory visible, and then
+// pdl_trigger(), which lets the next kernel of the stream be placed. A kernel
+// passes pdl_trigger() only after its own pdl_wait(), so when a kernel starts,
+// every kernel two or more places before it has completed.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = grid;
+    lc.blockDim = block;
+    lc.dynamicSmemBytes = smem;
+    lc.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+    return cudaLaunchKernelEx(&lc, kernel, std::forward<Args>(args)...);
+}
+
 // ---- shape and workspace layout, defined in api.cu ----
 bool aligned16(const void* p);
 // Validates cfg and fills the derived shape: INVALID_ARG for an ill-formed
@@ -143,11 +171,20 @@ cudaError_t launch_combine(const Shape& s, const void* yp, const float* w, void*
 cudaError_t launch_ffn_simt(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                             const WsPtrs& ws, cudaStream_t st);
 cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaStream_t st);
+// The combine folded into FC2: the top-k weights [T, K], the layer output
+// y [T, d] and one arrival counter per (token, 32 columns of y), [T, d/32],
+// all zero before the launch (the launch leaves them zero when it completes).
+struct FoldArgs {
+    const float* topk_w;
+    void* y;
+    int32_t* arrivals;
+};
 // The grouped GEMM with the token rows as the MMA's N (which = 1: FC1 + SwiGLU,
-// 2: FC2; bf16): the MMA covers each block's valid rows rounded up to 16; rows
-// of h and yp past a block's valid ones are not written.
+// 2: FC2, with fold also the combine; bf16): the MMA covers each block's valid
+// rows rounded up to 16; rows of h and yp past a block's valid ones are not written.
 cudaError_t launch_ffn_tn(const Shape& s, int which, const void* a_mat, const void* w, void* out,
-                          const WsPtrs& ws, cudaStream_t st, long long spin_budget);
+                          const WsPtrs& ws, cudaStream_t st, long long spin_budget,
+                          const FoldArgs* fold = nullptr);
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact = nullptr);
 // FC1 then FC2 in one launch (bf16): h and yp as launch_ffn_tc's which = 1 and 2;

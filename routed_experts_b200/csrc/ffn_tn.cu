@@ -133,6 +133,15 @@ struct TnArgs {
     uint32_t* header;
     int32_t* queue;               // [3]: head of queue 0, head of queue 1, clusters finished
     __nv_bfloat16* out;
+    // FC2 with the combine folded in (MODE 2)
+    int K;                        // experts per token
+    int T;
+    int64_t rows_cap;
+    const float* topk_w;          // [T, K]
+    const int32_t* row_of;        // [T*K] token entry -> row of yp
+    const int32_t* src_of;        // [rows_cap] row of yp -> token
+    int32_t* arrivals;            // [T, d/32] rows of the token stored, per 32-column chunk (zero between launches)
+    __nv_bfloat16* y;             // [T, d] the layer's output
 };
 
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
@@ -242,11 +251,113 @@ __device__ __forceinline__ void tn_chunk(uint32_t t_acc, int c0, int lane, float
     __syncwarp();   // the staging tile is free for the next chunk
 }
 
-// MODE 0: FC1 + SwiGLU (B = xp, out = h); MODE 1: FC2 (B = h, out = yp).
+// The combine folded into FC2 (MODE 2), after one epilogue warp has stored
+// its 32 yp columns (chunk col / 32) of every valid token row of an item:
+// each of those rows counts itself on its token's arrival counter of the
+// chunk, and the warp whose count completes a token's K rows forms
+// y[t, col .. col + 31] = sum over k = 0..K-1, in that order, of
+// w[t,k] * yp[row_of(t,k), col ..] in fp32 (fmaf from 0, one rounding to
+// bf16: the arithmetic of combine.cu, so the result is bit-identical), then
+// clears the counter for the next launch. The warp's stores, a warp barrier
+// and a GPU-scope fence come before its counts (the release side); a warp
+// that completes tokens fences once after its counts and reads the rows
+// through L2 (ld.global.cg: another SM stored them during this launch).
+// Eight completed tokens at a time, four lanes per token, 16 bytes (8
+// columns) per lane.
+__device__ __forceinline__ void tn_fold_combine(const TnArgs& a, int lane, int col, int r0, int r1, int n, int v0,
+                                                int v1) {
+    __syncwarp();
+    __threadfence();
+    const int n_chunks = a.d >> 5, chunk = col >> 5;
+    const int rows = 2 * n;   // token columns of the item: block 0 then block 1 (or one block's 2n rows)
+    int tok[8], old[8];
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        tok[i] = -1;
+        old[i] = -1;
+        const int s_ = 32 * i + lane;
+        if (s_ < rows) {
+            const bool in0 = s_ < n || r1 < 0;
+            const int r = in0 ? s_ : s_ - n;
+            if (r < (in0 ? v0 : v1)) {
+                const int t = __ldg(a.src_of + (int64_t)(in0 ? r0 : r1) + r);
+                if (t >= 0 && t < a.T) tok[i] = t; else bad = true;
+            }
+        }
+        if (tok[i] >= 0) old[i] = atomicAdd(a.arrivals + (int64_t)tok[i] * n_chunks + chunk, 1);
+    }
+    const int g = lane >> 2, q = lane & 3;
+    if (__any_sync(0xffffffffu, (old[0] == a.K - 1) | (old[1] == a.K - 1) | (old[2] == a.K - 1) |
+                                    (old[3] == a.K - 1) | (old[4] == a.K - 1) | (old[5] == a.K - 1) |
+                                    (old[6] == a.K - 1) | (old[7] == a.K - 1))) {
+        __threadfence();
+        __syncwarp();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        unsigned m = __ballot_sync(0xffffffffu, old[i] == a.K - 1);
+        while (m) {
+            // the g-th completed token of this group of (up to) 8 goes to lanes 4g .. 4g+3
+            unsigned mm = m;
+            for (int x = 0; x < g && mm; ++x) mm &= mm - 1;
+            const int src = mm ? __ffs(mm) - 1 : 0;
+            const int t = __shfl_sync(0xffffffffu, tok[i], src);
+            for (int x = 0; x < 8 && m; ++x) m &= m - 1;
+            if (!mm) continue;
+            if (q == 0) a.arrivals[(int64_t)t * n_chunks + chunk] = 0;
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+            for (int k0 = 0; k0 < a.K; k0 += 8) {
+                uint4 v[8];
+                float wk[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    wk[u] = 0.f;
+                    v[u] = make_uint4(0u, 0u, 0u, 0u);
+                    if (k0 + u < a.K) {
+                        const int64_t e = (int64_t)t * a.K + k0 + u;
+                        const int row = __ldg(a.row_of + e);
+                        if (row >= 0 && row < a.rows_cap) {
+                            wk[u] = __ldg(a.topk_w + e);
+                            v[u] = __ldcg(reinterpret_cast<const uint4*>(a.out + (int64_t)row * a.d + col + 8 * q));
+                        } else {
+                            bad = true;
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (k0 + u >= a.K) break;
+                    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v[u]);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float2 f = __bfloat1622float2(p[j]);
+                        acc[2 * j] = fmaf(wk[u], f.x, acc[2 * j]);
+                        acc[2 * j + 1] = fmaf(wk[u], f.y, acc[2 * j + 1]);
+                    }
+                }
+            }
+            uint4 o;
+            __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) po[j] = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+            *reinterpret_cast<uint4*>(a.y + (int64_t)t * a.d + col + 8 * q) = o;
+        }
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.header, MOE_DEV_BAD_INDEX);
+}
+
+// MODE 0: FC1 + SwiGLU (B = xp, out = h); MODE 1: FC2 (B = h, out = yp);
+// MODE 2: FC2 with the combine folded in (also y).
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
     constexpr bool kFC1 = MODE == 0;
+    constexpr bool kFold = MODE == 2;
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* epi_base = reinterpret_cast<float*>(base + kTnStages * kTnStageBytes);
@@ -559,6 +670,8 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
                 if (even) ptx::mbar_arrive(&S->acc_empty[acc]);
                 else ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->acc_empty[acc]), 0));
             }
+            // the accumulator is free: the next item's MMAs overlap the combine
+            if (kFold) tn_fold_combine(a, lane, col, item.z, item.w, n, v0, v1);
         }
     }
     ptx::tc_fence_before();
@@ -608,9 +721,10 @@ bool make_tmap_slabs(CUtensorMap* tm, const void* p, uint64_t K, uint64_t rows, 
 }  // namespace
 
 // which = 1: FC1 + SwiGLU, xp [rows_cap, d] x w_gate_up -> h [rows_cap, F];
-// which = 2: FC2, h [rows_cap, F] x w_down -> yp [rows_cap, d].
+// which = 2: FC2, h [rows_cap, F] x w_down -> yp [rows_cap, d], and with
+// fold also the weighted top-k sum of the yp rows into fold->y [T, d].
 cudaError_t launch_ffn_tn(const Shape& s, int which, const void* a_mat, const void* w, void* out,
-                          const WsPtrs& ws, cudaStream_t st, long long spin_budget) {
+                          const WsPtrs& ws, cudaStream_t st, long long spin_budget, const FoldArgs* fold) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -644,17 +758,29 @@ cudaError_t launch_ffn_tn(const Shape& s, int which, const void* a_mat, const vo
     a.header = ws.header;
     a.queue = ws.gemm_q + (fc1 ? 0 : 4);
     a.out = static_cast<__nv_bfloat16*>(out);
+    a.K = s.K;
+    a.T = s.T;
+    a.rows_cap = s.rows_cap;
+    a.row_of = ws.row_of;
+    a.src_of = ws.src_of;
+    a.topk_w = fold ? fold->topk_w : nullptr;
+    a.arrivals = fold ? fold->arrivals : nullptr;
+    a.y = fold ? static_cast<__nv_bfloat16*>(fold->y) : nullptr;
+    if (fold && (fc1 || !fold->topk_w || !fold->arrivals || !fold->y)) return cudaErrorInvalidValue;
     cudaError_t err;
     if (fc1) {
         err = cudaFuncSetAttribute(ffn_tn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTnSmemBytes);
         if (err != cudaSuccess) return err;
-        ffn_tn_kernel<0><<<sms, kThreads, kTnSmemBytes, st>>>(maps, a);
-    } else {
+        return launch_pdl(ffn_tn_kernel<0>, dim3(sms), dim3(kThreads), kTnSmemBytes, st, maps, a);
+    } else if (!fold) {
         err = cudaFuncSetAttribute(ffn_tn_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTnSmemBytes);
         if (err != cudaSuccess) return err;
-        ffn_tn_kernel<1><<<sms, kThreads, kTnSmemBytes, st>>>(maps, a);
+        return launch_pdl(ffn_tn_kernel<1>, dim3(sms), dim3(kThreads), kTnSmemBytes, st, maps, a);
+    } else {
+        err = cudaFuncSetAttribute(ffn_tn_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTnSmemBytes);
+        if (err != cudaSuccess) return err;
+        return launch_pdl(ffn_tn_kernel<2>, dim3(sms), dim3(kThreads), kTnSmemBytes, st, maps, a);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace moe

@@ -32,6 +32,8 @@ constexpr int kRmWarps = 4;
 
 __global__ void __launch_bounds__(kRmWarps * 32)
 row_maps_kernel(const int32_t* __restrict__ idx, int T, int K, int E, int n_chunks, int max_pieces, WsPtrs ws) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ int32_t sm_rm[];
     int32_t* s_poff = sm_rm;                       // [E+1] first piece of each expert (start order)
     int4* s_piece = reinterpret_cast<int4*>(s_poff + ((E + 1 + 3) & ~3));   // [n_pieces]: start, len, row0
@@ -99,6 +101,8 @@ constexpr int kUnroll = 8;
 __global__ void __launch_bounds__(kGWarps * 32)
 dispatch_kernel(const uint4* __restrict__ x, uint4* __restrict__ xp, int T, int K, int nvec, int64_t rows_cap,
                 WsPtrs ws) {
+    pdl_wait();
+    pdl_trigger();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint32_t bad = 0;
     for (int t = blockIdx.x * kGWarps + warp; t < T; t += gridDim.x * kGWarps) {
@@ -139,8 +143,8 @@ cudaError_t launch_row_maps(const Shape& s, const int32_t* idx, const WsPtrs& ws
         cudaError_t err = cudaFuncSetAttribute(row_maps_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (err != cudaSuccess) return err;
     }
-    row_maps_kernel<<<grid, kRmWarps * 32, smem, st>>>(idx, s.T, s.K, s.E, s.n_chunks, (int)s.max_pieces, ws);
-    return cudaGetLastError();
+    return launch_pdl(row_maps_kernel, dim3(grid), dim3(kRmWarps * 32), smem, st, idx, s.T, s.K, s.E, s.n_chunks,
+                      (int)s.max_pieces, ws);
 }
 
 cudaError_t launch_gather(const Shape& s, const void* x, void* xp, const WsPtrs& ws,
@@ -153,9 +157,8 @@ cudaError_t launch_gather(const Shape& s, const void* x, void* xp, const WsPtrs&
     int64_t cap = (int64_t)sms * 8;
     const int grid = (int)(want < cap ? want : cap);
     if (grid == 0) return cudaSuccess;
-    dispatch_kernel<<<grid, kGWarps * 32, 0, st>>>(static_cast<const uint4*>(x), static_cast<uint4*>(xp), s.T,
-                                                  s.K, nvec, s.rows_cap, ws);
-    return cudaGetLastError();
+    return launch_pdl(dispatch_kernel, dim3(grid), dim3(kGWarps * 32), 0, st, static_cast<const uint4*>(x),
+                      static_cast<uint4*>(xp), s.T, s.K, nvec, s.rows_cap, ws);
 }
 
 }  // namespace moe

@@ -194,6 +194,8 @@ __device__ void block_candidate(int prio, int fan, const int32_t* b, int E, int 
 
 __global__ void __launch_bounds__(kThreads, 1)
 plan_kernel(PlanArgs a, int32_t* __restrict__ counts_out, WsPtrs ws) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ int32_t sm[];
     const int E = a.E, R = a.R;
     int32_t* part = sm;                              // [G*E]
@@ -697,8 +699,7 @@ cudaError_t launch_plan(const Shape& s, int32_t* counts_out, const WsPtrs& ws, c
     cudaError_t err = cudaFuncSetAttribute(plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            (int)smem);
     if (err != cudaSuccess) return err;
-    plan_kernel<<<1, kThreads, smem, st>>>(a, counts_out, ws);
-    return cudaGetLastError();
+    return launch_pdl(plan_kernel, dim3(1), dim3(kThreads), smem, st, a, counts_out, ws);
 }
 
 }  // namespace moe

@@ -9,7 +9,9 @@
 //
 // One warp per token (a CTA per 32-token chunk). Lane l holds logits of experts l, l+32, l+64, ...
 // (coalesced 128-byte rows). K rounds of a warp arg-max pick the experts in
-// descending logit order, ties to the lower expert id. Gating: softmax over
+// descending logit order, ties to the lower expert id: each round is two
+// warp reductions (redux.sync), the largest order-preserving key of the
+// lanes' best logits, then the lowest expert among the lanes that hold it. Gating: softmax over
 // the chosen logits (equal to the full softmax renormalised over them), or
 // their sigmoids normalised over them. Every CTA covers kTokPerChunk tokens
 // and counts its chunk's entries per expert in shared memory; the planner
@@ -28,11 +30,24 @@ __device__ __forceinline__ bool better(float va, int ea, float vb, int eb) {
     return va > vb || (va == vb && ea < eb);
 }
 
+// An unsigned key in the order of the float (finite or -inf, -0 already
+// folded into +0, so equal values have equal keys), and back.
+__device__ __forceinline__ uint32_t order_key(float x) {
+    const uint32_t b = __float_as_uint(x);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Two CTAs per SM where the logits of a lane fit in few registers.
 template <int EPT>
-__global__ void __launch_bounds__(kWarps * 32, 1)
+__global__ void __launch_bounds__(kWarps * 32, EPT <= 4 ? 2 : 1)
 topk_hist_kernel(const float* __restrict__ logits, int32_t* __restrict__ idx,
                  float* __restrict__ wout, int T, int E, int K, int gating,
                  int32_t* __restrict__ chunk_counts, uint32_t* __restrict__ chunk_flags) {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ int32_t hist[];   // [E]
     __shared__ uint32_t flag;
     const int lane = threadIdx.x & 31;
@@ -54,14 +69,14 @@ topk_hist_kernel(const float* __restrict__ logits, int32_t* __restrict__ idx,
             float x = e < E ? __ldg(row + e) : -INFINITY;
             if (e < E && !isfinite(x)) bad = 1;
             if (x != x) x = -INFINITY;
+            if (x == 0.f) x = 0.f;   // -0 and +0 compare equal: one key for both
             v[j] = x;
         }
+        // lane k < K owns entry k
         uint32_t taken = 0;
-        float sel_v[kMaxK];
-        int sel_e[kMaxK];
-#pragma unroll
-        for (int k = 0; k < kMaxK; ++k) {
-            if (k >= K) break;
+        float my_v = 0.f, top = 0.f;
+        int my_e = 0;
+        for (int k = 0; k < K; ++k) {
             float bv = -INFINITY;
             int be = 0x7fffffff;
 #pragma unroll
@@ -69,25 +84,17 @@ topk_hist_kernel(const float* __restrict__ logits, int32_t* __restrict__ idx,
                 const int e = j * 32 + lane;
                 if (!(taken >> j & 1u) && e < E && better(v[j], e, bv, be)) { bv = v[j]; be = e; }
             }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-                const int oe = __shfl_xor_sync(0xffffffffu, be, off);
-                if (better(ov, oe, bv, be)) { bv = ov; be = oe; }
-            }
+            const uint32_t key = order_key(bv);
+            const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+            be = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)be : 0xffffffffu);
+            bv = key_value(kmax);
             if ((be & 31) == lane) taken |= 1u << (be >> 5);
-            sel_v[k] = bv;
-            sel_e[k] = be;
+            if (k == 0) top = bv;
+            if (k == lane) { my_v = bv; my_e = be; }
         }
-        // lane k < K owns entry k
-        float my_v = 0.f;
-        int my_e = 0;
-#pragma unroll
-        for (int k = 0; k < kMaxK; ++k)
-            if (k == lane) { my_v = sel_v[k]; my_e = sel_e[k]; }
         float g = 0.f;
         if (lane < K) {
-            g = gating == MOE_GATE_SOFTMAX_TOPK ? expf(my_v - sel_v[0]) : 1.f / (1.f + expf(-my_v));
+            g = gating == MOE_GATE_SOFTMAX_TOPK ? expf(my_v - top) : 1.f / (1.f + expf(-my_v));
         }
         float sum = g;
 #pragma unroll
@@ -109,9 +116,8 @@ template <int EPT>
 cudaError_t launch_ept(const Shape& s, const float* logits, int32_t* idx, float* w,
                        const WsPtrs& ws, cudaStream_t st) {
     const size_t smem = sizeof(int32_t) * s.E;
-    topk_hist_kernel<EPT><<<s.n_chunks, kWarps * 32, smem, st>>>(
-        logits, idx, w, s.T, s.E, s.K, s.gating, ws.chunk_counts, ws.chunk_flags);
-    return cudaGetLastError();
+    return launch_pdl(topk_hist_kernel<EPT>, dim3(s.n_chunks), dim3(kWarps * 32), smem, st, logits, idx, w, s.T,
+                      s.E, s.K, s.gating, ws.chunk_counts, ws.chunk_flags);
 }
 
 }  // namespace

@@ -65,6 +65,7 @@ def lib() -> ctypes.CDLL:
         L.moe_expert_fc2.argtypes = [C, P, P, P, P, S, P]
         L.moe_expert_fc1_gather.argtypes = [C, P, P, P, P, S, P]
         L.moe_combine.argtypes = [C, P, P, P, P, S, P]
+        L.moe_expert_fc2_combine.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_bwd.argtypes = [C, P, P, P, P, P, P, P, P, P, S, P]
@@ -84,6 +85,7 @@ def lib() -> ctypes.CDLL:
         L.moe_status_string.restype = ctypes.c_char_p
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_ffn_fused", "moe_expert_ffn_fused_gather", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
+                  "moe_expert_fc2_combine",
                   "moe_layer_fwd", "moe_layer_bwd", "moe_layer_fwd_train",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait",
                   "moe_probe_expert_ffn_timeout",
@@ -196,6 +198,13 @@ def moe_expert_fc2(c, h, w_down, yp, ws, stream=None):
     p, n = _ws(ws)
     _check(lib().moe_expert_fc2(ctypes.byref(config(c)), _ptr(h), _ptr(w_down), _ptr(yp), p, n, _stream(stream)),
            "moe_expert_fc2")
+
+
+def moe_expert_fc2_combine(c, h, w_down, topk_w, yp, out, ws, stream=None):
+    """FC2 with the weighted top-k sum folded in: yp as moe_expert_fc2, out as moe_combine."""
+    p, n = _ws(ws)
+    _check(lib().moe_expert_fc2_combine(ctypes.byref(config(c)), _ptr(h), _ptr(w_down), _ptr(topk_w), _ptr(yp),
+                                        _ptr(out), p, n, _stream(stream)), "moe_expert_fc2_combine")
 
 
 def moe_combine(c, yp, topk_w, out, ws, stream=None):

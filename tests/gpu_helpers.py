@@ -49,7 +49,7 @@ def sentinel_like(shape, cfg, device) -> torch.Tensor:
     return torch.full(shape, SENTINEL[C.FP32], dtype=torch.int32, device=device).view(torch.float32)
 
 
-PATHS = ("staged", "fused", "fused_gather", "fc1_gather", "layer")
+PATHS = ("staged", "fused", "fused_gather", "fc1_gather", "fc2_combine", "layer")
 
 
 def run_path(cfg, inp: dict, path: str = "staged") -> dict:
@@ -59,6 +59,9 @@ def run_path(cfg, inp: dict, path: str = "staged") -> dict:
       fused         moe_dispatch, moe_expert_ffn_fused (FC1 and FC2 in one launch)
       fused_gather  moe_expert_ffn_fused_gather (dispatch, FC1 and FC2 in one launch)
       fc1_gather    moe_expert_fc1_gather (dispatch and FC1 in one launch), moe_expert_fc2
+      fc2_combine   moe_dispatch, moe_expert_fc1, moe_expert_fc2_combine (FC2 and the combine
+                    in one launch; no moe_combine), on a MOE_WS_LAYER workspace whose layer
+                    part starts as 0xff bytes, so its arrival counters must be cleared
       layer         moe_layer_fwd alone (h and yp stay inside its workspace)."""
     dev = inp["x"].device
     T, K, E, d, F = cfg.T, cfg.K, cfg.E, cfg.d, cfg.F
@@ -73,13 +76,17 @@ def run_path(cfg, inp: dict, path: str = "staged") -> dict:
     idx = torch.empty(T, K, dtype=torch.int32, device=dev)
     w = torch.empty(T, K, dtype=torch.float32, device=dev)
     counts = torch.empty(E, dtype=torch.int32, device=dev)
-    ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
+    if path == "fc2_combine":
+        ws = M.alloc_workspace(cfg, M.WS_LAYER, dev)
+        ws[M.moe_workspace_size(cfg, M.WS_PLAN):].fill_(255)
+    else:
+        ws = M.alloc_workspace(cfg, M.WS_PLAN, dev)
     h = sentinel_like((cap, F), cfg, dev)
     yp = sentinel_like((cap, d), cfg, dev)
     out = torch.empty(T, d, dtype=dt, device=dev)
     M.moe_plan(cfg, inp["logits"], idx, w, counts, ws)
     xp = None
-    if path in ("staged", "fused"):
+    if path in ("staged", "fused", "fc2_combine"):
         # dispatch leaves padding rows of xp alone: NaN there must not reach h, yp or out
         xp = torch.full((cap, d), float("nan"), dtype=dt, device=dev)
         M.moe_dispatch(cfg, inp["x"], xp, ws)
@@ -92,9 +99,13 @@ def run_path(cfg, inp: dict, path: str = "staged") -> dict:
     elif path == "fc1_gather":
         M.moe_expert_fc1_gather(cfg, inp["x"], inp["w_gate_up"], h, ws)
         M.moe_expert_fc2(cfg, h, inp["w_down"], yp, ws)
+    elif path == "fc2_combine":
+        M.moe_expert_fc1(cfg, xp, inp["w_gate_up"], h, ws)
+        M.moe_expert_fc2_combine(cfg, h, inp["w_down"], w, yp, out, ws)
     else:
         raise ValueError(path)
-    M.moe_combine(cfg, yp, w, out, ws)
+    if path != "fc2_combine":
+        M.moe_combine(cfg, yp, w, out, ws)
     status = M.moe_read_status(ws)
     plan = M.read_plan(cfg, ws)
     return {"idx": idx, "w": w, "counts": counts, "xp": xp, "h": h, "yp": yp, "out": out,

@@ -197,7 +197,7 @@ def test_qwen3_skew_sweep(cfg):
     torch.cuda.empty_cache()
 
 
-FUSED_PATHS = ["fused", "fused_gather", "fc1_gather", "layer"]
+FUSED_PATHS = ["fused", "fused_gather", "fc1_gather", "fc2_combine", "layer"]
 
 
 @pytest.mark.parametrize("path", FUSED_PATHS)
@@ -209,16 +209,77 @@ def test_full_size_other_paths(cfg, path):
     torch.cuda.empty_cache()
 
 
-@pytest.mark.parametrize("path", ["staged", "fused", "fused_gather", "fc1_gather"])
+@pytest.mark.parametrize("path", ["staged", "fused", "fused_gather", "fc1_gather", "fc2_combine"])
 def test_every_element_of_a_layer_whose_clusters_take_several_items(path):
     check_full_small(RING_BF16, 0, path=path, threads=True)
     torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, WIDE_BF16], ids=lambda c: c.name)
-@pytest.mark.parametrize("path", ["fused", "fused_gather", "fc1_gather"])
+@pytest.mark.parametrize("path", ["fused", "fused_gather", "fc1_gather", "fc2_combine"])
 def test_small_layers_other_paths(cfg, path):
     check_full_small(cfg, 3, path=path)
+
+
+# The combine folded into FC2: one row per token (K = 1), K = 16 (two
+# batches of eight rows in the summing lanes), one token per rank.
+FOLD_EDGE = [SMALL_BF16.replace(name="k1", K=1), EDGE[5], EDGE[3], EDGE[0]]
+
+
+@pytest.mark.parametrize("cfg", FOLD_EDGE, ids=lambda c: c.name)
+def test_fc2_combine_edge_shapes(cfg):
+    check_full_small(cfg, 2, path="fc2_combine")
+
+
+@pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, WIDE_BF16, RING_BF16, C.OLMOE, C.DSV3],
+                         ids=lambda c: c.name)
+def test_fc2_combine_is_bit_identical_to_fc2_then_combine(cfg):
+    """FC2 with the combine folded in stores the same yp bits as moe_expert_fc2
+    and the same out bits as moe_combine (the same fixed k order, fp32 sum
+    and rounding), and a second call on the same workspace gives them again."""
+    inp = I.make_inputs(cfg, 6, "cuda")
+    a = run_path(cfg, inp, "staged")
+    b = run_path(cfg, inp, "fc2_combine")
+    assert b["status"] & ~M.DEV_PLAN_INEXACT == 0
+    valid = torch.as_tensor(np.nonzero(a["plan"]["src_of"].numpy() >= 0)[0], device="cuda")
+    assert torch.equal(b["yp"][valid], a["yp"][valid])
+    assert torch.equal(b["out"], a["out"])
+    out2 = torch.full_like(b["out"], float("nan"))
+    M.moe_expert_fc2_combine(cfg, b["h"], inp["w_down"], b["w"], b["yp"], out2, b["ws"])
+    assert M.moe_read_status(b["ws"]) & ~M.DEV_PLAN_INEXACT == 0
+    assert torch.equal(out2, a["out"])
+    del a, b, inp
+    torch.cuda.empty_cache()
+
+
+def test_fc2_combine_needs_a_layer_workspace_and_bf16():
+    cfg = SMALL_BF16
+    ws = M.alloc_workspace(cfg, M.WS_PLAN)
+    z = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    w = torch.zeros(16, dtype=torch.float32, device="cuda")
+    with pytest.raises(M.MoeError) as e:
+        M.moe_expert_fc2_combine(cfg, z, z, w, z, z, ws)
+    assert e.value.code == M.MOE_ERR_WORKSPACE
+    with pytest.raises(M.MoeError) as e:
+        M.moe_expert_fc2_combine(C.TINY, z, z, w, z, z, M.alloc_workspace(C.TINY, M.WS_LAYER))
+    assert e.value.code == M.MOE_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("cfg", [MED_BF16, C.OLMOE], ids=lambda c: c.name)
+def test_layer_clears_what_an_earlier_call_left(cfg):
+    """moe_layer_fwd on a workspace whose layer part holds garbage (as after a
+    call that stopped at a timeout) gives the bits of the staged launches:
+    every word it reads there is written earlier in the same call."""
+    inp = I.make_inputs(cfg, 7, "cuda")
+    staged = run_stages(cfg, inp)["out"]
+    layer = M.Layer(cfg)
+    for fill in (255, 1):
+        layer.ws[M.moe_workspace_size(cfg, M.WS_PLAN):].fill_(fill)
+        out = layer.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"])
+        assert layer.status() & ~M.DEV_PLAN_INEXACT == 0
+        assert torch.equal(out, staged), fill
+    del layer, inp
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, C.OLMOE], ids=lambda c: c.name)
