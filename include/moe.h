@@ -243,15 +243,15 @@ moe_status moe_expert_ffn_fused_gather(const moe_config* cfg, const void* x, con
                                        moe_stream_t stream);
 
 /*
- * moe_expert_fc1_gather - steps A6 and A7 in one pass (bf16 layers only):
- * FC1 + SwiGLU whose activation rows are gathered straight from x [T, d]
+ * moe_expert_fc1_gather - steps A6 and A7 in one launch (bf16 layers only):
+ * FC1 + SwiGLU whose activation rows are read straight from x [T, d]
  * (device) through the plan's row map, so no xp buffer is written or read
  * ([MegaFlux] §2.1: token movement overlapped with the tiled FC1 work).
- * h [rows_cap, F] (device, out) holds what moe_dispatch + moe_expert_fc1
- * give on valid rows (the same formula and rounding; padding rows are
- * written as zero). It needs no xp buffer (rows_cap * d elements less memory)
- * but runs FC1 at about half the speed of moe_expert_fc1: each 16 KB
- * activation tile takes 32 four-row gathers instead of one tile copy.
+ * h [rows_cap, F] (device, out) holds, on valid rows, the bits
+ * moe_dispatch + moe_expert_fc1 give; padding rows of h are not written.
+ * It needs no xp buffer (rows_cap * d elements less memory) but is slower
+ * than the two launches: its rows arrive by 16-byte copies from scattered
+ * token rows instead of one tensor copy of consecutive rows.
  * fp32 layers return MOE_ERR_UNSUPPORTED.
  */
 moe_status moe_expert_fc1_gather(const moe_config* cfg, const void* x, const void* w_gate_up, void* h, void* ws,

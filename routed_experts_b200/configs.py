@@ -70,7 +70,11 @@ EXTREME = LayerConfig("extreme", T=32768, d=4096, E=64, K=4, F=1536, R=8, tile=1
 DSV3 = LayerConfig("dsv3", T=8192, d=7168, E=256, K=8, F=2048, R=32, tile=128, budget=4,
                    gating=GATE_SIGMOID_TOPK, logits="normal", zipf_s=1.2)
 
-NAMED = {c.name: c for c in (TINY, OLMOE, QWEN3, EXTREME, DSV3)}
+# A reduced DeepSeek-V3-like shape for profiler captures of the GEMM: the
+# full shape's d and F with about 256 rows per expert and 2.8 GB of weights.
+DSV3_SMALL = DSV3.replace(name="dsv3_small", T=1024, E=32, R=4, budget=4)
+
+NAMED = {c.name: c for c in (TINY, OLMOE, QWEN3, EXTREME, DSV3, DSV3_SMALL)}
 
 # The Qwen3-shaped skew sweep.
 QWEN3_SWEEP = tuple(QWEN3.replace(name=f"qwen3_s{s}", zipf_s=s) for s in (0.0, 0.5, 1.0, 1.5))

@@ -2,11 +2,11 @@
 // (steps A7, A8 for bf16 layers) with the token rows as the MMA's M: a
 // persistent, warp-specialised tcgen05 GEMM over the planned token blocks, run
 // by CTA pairs, fed by TMA, accumulating in TMEM. It computes whole 128-row
-// blocks, and serves the launches that need that: FC1 gathering x through the
-// row map, the training forward (which keeps the pre-activations and zero
-// padding rows for the backward) and the fused FC1 -> FC2 launches. The
-// staged FC1 and FC2 of the layer run on ffn_tn.cu, which covers each
-// block's valid rows rounded up to 16 instead.
+// blocks, and serves the launches that need that: the training forward (which
+// keeps the pre-activations and zero padding rows for the backward) and the
+// fused FC1 -> FC2 launches. The layer's FC1 (also the one gathering x) and
+// FC2 run on ffn_tn.cu, which covers each block's valid rows rounded up to 16
+// instead.
 //
 // [MegaFlux] "MegaFlux: Skew-Resilient MoE Megakernels via Pipelined Expert
 // Replication", §2.1 'Persistent MoE execution': persistent CTAs with
@@ -30,10 +30,11 @@
 // block past its valid ones (padding) are stored as zero, whatever the
 // activation rows held there.
 //
-// FC1 can also read its activation rows straight from x (dispatch fused into
-// FC1): each 128-row A tile is built by 32 four-row TMA gathers
-// (tile::gather4, one per lane of the TMA warp) of the token rows the plan's
-// row map names; padding rows repeat the block's first token.
+// The fused launch with the dispatch folded in (mode 5) reads FC1's
+// activation rows straight from x: each 128-row A tile is built by 32
+// four-row TMA gathers (tile::gather4, one per lane of the TMA warp) of the
+// token rows the plan's row map names; padding rows repeat the block's first
+// token.
 //
 // Scheduling is dynamic. Items are listed expert-major (then column tile,
 // then block pair), so consecutive items share an expert's weight tiles and a
@@ -835,7 +836,7 @@ cudaError_t launch_bounded_wait_probe(uint32_t* status, long long budget, cudaSt
 cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget, void* preact) {
     // FC1 + SwiGLU (which = 1) and FC2 (which = 2) run on the token-N kernel (ffn_tn.cu)
-    if (which == 1 || which == 2) return launch_ffn_tn(s, which, a_mat, w, out, ws, st, spin_budget);
+    if (which == 1 || which == 2 || which == 3) return launch_ffn_tn(s, which, a_mat, w, out, ws, st, spin_budget);
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -850,18 +851,6 @@ cudaError_t launch_ffn_tc(const Shape& s, int which, const void* a_mat, const vo
     a.queue = ws.gemm_q + (which == 2 ? 4 : 0);
     a.src_of = ws.src_of;
     CUtensorMap tA, tB, tO, tP;
-    if (which == 3) {
-        // FC1 + SwiGLU with A gathered from x [T, d] by the row map -> h [rows_cap, F]
-        if (!make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.T, 1) ||
-            !make_tmap(&tB, w, (uint64_t)s.d, (uint64_t)s.E * 2 * s.F, kHalfN) ||
-            !make_tmap_out(&tO, out, (uint64_t)s.F, (uint64_t)s.rows_cap))
-            return cudaErrorInvalidValue;
-        a.Kdim = s.d;
-        a.n_tiles = s.F / 128;
-        a.F = s.F;
-        a.b_rows = 2 * s.F;
-        return launch_mode<2>(tA, tB, tO, tO, a, sms, st, nullptr);
-    }
     if (which == 4) {
         // FC1 + SwiGLU -> h [rows_cap, F], and the pre-activations -> preact [rows_cap, 2F]
         if (!preact || !make_tmap(&tA, a_mat, (uint64_t)s.d, (uint64_t)s.rows_cap, kBM) ||

@@ -67,6 +67,17 @@
 // is bounded; a wait that runs out sets MOE_DEV_TIMEOUT, raises the CTA's
 // abort flag, lets its in-flight copies and MMAs finish and returns; both
 // CTAs then meet at the cluster barrier and free TMEM.
+//
+// MODE 3 is FC1 + SwiGLU with the token rows read straight from x [T, d]
+// through the row map, so no dispatched copy xp is written or read: four
+// more warps per CTA copy each k-step's rows (16-byte cp.async into the
+// 128-byte-swizzled layout the TMA box would have produced) and arrive on the
+// stage's local gather barrier as their copies land (cp.async.mbarrier
+// arrive); a fifth warp waits on it, fences the async proxy and signals the
+// stage's row barrier on the even CTA, which the MMA thread waits on beside
+// the weights' TMA barrier. The copying warps never wait for their own
+// copies, so all stages of the ring can be in flight, as with TMA. Padding
+// rows are not copied: their accumulator columns are never stored.
 #include <cudaTypedefs.h>
 #include <string.h>
 
@@ -102,6 +113,12 @@ struct TnSmem {
     // count of fills, then arrives on odd_done; peer_bytes holds the odd
     // CTA's bytes the even CTA expected for its own latest fill of each stage.
     uint64_t odd_done;
+    uint64_t bfull[kTnStages];    // MODE 3 (even CTA): both CTAs' gathered rows of the stage have landed
+    uint64_t gfull[kTnStages];    // MODE 3: this CTA's gathered rows of the stage have landed
+    int4 g_item;                  // MODE 3: the item the gather warps work on (x = -2: stop)
+    uint32_t g_valid;
+    int g_ok;
+    int32_t g_tok[128];           // MODE 3: token of each of this CTA's rows of the item (-1: padding)
     uint32_t odd_bytes[kTnStages], peer_bytes[kTnStages];
     long long odd_fills;
     uint32_t tmem_base;
@@ -142,7 +159,14 @@ struct TnArgs {
     const int32_t* src_of;        // [rows_cap] row of yp -> token
     int32_t* arrivals;            // [T, d/32] rows of the token stored, per 32-column chunk (zero between launches)
     __nv_bfloat16* y;             // [T, d] the layer's output
+    const __nv_bfloat16* x;       // MODE 3: the token rows [T, d]
 };
+
+constexpr int kGatherWarp = 7;    // MODE 3: warps 7 .. 10 gather the token rows
+constexpr int kGatherThreads = 128;
+constexpr int kSignalWarp = 11;   // MODE 3: turns landed gathers into row-barrier arrivals
+constexpr int kGatherExtra = kGatherThreads + 32;
+static_assert(kTnSlabs == 2, "the row gather splits a 16-byte chunk index as (row, slab, chunk) = (i/16, i/8%2, i%8)");
 
 __device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
 
@@ -350,12 +374,14 @@ __device__ __forceinline__ void tn_fold_combine(const TnArgs& a, int lane, int c
 }
 
 // MODE 0: FC1 + SwiGLU (B = xp, out = h); MODE 1: FC2 (B = h, out = yp);
-// MODE 2: FC2 with the combine folded in (also y).
+// MODE 2: FC2 with the combine folded in (also y); MODE 3: FC1 + SwiGLU with
+// B gathered from x.
 template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(MODE == 3 ? kThreads + kGatherExtra : kThreads, 1)
 ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
-    constexpr bool kFC1 = MODE == 0;
+    constexpr bool kFC1 = MODE == 0 || MODE == 3;
     constexpr bool kFold = MODE == 2;
+    constexpr bool kGather = MODE == 3;
     pdl_wait();
     pdl_trigger();
     extern __shared__ uint8_t smem_raw[];
@@ -374,15 +400,20 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
         for (int q = 0; q < 2; ++q) { ptx::mbar_init(&S->acc_full[q], 1); ptx::mbar_init(&S->acc_empty[q], 8); }
         for (int q = 0; q < kItemSlots; ++q) {
             ptx::mbar_init(&S->item_full[q], 1);
-            ptx::mbar_init(&S->item_empty[q], kItemConsumers);
-            ptx::mbar_init(&S->fwd_empty[q], kOddConsumers);
+            // + the gather leader and the signal thread
+            ptx::mbar_init(&S->item_empty[q], kItemConsumers + (kGather ? 2 : 0));
+            ptx::mbar_init(&S->fwd_empty[q], kOddConsumers + (kGather ? 2 : 0));
+        }
+        for (int s_ = 0; s_ < kTnStages; ++s_) {
+            ptx::mbar_init(&S->bfull[s_], 2);                 // one arrival per CTA
+            ptx::mbar_init(&S->gfull[s_], kGatherThreads);    // one per gather thread
         }
         ptx::mbar_init(&S->drain, 1);
         ptx::mbar_init(&S->odd_done, 1);
         S->abort_flag = 0;
         ptx::fence_barrier_init();
     }
-    for (int i = threadIdx.x; i <= a.E; i += kThreads) s_off[i] = a.sched_off[i];
+    for (int i = threadIdx.x; i <= a.E; i += blockDim.x) s_off[i] = a.sched_off[i];
     __syncthreads();
     if (warp == 0) {
         // pair offsets: p_off[e] = sum over e' < e of ceil(blocks of e' / 2)
@@ -519,7 +550,7 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
                 // this CTA's token rows: block 0's first n, then block 1's (or the single block's next n)
                 const int brow = rank == 0 ? item.z : (item.w >= 0 ? item.w : item.z + n);
                 const CUtensorMap* bmap = &maps.b[(n >> 4) - 1];
-                const uint32_t cta_bytes = (uint32_t)(kTnBytesA + kTnSlabs * n * kBK * 2);
+                const uint32_t cta_bytes = (uint32_t)(kTnBytesA + (kGather ? 0 : kTnSlabs * n * kBK * 2));
                 const uint32_t tx = 2 * cta_bytes;   // both CTAs' copies count on the even CTA's barrier
                 // FC1: the 64 h columns 128j + 64 rank .. as 4 groups of (16 gate rows, 16 up rows),
                 // the first being 16-row group e*F/8 + (128j + 64 rank)/16 of w_gate_up
@@ -537,7 +568,7 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
                     }
                     if (kFC1) ptx::tma_load_5d_pair(st, &maps.w, 0, 0, 0, fg, kb * kTnSlabs, bar);
                     else ptx::tma_load_3d_pair(st, &maps.w, 0, wrow, kb * kTnSlabs, bar);
-                    ptx::tma_load_3d_pair(st + kTnBytesA, bmap, 0, brow, kb * kTnSlabs, bar);
+                    if (!kGather) ptx::tma_load_3d_pair(st + kTnBytesA, bmap, 0, brow, kb * kTnSlabs, bar);
                     ++fills;
                     if (++stage == kTnStages) { stage = 0; phase ^= 1; }
                 }
@@ -595,6 +626,10 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
                 const uint32_t d_tmem = tmem + (uint32_t)(acc * kN);
                 for (int kb = 0; kb < kb_count; ++kb) {
                     if (!role_wait(&S->full[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
+                    if (kGather && !role_wait_cluster(&S->bfull[stage], phase, a.spin, abort_flag, a.header)) {
+                        ok = false;
+                        break;
+                    }
                     ptx::tc_fence_after();
                     const uint32_t a_addr = ptx::smem_addr(base + stage * kTnStageBytes);
                     const uint32_t b_addr = a_addr + kTnBytesA;
@@ -626,6 +661,92 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
                 ptx::mbar_wait(&S->drain, 0, kDrainBudget);
             }
         }
+    } else if (kGather && warp == kSignalWarp) {
+        // ------------------------------------------------ gather signal (MODE 3), warp 11 of both CTAs
+        if (lane == 0) {
+            const uint32_t bfull0 = ptx::map_to_rank(ptx::smem_addr(&S->bfull[0]), 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                int4 item;
+                uint32_t valid;
+                if (!take_item(k, item, valid)) { ok = false; break; }
+                release_item(k);
+                if (item.x < 0) break;
+                for (int kb = 0; kb < kb_count; ++kb) {
+                    if (!role_wait(&S->gfull[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
+                    // the rows reached shared memory through the generic proxy; the MMAs read them
+                    // through the async proxy
+                    ptx::fence_proxy_async_shared();
+                    if (even) ptx::mbar_arrive(&S->bfull[stage]);
+                    else ptx::mbar_arrive_cluster(bfull0 + (uint32_t)(stage * sizeof(uint64_t)));
+                    if (++stage == kTnStages) { stage = 0; phase ^= 1; }
+                }
+            }
+            if (!ok) abort_pair();
+        }
+    } else if (kGather && warp >= kGatherWarp) {
+        // ------------------------------------------------ row gather (MODE 3), warps 7..10 of both CTAs
+        const int gt = threadIdx.x - kGatherWarp * 32;
+        auto gsync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kGatherThreads) : "memory"); };
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true, bad = false;
+        for (int k = 0; ok; ++k) {
+            if (gt == 0) {
+                int4 item = make_int4(-2, 0, -1, -1);
+                uint32_t valid = 0;
+                const bool got = take_item(k, item, valid);
+                if (got) release_item(k);
+                S->g_item = got ? item : make_int4(-2, 0, -1, -1);
+                S->g_valid = valid;
+            }
+            gsync();   // also: every thread is done with the previous item's g_tok
+            const int4 item = S->g_item;
+            const uint32_t valid = S->g_valid;
+            if (item.x == -2) { ok = false; break; }
+            if (item.x < 0) break;
+            const int n = item_rows((int)(valid & 0xffffu), (int)(valid >> 16), item.w >= 0);
+            const int brow = rank == 0 ? item.z : (item.w >= 0 ? item.w : item.z + n);
+            for (int r = gt; r < n; r += kGatherThreads) {
+                int t = __ldg(a.src_of + brow + r);
+                if (t >= a.T) { bad = true; t = -1; }
+                S->g_tok[r] = t;
+            }
+            gsync();
+            // this thread's 16-byte chunks of the item, the same in every k-step: source row
+            // (null for a padding row) and place in the B tile
+            constexpr int kPer = 128 * 8 * kTnSlabs / kGatherThreads;
+            const __nv_bfloat16* srcp[kPer];
+            uint32_t dsto[kPer];
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int i = gt + j * kGatherThreads;
+                const int r = i >> 4, sl = (i >> 3) & 1, c = i & 7;
+                const int t = i < n * 16 ? S->g_tok[r] : -1;
+                srcp[j] = t >= 0 ? a.x + (int64_t)t * a.d + sl * kBK + c * 8 : nullptr;
+                dsto[j] = (uint32_t)((sl * n + r) * 128 + ((c ^ (r & 7)) << 4));
+            }
+            for (int kb = 0; kb < kb_count; ++kb) {
+                if (gt == 0) S->g_ok = role_wait(&S->empty[stage], phase ^ 1, a.spin, abort_flag, a.header) ? 1 : 0;
+                gsync();
+                if (!S->g_ok) { ok = false; break; }
+                // n rows x kTnSlabs slabs x 8 chunks of 16 bytes; slab sl of row r at
+                // (sl*n + r)*128, chunk c at position c ^ (r % 8) (128-byte swizzle)
+                const uint32_t bs = ptx::smem_addr(base + stage * kTnStageBytes + kTnBytesA);
+                const __nv_bfloat16* xk = a.x + (int64_t)kb * kTnK;
+#pragma unroll
+                for (int j = 0; j < kPer; ++j)
+                    if (srcp[j]) ptx::cp_async16(bs + dsto[j], srcp[j] + (int64_t)kb * kTnK);
+                ptx::cp_async_mbar_arrive_noinc(&S->gfull[stage]);
+                if (++stage == kTnStages) { stage = 0; phase ^= 1; }
+            }
+        }
+        ptx::cp_async_commit();
+        ptx::cp_async_wait<0>();   // nothing may land after the CTA leaves
+        if (!ok && gt == 0) abort_pair();
+        if (bad) set_status(a.header, MOE_DEV_BAD_INDEX);
     } else {
         // ------------------------------------------------ epilogue, warps 2..5 of both CTAs
         const int quad = warp & 3;                 // TMEM lanes 32*quad .. 32*quad+31
@@ -722,18 +843,20 @@ bool make_tmap_slabs(CUtensorMap* tm, const void* p, uint64_t K, uint64_t rows, 
 
 // which = 1: FC1 + SwiGLU, xp [rows_cap, d] x w_gate_up -> h [rows_cap, F];
 // which = 2: FC2, h [rows_cap, F] x w_down -> yp [rows_cap, d], and with
-// fold also the weighted top-k sum of the yp rows into fold->y [T, d].
+// fold also the weighted top-k sum of the yp rows into fold->y [T, d];
+// which = 3: FC1 + SwiGLU with the token rows gathered from x [T, d].
 cudaError_t launch_ffn_tn(const Shape& s, int which, const void* a_mat, const void* w, void* out,
                           const WsPtrs& ws, cudaStream_t st, long long spin_budget, const FoldArgs* fold) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     sms &= ~1;   // whole CTA pairs
-    const bool fc1 = which == 1;
+    const bool gather = which == 3;
+    const bool fc1 = which == 1 || gather;
     const int K = fc1 ? s.d : s.F;
     TnMaps maps;
     memset(&maps, 0, sizeof(maps));
-    for (int m = 0; m < kTnMaps; ++m)
+    for (int m = 0; m < kTnMaps && !gather; ++m)
         if (!make_tmap_slabs(&maps.b[m], a_mat, (uint64_t)K, (uint64_t)s.rows_cap, 16u * (m + 1)))
             return cudaErrorInvalidValue;
     if (fc1 ? !make_tmap_w1_groups(&maps.w, w, s.E, s.F, s.d)
@@ -766,8 +889,14 @@ cudaError_t launch_ffn_tn(const Shape& s, int which, const void* a_mat, const vo
     a.topk_w = fold ? fold->topk_w : nullptr;
     a.arrivals = fold ? fold->arrivals : nullptr;
     a.y = fold ? static_cast<__nv_bfloat16*>(fold->y) : nullptr;
+    a.x = gather ? static_cast<const __nv_bfloat16*>(a_mat) : nullptr;
     if (fold && (fc1 || !fold->topk_w || !fold->arrivals || !fold->y)) return cudaErrorInvalidValue;
     cudaError_t err;
+    if (gather) {
+        err = cudaFuncSetAttribute(ffn_tn_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTnSmemBytes);
+        if (err != cudaSuccess) return err;
+        return launch_pdl(ffn_tn_kernel<3>, dim3(sms), dim3(kThreads + kGatherExtra), kTnSmemBytes, st, maps, a);
+    }
     if (fc1) {
         err = cudaFuncSetAttribute(ffn_tn_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kTnSmemBytes);
         if (err != cudaSuccess) return err;
