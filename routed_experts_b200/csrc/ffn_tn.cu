@@ -735,7 +735,6 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
                 // n rows x kTnSlabs slabs x 8 chunks of 16 bytes; slab sl of row r at
                 // (sl*n + r)*128, chunk c at position c ^ (r % 8) (128-byte swizzle)
                 const uint32_t bs = ptx::smem_addr(base + stage * kTnStageBytes + kTnBytesA);
-                const __nv_bfloat16* xk = a.x + (int64_t)kb * kTnK;
 #pragma unroll
                 for (int j = 0; j < kPer; ++j)
                     if (srcp[j]) ptx::cp_async16(bs + dsto[j], srcp[j] + (int64_t)kb * kTnK);
