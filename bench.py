@@ -3,10 +3,12 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config olmoe] [--impl mine|reference]
 
 One step = one pass of the whole layer (top-k and gating, histogram, planner,
-row maps, dispatch, FC1 + SwiGLU, FC2, combine) over one batch of seeded
+row maps, dispatch, FC1 + SwiGLU, FC2, combine; FC1 reads x itself in place
+of the dispatch when moe_layer_path says so) over one batch of seeded
 synthetic inputs already resident in HBM: one moe_layer_fwd call through the
 C ABI. The stages are timed in a second pass, one ABI call per stage, and
-FC2 with the combine folded in (moe_expert_fc2_combine) in a third. Under torchrun
+FC2 with the combine folded in (moe_expert_fc2_combine) and the other FC1
+input path in further passes. Under torchrun
 every rank runs its own independent layer (its own tokens, replicated
 weights, no collective on the data path: weak scaling); the timed region is
 bracketed by a barrier and a device synchronisation, and the time is the
@@ -38,7 +40,7 @@ from routed_experts_b200 import configs as C  # noqa: E402
 from routed_experts_b200 import inputs as I  # noqa: E402
 
 METRIC = "routed MoE layer tokens/s at 1 B200; % of bf16 tensor / HBM roofline"
-LAUNCHES_PER_STEP = 7   # moe_layer_fwd: topk_hist, plan, row_maps, gather, fc1, fc2, combine
+LAUNCHES_PER_STEP = 7   # moe_layer_fwd: topk_hist, plan, row_maps, dispatch, fc1, fc2, combine (6 when FC1 reads x)
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -607,14 +609,21 @@ def run_mine(args, world, rank, local):
         raise RuntimeError(f"device status {st} after the timed steps")
     del layer
 
-    # the same kernels, one ABI call per stage, so that each stage can be timed
-    def stages(evs, fold_fc2=False):
+    # the same kernels, one ABI call per stage, so that each stage can be timed;
+    # the FC1 input path is the one moe_layer_fwd takes for this shape (no
+    # dispatch stage when FC1 reads x itself), or with dispatch=True the other
+    gather = M.moe_layer_path(cfg) == M.PATH_GATHER_FC1
+    def stages(evs, fold_fc2=False, dispatch=False):
         evs[0].record(stream)
         M.moe_plan(cfg, lg, idx, w, counts, ws, stream)
         evs[1].record(stream)
-        M.moe_dispatch(cfg, x, xp, ws, stream)
-        evs[2].record(stream)
-        M.moe_expert_fc1(cfg, xp, wgu, h, ws, stream)
+        if gather and not dispatch:
+            evs[2].record(stream)
+            M.moe_expert_fc1_gather(cfg, x, wgu, h, ws, stream)
+        else:
+            M.moe_dispatch(cfg, x, xp, ws, stream)
+            evs[2].record(stream)
+            M.moe_expert_fc1(cfg, xp, wgu, h, ws, stream)
         evs[3].record(stream)
         if fold_fc2:
             M.moe_expert_fc2_combine(cfg, h, wdn, w, yp, out, ws, stream)
@@ -625,12 +634,12 @@ def run_mine(args, world, rank, local):
         M.moe_combine(cfg, yp, w, out, ws, stream)
         evs[5].record(stream)
 
-    def time_stages(fold_fc2):
+    def time_stages(fold_fc2, dispatch=False):
         n = 5 if fold_fc2 else 6
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps + args.warmup)]
         torch.cuda.synchronize(dev)
         for e in evs:
-            stages(e, fold_fc2)
+            stages(e, fold_fc2, dispatch)
         torch.cuda.synchronize(dev)
         st_ = M.moe_read_status(ws, stream)
         if st_ & (M.DEV_TIMEOUT | M.DEV_BAD_INDEX):
@@ -638,6 +647,7 @@ def run_mine(args, world, rank, local):
         return np.array([[e[i].elapsed_time(e[i + 1]) for i in range(n - 1)] for e in evs[args.warmup:]])
 
     fold_ms = time_stages(True) if fold else None
+    disp_ms = time_stages(False, dispatch=True) if gather else None
     stage_ms = time_stages(False)
     plan = M.read_plan(cfg, ws)
 
@@ -686,13 +696,16 @@ def run_mine(args, world, rank, local):
     torch.cuda.synchronize(dev)
     e2e_serial_ms = e0.elapsed_time(e1)
 
-    # the same calls as a serving loop issues them: two workspaces on two
-    # streams, steps alternating, so one step's copies overlap the other's kernels
-    layers = [layer_h, M.Layer(cfg, dev, host_io=True)]
-    streams = [torch.cuda.Stream(dev), torch.cuda.Stream(dev)]
-    outs = [out_h, torch.empty(T, d, dtype=dt).pin_memory()]
+    # the same calls as a serving loop issues them: three workspaces on three
+    # streams, steps in turn, so a step's input copy, another's kernels and a
+    # third's output copy run at once (with two, a stream's next input copy
+    # waits for its previous output copy)
+    NS = 3
+    layers = [layer_h] + [M.Layer(cfg, dev, host_io=True) for _ in range(NS - 1)]
+    streams = [torch.cuda.Stream(dev) for _ in range(NS)]
+    outs = [out_h] + [torch.empty(T, d, dtype=dt).pin_memory() for _ in range(NS - 1)]
     for k in range(args.warmup):
-        layers[k % 2].forward_host(lg_h, x_h, wgu, wdn, outs[k % 2], streams[k % 2])
+        layers[k % NS].forward_host(lg_h, x_h, wgu, wdn, outs[k % NS], streams[k % NS])
     if pg is not None:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
@@ -700,7 +713,7 @@ def run_mine(args, world, rank, local):
     for s_ in streams:
         s_.wait_event(e0)
     for k in range(args.steps):
-        layers[k % 2].forward_host(lg_h, x_h, wgu, wdn, outs[k % 2], streams[k % 2])
+        layers[k % NS].forward_host(lg_h, x_h, wgu, wdn, outs[k % NS], streams[k % NS])
     for s_ in streams:
         done = torch.cuda.Event()
         done.record(s_)
@@ -774,17 +787,24 @@ def run_mine(args, world, rank, local):
         "dtype": "bf16" if cfg.dtype == C.BF16 else "fp32",
         "data": "synthetic (seeded SplitMix64 + Box-Muller inputs, the recipe in routed_experts_b200/inputs.py)",
         "config": bench_config(cfg, args.seed, world),
-        "roofline": {"bound": "tensor", "kernel": "ffn_tn_kernel<0> (FC1 + SwiGLU)",
+        "roofline": {"bound": "tensor",
+                     "kernel": "ffn_tn_kernel<3> (FC1 + SwiGLU reading x)" if gather else "ffn_tn_kernel<0> (FC1 + SwiGLU)",
                      "achieved": fc1_flop / fc1_s / 1e12, "peak": tensor_peak, "unit": "TFLOP/s",
                      "frac": fc1_flop / fc1_s / 1e12 / tensor_peak,
-                     "traffic": ncu_traffic(f"fc1@{cfg.name}"),
+                     "traffic": ncu_traffic(f"{'fc1_gather' if gather else 'fc1'}@{cfg.name}"),
                      "peak_kind": f"{pk_kind} bf16 burst",
                      "flop_per_launch": fc1_flop, "launch_ms": mean[2]},
         "layer_roofline": {"frac": (t_roof * 1e3) / ms_per_step, "roofline_ms": t_roof * 1e3,
                            "flop": layer_flop, "alg_bytes": alg_bytes,
                            "peaks": {"bf16_tflops": tensor_peak, "hbm_gbs": pk["hbm_gbs"], "kind": pk_kind}},
-        "stages_ms": {"plan(topk+hist+plan+rowmaps)": med[0], "dispatch": med[1], "fc1": med[2], "fc2": med[3],
-                      "combine": med[4]},
+        "stages_ms": ({"plan(topk+hist+plan+rowmaps)": med[0], "fc1 (reading x, no dispatch)": med[2],
+                       "fc2": med[3], "combine": med[4]} if gather else
+                      {"plan(topk+hist+plan+rowmaps)": med[0], "dispatch": med[1], "fc1": med[2], "fc2": med[3],
+                       "combine": med[4]}),
+        "fc1_input_paths_ms": None if disp_ms is None else {
+            "fc1_reading_x": float(med[2]), "dispatch": float(np.median(disp_ms[:, 1])),
+            "fc1_after_dispatch": float(np.median(disp_ms[:, 2])),
+            "note": "moe_expert_fc1_gather (the layer's path for this shape) against moe_dispatch + moe_expert_fc1"},
         "fc2_combine_fold_ms": None if fold_ms is None else {
             "median": float(np.median(fold_ms[:, 3])), "separate_fc2_plus_combine": float(med[3] + med[4]),
             "note": "moe_expert_fc2_combine (FC2 with the top-k sum in its epilogue, bit-identical; its call "
@@ -792,7 +812,8 @@ def run_mine(args, world, rank, local):
         "step_ms": {"median": float(np.median(step_ms)), "min": float(step_ms.min()),
                     "max": float(step_ms.max())},
         "stage_rates": {"fc1_tflops": fc1_flop / fc1_s / 1e12, "fc2_tflops": fc2_flop / fc2_s / 1e12,
-                        "dispatch_gbs": gather_bytes / (mean[1] * 1e-3) / 1e9,
+                        "dispatch_gbs": (gather_bytes / (float(disp_ms[:, 1].mean()) * 1e-3) / 1e9 if gather else
+                                         gather_bytes / (mean[1] * 1e-3) / 1e9),
                         "combine_gbs": combine_bytes / (mean[4] * 1e-3) / 1e9},
         "plan": {"moves": plan["moves"], "replicas": plan["replicas"], "status": plan["status"],
                  "padded_rows": plan["total_rows"] - N, "blocks": plan["n_blocks"]},
@@ -802,11 +823,13 @@ def run_mine(args, world, rank, local):
                 "h2d_bytes_per_step": 4 * T * E + T * d * eb, "d2h_bytes_per_step": T * d * eb,
                 "ms_per_step": e2e_ms / args.steps,
                 "path": "moe_layer_fwd_host per step (H2D of logits and x from pinned memory, the layer, D2H of "
-                        "out), two workspaces on two streams with steps alternating",
+                        "out), three workspaces on three streams with steps in turn",
                 "one_stream_value": world * T / (e2e_serial_ms / args.steps * 1e-3),
                 "one_stream_ms_per_step": e2e_serial_ms / args.steps},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
-        "layer_path": "moe_layer_fwd: top-k + histogram, plan, row maps, dispatch, FC1 + SwiGLU, FC2, combine",
+        "gpu_launches": (LAUNCHES_PER_STEP - (1 if gather else 0)) * args.steps,
+        "layer_path": ("moe_layer_fwd: top-k + histogram, plan, row maps, FC1 + SwiGLU reading x through the row "
+                       "map, FC2, combine" if gather else
+                       "moe_layer_fwd: top-k + histogram, plan, row maps, dispatch, FC1 + SwiGLU, FC2, combine"),
         "backward": bwd,
         "mx": mx,
         "mx_fp4_weights": mx4,

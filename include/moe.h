@@ -289,10 +289,22 @@ moe_status moe_combine(const moe_config* cfg, const void* yp, const float* topk_
 moe_status moe_expert_fc2_combine(const moe_config* cfg, const void* h, const void* w_down, const float* topk_w,
                                   void* yp, void* out, void* ws, size_t ws_bytes, moe_stream_t stream);
 
+/* Which FC1 input path moe_layer_fwd takes for a shape. */
+enum {
+    MOE_PATH_DISPATCH = 0,   /* moe_dispatch, then moe_expert_fc1 */
+    MOE_PATH_GATHER_FC1 = 1  /* moe_expert_fc1_gather (no dispatch launch, xp unused) */
+};
+/* moe_layer_path - *path = the moe_layer_fwd FC1 input path of cfg (host only). */
+moe_status moe_layer_path(const moe_config* cfg, int32_t* path);
+
 /*
  * moe_layer_fwd - the whole layer, A1 to A9, on device buffers, with
  * top-k, xp, h and yp carved from a MOE_WS_LAYER workspace: the kernels of
- * moe_plan, moe_dispatch, moe_expert_fc1, moe_expert_fc2 and moe_combine.
+ * moe_plan, then moe_dispatch and moe_expert_fc1 or, for bf16 layers whose
+ * x [T, d] takes at most 64 MiB, moe_expert_fc1_gather in their place (x
+ * then stays in L2 and the gathered FC1 is as fast or faster; the result is
+ * bit-identical either way), then moe_expert_fc2 and moe_combine. The
+ * launches are chained (programmatic dependent launch) on the stream.
  */
 moe_status moe_layer_fwd(const moe_config* cfg, const float* logits, const void* x,
                          const void* w_gate_up, const void* w_down, void* out, void* ws,

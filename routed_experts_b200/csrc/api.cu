@@ -125,6 +125,13 @@ moe_status ffn_impl(const Shape& s, const WsLayout& L, const void* xp, const voi
     return fc_impl(s, L, 2, h, wdn, yp, ws, st);
 }
 
+// moe_layer_fwd reads FC1's token rows straight from x (no dispatch launch,
+// no xp) when x is small enough to stay in L2 beside the streaming weights:
+// there the gathered FC1 measured as fast as dispatch + FC1 or faster, and
+// with a larger x (whose rows it reads scattered from DRAM) slower.
+constexpr int64_t kGatherMaxXBytes = (int64_t)64 << 20;
+bool layer_gathers(const Shape& s) { return s.dtype == MOE_BF16 && (int64_t)s.T * s.d * s.eb <= kGatherMaxXBytes; }
+
 moe_status mx_shape(const moe_config* cfg, Shape* s) {
     moe_status r = make_shape(cfg, s);
     if (r != MOE_OK) return r;
@@ -357,9 +364,24 @@ moe_status moe_layer_fwd(const moe_config* cfg, const float* logits, const void*
     void* yp = b + L.yp;
     if ((r = plan_impl(s, L, logits, idx, w, counts, ws, st)) != MOE_OK) return r;
     const WsPtrs P = ws_ptrs(ws, L);
+    if (layer_gathers(s)) {
+        cudaError_t e = launch_ffn_tc(s, 3, x, w_gate_up, h, P, st, kSpinBudget);   // FC1 reading x
+        if (e == cudaSuccess) e = launch_ffn_tc(s, 2, h, w_down, yp, P, st, kSpinBudget);
+        if (e == cudaSuccess) e = launch_combine(s, yp, w, out, P, st);
+        return from_cuda(e);
+    }
     if ((r = from_cuda(launch_gather(s, x, xp, P, st))) != MOE_OK) return r;
     if ((r = ffn_impl(s, L, xp, w_gate_up, w_down, h, yp, ws, st)) != MOE_OK) return r;
     return from_cuda(launch_combine(s, yp, w, out, P, st));
+}
+
+moe_status moe_layer_path(const moe_config* cfg, int32_t* path) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (!path) return MOE_ERR_INVALID_ARG;
+    *path = layer_gathers(s) ? MOE_PATH_GATHER_FC1 : MOE_PATH_DISPATCH;
+    return MOE_OK;
 }
 
 moe_status moe_layer_fwd_train(const moe_config* cfg, const float* logits, const void* x, const void* w_gate_up,

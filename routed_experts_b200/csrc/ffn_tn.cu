@@ -76,8 +76,13 @@
 // arrive); a fifth warp waits on it, fences the async proxy and signals the
 // stage's row barrier on the even CTA, which the MMA thread waits on beside
 // the weights' TMA barrier. The copying warps never wait for their own
-// copies, so all stages of the ring can be in flight, as with TMA. Padding
-// rows are not copied: their accumulator columns are never stored.
+// copies, so all stages of the ring can be in flight, as with TMA. The even
+// CTA's signal is a local arrive that also expects 16 bytes; the odd CTA's is
+// a 16-byte shared-to-shared bulk copy into the even CTA that completes those
+// bytes on the same barrier. (A cluster-scope release arrive from the odd
+// CTA cost about a microsecond per stage, and the MMA waited on it nearly
+// half of the time.) Padding rows are not copied: their accumulator columns
+// are never stored.
 #include <cudaTypedefs.h>
 #include <string.h>
 
@@ -119,6 +124,10 @@ struct TnSmem {
     uint32_t g_valid;
     int g_ok;
     int32_t g_tok[128];           // MODE 3: token of each of this CTA's rows of the item (-1: padding)
+    alignas(16) uint32_t sig_src[4];              // MODE 3 (odd CTA): source of the 16-byte signal copies
+    alignas(16) uint32_t sig_dst[kTnStages][4];   // MODE 3 (even CTA): their destinations, one per stage
+    uint64_t sig_done;            // MODE 3 (even CTA): the odd CTA's signal thread has stopped
+    long long sig_fills;          // MODE 3 (even CTA): how many signal copies it issued
     uint32_t odd_bytes[kTnStages], peer_bytes[kTnStages];
     long long odd_fills;
     uint32_t tmem_base;
@@ -405,11 +414,12 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
             ptx::mbar_init(&S->fwd_empty[q], kOddConsumers + (kGather ? 2 : 0));
         }
         for (int s_ = 0; s_ < kTnStages; ++s_) {
-            ptx::mbar_init(&S->bfull[s_], 2);                 // one arrival per CTA
+            ptx::mbar_init(&S->bfull[s_], 1);                 // the even signal, + 16 bytes from the odd CTA
             ptx::mbar_init(&S->gfull[s_], kGatherThreads);    // one per gather thread
         }
         ptx::mbar_init(&S->drain, 1);
         ptx::mbar_init(&S->odd_done, 1);
+        ptx::mbar_init(&S->sig_done, 1);
         S->abort_flag = 0;
         ptx::fence_barrier_init();
     }
@@ -668,23 +678,51 @@ ffn_tn_kernel(const __grid_constant__ TnMaps maps, TnArgs a) {
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
+            long long fills = 0;   // stages signalled
             for (int k = 0; ok; ++k) {
                 int4 item;
                 uint32_t valid;
                 if (!take_item(k, item, valid)) { ok = false; break; }
                 release_item(k);
                 if (item.x < 0) break;
-                for (int kb = 0; kb < kb_count; ++kb) {
+                for (int kb = 0; kb < kb_count; ++kb, ++fills) {
                     if (!role_wait(&S->gfull[stage], phase, a.spin, abort_flag, a.header)) { ok = false; break; }
                     // the rows reached shared memory through the generic proxy; the MMAs read them
                     // through the async proxy
                     ptx::fence_proxy_async_shared();
-                    if (even) ptx::mbar_arrive(&S->bfull[stage]);
-                    else ptx::mbar_arrive_cluster(bfull0 + (uint32_t)(stage * sizeof(uint64_t)));
+                    if (even) {
+                        ptx::mbar_arrive_expect_tx(&S->bfull[stage], 16u);
+                    } else {
+                        ptx::bulk_copy_s2c(ptx::map_to_rank(ptx::smem_addr(&S->sig_dst[stage][0]), 0),
+                                           ptx::smem_addr(&S->sig_src[0]), 16u,
+                                           bfull0 + (uint32_t)(stage * sizeof(uint64_t)));
+                    }
                     if (++stage == kTnStages) { stage = 0; phase ^= 1; }
                 }
             }
             if (!ok) abort_pair();
+            if (!even) {
+                // tell the even CTA how many signal copies this CTA issued
+                const uint32_t fa = ptx::map_to_rank(ptx::smem_addr(&S->sig_fills), 0);
+                ptx::st_cluster_u32(fa, (uint32_t)(fills & 0xffffffffll));
+                ptx::st_cluster_u32(fa + 4, (uint32_t)(fills >> 32));
+                ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_addr(&S->sig_done), 0));
+            } else {
+                // Every signal copy of the odd CTA lands before the CTAs leave. After a
+                // complete run the MMA thread has waited for every stage; after a stop,
+                // wait for the phases the odd CTA sent bytes to: this thread's last
+                // arrival on each stage, and (armed here) the odd CTA's signals past them.
+                if (ptx::mbar_wait_cluster(&S->sig_done, 0, kDrainBudget)) {
+                    const long long fo = *reinterpret_cast<volatile long long*>(&S->sig_fills);
+                    const long long first = fills > kTnStages ? fills - kTnStages : 0;
+                    for (long long f = first; f < fills && f < fo; ++f)
+                        ptx::mbar_wait(&S->bfull[f % kTnStages], (uint32_t)((f / kTnStages) & 1), kDrainBudget);
+                    for (long long f = fills; f < fo; ++f) {
+                        ptx::mbar_arrive_expect_tx(&S->bfull[f % kTnStages], 16u);
+                        ptx::mbar_wait(&S->bfull[f % kTnStages], (uint32_t)((f / kTnStages) & 1), kDrainBudget);
+                    }
+                }
+            }
         }
     } else if (kGather && warp >= kGatherWarp) {
         // ------------------------------------------------ row gather (MODE 3), warps 7..10 of both CTAs

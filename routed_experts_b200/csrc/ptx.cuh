@@ -134,6 +134,16 @@ __device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned)
+// from this CTA's shared memory to a CTA of the cluster (shared::cluster
+// addresses of the destination and of its mbarrier), completing the bytes
+// on that mbarrier.
+__device__ __forceinline__ void bulk_copy_s2c(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(dst), "r"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
 // 16-byte asynchronous copy global -> shared, cached in L2 only; completion
 // is tracked per thread by commit groups.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {

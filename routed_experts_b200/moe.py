@@ -21,6 +21,7 @@ DEV_PLAN_INEXACT, DEV_TIMEOUT, DEV_BAD_INDEX = 1, 2, 4
 WS_PLAN, WS_LAYER, WS_LAYER_HOST, WS_LAYER_TRAIN = 0, 1, 2, 3
 MX_XQ, MX_XS, MX_HQ, MX_HS, MX_W1Q, MX_W1S, MX_W2Q, MX_W2S = range(8)
 MX_W_E4M3, MX_W_E2M1 = 0, 1   # weight element formats: MXFP8, MXFP4
+PATH_DISPATCH, PATH_GATHER_FC1 = 0, 1   # moe_layer_fwd's FC1 input path
 
 
 class MoeError(RuntimeError):
@@ -67,6 +68,7 @@ def lib() -> ctypes.CDLL:
         L.moe_combine.argtypes = [C, P, P, P, P, S, P]
         L.moe_expert_fc2_combine.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd.argtypes = [C, P, P, P, P, P, P, S, P]
+        L.moe_layer_path.argtypes = [C, ctypes.POINTER(ctypes.c_int32)]
         L.moe_layer_fwd_host.argtypes = [C, P, P, P, P, P, P, S, P]
         L.moe_layer_bwd.argtypes = [C, P, P, P, P, P, P, P, P, P, S, P]
         L.moe_layer_fwd_train.argtypes = [C, P, P, P, P, P, P, S, P]
@@ -86,7 +88,7 @@ def lib() -> ctypes.CDLL:
         for f in ("moe_workspace_size", "moe_rows_capacity", "moe_plan_view", "moe_plan", "moe_dispatch",
                   "moe_expert_ffn", "moe_expert_ffn_fused", "moe_expert_ffn_fused_gather", "moe_expert_fc1", "moe_expert_fc2", "moe_expert_fc1_gather", "moe_combine",
                   "moe_expert_fc2_combine",
-                  "moe_layer_fwd", "moe_layer_bwd", "moe_layer_fwd_train",
+                  "moe_layer_fwd", "moe_layer_path", "moe_layer_bwd", "moe_layer_fwd_train",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait",
                   "moe_probe_expert_ffn_timeout",
                   "moe_mx_buffer_bytes", "moe_mx_quantize_weights", "moe_dispatch_mx", "moe_expert_fc1_mx",
@@ -132,6 +134,13 @@ def _ws(ws: torch.Tensor):
 
 
 # ---------------------------------------------------------------- the C calls
+
+def moe_layer_path(c) -> int:
+    """PATH_GATHER_FC1 when moe_layer_fwd reads FC1's rows straight from x, else PATH_DISPATCH."""
+    p = ctypes.c_int32(-1)
+    _check(lib().moe_layer_path(ctypes.byref(config(c)), ctypes.byref(p)), "moe_layer_path")
+    return p.value
+
 
 def moe_workspace_size(c, kind: int = WS_PLAN) -> int:
     n = ctypes.c_size_t(0)

@@ -225,3 +225,14 @@ def test_binding_refuses_to_run_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(moe, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         moe.lib()
+
+
+@pytest.mark.parametrize("cfg", list(C.NAMED.values()), ids=lambda c: c.name)
+def test_layer_path_of_named_configs(M, cfg):
+    """moe_layer_fwd reads FC1's rows straight from x for bf16 layers whose x
+    takes at most 64 MiB (OLMoE and Qwen3 here), through the dispatch otherwise."""
+    small_x = cfg.T * cfg.d * cfg.elem_bytes <= 64 << 20
+    want = M.PATH_GATHER_FC1 if cfg.dtype == C.BF16 and small_x else M.PATH_DISPATCH
+    assert M.moe_layer_path(cfg) == want
+    assert {"olmoe": M.PATH_GATHER_FC1, "qwen3": M.PATH_GATHER_FC1, "extreme": M.PATH_DISPATCH,
+            "dsv3": M.PATH_DISPATCH}.get(cfg.name, want) == want
