@@ -525,6 +525,17 @@ moe_status moe_probe_expert_ffn_timeout(const moe_config* cfg, const void* xp, c
                                         const void* w_down, void* h, void* yp, void* ws, size_t ws_bytes,
                                         int64_t budget_cycles, moe_stream_t stream);
 
+/*
+ * moe_probe_fc1_gather_timeout - the same check for moe_expert_fc1_gather
+ * (FC1 reading x [T, d] through the row map; bf16 layers): every
+ * device-side wait of its kernel, including those of its row-gather and
+ * signal warps, gets budget_cycles clock cycles (1 .. 2^34). A stop drains
+ * the row copies and the stage signals in flight before the CTAs leave. h
+ * is then undefined; the next call runs normally. No papers' counterpart.
+ */
+moe_status moe_probe_fc1_gather_timeout(const moe_config* cfg, const void* x, const void* w_gate_up, void* h,
+                                        void* ws, size_t ws_bytes, int64_t budget_cycles, moe_stream_t stream);
+
 /* A static string naming a moe_status. */
 const char* moe_status_string(moe_status s);
 

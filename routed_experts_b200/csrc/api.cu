@@ -618,6 +618,20 @@ moe_status moe_probe_expert_ffn_timeout(const moe_config* cfg, const void* xp, c
     return from_cuda(e);
 }
 
+moe_status moe_probe_fc1_gather_timeout(const moe_config* cfg, const void* x, const void* w_gate_up, void* h,
+                                        void* ws, size_t ws_bytes, int64_t budget_cycles, moe_stream_t stream) {
+    Shape s;
+    moe_status r = make_shape(cfg, &s);
+    if (r != MOE_OK) return r;
+    if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (budget_cycles < 1 || budget_cycles > ((int64_t)1 << 34)) return MOE_ERR_INVALID_ARG;
+    if (!x || !w_gate_up || !h || !aligned16(x) || !aligned16(w_gate_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
+    const WsLayout L = make_layout(s);
+    if ((r = check_ws(ws, ws_bytes, L.plan_end)) != MOE_OK) return r;
+    return from_cuda(launch_ffn_tn(s, 3, x, w_gate_up, h, ws_ptrs(ws, L), reinterpret_cast<cudaStream_t>(stream),
+                                   (long long)budget_cycles));
+}
+
 const char* moe_status_string(moe_status s) {
     switch (s) {
         case MOE_OK: return "MOE_OK";

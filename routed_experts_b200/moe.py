@@ -76,6 +76,7 @@ def lib() -> ctypes.CDLL:
         L.moe_plan_noalloc.argtypes = [C, P, P, P, P, P, P, P]
         L.moe_probe_bounded_wait.argtypes = [P, ctypes.c_int64, P]
         L.moe_probe_expert_ffn_timeout.argtypes = [C, P, P, P, P, P, P, S, ctypes.c_int64, P]
+        L.moe_probe_fc1_gather_timeout.argtypes = [C, P, P, P, P, S, ctypes.c_int64, P]
         L.moe_status_string.argtypes = [ctypes.c_int]
         I32 = ctypes.c_int32
         L.moe_mx_buffer_bytes.argtypes = [C, I32, I32, ctypes.POINTER(ctypes.c_size_t)]
@@ -90,7 +91,7 @@ def lib() -> ctypes.CDLL:
                   "moe_expert_fc2_combine",
                   "moe_layer_fwd", "moe_layer_path", "moe_layer_bwd", "moe_layer_fwd_train",
                   "moe_layer_fwd_host", "moe_read_status", "moe_plan_noalloc", "moe_probe_bounded_wait",
-                  "moe_probe_expert_ffn_timeout",
+                  "moe_probe_expert_ffn_timeout", "moe_probe_fc1_gather_timeout",
                   "moe_mx_buffer_bytes", "moe_mx_quantize_weights", "moe_dispatch_mx", "moe_expert_fc1_mx",
                   "moe_expert_fc2_mx", "moe_layer_fwd_mx"):
             getattr(L, f).restype = ctypes.c_int
@@ -267,6 +268,14 @@ def moe_probe_expert_ffn_timeout(c, xp, w_gate_up, w_down, h, yp, ws, budget_cyc
     _check(lib().moe_probe_expert_ffn_timeout(ctypes.byref(config(c)), _ptr(xp), _ptr(w_gate_up), _ptr(w_down),
                                               _ptr(h), _ptr(yp), p, n, ctypes.c_int64(int(budget_cycles)),
                                               _stream(stream)), "moe_probe_expert_ffn_timeout")
+
+
+def moe_probe_fc1_gather_timeout(c, x, w_gate_up, h, ws, budget_cycles: int, stream=None):
+    """moe_expert_fc1_gather with every device-side wait limited to budget_cycles (a failure-handling check)."""
+    p, n = _ws(ws)
+    _check(lib().moe_probe_fc1_gather_timeout(ctypes.byref(config(c)), _ptr(x), _ptr(w_gate_up), _ptr(h), p, n,
+                                              ctypes.c_int64(int(budget_cycles)), _stream(stream)),
+           "moe_probe_fc1_gather_timeout")
 
 
 def moe_read_status(ws, stream=None) -> int:

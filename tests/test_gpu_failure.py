@@ -101,3 +101,28 @@ def test_expert_ffn_timeout_probe_rejects_bad_arguments():
             M.moe_probe_expert_ffn_timeout(SMALL, x, x, x, x, x, ws, budget)
     with pytest.raises(M.MoeError):
         M.moe_probe_expert_ffn_timeout(C.TINY, x, x, x, x, x, ws, 100)
+
+
+@pytest.mark.parametrize("budget", [1, 300, 3000])
+def test_fc1_gather_timeout_path_returns_and_recovers(budget):
+    """The FC1 that reads x (row-gather and signal warps besides the TMA and
+    MMA threads) with every wait cut short: it stops, drains its row copies
+    and stage signals, and the next call on the same workspace is right."""
+    from routed_experts_b200 import inputs as I
+    from .gpu_helpers import run_path
+    inp = I.make_inputs(MED, 8, "cuda")
+    ref = run_path(MED, inp, "fc1_gather")
+    assert ref["status"] & M.DEV_TIMEOUT == 0
+    h = torch.zeros_like(ref["h"])
+    t0 = time.perf_counter()
+    for _ in range(3):
+        M.moe_probe_fc1_gather_timeout(MED, inp["x"], inp["w_gate_up"], h, ref["ws"], budget)
+    status = M.moe_read_status(ref["ws"])
+    assert time.perf_counter() - t0 < 60.0
+    if budget == 1:
+        assert status & M.DEV_TIMEOUT
+    M.moe_plan(MED, inp["logits"], ref["idx"], ref["w"], ref["counts"], ref["ws"])
+    M.moe_expert_fc1_gather(MED, inp["x"], inp["w_gate_up"], h, ref["ws"])
+    assert M.moe_read_status(ref["ws"]) & ~M.DEV_PLAN_INEXACT == 0
+    valid = torch.as_tensor((ref["plan"]["src_of"].numpy() >= 0).nonzero()[0], device="cuda")
+    assert torch.equal(h[valid], ref["h"][valid])
