@@ -200,6 +200,15 @@ def test_qwen3_skew_sweep(cfg):
 FUSED_PATHS = ["fused", "fused_gather", "fc1_gather", "fc2_combine", "layer"]
 
 
+@pytest.mark.parametrize("path", ["layer", "fc1_gather"])
+def test_full_size_qwen3_layer_reading_x(path):
+    """The Qwen3-shaped layer's x takes exactly 64 MiB: moe_layer_fwd reads
+    FC1's rows from x there too."""
+    assert M.moe_layer_path(C.QWEN3) == M.PATH_GATHER_FC1
+    check_full_size(C.QWEN3, 3, path=path, n_tokens=32)
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("path", FUSED_PATHS)
 @pytest.mark.parametrize("cfg", [C.OLMOE, C.DSV3], ids=lambda c: c.name)
 def test_full_size_other_paths(cfg, path):
@@ -229,6 +238,28 @@ FOLD_EDGE = [SMALL_BF16.replace(name="k1", K=1), EDGE[5], EDGE[3], EDGE[0]]
 @pytest.mark.parametrize("cfg", FOLD_EDGE, ids=lambda c: c.name)
 def test_fc2_combine_edge_shapes(cfg):
     check_full_small(cfg, 2, path="fc2_combine")
+
+
+# FC1 reading x (the layer's path for bf16 layers whose x is at most 64 MiB)
+# on the edge shapes: ragged chunks, K = E, E = R, one token per rank, a hot
+# expert, E = 1024 with K = 16.
+EDGE_BF16 = [c for c in EDGE if c.dtype == C.BF16]
+
+
+@pytest.mark.parametrize("cfg", EDGE_BF16, ids=lambda c: c.name)
+def test_fc1_gather_edge_shapes(cfg):
+    check_full_small(cfg, 2, path="fc1_gather")
+
+
+@pytest.mark.parametrize("cfg", EDGE_BF16, ids=lambda c: c.name)
+def test_layer_matches_staged_calls_on_edge_shapes(cfg):
+    assert M.moe_layer_path(cfg) == M.PATH_GATHER_FC1
+    inp = I.make_inputs(cfg, 4, "cuda")
+    staged = run_stages(cfg, inp)["out"]
+    layer = M.Layer(cfg)
+    out = layer.forward(inp["logits"], inp["x"], inp["w_gate_up"], inp["w_down"])
+    assert layer.status() & ~M.DEV_PLAN_INEXACT == 0
+    assert torch.equal(out, staged)
 
 
 @pytest.mark.parametrize("cfg", [SMALL_BF16, MED_BF16, WIDE_BF16, RING_BF16, C.OLMOE, C.DSV3],
